@@ -1,0 +1,247 @@
+"""CPU oracle for the bit-packed VQ/RVQ linear layer -- TEST INFRASTRUCTURE.
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg may import this package.  The product (``bit_packed_index_b200``) never
+does, and nothing here imports the product: the two share only the seeded
+input generators in ``synth``.
+
+The arithmetic lives in ``vq_oracle.c`` (plain C, built here with gcc into
+``liboracle.so``); this module marshals numpy arrays for it.  What each
+routine computes, and the page passage it follows, is documented in the C
+file.  Functions pinned by the not-gpu tests: the conversions, unpack/pack,
+dequant, matmul/linear and the encoders.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+import threading
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "vq_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+GCC_FLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+             "-shared", "-fPIC", "-Wall", "-Wextra"]
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so next to its source (skipped when up to date)."""
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    tmp = _LIB + f".tmp{os.getpid()}"
+    subprocess.run(["gcc", *GCC_FLAGS, "-o", tmp, _SRC, "-lm"], check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Layer(C.Structure):
+    _fields_ = [
+        ("out_features", C.c_int64), ("in_features", C.c_int64),
+        ("d", C.c_int32), ("n_books", C.c_int32), ("log2k", C.c_int32 * 2),
+        ("idx", C.c_void_p * 2), ("row_words", C.c_int64 * 2),
+        ("codebook", C.c_void_p * 2), ("scale", C.c_void_p), ("bias", C.c_void_p),
+    ]
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = C.CDLL(build())
+            P, I64, I32 = C.c_void_p, C.c_int64, C.c_int
+            sig = {
+                "vqo_f32_to_f16_array": [P, P, I64], "vqo_f16_to_f32_array": [P, P, I64],
+                "vqo_f32_to_bf16_array": [P, P, I64], "vqo_bf16_to_f32_array": [P, P, I64],
+                "vqo_unpack": [P, I64, I64, I32, I64, P],
+                "vqo_pack": [P, I64, I64, I32, I64, P],
+                "vqo_dequant": [P, P, I64],
+                "vqo_dequant_rows": [P, P, I64, P, I64],
+                "vqo_matmul": [I64, I64, I64, P, I32, I64, P, I64, P, I64],
+                "vqo_linear": [P, P, I32, I64, I64, P, I64, P, I64],
+                "vqo_encode": [P, I64, I32, P, I64, P],
+                "vqo_encode_residual": [P, I64, I32, P, I64, P, I64, P, P],
+                "vqo_encode_joint": [P, I64, I32, P, I64, P, I64, P, P],
+                "vqo_num_threads": [],
+            }
+            for name, args in sig.items():
+                fn = getattr(lib, name)
+                fn.argtypes = args
+                fn.restype = None if name.endswith("_array") else C.c_int
+            _lib = lib
+    return _lib
+
+
+def _p(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+def _check(rc: int, what: str):
+    if rc:
+        raise ValueError(f"oracle {what} rejected its arguments (code {rc})")
+
+
+# -- conversions ------------------------------------------------------------
+
+def f32_to_f16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a, np.float32)
+    out = np.empty(a.shape, np.uint16)
+    _load().vqo_f32_to_f16_array(_p(a), _p(out), a.size)
+    return out
+
+
+def f16_to_f32(h) -> np.ndarray:
+    h = np.ascontiguousarray(h, np.uint16)
+    out = np.empty(h.shape, np.float32)
+    _load().vqo_f16_to_f32_array(_p(h), _p(out), h.size)
+    return out
+
+
+def f32_to_bf16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a, np.float32)
+    out = np.empty(a.shape, np.uint16)
+    _load().vqo_f32_to_bf16_array(_p(a), _p(out), a.size)
+    return out
+
+
+def bf16_to_f32(h) -> np.ndarray:
+    h = np.ascontiguousarray(h, np.uint16)
+    out = np.empty(h.shape, np.float32)
+    _load().vqo_bf16_to_f32_array(_p(h), _p(out), h.size)
+    return out
+
+
+# -- index streams ----------------------------------------------------------
+
+def unpack(words: np.ndarray, b: int, nvec: int) -> np.ndarray:
+    words = np.ascontiguousarray(words, np.uint32)
+    n, rw = words.shape
+    out = np.empty((n, nvec), np.uint32)
+    _check(_load().vqo_unpack(_p(words), n, rw, b, nvec, _p(out)), "unpack")
+    return out
+
+
+def pack(idx: np.ndarray, b: int, row_words: Optional[int] = None) -> np.ndarray:
+    idx = np.ascontiguousarray(idx, np.uint32)
+    n, nvec = idx.shape
+    if row_words is None:
+        row_words = -(-(nvec * b) // 128) * 4
+    out = np.empty((n, row_words), np.uint32)
+    _check(_load().vqo_pack(_p(idx), n, nvec, b, row_words, _p(out)), "pack")
+    return out
+
+
+# -- the layer --------------------------------------------------------------
+
+def _layer_struct(layer):
+    s = layer.spec
+    keep = []
+    L = _Layer()
+    L.out_features, L.in_features, L.d, L.n_books = s.out_features, s.in_features, s.d, s.n_books
+    for m in range(s.n_books):
+        w = np.ascontiguousarray(layer.idx_words[m], np.uint32)
+        c = np.ascontiguousarray(layer.codebooks[m], np.uint16)
+        keep += [w, c]
+        L.log2k[m] = s.log2k[m]
+        L.idx[m] = w.ctypes.data
+        L.row_words[m] = layer.row_words[m]
+        L.codebook[m] = c.ctypes.data
+    for name in ("scale", "bias"):
+        a = getattr(layer, name)
+        if a is not None:
+            a = np.ascontiguousarray(a, np.uint16)
+            keep.append(a)
+            setattr(L, name, a.ctypes.data)
+    return L, keep
+
+
+def dequant(layer, rows: Optional[Sequence[int]] = None) -> np.ndarray:
+    """W_hat as fp16 bits [N][Kin] (or [len(rows)][Kin])."""
+    L, keep = _layer_struct(layer)
+    kin = layer.spec.in_features
+    if rows is None:
+        w = np.zeros((layer.spec.out_features, kin), np.uint16)
+        _check(_load().vqo_dequant(C.byref(L), _p(w), kin), "dequant")
+    else:
+        r = np.ascontiguousarray(rows, np.int64)
+        w = np.zeros((r.size, kin), np.uint16)
+        _check(_load().vqo_dequant_rows(C.byref(L), _p(r), r.size, _p(w), kin), "dequant_rows")
+    del keep
+    return w
+
+
+def matmul(x: np.ndarray, w: np.ndarray, kin: Optional[int] = None, x_is_fp16: bool = False) -> np.ndarray:
+    """fp64 y[M][N] = x[M][:kin] . w[N][:kin]^T (x bf16 or fp16 bits, w fp16 bits)."""
+    x = np.ascontiguousarray(x, np.uint16)
+    w = np.ascontiguousarray(w, np.uint16)
+    kin = w.shape[1] if kin is None else kin
+    M, N = x.shape[0], w.shape[0]
+    y = np.empty((M, N), np.float64)
+    _check(_load().vqo_matmul(M, N, kin, _p(x), int(x_is_fp16), x.shape[1], _p(w), w.shape[1],
+                              _p(y), N), "matmul")
+    return y
+
+
+def linear(layer, x: np.ndarray, rows: Optional[Sequence[int]] = None,
+           x_is_fp16: bool = False) -> np.ndarray:
+    """Forward pass in fp64: y[M][n] for all output rows, or for ``rows``."""
+    L, keep = _layer_struct(layer)
+    x = np.ascontiguousarray(x, np.uint16)
+    M = x.shape[0]
+    if rows is None:
+        n_out, rp = layer.spec.out_features, None
+    else:
+        r = np.ascontiguousarray(rows, np.int64)
+        keep.append(r)
+        n_out, rp = r.size, _p(r)
+    y = np.empty((M, n_out), np.float64)
+    _check(_load().vqo_linear(C.byref(L), _p(x), int(x_is_fp16), M, x.shape[1], rp, n_out,
+                              _p(y), n_out), "linear")
+    del keep
+    return y
+
+
+# -- encoders (tests only) --------------------------------------------------
+
+def encode(v: np.ndarray, book: np.ndarray) -> np.ndarray:
+    v = np.ascontiguousarray(v, np.float64)
+    book = np.ascontiguousarray(book, np.uint16)
+    nv, d = v.shape
+    idx = np.empty(nv, np.uint32)
+    _check(_load().vqo_encode(_p(v), nv, d, _p(book), book.shape[0], _p(idx)), "encode")
+    return idx
+
+
+def encode_residual(v: np.ndarray, book1: np.ndarray, book2: np.ndarray):
+    v = np.ascontiguousarray(v, np.float64)
+    b1 = np.ascontiguousarray(book1, np.uint16)
+    b2 = np.ascontiguousarray(book2, np.uint16)
+    nv, d = v.shape
+    i1 = np.empty(nv, np.uint32)
+    i2 = np.empty(nv, np.uint32)
+    _check(_load().vqo_encode_residual(_p(v), nv, d, _p(b1), b1.shape[0], _p(b2), b2.shape[0],
+                                       _p(i1), _p(i2)), "encode_residual")
+    return i1, i2
+
+
+def encode_joint(v: np.ndarray, book1: np.ndarray, book2: np.ndarray):
+    v = np.ascontiguousarray(v, np.float64)
+    b1 = np.ascontiguousarray(book1, np.uint16)
+    b2 = np.ascontiguousarray(book2, np.uint16)
+    nv, d = v.shape
+    i1 = np.empty(nv, np.uint32)
+    i2 = np.empty(nv, np.uint32)
+    _check(_load().vqo_encode_joint(_p(v), nv, d, _p(b1), b1.shape[0], _p(b2), b2.shape[0],
+                                    _p(i1), _p(i2)), "encode_joint")
+    return i1, i2
+
+
+def num_threads() -> int:
+    return int(_load().vqo_num_threads())

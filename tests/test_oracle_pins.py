@@ -1,0 +1,306 @@
+"""Pins for the CPU oracle: each test checks it against something other than
+itself -- library conversions, a hand-derived fixture, closed forms,
+identities with a known answer, an independent numpy restatement, and brute
+force on tiny inputs.  A plausible slip in the oracle (a wrong bit order, a
+dropped residual term, a swapped scale/bias order, a transposed product, a
+tie broken the wrong way) fails at least one of them."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth import LayerData, LayerSpec
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# -- fp16 / bf16 conversions against numpy and torch --------------------------
+
+def test_f16_to_f32_all_patterns():
+    h = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = h.view(np.float16).astype(np.float32)
+    got = oracle.f16_to_f32(h)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+
+
+def test_f32_to_f16_matches_numpy():
+    rng = np.random.default_rng(7)
+    parts = [
+        rng.standard_normal(400_000).astype(np.float32) * 0.02,
+        rng.standard_normal(200_000).astype(np.float32) * 3e4,
+        (rng.standard_normal(200_000) * 1e-5).astype(np.float32),      # subnormal range
+        (rng.standard_normal(100_000) * 1e-8).astype(np.float32),      # underflow
+        rng.uniform(65400, 65600, 50_000).astype(np.float32),           # overflow edge
+        np.array([0.0, -0.0, np.inf, -np.inf, 65504, 65519.99, 65520, 65536,
+                  2 ** -24, 2 ** -25, 3 * 2 ** -26, 2 ** -14, 2 ** -14 - 2 ** -25],
+                 np.float32),
+    ]
+    # exact midpoints between neighbouring fp16 values (ties to even)
+    h = np.arange(0x0001, 0x7bff, dtype=np.uint16)
+    lo = h.view(np.float16).astype(np.float64)
+    hi = (h + 1).view(np.float16).astype(np.float64)
+    mid = ((lo + hi) / 2).astype(np.float32)
+    parts += [mid, -mid]
+    a = np.concatenate(parts)
+    with np.errstate(over="ignore"):
+        ref = a.astype(np.float16).view(np.uint16)
+    got = oracle.f32_to_f16(a)
+    assert np.array_equal(got, ref), np.flatnonzero(got != ref)[:10]
+
+
+def test_bf16_conversions_match_torch():
+    h = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = (h.astype(np.uint32) << 16).view(np.float32)
+    got = oracle.bf16_to_f32(h)
+    nan = np.isnan(ref)
+    assert np.array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+    rng = np.random.default_rng(8)
+    a = np.concatenate([
+        rng.standard_normal(300_000).astype(np.float32),
+        (rng.standard_normal(100_000) * 1e-39).astype(np.float32),     # fp32 subnormals
+        np.array([0.0, -0.0, np.inf, -np.inf, 3.3895314e38, 3.4e38], np.float32),
+    ])
+    # exact ties between neighbouring bf16 values
+    hb = np.arange(0x0001, 0x7f7f, 97, dtype=np.uint32)
+    mid = ((hb << 16) + (1 << 15)).astype(np.uint32).view(np.float32)
+    a = np.concatenate([a, mid, -mid])
+    ref = torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = oracle.f32_to_bf16(a)
+    assert np.array_equal(got, ref)
+
+
+# -- index streams ------------------------------------------------------------
+
+def _numpy_unpack(words: np.ndarray, b: int, nvec: int) -> np.ndarray:
+    """Independent restatement: expand words to bits (LSB first), regroup."""
+    bits = np.unpackbits(words.view(np.uint8), axis=1, bitorder="little")
+    f = bits[:, : nvec * b].reshape(words.shape[0], nvec, b).astype(np.uint32)
+    return (f << np.arange(b, dtype=np.uint32)).sum(axis=2).astype(np.uint32)
+
+
+def test_golden_layout():
+    with open(os.path.join(GOLDEN, "index_stream_layout.txt")) as fh:
+        rows = [ln for ln in fh if ln.strip() and not ln.startswith("#")]
+    assert len(rows) == 3
+    for ln in rows:
+        b, fields, words = (p.split() for p in ln.split("|"))
+        b = int(b[0])
+        fields = np.array([[int(v) for v in fields]], np.uint32)
+        words = np.array([[int(v, 16) for v in words]], np.uint32)
+        assert np.array_equal(oracle.pack(fields, b), words)
+        assert np.array_equal(oracle.unpack(words, b, fields.shape[1]), fields)
+
+
+@pytest.mark.parametrize("b", range(1, 17))
+def test_unpack_matches_numpy_and_roundtrips(b):
+    rng = np.random.default_rng(100 + b)
+    for nvec in (1, 7, 31, 32, 33, 129, 1000):
+        rw = synth.row_words_for(nvec, b) + 4 * int(rng.integers(0, 3))
+        words = rng.integers(0, 1 << 32, size=(5, rw), dtype=np.uint64).astype(np.uint32)
+        idx = oracle.unpack(words, b, nvec)
+        assert np.array_equal(idx, _numpy_unpack(words, b, nvec))
+        assert idx.max() < (1 << b)
+        again = oracle.unpack(oracle.pack(idx, b, rw), b, nvec)
+        assert np.array_equal(again, idx)
+
+
+def test_pack_rejects_wide_fields():
+    with pytest.raises(ValueError):
+        oracle.pack(np.array([[8]], np.uint32), 3)
+
+
+# -- dequantisation -----------------------------------------------------------
+
+ONE = np.float16(1.0).view(np.uint16)
+
+
+def _layer(n, kin, d, books, streams_idx, scale=None, bias=None):
+    """A LayerData from explicit books and index arrays (packed by the oracle)."""
+    log2k = tuple(int(np.log2(bk.shape[0])) for bk in books)
+    spec = LayerSpec(n, kin, d, log2k, tuple(0.0 for _ in books), None, None)
+    words = [oracle.pack(ix, b) for ix, b in zip(streams_idx, log2k)]
+    return LayerData(spec, words, [w.shape[1] for w in words], list(books), scale, bias)
+
+
+def test_binary_codebook_identity():
+    """d=8, K=256, C[k][e] = bit e of k: W_hat spells out every index's bits."""
+    d, n, kin = 8, 37, 8 * 41
+    k = np.arange(256, dtype=np.uint32)
+    book = np.where((k[:, None] >> np.arange(8)) & 1, ONE, 0).astype(np.uint16)
+    rng = np.random.default_rng(1)
+    idx = rng.integers(0, 256, size=(n, kin // d), dtype=np.uint32)
+    w = oracle.dequant(_layer(n, kin, d, [book], [idx]))
+    bits = ((idx[:, :, None] >> np.arange(8)) & 1).reshape(n, kin)
+    assert np.array_equal(w, np.where(bits, ONE, 0).astype(np.uint16))
+
+
+def test_one_hot_identity_and_product():
+    """d=8, K=8, C[k] = e_k: y[o] = sum_j x[8j + idx[o][j]]."""
+    d, n, nvec = 8, 23, 50
+    kin = d * nvec
+    book = np.where(np.eye(8, dtype=bool), ONE, 0).astype(np.uint16)
+    rng = np.random.default_rng(2)
+    idx = rng.integers(0, 8, size=(n, nvec), dtype=np.uint32)
+    layer = _layer(n, kin, d, [book], [idx])
+    x = synth.make_x(11, 3, kin)
+    y = oracle.linear(layer, x)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    cols = np.arange(nvec) * 8 + idx                      # [n][nvec]
+    ref = np.stack([xf[:, cols[o]].sum(axis=1) for o in range(n)], axis=1)
+    assert np.allclose(y, ref, rtol=1e-13, atol=1e-13)
+
+
+def test_affine_special_case():
+    """All-zero book: W_hat[o][:] = fp16(0 * s[o] + t[o]) = t[o]; y = t[o] * sum(x)."""
+    d, n, kin = 6, 19, 6 * 9 + 4
+    book = np.zeros((16, d), np.uint16)
+    rng = np.random.default_rng(3)
+    idx = rng.integers(0, 16, size=(n, -(-kin // d)), dtype=np.uint32)
+    scale = synth.to_f16_bits(rng.uniform(0.5, 1.5, n).astype(np.float32))
+    bias = synth.to_f16_bits(rng.standard_normal(n).astype(np.float32))
+    layer = _layer(n, kin, d, [book], [idx], scale, bias)
+    w = oracle.dequant(layer)
+    assert np.array_equal(w, np.repeat(bias[:, None], kin, axis=1))
+    x = synth.make_x(12, 2, kin)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    tf = bias.view(np.float16).astype(np.float64)
+    assert np.allclose(oracle.linear(layer, x), xf.sum(1)[:, None] * tf[None, :], rtol=1e-12)
+
+
+def _numpy_dequant(layer) -> np.ndarray:
+    """Independent float32 restatement, vectorised: same operation order."""
+    s = layer.spec
+    nvec = s.nvec
+    acc = None
+    for m in range(s.n_books):
+        idx = _numpy_unpack(layer.idx_words[m], s.log2k[m], nvec)
+        c = layer.codebooks[m].view(np.float16).astype(np.float32)[idx]   # [n][nvec][d]
+        acc = c if acc is None else (acc + c).astype(np.float32)
+    acc = acc.reshape(s.out_features, nvec * s.d)[:, : s.in_features]
+    if layer.scale is not None:
+        acc = (acc * layer.scale.view(np.float16).astype(np.float32)[:, None]).astype(np.float32)
+    if layer.bias is not None:
+        acc = (acc + layer.bias.view(np.float16).astype(np.float32)[:, None]).astype(np.float32)
+    return acc.astype(np.float16).view(np.uint16)
+
+
+@pytest.mark.parametrize("d,log2k,kin,scale,bias", [
+    (8, (16,), 512, True, True),
+    (8, (12, 8), 1024, True, True),
+    (6, (12, 4), 6 * 50 + 4, True, True),
+    (6, (12, 4), 6 * 50 + 1, False, True),
+    (8, (8, 8), 8 * 33, True, False),
+    (5, (7, 3), 5 * 20 + 3, False, False),
+    (16, (16,), 16 * 8 + 15, True, True),
+    (1, (4, 2), 77, True, True),
+])
+def test_dequant_matches_numpy_restatement(d, log2k, kin, scale, bias):
+    spec = LayerSpec(61, kin, d, log2k, (0.02, 0.005)[: len(log2k)],
+                     (0.5, 1.5) if scale else None, 1e-3 if bias else None)
+    layer = synth.make_layer(spec, seed=d * 1000 + kin, pad_garbage=True)
+    assert np.array_equal(oracle.dequant(layer), _numpy_dequant(layer))
+
+
+def test_dequant_semantics_are_distinguishable():
+    """The restatement pin separates the reading s*(c1+c2)+t from plausible
+    slips: bias applied before the scale, or the residual book dropped."""
+    spec = LayerSpec(64, 512, 8, (12, 8), (0.02, 0.005))
+    layer = synth.make_layer(spec, seed=5)
+    w = oracle.dequant(layer)
+    s = spec
+    i1 = _numpy_unpack(layer.idx_words[0], 12, s.nvec)
+    i2 = _numpy_unpack(layer.idx_words[1], 8, s.nvec)
+    c1 = layer.codebooks[0].view(np.float16).astype(np.float32)[i1].reshape(64, 512)
+    c2 = layer.codebooks[1].view(np.float16).astype(np.float32)[i2].reshape(64, 512)
+    sc = layer.scale.view(np.float16).astype(np.float32)[:, None]
+    t = layer.bias.view(np.float16).astype(np.float32)[:, None]
+    bias_first = ((c1 + c2 + t) * sc).astype(np.float16).view(np.uint16)
+    no_residual = (c1 * sc + t).astype(np.float16).view(np.uint16)
+    assert (w != bias_first).mean() > 0.5
+    assert (w != no_residual).mean() > 0.5
+
+
+def test_rows_and_linear_consistent():
+    spec = LayerSpec(40, 200, 8, (12, 8), (0.02, 0.005))
+    layer = synth.make_layer(spec, seed=9)
+    w = oracle.dequant(layer)
+    rows = [3, 0, 39, 17]
+    assert np.array_equal(oracle.dequant(layer, rows), w[rows])
+    x = synth.make_x(13, 4, 200)
+    assert np.array_equal(oracle.linear(layer, x, rows), oracle.linear(layer, x)[:, rows])
+
+
+# -- products -----------------------------------------------------------------
+
+def test_matmul_matches_numpy_float64():
+    rng = np.random.default_rng(4)
+    for M, N, K in [(1, 33, 100), (7, 64, 257), (16, 5, 1000)]:
+        x = synth.make_x(int(rng.integers(1 << 30)), M, K)
+        w = synth.to_f16_bits(rng.standard_normal((N, K)).astype(np.float32) * 0.02)
+        y = oracle.matmul(x, w)
+        xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        ref = xf @ w.view(np.float16).astype(np.float64).T
+        assert np.allclose(y, ref, rtol=1e-12, atol=1e-14 * np.abs(ref).max())
+        # fp16 activations
+        xh = synth.make_x(5, M, K, as_fp16=True)
+        ref = xh.view(np.float16).astype(np.float64) @ w.view(np.float16).astype(np.float64).T
+        assert np.allclose(oracle.matmul(xh, w, x_is_fp16=True), ref, rtol=1e-12,
+                           atol=1e-14 * np.abs(ref).max())
+
+
+def test_linear_is_x_times_dequant_transpose_and_rows_independent():
+    spec = LayerSpec(50, 6 * 30 + 2, 6, (12, 4), (0.02, 0.005))
+    layer = synth.make_layer(spec, seed=6)
+    x = synth.make_x(14, 6, spec.in_features, outlier_frac=0.01)
+    w = oracle.dequant(layer)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    ref = xf @ w.view(np.float16).astype(np.float64).T
+    y = oracle.linear(layer, x)
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-14 * np.abs(ref).max())
+    for b in range(6):      # batch-row independence
+        assert np.array_equal(oracle.linear(layer, x[b:b + 1])[0], y[b])
+
+
+# -- encoders -----------------------------------------------------------------
+
+def test_encode_recovers_generating_indices():
+    spec = LayerSpec(32, 64, 8, (8,), (0.02,))
+    book = synth.make_layer(spec, seed=21).codebooks[0]
+    rng = np.random.default_rng(22)
+    idx = rng.integers(0, 256, size=512, dtype=np.uint32)
+    v = book.view(np.float16).astype(np.float64)[idx]
+    assert np.array_equal(oracle.encode(v, book), idx)
+    # a perturbed copy agrees with numpy's argmin (first minimum on ties)
+    v2 = v + rng.standard_normal(v.shape) * 0.004
+    dist = ((v2[:, None, :] - book.view(np.float16).astype(np.float64)[None]) ** 2).sum(-1)
+    assert np.array_equal(oracle.encode(v2, book), dist.argmin(1).astype(np.uint32))
+
+
+def test_encode_ties_go_to_lowest_index():
+    book = np.array([[ONE, 0], [0, ONE], [ONE, 0]], np.uint16)     # rows 0 and 2 equal
+    v = np.array([[1.0, 0.0], [0.5, 0.5]])
+    assert list(oracle.encode(v, book)) == [0, 0]
+
+
+def test_two_book_encoders():
+    spec = LayerSpec(8, 8, 4, (4, 3), (0.3, 0.01))
+    L = synth.make_layer(spec, seed=23)
+    b1, b2 = L.codebooks
+    rng = np.random.default_rng(24)
+    i1 = rng.integers(0, 16, 300, dtype=np.uint32)
+    i2 = rng.integers(0, 8, 300, dtype=np.uint32)
+    c1 = b1.view(np.float16).astype(np.float64)
+    c2 = b2.view(np.float16).astype(np.float64)
+    v = c1[i1] + c2[i2]
+    j1, j2 = oracle.encode_joint(v, b1, b2)
+    assert np.array_equal(c1[j1] + c2[j2], v)           # the generating W_hat
+    g1, g2 = oracle.encode_residual(v, b1, b2)           # greedy cascade
+    assert np.array_equal(g1, oracle.encode(v, b1))
+    r = v - c1[g1]
+    dist = ((r[:, None, :] - c2[None]) ** 2).sum(-1)
+    assert np.array_equal(g2, dist.argmin(1).astype(np.uint32))
