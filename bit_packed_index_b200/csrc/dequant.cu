@@ -1,0 +1,127 @@
+// dequant.cu -- vq_dequant: W_hat = fp16((C1[i1] + C2[i2]) * s + t), bit-exact.
+//
+// Follows "VPTQ Guide: Extreme 2-Bit Vector Quantization", section "Step 2"
+// (dequantize: gather both codebooks, add, reshape to (out, in)) with the
+// per-row scale and bias of the layer, in the fixed fp32 order documented in
+// include/vq.h.  Every fp32 operation is an explicitly rounded intrinsic
+// (__fadd_rn / __fmul_rn), so no multiply-add contraction can change a bit.
+//
+// Work split: persistent blocks loop over output rows; each thread owns whole
+// d-vectors (consecutive threads -> consecutive vectors, so index reads and
+// W_hat stores are coalesced).  Books that fit are staged once per block in
+// shared memory; 2^16-entry books are read through L1/L2.  For d = 8 with an
+// aligned destination a vector is written with one 16-byte store.
+#include <algorithm>
+
+#include "codebook.cuh"
+
+namespace vqk {
+namespace {
+
+constexpr int kDqThreads = 256;
+constexpr size_t kDqSmemBooks = 96 * 1024;   // stage books up to this size
+
+template <int D, int NB>
+__global__ void __launch_bounds__(kDqThreads) dequant_kernel(Layer L, uint16_t* __restrict__ w,
+                                                             int64_t ldw, int smem_mask,
+                                                             int vec_store) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  BookView bv[2];
+  {
+    size_t off = 0;
+#pragma unroll
+    for (int m = 0; m < NB; ++m) {
+      if (smem_mask & (1 << m)) {
+        const int pad = L.d <= 8 ? 8 : 16;
+        uint16_t* dst = reinterpret_cast<uint16_t*>(smem + off);
+        stage_book(dst, L.book[m], 1 << L.b[m], L.d, pad);
+        bv[m] = {dst, pad};
+        off += (static_cast<size_t>(1) << L.b[m]) * pad * sizeof(uint16_t);
+      } else {
+        bv[m] = {L.book[m], L.d};
+      }
+    }
+    if (smem_mask) __syncthreads();
+  }
+  const int d = (D > 0) ? D : L.d;
+  for (int64_t o = blockIdx.x; o < L.n; o += gridDim.x) {
+    const bool has_s = L.scale != nullptr, has_t = L.bias != nullptr;
+    const float s = has_s ? h2f(L.scale[o]) : 1.0f;
+    const float t = has_t ? h2f(L.bias[o]) : 0.0f;
+    const uint32_t* row0 = L.idx[0] + o * L.rw[0];
+    const uint32_t* row1 = (NB == 2) ? L.idx[1] + o * L.rw[1] : nullptr;
+    uint16_t* wrow = w + o * ldw;
+    for (int j = threadIdx.x; j < L.nvec; j += blockDim.x) {
+      float c[kMaxVecDim];
+      load_centroid<D>(bv[0], load_field(row0, static_cast<int64_t>(j) * L.b[0], L.b[0]), d, c);
+      if constexpr (NB == 2) {
+        float c2[kMaxVecDim];
+        load_centroid<D>(bv[1], load_field(row1, static_cast<int64_t>(j) * L.b[1], L.b[1]), d, c2);
+#pragma unroll
+        for (int e = 0; e < kMaxVecDim; ++e)
+          if (e < d) c[e] = __fadd_rn(c[e], c2[e]);
+      }
+      uint16_t h[kMaxVecDim];
+#pragma unroll
+      for (int e = 0; e < kMaxVecDim; ++e) {
+        if (e < d) {
+          float v = c[e];
+          if (has_s) v = __fmul_rn(v, s);
+          if (has_t) v = __fadd_rn(v, t);
+          h[e] = f2h(v);
+        }
+      }
+      const int64_t k0 = static_cast<int64_t>(j) * d;
+      if (D == 8 && vec_store && k0 + 8 <= L.kin) {
+        uint4 v;
+        v.x = h[0] | (static_cast<uint32_t>(h[1]) << 16);
+        v.y = h[2] | (static_cast<uint32_t>(h[3]) << 16);
+        v.z = h[4] | (static_cast<uint32_t>(h[5]) << 16);
+        v.w = h[6] | (static_cast<uint32_t>(h[7]) << 16);
+        *reinterpret_cast<uint4*>(wrow + k0) = v;
+      } else {
+#pragma unroll
+        for (int e = 0; e < kMaxVecDim; ++e)
+          if (e < d && k0 + e < L.kin) wrow[k0 + e] = h[e];
+      }
+    }
+  }
+}
+
+template <int D, int NB>
+cudaError_t launch_dq(const Layer& L, uint16_t* w, int64_t ldw, int smem_mask, size_t smem,
+                      int vec_store, int grid, cudaStream_t stream) {
+  auto k = dequant_kernel<D, NB>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  k<<<grid, kDqThreads, smem, stream>>>(L, w, ldw, smem_mask, vec_store);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+vq_status launch_dequant(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream) {
+  if (L.n == 0 || L.kin == 0) return VQ_OK;
+  int smem_mask = 0;
+  const size_t smem = stage_plan(L, std::min<size_t>(kDqSmemBooks, device_smem_optin()), &smem_mask);
+  const int vec_store = aligned(w, 16) && (ldw % 8 == 0);
+  const int per_sm = smem ? std::max(1, std::min(8, static_cast<int>((228 * 1024) / (smem + 1024)))) : 8;
+  const int grid = static_cast<int>(std::min<int64_t>(L.n, static_cast<int64_t>(device_sm_count()) * per_sm));
+  cudaError_t e;
+  const int D = (L.d == 8) ? 8 : (L.d == 6 ? 6 : 0);
+  if (L.nb == 1) {
+    e = D == 8 ? launch_dq<8, 1>(L, w, ldw, smem_mask, smem, vec_store, grid, stream)
+      : D == 6 ? launch_dq<6, 1>(L, w, ldw, smem_mask, smem, vec_store, grid, stream)
+               : launch_dq<0, 1>(L, w, ldw, smem_mask, smem, vec_store, grid, stream);
+  } else {
+    e = D == 8 ? launch_dq<8, 2>(L, w, ldw, smem_mask, smem, vec_store, grid, stream)
+      : D == 6 ? launch_dq<6, 2>(L, w, ldw, smem_mask, smem, vec_store, grid, stream)
+               : launch_dq<0, 2>(L, w, ldw, smem_mask, smem, vec_store, grid, stream);
+  }
+  return cuda_status(e);
+}
+
+}  // namespace vqk

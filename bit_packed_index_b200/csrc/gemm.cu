@@ -1,0 +1,550 @@
+// gemm.cu -- vq_gemm: prefill y = x . W_hat^T on the tcgen05 tensor cores.
+//
+// The pages place prefill in the compute-bound regime, where table lookups
+// compete with the matrix multiply ("Vector Quantization for LLM Weights in
+// Production", section "1. Prefill vs. Decode Bottlenecks"; its dequantisation
+// diagram feeds dequantised fp16/bf16 vectors to "GEMV / Tensor Core Dot
+// Products").  The B200 design:
+//
+//  * One CTA per 128 x 256 output tile, K in steps of 64 (fp16 operands, 128-
+//    byte rows, 128-byte swizzle), a multi-stage shared-memory pipeline driven
+//    by mbarriers, one elected thread issuing tcgen05.mma (M=128, N=256, K=16)
+//    into an fp32 accumulator in tensor memory, and a tcgen05.ld epilogue.
+//  * A tiles (activations) arrive by TMA from an fp16 copy of x that a small
+//    pre-pass writes into the workspace, together with the row sums of x.
+//    bf16 -> fp16 is exact for |x| in [2^-14, 65504].
+//  * B tiles (weights) come from one of two sources:
+//      - fused: eight producer warps unpack the index streams, gather the
+//        centroids (shared memory for small books, L1/L2 for 2^16-entry
+//        books), add the residual centroid in fp16 and write the swizzled
+//        tile directly; W_hat never reaches global memory.  Scale and bias
+//        are applied in the epilogue: y = s[n] * acc + t[n] * sum_k x[m][k].
+//      - staged: vq_dequant writes W_hat (fp16, bit-exact) into the
+//        workspace once and TMA streams its tiles; the epilogue is y = acc.
+//    Each W_hat element costs one centroid gather per 128 rows of x in the
+//    fused form but one gather in total in the staged form, so the staged
+//    form wins when gathers are served from L2 and M is large.
+//  * Every mbarrier wait is bounded; a wait that runs out of budget raises
+//    the block's abort flag, records VQ_ERR_TIMEOUT in the workspace's status
+//    word and lets every warp fall through to the teardown.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "codebook.cuh"
+#include "sm100.cuh"
+
+namespace vqk {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int kATile = BM * BK * 2;             // 16 KB
+constexpr int kBTile = BN * BK * 2;             // 32 KB
+constexpr int kStageBytes = kATile + kBTile;    // 48 KB
+constexpr int kThreads = 384;                   // 12 warps
+constexpr int kProducerThread0 = 128;           // warps 4..11 produce B tiles
+constexpr int kProducers = 256;
+constexpr uint32_t kTmemCols = 256;
+constexpr int kCtrlBytes = 3072;                // barriers, flags, scale/bias staging
+constexpr long long kWaitBudget = 4000000000LL; // SM clocks (about 2 s)
+constexpr int kMaxStages = 8;
+
+enum Mode { kFused = 0, kStaged = 1 };
+
+struct GemmArgs {
+  Layer L;
+  int m;
+  int num_kt;
+  int stages;
+  int smem_mask;
+  int book_bytes;
+  const float* rowsum;
+  void* y;
+  vq_dtype yt;
+  int64_t ldy;
+  int* status;
+};
+
+// Control block at the start of (1024-aligned) dynamic shared memory.
+struct Ctrl {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  uint64_t acc_full;
+  uint32_t tmem_base;
+  int abort_flag;
+  float sb[2 * BN];   // per-column scale, then bias, of this tile
+};
+static_assert(sizeof(Ctrl) <= kCtrlBytes, "control block");
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Byte offset of 16-byte chunk c of row r in a 128-byte-swizzled tile.
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
+  return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+// Eight consecutive B-bit fields starting at field j0 (a multiple of 8, so
+// the first bit is word aligned for B in {4, 8, 12, 16}).  Words past the row
+// are read as zero (their fields lie past the last vector and are masked).
+template <int B>
+__device__ __forceinline__ void fields8(const uint32_t* __restrict__ row, int64_t rw, int j0,
+                                        uint32_t (&f)[8]) {
+  constexpr int NW = (8 * B) / 32;
+  const int64_t w0 = (static_cast<int64_t>(j0) * B) >> 5;
+  uint32_t w[NW + 1];
+  if (B == 16 && w0 + 4 <= rw) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + w0));
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if (B == 8 && w0 + 2 <= rw) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(row + w0));
+    w[0] = v.x; w[1] = v.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < NW; ++i) w[i] = (w0 + i < rw) ? __ldg(row + w0 + i) : 0u;
+  }
+  w[NW] = 0u;
+#pragma unroll
+  for (int v = 0; v < 8; ++v) {
+    constexpr uint32_t mask = (1u << B) - 1u;
+    const int bit = v * B;
+    f[v] = __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31) & mask;
+  }
+}
+
+__device__ __forceinline__ uint4 hadd8(uint4 a, uint4 b) {
+  uint4 r;
+  const __half2* x = reinterpret_cast<const __half2*>(&a);
+  const __half2* y = reinterpret_cast<const __half2*>(&b);
+  __half2* z = reinterpret_cast<__half2*>(&r);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) z[i] = __hadd2(x[i], y[i]);
+  return r;
+}
+
+__device__ __forceinline__ uint4 zero_tail8(uint4 v, int valid) {   // keep `valid` of 8 halves
+  uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (2 * i >= valid) w[i] = 0u;
+    else if (2 * i + 1 >= valid) w[i] &= 0xFFFFu;
+  }
+  return v;
+}
+
+// Fused B-tile row (d = 8, compile-time index widths; B2 = 0: one book).
+template <int B1, int B2>
+__device__ __forceinline__ void produce_row_d8(const Layer& L, const BookView (&bv)[2], int n,
+                                               int kt, uint8_t* btile, int r) {
+  if (n >= L.n) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(btile + sw128_off(r, c)) = make_uint4(0, 0, 0, 0);
+    return;
+  }
+  const int j0 = kt * 8;
+  uint32_t f1[8], f2[8];
+  fields8<B1>(L.idx[0] + static_cast<int64_t>(n) * L.rw[0], L.rw[0], j0, f1);
+  if constexpr (B2 > 0) fields8<B2>(L.idx[1] + static_cast<int64_t>(n) * L.rw[1], L.rw[1], j0, f2);
+  uint4 c[8];
+#pragma unroll
+  for (int v = 0; v < 8; ++v) c[v] = *reinterpret_cast<const uint4*>(bv[0].base + static_cast<size_t>(f1[v]) * 8);
+  if constexpr (B2 > 0) {
+#pragma unroll
+    for (int v = 0; v < 8; ++v)
+      c[v] = hadd8(c[v], *reinterpret_cast<const uint4*>(bv[1].base + static_cast<size_t>(f2[v]) * 8));
+  }
+  const int k0 = kt * BK;
+#pragma unroll
+  for (int v = 0; v < 8; ++v) {
+    const int valid = L.kin - (k0 + 8 * v);
+    uint4 x = c[v];
+    if (valid < 8) x = zero_tail8(x, valid < 0 ? 0 : valid);
+    *reinterpret_cast<uint4*>(btile + sw128_off(r, v)) = x;
+  }
+}
+
+// Fused B-tile row, any d <= 8 and any index widths.
+template <int NB>
+__device__ __forceinline__ void produce_row_generic(const Layer& L, const BookView (&bv)[2], int n,
+                                                    int kt, uint8_t* btile, int r) {
+  const int k0 = kt * BK;
+  if (n >= L.n || k0 + BK > L.kin) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(btile + sw128_off(r, c)) = make_uint4(0, 0, 0, 0);
+    if (n >= L.n) return;
+  }
+  const int d = L.d;
+  const int j_lo = k0 / d;
+  const int j_hi = min(L.nvec - 1, (k0 + BK - 1) / d);
+  const uint32_t* row0 = L.idx[0] + static_cast<int64_t>(n) * L.rw[0];
+  const uint32_t* row1 = L.idx[1] + static_cast<int64_t>(n) * L.rw[1];
+  for (int j = j_lo; j <= j_hi; ++j) {
+    const uint32_t i1 = load_field(row0, static_cast<int64_t>(j) * L.b[0], L.b[0]);
+    const uint16_t* c1 = bv[0].base + static_cast<size_t>(i1) * bv[0].stride;
+    const uint16_t* c2 = nullptr;
+    if (NB == 2) {
+      const uint32_t i2 = load_field(row1, static_cast<int64_t>(j) * L.b[1], L.b[1]);
+      c2 = bv[1].base + static_cast<size_t>(i2) * bv[1].stride;
+    }
+    for (int e = 0; e < d; ++e) {
+      const int k = j * d + e;
+      if (k < k0 || k >= k0 + BK || k >= L.kin) continue;
+      __half h = __ushort_as_half(c1[e]);
+      if (NB == 2) h = __hadd(h, __ushort_as_half(c2[e]));
+      const int kk = k - k0;
+      *reinterpret_cast<__half*>(btile + sw128_off(r, kk >> 3) + (kk & 7) * 2) = h;
+    }
+  }
+}
+
+template <int MODE, int B1, int B2>
+__global__ void __launch_bounds__(kThreads, 1)
+    vq_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                   const __grid_constant__ CUtensorMap tmap_b, GemmArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem);
+  uint8_t* stages = smem + kCtrlBytes + (1024 - kCtrlBytes % 1024) % 1024;
+  uint16_t* books = reinterpret_cast<uint16_t*>(stages + g.stages * kStageBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
+  const Layer& L = g.L;
+  volatile int* abort_flag = &ctrl->abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < g.stages; ++s) {
+      mbar_init(&ctrl->full[s], MODE == kFused ? kProducers + 1 : 1);
+      mbar_init(&ctrl->empty[s], 1);
+    }
+    mbar_init(&ctrl->acc_full, 1);
+    ctrl->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctrl->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch(&tmap_a);
+    if (MODE == kStaged) tma_prefetch(&tmap_b);
+  }
+  // Per-column scale and bias of this tile (fused form applies them).
+  for (int i = threadIdx.x; i < BN; i += kThreads) {
+    const int n = n0 + i;
+    float s = 1.0f, t = 0.0f;
+    if (MODE == kFused && n < L.n) {
+      if (L.scale) s = h2f(L.scale[n]);
+      if (L.bias) t = h2f(L.bias[n]);
+    }
+    ctrl->sb[i] = s;
+    ctrl->sb[BN + i] = t;
+  }
+  BookView bv[2];
+  if (MODE == kFused) {
+    size_t off = 0;
+    for (int m = 0; m < L.nb; ++m) {
+      if (g.smem_mask & (1 << m)) {
+        uint16_t* dst = books + off / 2;
+        stage_book(dst, L.book[m], 1 << L.b[m], L.d, 8);
+        bv[m] = {dst, 8};
+        off += padded_book_bytes(L.b[m], L.d);
+      } else {
+        bv[m] = {L.book[m], L.d};
+      }
+    }
+    if (L.nb == 1) bv[1] = bv[0];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {                                   // TMA producer
+      int issued = 0;
+      for (int kt = 0; kt < g.num_kt; ++kt) {
+        const int s = kt % g.stages;
+        const uint32_t ph = (kt / g.stages) & 1;
+        if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, kWaitBudget)) break;
+        uint8_t* a = stages + s * kStageBytes;
+        mbar_arrive_expect_tx(&ctrl->full[s], MODE == kStaged ? kATile + kBTile : kATile);
+        tma_load_2d(a, &tmap_a, &ctrl->full[s], kt * BK, m0);
+        if (MODE == kStaged) tma_load_2d(a + kATile, &tmap_b, &ctrl->full[s], kt * BK, n0);
+        issued = kt + 1;
+      }
+      if (*abort_flag) {   // let loads already in flight land before the block exits
+        for (int kt = max(0, issued - g.stages); kt < issued; ++kt)
+          bounded_wait(&ctrl->full[kt % g.stages], (kt / g.stages) & 1, abort_flag, nullptr,
+                       kWaitBudget / 8);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {                                   // MMA issuer
+      constexpr uint32_t idesc = f16_idesc(BM, BN);
+      for (int kt = 0; kt < g.num_kt; ++kt) {
+        const int s = kt % g.stages;
+        const uint32_t ph = (kt / g.stages) & 1;
+        if (!bounded_wait(&ctrl->full[s], ph, abort_flag, g.status, kWaitBudget)) break;
+        tc_fence_after();
+        const uint32_t a = smem_addr(stages + s * kStageBytes);
+        const uint32_t b = a + kATile;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          umma_f16(tmem, sw128_kmajor_desc(a + kk * 32), sw128_kmajor_desc(b + kk * 32), idesc,
+                   (kt | kk) != 0);
+        umma_commit(&ctrl->empty[s]);
+      }
+      umma_commit(&ctrl->acc_full);
+    }
+  } else if (warp >= 4) {
+    if (MODE == kFused) {                              // B-tile producers
+      const int r = threadIdx.x - kProducerThread0;
+      for (int kt = 0; kt < g.num_kt; ++kt) {
+        const int s = kt % g.stages;
+        const uint32_t ph = (kt / g.stages) & 1;
+        if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, kWaitBudget)) break;
+        uint8_t* btile = stages + s * kStageBytes + kATile;
+        if constexpr (B1 > 0) produce_row_d8<B1, B2>(L, bv, n0 + r, kt, btile, r);
+        else if (L.nb == 2) produce_row_generic<2>(L, bv, n0 + r, kt, btile, r);
+        else produce_row_generic<1>(L, bv, n0 + r, kt, btile, r);
+        fence_proxy_async_smem();
+        mbar_arrive(&ctrl->full[s]);
+      }
+    }
+    if (warp < 8) {                                    // epilogue: warps 4..7 = TMEM lane quarters
+      const int q = warp & 3;
+      if (bounded_wait(&ctrl->acc_full, 0, abort_flag, g.status, kWaitBudget)) {
+        tc_fence_after();
+        const int row = m0 + q * 32 + lane;
+        const float rs = (MODE == kFused && row < g.m) ? g.rowsum[row] : 0.0f;
+        const size_t es = g.yt == VQ_FP32 ? 4 : 2;
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t acc[32];
+          tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c * 32, acc);
+          tmem_wait_ld();
+          const int nb = n0 + c * 32;
+          if (row >= g.m || nb >= L.n) continue;
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            v[i] = ctrl->sb[c * 32 + i] * __uint_as_float(acc[i]) + ctrl->sb[BN + c * 32 + i] * rs;
+          const int ncols = min(32, L.n - nb);
+          uint8_t* dst = reinterpret_cast<uint8_t*>(g.y) + (static_cast<int64_t>(row) * g.ldy + nb) * es;
+          if (ncols == 32 && aligned(dst, 16)) {
+            if (g.yt == VQ_FP32) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                reinterpret_cast<float4*>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            } else {
+              uint32_t p[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const uint16_t lo = g.yt == VQ_FP16 ? f2h(v[2 * i]) : f2bf(v[2 * i]);
+                const uint16_t hi = g.yt == VQ_FP16 ? f2h(v[2 * i + 1]) : f2bf(v[2 * i + 1]);
+                p[i] = lo | (static_cast<uint32_t>(hi) << 16);
+              }
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                reinterpret_cast<uint4*>(dst)[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+            }
+          } else {
+            for (int i = 0; i < ncols; ++i) store_out(dst, g.yt, i, v[i]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// x -> fp16 copy [m][kp] (zeros past kin) and fp32 row sums of the fp16 values.
+__global__ void gemm_prep(const uint16_t* __restrict__ x, int x_fp16, int m, int kin, int64_t ldx,
+                          uint16_t* __restrict__ x16, int kp, float* __restrict__ rowsum,
+                          int* __restrict__ status) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
+  const int warps = blockDim.x >> 5;
+  const int row = blockIdx.x * warps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= m) return;
+  const uint16_t* xr = x + static_cast<int64_t>(row) * ldx;
+  uint16_t* outr = x16 + static_cast<int64_t>(row) * kp;
+  float s = 0.0f;
+  for (int k = lane; k < kp; k += 32) {
+    float v = 0.0f;
+    if (k < kin) v = x_fp16 ? h2f(xr[k]) : bf2f(xr[k]);
+    const uint16_t h = f2h(v);
+    outr[k] = h;
+    s += h2f(h);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (lane == 0) rowsum[row] = s;
+}
+
+// ---- host side ---------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D fp16 tensor [rows][cols] with row stride ld elements, box {64, box_rows},
+// 128-byte swizzle; reads past cols / rows return zeros.
+bool make_map(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int64_t ld,
+              int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+struct GemmLayout {
+  int mode;
+  int kp;
+  size_t off_rowsum, off_x16, off_w, total;
+};
+
+int choose_mode(const Layer& L, int m) {
+  const char* env = std::getenv("VQ_GEMM_MODE");
+  if (env && std::strcmp(env, "fused") == 0) return kFused;
+  if (env && std::strcmp(env, "staged") == 0) return kStaged;
+  // The staged form gathers each centroid once; the fused form once per 128
+  // rows of x.  Prefer it once the gathers of the fused form would outweigh
+  // writing and re-reading W_hat.
+  bool l2_book = false;
+  for (int i = 0; i < L.nb; ++i) l2_book |= L.b[i] > 12;
+  return (l2_book && m > 256) || m >= 2048 ? kStaged : kFused;
+}
+
+GemmLayout layout_for(const Layer& L, int m) {
+  GemmLayout g;
+  g.mode = choose_mode(L, m);
+  g.kp = (L.kin + 7) / 8 * 8;
+  g.off_rowsum = 256;
+  g.off_x16 = g.off_rowsum + round256(static_cast<size_t>(m) * 4);
+  g.off_w = g.off_x16 + round256(static_cast<size_t>(m) * g.kp * 2);
+  g.total = g.off_w + (g.mode == kStaged ? round256(static_cast<size_t>(L.n) * g.kp * 2) : 0);
+  return g;
+}
+
+template <int MODE, int B1, int B2>
+cudaError_t launch_kernel(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g,
+                          size_t smem, dim3 grid, cudaStream_t stream) {
+  auto k = vq_gemm_kernel<MODE, B1, B2>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  k<<<grid, kThreads, smem, stream>>>(ma, mb, g);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t gemm_workspace_bytes(const Layer& L, int m, bool) { return layout_for(L, m).total; }
+
+vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t ldx, void* y,
+                      vq_dtype yt, int64_t ldy, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const size_t es = yt == VQ_FP32 ? 4 : 2;
+  if (L.kin == 0)
+    return cuda_status(cudaMemset2DAsync(y, ldy * es, 0, static_cast<size_t>(L.n) * es, m, stream));
+  const GemmLayout lay = layout_for(L, m);
+  if (ws_bytes < lay.total) return VQ_ERR_WORKSPACE;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(w8);
+  float* rowsum = reinterpret_cast<float*>(w8 + lay.off_rowsum);
+  uint16_t* x16 = reinterpret_cast<uint16_t*>(w8 + lay.off_x16);
+  uint16_t* what = reinterpret_cast<uint16_t*>(w8 + lay.off_w);
+
+  {
+    const int warps = 8;
+    gemm_prep<<<(m + warps - 1) / warps, warps * 32, 0, stream>>>(
+        static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, m, L.kin, ldx, x16, lay.kp, rowsum, status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  if (lay.mode == kStaged) {
+    vq_status st = launch_dequant(L, what, lay.kp, stream);
+    if (st != VQ_OK) return st;
+  }
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, x16, L.kin, m, lay.kp, BM)) return VQ_ERR_CUDA;
+  if (lay.mode == kStaged) {
+    if (!make_map(&mb, what, L.kin, L.n, lay.kp, BN)) return VQ_ERR_CUDA;
+  } else {
+    mb = ma;
+  }
+
+  GemmArgs g;
+  g.L = L;
+  g.m = m;
+  g.num_kt = (L.kin + BK - 1) / BK;
+  g.rowsum = rowsum;
+  g.y = y;
+  g.yt = yt;
+  g.ldy = ldy;
+  g.status = status;
+  g.smem_mask = 0;
+  g.book_bytes = 0;
+  const int optin = device_smem_optin();
+  const size_t fixed = 1024 + 3072;   // alignment slack + control block
+  if (lay.mode == kFused) {
+    // Stage the books that fit next to at least three pipeline stages.
+    const size_t budget = static_cast<size_t>(optin) - fixed - 3 * kStageBytes;
+    int mask = 0;
+    size_t used = 0;
+    for (int i = 0; i < L.nb; ++i) {
+      const size_t b = padded_book_bytes(L.b[i], L.d);
+      if (used + b <= budget) { used += b; mask |= 1 << i; }
+    }
+    g.smem_mask = mask;
+    g.book_bytes = static_cast<int>(used);
+  }
+  g.stages = static_cast<int>(std::min<size_t>(kMaxStages, (optin - fixed - g.book_bytes) / kStageBytes));
+  g.stages = std::min(g.stages, 4);
+  const size_t smem = fixed + static_cast<size_t>(g.stages) * kStageBytes + g.book_bytes;
+  dim3 grid((m + BM - 1) / BM, (L.n + BN - 1) / BN);
+
+  cudaError_t e;
+  if (lay.mode == kStaged) {
+    e = launch_kernel<kStaged, 0, 0>(ma, mb, g, smem, grid, stream);
+  } else if (L.d == 8 && L.nb == 1 && L.b[0] == 16) {
+    e = launch_kernel<kFused, 16, 0>(ma, mb, g, smem, grid, stream);
+  } else if (L.d == 8 && L.nb == 2 && L.b[0] == 16 && L.b[1] == 8) {
+    e = launch_kernel<kFused, 16, 8>(ma, mb, g, smem, grid, stream);
+  } else if (L.d == 8 && L.nb == 2 && L.b[0] == 12 && L.b[1] == 8) {
+    e = launch_kernel<kFused, 12, 8>(ma, mb, g, smem, grid, stream);
+  } else if (L.d == 8 && L.nb == 2 && L.b[0] == 8 && L.b[1] == 8) {
+    e = launch_kernel<kFused, 8, 8>(ma, mb, g, smem, grid, stream);
+  } else {
+    e = launch_kernel<kFused, 0, 0>(ma, mb, g, smem, grid, stream);
+  }
+  return cuda_status(e);
+}
+
+}  // namespace vqk

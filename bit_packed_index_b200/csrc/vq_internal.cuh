@@ -1,0 +1,113 @@
+// vq_internal.cuh -- shared pieces of libvq's kernels and host entry points.
+//
+// The storage format, the layer description and what each call computes are
+// documented in include/vq.h.  This header holds the validated, by-value copy
+// of a layer that kernels receive, the index-field extraction, and the fp16 /
+// bf16 conversions (CUDA's own intrinsics).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "vq.h"
+
+namespace vqk {
+
+constexpr int kMaxVecDim = 16;
+constexpr int kMaxBatch = 16;
+
+// A validated layer, passed to kernels by value.
+struct Layer {
+  int n;            // out_features
+  int kin;          // in_features
+  int d;            // vector length
+  int nb;           // number of codebooks (1 or 2)
+  int nvec;         // ceil(kin / d)
+  int b[2];         // index width per book
+  int64_t rw[2];    // stream row stride, 32-bit words
+  const uint32_t* idx[2];
+  const uint16_t* book[2];
+  const uint16_t* scale;  // may be null
+  const uint16_t* bias;   // may be null
+};
+
+// ---------------------------------------------------------------------------
+// Host helpers (vq_api.cu).
+// ---------------------------------------------------------------------------
+vq_status check_layer(const vq_layer_desc* desc, Layer* out);
+vq_status cuda_status(cudaError_t e);  // records e, returns VQ_ERR_CUDA (or VQ_OK)
+int device_sm_count();
+int device_smem_optin();               // max dynamic shared memory per block, bytes
+
+__host__ __device__ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ---------------------------------------------------------------------------
+// Kernel launchers (one per .cu file).
+// ---------------------------------------------------------------------------
+vq_status launch_dequant(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream);
+
+struct GemvPlan {
+  int bt;        // batch tile (power of two >= batch)
+  int nsplit;    // K splits
+  int vps;       // vectors per split (multiple of 32)
+  int rpb;       // rows per work item
+  int grid_x;    // blocks per split
+  int smem;      // dynamic shared memory bytes
+  int books_in_smem;  // bit m set: book m staged in shared memory
+  int book_bytes;     // shared memory taken by the staged books
+  size_t ws_bytes;
+};
+vq_status plan_gemv(const Layer& L, int batch, GemvPlan* plan);
+vq_status launch_gemv(const Layer& L, const GemvPlan& plan, const void* x, bool x_fp16, int batch,
+                      int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy, float* ws,
+                      cudaStream_t stream);
+
+size_t gemm_workspace_bytes(const Layer& L, int m, bool x_fp16);
+vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t ldx, void* y,
+                      vq_dtype y_dtype, int64_t ldy, void* ws, size_t ws_bytes,
+                      cudaStream_t stream);
+
+// ---------------------------------------------------------------------------
+// Device helpers.
+// ---------------------------------------------------------------------------
+
+// Field j of a stream row: bits [j*b, j*b+b), LSB-first in 32-bit words.  A
+// field of b <= 16 bits spans at most two words; the second is read only
+// when the field crosses into it, so no read goes past the row.
+__device__ __forceinline__ uint32_t load_field(const uint32_t* __restrict__ row, int64_t bit, int b) {
+  const int64_t w = bit >> 5;
+  const int sh = static_cast<int>(bit & 31);
+  const uint32_t lo = __ldg(row + w);
+  const uint32_t hi = (sh + b > 32) ? __ldg(row + w + 1) : 0u;
+  return __funnelshift_r(lo, hi, sh) & ((1u << b) - 1u);
+}
+
+__device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+__device__ __forceinline__ float bf2f(uint16_t h) {
+  return __bfloat162float(__ushort_as_bfloat16(h));
+}
+__device__ __forceinline__ uint16_t f2h(float f) { return __half_as_ushort(__float2half_rn(f)); }
+__device__ __forceinline__ uint16_t f2bf(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+__device__ __forceinline__ void store_out(void* y, vq_dtype t, int64_t i, float v) {
+  if (t == VQ_FP32) reinterpret_cast<float*>(y)[i] = v;
+  else if (t == VQ_FP16) reinterpret_cast<uint16_t*>(y)[i] = f2h(v);
+  else reinterpret_cast<uint16_t*>(y)[i] = f2bf(v);
+}
+
+// Copy codebook m into shared memory with rows padded to `pad` halves
+// (8 for d <= 8, 16 above), zeros in the padding.
+__device__ __forceinline__ void stage_book(uint16_t* dst, const uint16_t* __restrict__ src, int k,
+                                           int d, int pad) {
+  const int total = k * pad;
+  for (int i = threadIdx.x; i < total; i += blockDim.x) {
+    const int r = i / pad, e = i - r * pad;
+    dst[i] = (e < d) ? src[static_cast<int64_t>(r) * d + e] : static_cast<uint16_t>(0);
+  }
+}
+
+}  // namespace vqk

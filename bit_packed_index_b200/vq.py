@@ -1,0 +1,243 @@
+"""Python binding of libvq (include/vq.h): argument marshalling only.
+
+Every computation runs in the CUDA kernels behind the C ABI; this module only
+turns torch tensors into pointers, sizes and the current CUDA stream.  There
+is no fallback: if ``libvq.so`` is missing or fails to load, every call raises.
+
+Names follow the C ABI: ``dequant``, ``gemv``, ``gemm``, plus the workspace
+size queries.  A ``Layer`` holds the device tensors of one quantised layer
+(packed index streams, fp16 codebooks, optional fp16 scale and bias).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import re
+import threading
+from dataclasses import dataclass, field
+from typing import List, Optional, Sequence
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libvq.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "vq.h")
+
+VQ_OK, VQ_ERR_INVALID_ARG, VQ_ERR_UNSUPPORTED, VQ_ERR_ALIGNMENT = 0, 1, 2, 3
+VQ_ERR_WORKSPACE, VQ_ERR_CUDA, VQ_ERR_TIMEOUT = 4, 5, 6
+VQ_BF16, VQ_FP16, VQ_FP32 = 0, 1, 2
+
+_DTYPE = {torch.bfloat16: VQ_BF16, torch.float16: VQ_FP16, torch.float32: VQ_FP32}
+
+
+class VQError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str, cuda_error: int = 0):
+        super().__init__(f"{fn}: {msg} (status {status}"
+                         + (f", cudaError {cuda_error})" if status == VQ_ERR_CUDA else ")"))
+        self.status = status
+        self.cuda_error = cuda_error
+
+
+class _Desc(C.Structure):
+    _fields_ = [
+        ("out_features", C.c_int32), ("in_features", C.c_int32),
+        ("vec_dim", C.c_int32), ("n_books", C.c_int32), ("log2k", C.c_int32 * 2),
+        ("idx", C.c_void_p * 2), ("idx_row_words", C.c_int64 * 2),
+        ("codebook", C.c_void_p * 2), ("scale", C.c_void_p), ("bias", C.c_void_p),
+    ]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def exported_names() -> List[str]:
+    """Function names the header declares (VQ_API ...)."""
+    with open(HEADER) as fh:
+        text = fh.read()
+    return re.findall(r"VQ_API\s+[\w\s\*]+?\b(vq_\w+)\s*\(", text)
+
+
+def lib():
+    """Load libvq.so (raises if it is missing: there is no other code path)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"libvq.so not found at {LIB_PATH}; build it with "
+                                   "`python bit_packed_index_b200/build.py`")
+            L = C.CDLL(LIB_PATH)
+            P, I32, I64, SZ = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t
+            L.vq_dequant.argtypes = [P, P, I64, P]
+            L.vq_gemv_workspace_size.argtypes = [P, I32, C.POINTER(SZ)]
+            L.vq_gemv.argtypes = [P, P, C.c_int, I32, I64, P, C.c_int, I64, P, SZ, P]
+            L.vq_gemm_workspace_size.argtypes = [P, I32, C.c_int, C.POINTER(SZ)]
+            L.vq_gemm.argtypes = [P, P, C.c_int, I32, I64, P, C.c_int, I64, P, SZ, P]
+            for fn in ("vq_dequant", "vq_gemv_workspace_size", "vq_gemv",
+                       "vq_gemm_workspace_size", "vq_gemm"):
+                getattr(L, fn).restype = C.c_int
+            L.vq_status_string.argtypes = [C.c_int]
+            L.vq_status_string.restype = C.c_char_p
+            L.vq_last_cuda_error.restype = C.c_int
+            L.vq_abi_version.restype = C.c_int
+            _lib = L
+    return _lib
+
+
+def _check(fn: str, status: int):
+    if status != VQ_OK:
+        L = lib()
+        raise VQError(fn, status, L.vq_status_string(status).decode(),
+                      L.vq_last_cuda_error() if status == VQ_ERR_CUDA else 0)
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+@dataclass
+class Layer:
+    """Device tensors of one quantised layer (see include/vq.h)."""
+    out_features: int
+    in_features: int
+    vec_dim: int
+    log2k: List[int]
+    idx: List[torch.Tensor]            # int32 views of uint32 words [N][row_words]
+    codebooks: List[torch.Tensor]      # float16 [K][d]
+    scale: Optional[torch.Tensor] = None   # float16 [N]
+    bias: Optional[torch.Tensor] = None    # float16 [N]
+    _desc: Optional[_Desc] = field(default=None, repr=False)
+
+    @property
+    def n_books(self) -> int:
+        return len(self.log2k)
+
+    @property
+    def device(self) -> torch.device:
+        return self.idx[0].device
+
+    def desc(self) -> _Desc:
+        if self._desc is None:
+            d = _Desc()
+            d.out_features, d.in_features = self.out_features, self.in_features
+            d.vec_dim, d.n_books = self.vec_dim, self.n_books
+            for m in range(self.n_books):
+                d.log2k[m] = self.log2k[m]
+                d.idx[m] = self.idx[m].data_ptr()
+                d.idx_row_words[m] = self.idx[m].stride(0) if self.idx[m].shape[1] > 0 else 0
+                d.codebook[m] = self.codebooks[m].data_ptr()
+            d.scale = None if self.scale is None else self.scale.data_ptr()
+            d.bias = None if self.bias is None else self.bias.data_ptr()
+            self._desc = d
+        return self._desc
+
+    @classmethod
+    def from_host(cls, out_features: int, in_features: int, vec_dim: int, log2k: Sequence[int],
+                  idx_words: Sequence, codebooks: Sequence, scale=None, bias=None,
+                  device="cuda") -> "Layer":
+        """From numpy arrays: uint32 streams, fp16-bit (uint16) codebooks/scale/bias."""
+        import numpy as np
+
+        def words(a):
+            a = np.ascontiguousarray(a, np.uint32).view(np.int32)
+            return torch.from_numpy(a).to(device)
+
+        def halves(a):
+            if a is None:
+                return None
+            a = np.ascontiguousarray(a, np.uint16).view(np.int16)
+            return torch.from_numpy(a).to(device).view(torch.float16)
+
+        return cls(out_features, in_features, vec_dim, list(log2k),
+                   [words(w) for w in idx_words], [halves(c) for c in codebooks],
+                   halves(scale), halves(bias))
+
+    @classmethod
+    def from_synth(cls, data, device="cuda") -> "Layer":
+        s = data.spec
+        return cls.from_host(s.out_features, s.in_features, s.d, s.log2k, data.idx_words,
+                             data.codebooks, data.scale, data.bias, device)
+
+    def nbytes(self) -> int:
+        n = sum(t.numel() * t.element_size() for t in self.idx + self.codebooks)
+        for t in (self.scale, self.bias):
+            n += 0 if t is None else t.numel() * 2
+        return n
+
+
+def dequant(layer: Layer, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """W_hat, float16 [N][Kin] (or into ``out``, whose row stride is honoured)."""
+    if out is None:
+        out = torch.empty((layer.out_features, layer.in_features), dtype=torch.float16,
+                          device=layer.device)
+    ldw = out.stride(0) if out.dim() == 2 and out.shape[0] > 0 else layer.in_features
+    _check("vq_dequant", lib().vq_dequant(C.byref(layer.desc()), _ptr(out), ldw,
+                                          C.c_void_p(_stream(layer.device))))
+    return out
+
+
+def gemv_workspace_size(layer: Layer, batch: int) -> int:
+    n = C.c_size_t(0)
+    _check("vq_gemv_workspace_size", lib().vq_gemv_workspace_size(C.byref(layer.desc()), batch,
+                                                                  C.byref(n)))
+    return n.value
+
+
+def gemm_workspace_size(layer: Layer, m: int, x_dtype=torch.bfloat16) -> int:
+    n = C.c_size_t(0)
+    _check("vq_gemm_workspace_size", lib().vq_gemm_workspace_size(
+        C.byref(layer.desc()), m, _DTYPE[x_dtype], C.byref(n)))
+    return n.value
+
+
+def _workspace(nbytes: int, device, given: Optional[torch.Tensor]):
+    if nbytes == 0:
+        return None, 0
+    if given is not None:
+        return given, given.numel() * given.element_size()
+    t = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return t, nbytes
+
+
+def gemv(layer: Layer, x: torch.Tensor, out_dtype=torch.bfloat16,
+         out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y [B][N] = x [B][Kin] . W_hat^T for B <= 16 (x bf16 or fp16 on the device)."""
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    batch = x.shape[0]
+    if out is None:
+        out = torch.empty((batch, layer.out_features), dtype=out_dtype, device=layer.device)
+    ws, ws_bytes = _workspace(gemv_workspace_size(layer, batch), layer.device, workspace)
+    ldx = x.stride(0) if batch > 1 else max(x.shape[1], layer.in_features)
+    ldy = out.stride(0) if batch > 1 else max(out.shape[1], layer.out_features)
+    _check("vq_gemv", lib().vq_gemv(C.byref(layer.desc()), _ptr(x), _DTYPE[x.dtype], batch, ldx,
+                                    _ptr(out), _DTYPE[out.dtype], ldy, _ptr(ws), ws_bytes,
+                                    C.c_void_p(_stream(layer.device))))
+    return out
+
+
+def gemm(layer: Layer, x: torch.Tensor, out_dtype=torch.bfloat16,
+         out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y [M][N] = x [M][Kin] . W_hat^T on the tensor cores (x bf16 or fp16)."""
+    m = x.shape[0]
+    if out is None:
+        out = torch.empty((m, layer.out_features), dtype=out_dtype, device=layer.device)
+    ws, ws_bytes = _workspace(gemm_workspace_size(layer, m, x.dtype), layer.device, workspace)
+    ldx = x.stride(0) if m > 1 else max(x.shape[1], layer.in_features)
+    ldy = out.stride(0) if m > 1 else max(out.shape[1], layer.out_features)
+    _check("vq_gemm", lib().vq_gemm(C.byref(layer.desc()), _ptr(x), _DTYPE[x.dtype], m, ldx,
+                                    _ptr(out), _DTYPE[out.dtype], ldy, _ptr(ws), ws_bytes,
+                                    C.c_void_p(_stream(layer.device))))
+    return out
+
+
+def abi_version() -> int:
+    return lib().vq_abi_version()
+
+
+def status_string(status: int) -> str:
+    return lib().vq_status_string(status).decode()

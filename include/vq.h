@@ -1,0 +1,200 @@
+/*
+ * vq.h -- C ABI of libvq: B200 (sm_100a) kernels for linear layers whose
+ * weights are stored as bit-packed codebook indices (VQ / residual VQ).
+ *
+ * The method (what the calls compute)
+ * -----------------------------------
+ * A weight matrix W (out_features N x in_features Kin) is cut, row by row,
+ * into vectors of d consecutive input-dimension weights ("VPTQ Guide: Extreme
+ * 2-Bit Vector Quantization", section "The Information-Theoretic Superiority
+ * of Vector Quantization"; section "Step 2", which slices W.view(-1, v)).
+ * Row o has nvec = ceil(Kin / d) vectors; vector j of row o is replaced by a
+ * b_m-bit index i_m[o][j] into codebook m, C_m in fp16 [K_m = 2^b_m][d], for
+ * one or two codebooks (section "2. Multi-Stage Residual Vector Quantization
+ * (RVQ)": w_hat = C1[idx1] + C2[idx2]; "Vector Quantization for LLM Weights in
+ * Production", section "2. AQLM: Additive Multi-Codebook Vector Quantization":
+ * a sum of M = 1 or 2 centroids).  An optional per-output-row fp16 scale s and
+ * bias t complete the layer (section "1. QuIP#": per-channel scaling).  The
+ * dequantised weight is
+ *
+ *     W_hat[o][j*d + e] = fp16( (C1[i1][e] + C2[i2][e]) * s[o] + t[o] )
+ *
+ * for j*d + e < Kin, each of +, *, + an fp32 operation rounded to nearest even
+ * in that order, then one rounding to fp16 (with one codebook the first sum is
+ * just C1[i1][e]; a missing scale skips the multiply, a missing bias skips the
+ * add).  Components of the last vector past Kin are ignored.  The products are
+ * y = x . W_hat^T ("VPTQ Guide", section "Step 3: Fused Low-Bit VPTQ Linear
+ * Layer"), computed without writing W_hat to global memory, as the pages
+ * describe for production kernels ("Vector Quantization for LLM Weights in
+ * Production", section "2. Lookup Table (LUT) Overhead vs. Bit-Shifting":
+ * fused lookup and accumulation, no intermediate fp16 global writes).
+ *
+ * Storage format of the indices (this library's reading; the pages fix only
+ * the field width b = log2 K, e.g. "16-bit uint per 8 weights")
+ * ---------------------------------------------------------------
+ * One stream per codebook, one stream row per output row, rows idx_row_words
+ * 32-bit words apart.  Field j of a row occupies bits [j*b, j*b + b), bits
+ * numbered least-significant first inside little-endian 32-bit words.  Rows
+ * start 16-byte aligned: idx_row_words is a multiple of 4 and at least
+ * ceil(nvec*b / 128) * 4.  Bits past nvec*b in a row are ignored.  Indices are
+ * unsigned and K = 2^b exactly, so every index is inside its codebook.
+ *
+ * Conventions for every call
+ * --------------------------
+ * - Pointers named "device" must be CUDA device (or managed) memory visible
+ *   to the current device; the caller allocates and owns them.  The library
+ *   keeps no allocation between calls (it caches per-device attributes only).
+ * - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *   default stream).  Argument errors are detected on the host and returned
+ *   before anything is launched; nothing is written then.
+ * - Launch failures return VQ_ERR_CUDA; vq_last_cuda_error() gives the
+ *   cudaError_t.  Kernels never trap and never wait on flags.
+ * - fp16 / bf16 values are passed as their 16-bit patterns.
+ * - All calls are thread-safe; concurrent calls on different streams may not
+ *   share an output or a workspace buffer.
+ */
+#ifndef VQ_H_
+#define VQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VQ_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define VQ_API __attribute__((visibility("default")))
+#else
+#define VQ_API
+#endif
+
+typedef enum vq_status {
+    VQ_OK = 0,
+    VQ_ERR_INVALID_ARG = 1,   /* a size, pointer or field is out of range       */
+    VQ_ERR_UNSUPPORTED = 2,   /* well-formed, but outside what is implemented   */
+    VQ_ERR_ALIGNMENT = 3,     /* a pointer or leading dimension is misaligned   */
+    VQ_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required     */
+    VQ_ERR_CUDA = 5,          /* a CUDA call or kernel launch failed            */
+    VQ_ERR_TIMEOUT = 6        /* reserved: a bounded device-side wait gave up   */
+} vq_status;
+
+typedef enum vq_dtype {
+    VQ_BF16 = 0,
+    VQ_FP16 = 1,
+    VQ_FP32 = 2
+} vq_dtype;
+
+/*
+ * One quantised layer.  All pointers are device pointers.
+ *   out_features   N >= 0
+ *   in_features    Kin >= 0 (need not be a multiple of vec_dim)
+ *   vec_dim        d, 1..16
+ *   n_books        1 or 2 (main codebook plus optional residual/additive one)
+ *   log2k[m]       b_m, 1..16; K_m = 2^b_m
+ *   idx[m]         packed stream of book m, [N][idx_row_words[m]] uint32,
+ *                  16-byte aligned
+ *   idx_row_words[m]  row stride in 32-bit words, a multiple of 4,
+ *                  >= ceil(nvec*b_m / 128) * 4
+ *   codebook[m]    fp16 [K_m][d] row-major, 16-byte aligned, finite values
+ *   scale          fp16 [N], or NULL for no scale
+ *   bias           fp16 [N], or NULL for no bias
+ * Entries for m >= n_books are ignored.
+ */
+typedef struct vq_layer_desc {
+    int32_t out_features;
+    int32_t in_features;
+    int32_t vec_dim;
+    int32_t n_books;
+    int32_t log2k[2];
+    const uint32_t* idx[2];
+    int64_t idx_row_words[2];
+    const uint16_t* codebook[2];
+    const uint16_t* scale;
+    const uint16_t* bias;
+} vq_layer_desc;
+
+/*
+ * vq_dequant -- write W_hat (fp16 [N][ldw], device) exactly as defined above:
+ * bit-exact with the fixed-order fp32 definition.  Columns >= Kin of each row
+ * are not written.  ldw >= Kin.  Follows "VPTQ Guide", section "Step 2"
+ * (ResidualVectorQuantizer.dequantize) with the scale and bias of the layer.
+ * Errors: VQ_ERR_INVALID_ARG (bad layer, NULL w_hat with N*Kin > 0, ldw < Kin),
+ * VQ_ERR_ALIGNMENT (misaligned idx/codebook), VQ_ERR_CUDA.
+ */
+VQ_API vq_status vq_dequant(const vq_layer_desc* layer, uint16_t* w_hat, int64_t ldw, void* stream);
+
+/*
+ * vq_gemv_workspace_size -- bytes of device workspace vq_gemv needs for this
+ * layer and batch (0 when it needs none).  Host-only; launches nothing.
+ */
+VQ_API vq_status vq_gemv_workspace_size(const vq_layer_desc* layer, int32_t batch, size_t* bytes);
+
+/*
+ * vq_gemv -- decode-time product y[b][o] = sum_k x[b][k] * W_hat[o][k] for
+ * b < batch (1..16), fp32 accumulation, without materialising W_hat.  The
+ * pages place this regime at B = 1 to 8, memory-bandwidth bound
+ * ("Vector Quantization for LLM Weights in Production", section "1. Prefill
+ * vs. Decode Bottlenecks"); the fused lookup-and-accumulate kernel is the one
+ * "VPTQ Guide", section "Step 3", describes.
+ *   x        device, x_dtype (VQ_BF16 or VQ_FP16) [batch][ldx], ldx >= Kin
+ *   y        device, y_dtype (VQ_BF16, VQ_FP16 or VQ_FP32) [batch][ldy], ldy >= N
+ *   workspace  device scratch of at least vq_gemv_workspace_size() bytes
+ *            (may be NULL when that size is 0), 256-byte aligned; its contents
+ *            on entry do not matter
+ * Scale and bias are applied as y = s[o] * sum_k x[k] (C1+C2)[o][k]
+ * + t[o] * sum_k x[k], equal to the definition up to the fp16 rounding of
+ * W_hat (well inside a 2e-3 normwise relative error).
+ * Errors: VQ_ERR_INVALID_ARG, VQ_ERR_UNSUPPORTED (batch > 16), VQ_ERR_ALIGNMENT
+ * (x or y not aligned to its element size), VQ_ERR_WORKSPACE, VQ_ERR_CUDA.
+ */
+VQ_API vq_status vq_gemv(const vq_layer_desc* layer, const void* x, vq_dtype x_dtype, int32_t batch,
+                  int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy, void* workspace,
+                  size_t workspace_bytes, void* stream);
+
+/*
+ * vq_gemm_workspace_size -- bytes of device workspace vq_gemm needs for this
+ * layer, row count m and activation type.  Host-only.
+ */
+VQ_API vq_status vq_gemm_workspace_size(const vq_layer_desc* layer, int32_t m, vq_dtype x_dtype,
+                                 size_t* bytes);
+
+/*
+ * vq_gemm -- prefill product y[i][o] = sum_k x[i][k] * W_hat[o][k] for
+ * i < m, on the tcgen05 tensor cores (fp16 x fp16 products, fp32 accumulation
+ * in tensor memory); W_hat tiles are produced on chip from the index streams
+ * and never written to global memory.  The pages call prefill the
+ * compute-bound regime where lookups compete with the matrix multiply
+ * ("Vector Quantization for LLM Weights in Production", section "1. Prefill
+ * vs. Decode Bottlenecks", and the "GEMV / Tensor Core Dot Products" stage of
+ * its dequantisation diagram).
+ *   x        device, x_dtype (VQ_BF16 or VQ_FP16) [m][ldx]; 16-byte aligned,
+ *            ldx a multiple of 8, ldx >= Kin.  bf16 activations are converted
+ *            to fp16 operands (exact for |x| in [2^-14, 65504]; smaller values
+ *            become fp16 subnormals, larger ones overflow).
+ *   y        device, y_dtype [m][ldy]; ldy >= N
+ *   workspace  device scratch of at least vq_gemm_workspace_size() bytes,
+ *            256-byte aligned
+ * Scale and bias are applied in the epilogue as for vq_gemv.
+ * Errors: as vq_gemv; VQ_ERR_UNSUPPORTED for vec_dim > 8 or m > 2^30.
+ */
+VQ_API vq_status vq_gemm(const vq_layer_desc* layer, const void* x, vq_dtype x_dtype, int32_t m,
+                  int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy, void* workspace,
+                  size_t workspace_bytes, void* stream);
+
+/* Static description of a status code (never NULL). */
+VQ_API const char* vq_status_string(vq_status status);
+
+/* The cudaError_t of the last VQ_ERR_CUDA returned on this host thread. */
+VQ_API int vq_last_cuda_error(void);
+
+/* VQ_ABI_VERSION of the loaded library. */
+VQ_API int vq_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VQ_H_ */
