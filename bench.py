@@ -1,0 +1,462 @@
+#!/usr/bin/env python
+"""Benchmark of the bit-packed VQ/RVQ hot path on B200 (one JSON line).
+
+Step = one decode pass of the Llama-3-70B-shaped MLP at 2.0 bits per weight:
+gate_proj and up_proj (28672 x 8192) and down_proj (8192 x 28672), d = 8, one
+K = 2^16 fp16 codebook, per-row fp16 scale and bias, batch B = 1, through
+vq_gemv.  Two copies of the three layers (352 MB of index streams) are used
+in turn, so every step reads its weights from HBM, not from the 126 MB L2.
+
+value  = algorithmic bytes moved per step (packed indices + codebook + scale
+         and bias + activations + outputs) x steps x ranks / timed region,
+         in GB/s; the timed region is bracketed by a barrier and a device
+         synchronise on both sides and is the max over ranks.
+e2e    = the same metric through the public Python API with the activations
+         in pinned host memory: each step copies x to the device, runs the
+         layer and copies y back.
+gemm   = the prefill GEMM (x [2048, 8192] bf16, 8192 x 8192 layer, K = 2^16
+         + residual K = 2^8, 3.0 bpw) through vq_gemm, in TFLOP/s.
+roofline, cpu_baseline, clocks and gpu_launches are described beside the
+keys they fill.  ``--impl reference`` times the CPU oracle on the same
+metric instead (a bounded sample of the same workload per step).
+
+Multi-GPU (torchrun): every rank runs its own copy of the step (the layer
+rows shard with no exchange), so scaling is weak and no collective touches
+the data path; NCCL is used only for the barrier and the max of the times.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+from synth import WORKLOADS  # noqa: E402
+
+METRIC = "VQ-GEMV µs/layer & achieved HBM GB/s (% of peak) at 2 bpw; GEMM TFLOP/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DECODE = "llama3_70b_mlp"
+PREFILL = "prefill_8192"
+PREFILL_M = 2048
+BATCH = 1
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK), "fallback"
+
+
+def alg_bytes(spec, batch: int) -> float:
+    """Bytes the layer must move once: packed indices (nvec * b bits per
+    row), each codebook once, fp16 scale and bias, bf16 x and y."""
+    idx = sum(spec.out_features * spec.nvec * b / 8.0 for b in spec.log2k)
+    books = sum((1 << b) * spec.d * 2 for b in spec.log2k)
+    affine = 2 * spec.out_features * (int(spec.scale_range is not None) + int(spec.bias_std is not None))
+    return idx + books + affine + 2.0 * batch * spec.in_features + 2.0 * batch * spec.out_features
+
+
+# -- distributed plumbing (timing only; no collective on the data path) ------
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_dist(world: int, backend: str):
+    if world <= 1:
+        return None
+    import torch.distributed as dist
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def reduce_max(value: float, dist_mod, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity on one rank)."""
+    if dist_mod is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist_mod, device=None):
+    if dist_mod is not None:
+        if device is not None:
+            dist_mod.barrier(device_ids=[device.index])
+        else:
+            dist_mod.barrier()
+
+
+# -- clocks during the timed region ------------------------------------------
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 50 ms while active."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as fh:
+                for ln in fh:
+                    parts = [p.strip() for p in ln.split(",")]
+                    if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                        rows.append(parts)
+        finally:
+            if self.path and os.path.exists(self.path):
+                os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+# -- the oracle on the host (reference arm and cpu_baseline) ------------------
+
+def oracle_rate(target_s: float, spec_seed_pairs, x_list):
+    """Run the CPU oracle on a growing sample of output rows of the decode
+    layers until one pass takes about target_s; return (GB/s, rows, seconds,
+    threads).  Bytes are the algorithmic bytes of the rows processed."""
+    import oracle
+    datas = [synth.make_layer(spec, seed) for spec, seed in spec_seed_pairs]
+    rows = 16
+    while True:
+        t0 = time.perf_counter()
+        nbytes = 0.0
+        for data, x in zip(datas, x_list):
+            r = min(rows, data.spec.out_features)
+            oracle.linear(data, x, rows=np.arange(r))
+            nbytes += alg_bytes(data.spec, x.shape[0]) * r / data.spec.out_features
+        dt = time.perf_counter() - t0
+        if dt >= target_s or rows >= max(d.spec.out_features for d in datas):
+            return nbytes / dt / 1e9, rows, dt, oracle.num_threads()
+        rows = int(rows * min(8.0, max(1.5, 1.2 * target_s / max(dt, 1e-3))))
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = WORKLOADS[DECODE]
+    xs = [synth.make_x(w.x_seed + i, BATCH, spec.in_features, w.outlier_frac)
+          for i, (spec, _) in enumerate(w.layers)]
+    per_step = max(0.02, min(6.0, 120.0 / max(1, args.steps + args.warmup)))
+    gbs, rows, dt, cores = oracle_rate(per_step, w.layers, xs)
+    import oracle
+    datas = [synth.make_layer(spec, seed) for spec, seed in w.layers]
+    for _ in range(args.warmup):
+        for d, x in zip(datas, xs):
+            oracle.linear(d, x, rows=np.arange(min(rows, d.spec.out_features)))
+    t0 = time.perf_counter()
+    nbytes = 0.0
+    for _ in range(args.steps):
+        for d, x in zip(datas, xs):
+            r = min(rows, d.spec.out_features)
+            oracle.linear(d, x, rows=np.arange(r))
+            nbytes += alg_bytes(d.spec, BATCH) * r / d.spec.out_features
+    dt = time.perf_counter() - t0
+    value = nbytes / dt / 1e9
+    sample = (f"first {rows} output rows of each of gate/up/down (B=1) per step, "
+              f"oracle dequantise + fp64 dot products")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / max(1, args.steps) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": decode_config(),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def decode_config():
+    w = WORKLOADS[DECODE]
+    return {
+        "workload": "llama3_70b_mlp decode, B=1: gate_proj + up_proj 28672x8192, down_proj "
+                    "8192x28672; d=8, one K=2^16 fp16 codebook (2.0 bpw), fp16 scale/bias",
+        "batch": BATCH, "layers": [s.name for s, _ in w.layers], "bpw": 2.0,
+        "x": "bf16 ~N(0,1), 0.1% outlier columns x20",
+        "l2": "inputs larger than L2: two copies of the three layers (352 MB of indices) used in turn",
+        "parallelism": "replicas (each rank runs its own step; no collective on the data path)",
+    }
+
+
+# -- the GPU arm ----------------------------------------------------------------
+
+def run_gpu(args):
+    import torch
+    from bit_packed_index_b200 import vq
+
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the CPU oracle runs with --impl reference)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_mod = init_dist(world, "nccl")
+    peaks, peak_src = load_peaks()
+
+    w = WORKLOADS[DECODE]
+    specs = [s for s, _ in w.layers]
+    copies = []
+    for c in range(2):
+        layers = []
+        for spec, seed in w.layers:
+            layers.append(vq.Layer.from_synth(synth.make_layer(spec, seed + 1000 * c + 17 * rank), dev))
+        copies.append(layers)
+    xs_host = [synth.make_x(w.x_seed + i, BATCH, s.in_features, w.outlier_frac) for i, s in enumerate(specs)]
+    xs = [torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16) for x in xs_host]
+    ys = [torch.empty((BATCH, s.out_features), dtype=torch.bfloat16, device=dev) for s in specs]
+    ws = []
+    for k in range(3):
+        need = max(vq.gemv_workspace_size(copies[c][k], BATCH) for c in range(2))
+        ws.append(torch.empty(max(need, 256), dtype=torch.uint8, device=dev))
+    step_bytes = sum(alg_bytes(s, BATCH) for s in specs)
+
+    def step(i, events=None):
+        layers = copies[i & 1]
+        for k in range(3):
+            if events is not None:
+                events[k][0].record()
+            vq.gemv(layers[k], xs[k], out=ys[k], workspace=ws[k])
+            if events is not None:
+                events[k][1].record()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+            for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    uuid = str(getattr(torch.cuda.get_device_properties(local), "uuid", "") or "")
+    gpu_id = ("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or str(local))
+    with ClockSampler(gpu_id) as clocks:
+        barrier(dist_mod, dev)
+        torch.cuda.synchronize()
+        launches0 = vq.kernel_launches()
+        t_start.record()
+        for i in range(args.steps):
+            step(i, evs[i])
+        t_end.record()
+        torch.cuda.synchronize()
+        launches = vq.kernel_launches() - launches0
+        barrier(dist_mod, dev)
+    ms_total = reduce_max(t_start.elapsed_time(t_end), dist_mod, dev)
+    ms_step = ms_total / args.steps
+    value = step_bytes * args.steps * world / (ms_total * 1e-3) / 1e9
+
+    # live per-layer roofline of the dominant kernel (vq_gemv's gemv_kernel)
+    per_layer_ms = [statistics.mean(evs[i][k][0].elapsed_time(evs[i][k][1]) for i in range(args.steps))
+                    for k in range(3)]
+    achieved = step_bytes / (sum(per_layer_ms) * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "kernel": "gemv_kernel", "peak_source": peak_src,
+                "per_layer_us": {s.name: ms * 1e3 for s, ms in zip(specs, per_layer_ms)},
+                "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS}
+
+    # e2e through the public API with pinned host activations and outputs
+    xh = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in xs_host]
+    yh = [torch.empty((BATCH, s.out_features), dtype=torch.bfloat16).pin_memory() for s in specs]
+
+    def e2e_step(i):
+        layers = copies[i & 1]
+        for k in range(3):
+            xs[k].copy_(xh[k], non_blocking=True)
+            vq.gemv(layers[k], xs[k], out=ys[k], workspace=ws[k])
+            yh[k].copy_(ys[k], non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(dist_mod, dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(args.steps):
+        e2e_step(i)
+    b.record()
+    torch.cuda.synchronize()
+    barrier(dist_mod, dev)
+    e2e_ms = reduce_max(a.elapsed_time(b), dist_mod, dev)
+    e2e = {"value": step_bytes * args.steps * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+           "h2d_bytes_per_step": sum(x.numel() * 2 for x in xh),
+           "d2h_bytes_per_step": sum(y.numel() * 2 for y in yh),
+           "ms_per_step": e2e_ms / args.steps}
+
+    gemm = run_gemm(dev, peaks, peak_src, vq)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": decode_config(),
+        "us_per_layer": ms_step * 1e3 / 3,
+        "hbm_pct_of_measured": 100.0 * value / world / peaks["hbm_gbs"],
+        "hbm_pct_of_nominal_8tbs": 100.0 * value / world / NOMINAL_HBM_GBS,
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clocks.summary(),
+        "gemm": gemm,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, rows, dt, cores = oracle_rate(10.0, w.layers, xs_host)
+        line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                "sample": f"first {rows} output rows of each of gate/up/down "
+                                          f"(B=1), {dt:.1f} s of oracle work"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_mod is not None:
+        dist_mod.destroy_process_group()
+    return 0
+
+
+def run_gemm(dev, peaks, peak_src, vq):
+    """Prefill GEMM through vq_gemm, L2 flushed between timed calls."""
+    import torch
+    w = WORKLOADS[PREFILL]
+    spec, seed = w.layers[0]
+    layer = vq.Layer.from_synth(synth.make_layer(spec, seed), dev)
+    x = torch.from_numpy(synth.make_x(w.x_seed, PREFILL_M, spec.in_features).view(np.int16)).to(dev)
+    x = x.view(torch.bfloat16)
+    y = torch.empty((PREFILL_M, spec.out_features), dtype=torch.bfloat16, device=dev)
+    wsp = torch.empty(vq.gemm_workspace_size(layer, PREFILL_M), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        vq.gemm(layer, x, out=y, workspace=wsp)
+    times = []
+    for _ in range(10):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        vq.gemm(layer, x, out=y, workspace=wsp)
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    torch.cuda.synchronize()
+    status = int(wsp[:4].view(torch.int32).item())
+    ms = statistics.median(times)
+    flops = 2.0 * PREFILL_M * spec.out_features * spec.in_features
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": f"prefill_8192: x [{PREFILL_M},8192] bf16, W 8192x8192, d=8, K=2^16 + "
+                        f"residual K=2^8 (3.0 bpw), fp16 operands, fp32 accumulate, bf16 out",
+            "tflops": tf, "us": ms * 1e3, "device_status": status,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"],
+                         "peak_source": peak_src + " (bf16 burst; fp16 nominal rate is the same)"}}
+
+
+def run_profile(args):
+    """A few launches of one call on its bench workload, nothing timed: the
+    command the committed ncu summaries were captured from."""
+    import torch
+    from bit_packed_index_b200 import vq
+    dev = torch.device("cuda", 0)
+    if args.profile in ("gemv", "dequant"):
+        w = WORKLOADS[DECODE]
+        spec, seed = w.layers[0]
+        layer = vq.Layer.from_synth(synth.make_layer(spec, seed), dev)
+        x = torch.from_numpy(synth.make_x(w.x_seed, BATCH, spec.in_features, w.outlier_frac)
+                             .view(np.int16)).to(dev).view(torch.bfloat16)
+        out = (torch.empty((spec.out_features, spec.in_features), dtype=torch.float16, device=dev)
+               if args.profile == "dequant" else
+               torch.empty((BATCH, spec.out_features), dtype=torch.bfloat16, device=dev))
+        ws = torch.empty(max(256, vq.gemv_workspace_size(layer, BATCH)), dtype=torch.uint8, device=dev)
+        for _ in range(args.profile_launches):
+            if args.profile == "dequant":
+                vq.dequant(layer, out=out)
+            else:
+                vq.gemv(layer, x, out=out, workspace=ws)
+    else:
+        w = WORKLOADS[PREFILL]
+        spec, seed = w.layers[0]
+        layer = vq.Layer.from_synth(synth.make_layer(spec, seed), dev)
+        x = torch.from_numpy(synth.make_x(w.x_seed, PREFILL_M, spec.in_features).view(np.int16))
+        x = x.to(dev).view(torch.bfloat16)
+        y = torch.empty((PREFILL_M, spec.out_features), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(vq.gemm_workspace_size(layer, PREFILL_M), dtype=torch.uint8, device=dev)
+        for _ in range(args.profile_launches):
+            vq.gemm(layer, x, out=y, workspace=ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": args.profile, "launches": args.profile_launches,
+                      "kernel_launches": vq.kernel_launches()}))
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["gemv", "gemm", "dequant"],
+                    help="run a few untimed launches of one call on its workload (for ncu)")
+    ap.add_argument("--profile-launches", type=int, default=3)
+    args = ap.parse_args(argv)
+    if args.profile:
+        return run_profile(args)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

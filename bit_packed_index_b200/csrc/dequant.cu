@@ -97,6 +97,7 @@ cudaError_t launch_dq(const Layer& L, uint16_t* w, int64_t ldw, int smem_mask, s
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
+  count_launch();
   k<<<grid, kDqThreads, smem, stream>>>(L, w, ldw, smem_mask, vec_store);
   return cudaGetLastError();
 }

@@ -460,6 +460,7 @@ cudaError_t launch_kernel(const CUtensorMap& ma, const CUtensorMap& mb, const Ge
   auto k = vq_gemm_kernel<MODE, B1, B2>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
+  count_launch();
   k<<<grid, kThreads, smem, stream>>>(ma, mb, g);
   return cudaGetLastError();
 }
@@ -483,6 +484,7 @@ vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t
 
   {
     const int warps = 8;
+    count_launch();
     gemm_prep<<<(m + warps - 1) / warps, warps * 32, 0, stream>>>(
         static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, m, L.kin, ldx, x16, lay.kp, rowsum, status);
     cudaError_t e = cudaGetLastError();

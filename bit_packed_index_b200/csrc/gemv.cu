@@ -183,6 +183,7 @@ cudaError_t launch_bt(const Layer& L, const GemvPlan& p, const void* x, bool x_f
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.grid_x, p.nsplit);
+  count_launch();
   k<<<grid, kGvThreads, p.smem, stream>>>(L, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, batch,
                                           ldx, p.vps, p.rpb, p.books_in_smem, p.book_bytes, y, yt,
                                           ldy, p.nsplit > 1 ? ws : nullptr);
@@ -204,6 +205,11 @@ cudaError_t launch_d(const Layer& L, const GemvPlan& p, const void* x, bool xf, 
 }  // namespace
 
 vq_status plan_gemv(const Layer& L, int batch, GemvPlan* p) {
+  if (batch == 1 && gemv1_supported(L)) {
+    plan_gemv1(L, p);
+    if (p->smem <= device_smem_optin()) return VQ_OK;
+  }
+  p->fast = 0;
   int bt = 1;
   while (bt < batch) bt <<= 1;
   p->bt = bt;
@@ -245,7 +251,9 @@ vq_status launch_gemv(const Layer& L, const GemvPlan& p, const void* x, bool x_f
   }
   const int D = (L.d == 8) ? 8 : (L.d == 6 ? 6 : 0);
   cudaError_t e;
-  if (L.nb == 1) {
+  if (p.fast) {
+    e = launch_gemv1(L, p, x, x_fp16, y, yt, ws, stream);
+  } else if (L.nb == 1) {
     e = D == 8 ? launch_d<8, 1>(L, p, x, x_fp16, batch, ldx, y, yt, ldy, ws, stream)
       : D == 6 ? launch_d<6, 1>(L, p, x, x_fp16, batch, ldx, y, yt, ldy, ws, stream)
                : launch_d<0, 1>(L, p, x, x_fp16, batch, ldx, y, yt, ldy, ws, stream);
@@ -257,6 +265,7 @@ vq_status launch_gemv(const Layer& L, const GemvPlan& p, const void* x, bool x_f
   if (e == cudaSuccess && p.nsplit > 1) {
     const int64_t total = static_cast<int64_t>(batch) * L.n;
     const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 4 * device_sm_count()));
+    count_launch();
     gemv_finalize<<<blocks, 256, 0, stream>>>(ws, p.nsplit, batch, L.n, y, yt, ldy);
     e = cudaGetLastError();
   }

@@ -1,6 +1,7 @@
 // vq_api.cu -- the extern "C" entry points of libvq (declared in include/vq.h):
 // argument validation on the host, then one launcher per call.  Nothing is
 // launched when an argument is rejected.
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -12,6 +13,7 @@ namespace vqk {
 namespace {
 
 thread_local int g_last_cuda_error = 0;
+std::atomic<uint64_t> g_launches{0};
 
 struct DeviceAttrs {
   int sms = 0;
@@ -46,6 +48,8 @@ vq_status cuda_status(cudaError_t e) {
   g_last_cuda_error = static_cast<int>(e);
   return VQ_ERR_CUDA;
 }
+
+void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
 int device_sm_count() { return attrs_for_current_device().sms; }
 int device_smem_optin() { return attrs_for_current_device().smem_optin; }
@@ -195,5 +199,7 @@ const char* vq_status_string(vq_status status) {
 int vq_last_cuda_error(void) { return g_last_cuda_error; }
 
 int vq_abi_version(void) { return VQ_ABI_VERSION; }
+
+uint64_t vq_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"

@@ -38,6 +38,7 @@ struct Layer {
 // ---------------------------------------------------------------------------
 vq_status check_layer(const vq_layer_desc* desc, Layer* out);
 vq_status cuda_status(cudaError_t e);  // records e, returns VQ_ERR_CUDA (or VQ_OK)
+void count_launch(int n = 1);          // adds to the process-wide kernel launch counter
 int device_sm_count();
 int device_smem_optin();               // max dynamic shared memory per block, bytes
 
@@ -58,8 +59,13 @@ struct GemvPlan {
   int books_in_smem;  // bit m set: book m staged in shared memory
   int book_bytes;     // shared memory taken by the staged books
   size_t ws_bytes;
+  int fast = 0;       // 1: the single-row kernel of gemv1.cu
 };
 vq_status plan_gemv(const Layer& L, int batch, GemvPlan* plan);
+bool gemv1_supported(const Layer& L);
+void plan_gemv1(const Layer& L, GemvPlan* plan);
+cudaError_t launch_gemv1(const Layer& L, const GemvPlan& plan, const void* x, bool x_fp16, void* y,
+                         vq_dtype y_dtype, float* ws, cudaStream_t stream);
 vq_status launch_gemv(const Layer& L, const GemvPlan& plan, const void* x, bool x_fp16, int batch,
                       int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy, float* ws,
                       cudaStream_t stream);

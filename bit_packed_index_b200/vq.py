@@ -80,6 +80,7 @@ def lib():
             L.vq_status_string.restype = C.c_char_p
             L.vq_last_cuda_error.restype = C.c_int
             L.vq_abi_version.restype = C.c_int
+            L.vq_kernel_launches.restype = C.c_uint64
             _lib = L
     return _lib
 
@@ -233,6 +234,11 @@ def gemm(layer: Layer, x: torch.Tensor, out_dtype=torch.bfloat16,
                                     _ptr(out), _DTYPE[out.dtype], ldy, _ptr(ws), ws_bytes,
                                     C.c_void_p(_stream(layer.device))))
     return out
+
+
+def kernel_launches() -> int:
+    """Kernels this library has launched in this process (host counter)."""
+    return int(lib().vq_kernel_launches())
 
 
 def abi_version() -> int:

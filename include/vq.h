@@ -193,6 +193,11 @@ VQ_API int vq_last_cuda_error(void);
 /* VQ_ABI_VERSION of the loaded library. */
 VQ_API int vq_abi_version(void);
 
+/* Host-only: number of CUDA kernels this library has launched in this process
+ * (all threads, all devices).  Lets a caller count the device work behind a
+ * sequence of calls. */
+VQ_API uint64_t vq_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif

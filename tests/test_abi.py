@@ -17,13 +17,14 @@ def test_every_declared_symbol_is_exported(lib):
     names = vq.exported_names()
     assert set(names) == {"vq_dequant", "vq_gemv_workspace_size", "vq_gemv",
                           "vq_gemm_workspace_size", "vq_gemm", "vq_status_string",
-                          "vq_last_cuda_error", "vq_abi_version"}
+                          "vq_last_cuda_error", "vq_abi_version", "vq_kernel_launches"}
     for n in names:
         assert hasattr(lib, n), n
 
 
 def test_host_only_calls(lib):
     assert lib.vq_abi_version() == 1
+    assert vq.kernel_launches() == 0          # nothing launched in this process
     for s in range(7):
         assert lib.vq_status_string(s)
     assert lib.vq_status_string(99) == b"unknown status"

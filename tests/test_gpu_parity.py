@@ -126,6 +126,35 @@ def test_gemv_output_types_and_fp16_input(out_dtype):
     assert np.array_equal(yb.view(torch.int16).cpu().numpy().view(np.uint16), oracle.f32_to_bf16(y32))
 
 
+# Single-row (batch 1) kernel: every supported (d, index widths) pair, ragged
+# rows and columns, partial 256-vector chunks, and narrow layers that take the
+# split along the input dimension.
+FAST_SPECS = [
+    LayerSpec(300, 8 * 300 + 5, 8, (16,), (0.02,)),
+    LayerSpec(300, 8 * 300 + 5, 8, (16, 8), (0.02, 0.005)),
+    LayerSpec(300, 8 * 300 + 5, 8, (12, 8), (0.02, 0.005)),
+    LayerSpec(300, 8 * 300 + 5, 8, (8, 8), (0.02, 0.005)),
+    LayerSpec(257, 8 * 700, 8, (8,), (0.02,), None, None),
+    LayerSpec(300, 6 * 600 + 4, 6, (12, 4), (0.02, 0.005)),
+    LayerSpec(129, 6 * 300 + 1, 6, (12,), (0.02,)),
+    LayerSpec(64, 8 * 4000, 8, (16,), (0.02,)),
+    LayerSpec(40, 6 * 3000 + 2, 6, (12, 4), (0.02, 0.005)),
+    LayerSpec(1, 8, 8, (16,), (0.02,)),
+]
+
+
+@pytest.mark.parametrize("i", range(len(FAST_SPECS)))
+def test_gemv_single_row_kernel(i):
+    spec = FAST_SPECS[i]
+    data = synth.make_layer(spec, seed=1300 + i, pad_garbage=True)
+    layer = _dev_layer(data)
+    for fp16 in (False, True):
+        x = synth.make_x(90 + i, 1, spec.in_features, outlier_frac=0.01, as_fp16=fp16)
+        ref = oracle.linear(data, x, x_is_fp16=fp16)
+        y = _vq().gemv(layer, _x_dev(x, fp16), out_dtype=torch.float32)
+        assert_close(_f64(y), ref, "float32")
+
+
 def test_gemv_strided_x_and_y():
     spec = LayerSpec(70, 600, 6, (12, 4), (0.02, 0.005))
     data = synth.make_layer(spec, seed=34)
