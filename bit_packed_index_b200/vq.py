@@ -71,9 +71,10 @@ def lib():
             L.vq_dequant.argtypes = [P, P, I64, P]
             L.vq_gemv_workspace_size.argtypes = [P, I32, C.POINTER(SZ)]
             L.vq_gemv.argtypes = [P, P, C.c_int, I32, I64, P, C.c_int, I64, P, SZ, P]
+            L.vq_gemv_noalloc.argtypes = [P, P, C.c_int, I32, I64, P, C.c_int, I64, P]
             L.vq_gemm_workspace_size.argtypes = [P, I32, C.c_int, C.POINTER(SZ)]
             L.vq_gemm.argtypes = [P, P, C.c_int, I32, I64, P, C.c_int, I64, P, SZ, P]
-            for fn in ("vq_dequant", "vq_gemv_workspace_size", "vq_gemv",
+            for fn in ("vq_dequant", "vq_gemv_workspace_size", "vq_gemv", "vq_gemv_noalloc",
                        "vq_gemm_workspace_size", "vq_gemm"):
                 getattr(L, fn).restype = C.c_int
             L.vq_status_string.argtypes = [C.c_int]
@@ -218,6 +219,28 @@ def gemv(layer: Layer, x: torch.Tensor, out_dtype=torch.bfloat16,
     _check("vq_gemv", lib().vq_gemv(C.byref(layer.desc()), _ptr(x), _DTYPE[x.dtype], batch, ldx,
                                     _ptr(out), _DTYPE[out.dtype], ldy, _ptr(ws), ws_bytes,
                                     C.c_void_p(_stream(layer.device))))
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def gemv_noalloc(layer: Layer, x: torch.Tensor, out_dtype=torch.bfloat16,
+                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """vq_gemv without a workspace, for callers that cannot allocate device
+    memory where they run the layer: the split-K scratch is a fixed
+    NOALLOC_SCRATCH_BYTES array inside the library (see vq_gemv_noalloc in
+    include/vq.h).  Pass ``out`` to keep the call free of allocations."""
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    batch = x.shape[0]
+    if out is None:
+        out = torch.empty((batch, layer.out_features), dtype=out_dtype, device=layer.device)
+    ldx = x.stride(0) if batch > 1 else max(x.shape[1], layer.in_features)
+    ldy = out.stride(0) if batch > 1 else max(out.shape[1], layer.out_features)
+    _check("vq_gemv_noalloc", lib().vq_gemv_noalloc(
+        C.byref(layer.desc()), _ptr(x), _DTYPE[x.dtype], batch, ldx, _ptr(out),
+        _DTYPE[out.dtype], ldy, C.c_void_p(_stream(layer.device))))
     return out
 
 

@@ -155,6 +155,31 @@ VQ_API vq_status vq_gemv(const vq_layer_desc* layer, const void* x, vq_dtype x_d
                   size_t workspace_bytes, void* stream);
 
 /*
+ * vq_gemv_noalloc -- vq_gemv for callers that cannot allocate device memory
+ * where they run the layer (a serving loop working inside a pre-reserved pool,
+ * a plug-in called from another framework's allocator-controlled context, or
+ * code with no CUDA allocation API at hand).  The pages have no counterpart:
+ * this is a deployment convenience of this library.  Same arguments and
+ * results as vq_gemv, minus the workspace: the split-K scratch comes from a
+ * fixed device array of VQ_NOALLOC_SCRATCH_BYTES inside the library, which
+ * every GPU that loads the library holds until the process exits.  The call
+ * allocates nothing (no cudaMalloc, no allocating library routine).
+ *   - Returns VQ_ERR_WORKSPACE when this layer and batch need more scratch than
+ *     VQ_NOALLOC_SCRATCH_BYTES (vq_gemv_workspace_size() tells in advance).
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the array; calls whose kernels overlap on
+ *     the GPU (e.g. on two streams at once) race on it and must be ordered by
+ *     the caller.  No part of the array needs to start at zero, so its
+ *     contents from an earlier call do not matter.
+ */
+#define VQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+VQ_API vq_status vq_gemv_noalloc(const vq_layer_desc* layer, const void* x, vq_dtype x_dtype,
+                                 int32_t batch, int64_t ldx, void* y, vq_dtype y_dtype,
+                                 int64_t ldy, void* stream);
+
+/*
  * vq_gemm_workspace_size -- bytes of device workspace vq_gemm needs for this
  * layer, row count m and activation type.  Host-only.
  */

@@ -15,7 +15,7 @@ def lib():
 
 def test_every_declared_symbol_is_exported(lib):
     names = vq.exported_names()
-    assert set(names) == {"vq_dequant", "vq_gemv_workspace_size", "vq_gemv",
+    assert set(names) == {"vq_dequant", "vq_gemv_workspace_size", "vq_gemv", "vq_gemv_noalloc",
                           "vq_gemm_workspace_size", "vq_gemm", "vq_status_string",
                           "vq_last_cuda_error", "vq_abi_version", "vq_kernel_launches"}
     for n in names:
