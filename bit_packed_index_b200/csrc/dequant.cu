@@ -44,6 +44,19 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(Layer L, uint16_t* 
     if (smem_mask) __syncthreads();
   }
   const int d = (D > 0) ? D : L.d;
+  // Centroid row k of book m: staged rows from shared memory; for an
+  // L2-served d = 8 book an evict-last load keeps its rows in L1.
+  auto fetch = [&](int m, uint32_t k, float* c) {
+    if (D == 8 && !(smem_mask & (1 << m))) {
+      uint4 v;
+      asm volatile("ld.global.nc.L1::evict_last.v4.u32 {%0,%1,%2,%3}, [%4];"
+                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                   : "l"(bv[m].base + static_cast<size_t>(k) * 8));
+      unpack8(v, c);
+    } else {
+      load_centroid<D>(bv[m], k, d, c);
+    }
+  };
   for (int64_t o = blockIdx.x; o < L.n; o += gridDim.x) {
     const bool has_s = L.scale != nullptr, has_t = L.bias != nullptr;
     const float s = has_s ? h2f(L.scale[o]) : 1.0f;
@@ -51,38 +64,57 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(Layer L, uint16_t* 
     const uint32_t* row0 = L.idx[0] + o * L.rw[0];
     const uint32_t* row1 = (NB == 2) ? L.idx[1] + o * L.rw[1] : nullptr;
     uint16_t* wrow = w + o * ldw;
-    for (int j = threadIdx.x; j < L.nvec; j += blockDim.x) {
-      float c[kMaxVecDim];
-      load_centroid<D>(bv[0], load_field(row0, static_cast<int64_t>(j) * L.b[0], L.b[0]), d, c);
+    // Two vectors per thread per step: both index fields and both gathers are
+    // issued before either result is used.
+    for (int j0 = threadIdx.x; j0 < L.nvec; j0 += 2 * blockDim.x) {
+      const int jv[2] = {j0, j0 + static_cast<int>(blockDim.x)};
+      const bool ok1 = jv[1] < L.nvec;
+      uint32_t i1[2], i2[2] = {0u, 0u};
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int j = ok1 || u == 0 ? jv[u] : jv[0];
+        i1[u] = load_field(row0, static_cast<int64_t>(j) * L.b[0], L.b[0]);
+        if constexpr (NB == 2) i2[u] = load_field(row1, static_cast<int64_t>(j) * L.b[1], L.b[1]);
+      }
+      float c[2][kMaxVecDim];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) fetch(0, i1[u], c[u]);
       if constexpr (NB == 2) {
-        float c2[kMaxVecDim];
-        load_centroid<D>(bv[1], load_field(row1, static_cast<int64_t>(j) * L.b[1], L.b[1]), d, c2);
+        float c2[2][kMaxVecDim];
 #pragma unroll
-        for (int e = 0; e < kMaxVecDim; ++e)
-          if (e < d) c[e] = __fadd_rn(c[e], c2[e]);
+        for (int u = 0; u < 2; ++u) fetch(1, i2[u], c2[u]);
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int e = 0; e < kMaxVecDim; ++e)
+            if (e < d) c[u][e] = __fadd_rn(c[u][e], c2[u][e]);
       }
-      uint16_t h[kMaxVecDim];
 #pragma unroll
-      for (int e = 0; e < kMaxVecDim; ++e) {
-        if (e < d) {
-          float v = c[e];
-          if (has_s) v = __fmul_rn(v, s);
-          if (has_t) v = __fadd_rn(v, t);
-          h[e] = f2h(v);
+      for (int u = 0; u < 2; ++u) {
+        if (u == 1 && !ok1) break;
+        uint16_t h[kMaxVecDim];
+#pragma unroll
+        for (int e = 0; e < kMaxVecDim; ++e) {
+          if (e < d) {
+            float v = c[u][e];
+            if (has_s) v = __fmul_rn(v, s);
+            if (has_t) v = __fadd_rn(v, t);
+            h[e] = f2h(v);
+          }
         }
-      }
-      const int64_t k0 = static_cast<int64_t>(j) * d;
-      if (D == 8 && vec_store && k0 + 8 <= L.kin) {
-        uint4 v;
-        v.x = h[0] | (static_cast<uint32_t>(h[1]) << 16);
-        v.y = h[2] | (static_cast<uint32_t>(h[3]) << 16);
-        v.z = h[4] | (static_cast<uint32_t>(h[5]) << 16);
-        v.w = h[6] | (static_cast<uint32_t>(h[7]) << 16);
-        *reinterpret_cast<uint4*>(wrow + k0) = v;
-      } else {
+        const int64_t k0 = static_cast<int64_t>(jv[u]) * d;
+        if (D == 8 && vec_store && k0 + 8 <= L.kin) {
+          uint4 v;
+          v.x = h[0] | (static_cast<uint32_t>(h[1]) << 16);
+          v.y = h[2] | (static_cast<uint32_t>(h[3]) << 16);
+          v.z = h[4] | (static_cast<uint32_t>(h[5]) << 16);
+          v.w = h[6] | (static_cast<uint32_t>(h[7]) << 16);
+          *reinterpret_cast<uint4*>(wrow + k0) = v;
+        } else {
 #pragma unroll
-        for (int e = 0; e < kMaxVecDim; ++e)
-          if (e < d && k0 + e < L.kin) wrow[k0 + e] = h[e];
+          for (int e = 0; e < kMaxVecDim; ++e)
+            if (e < d && k0 + e < L.kin) wrow[k0 + e] = h[e];
+        }
       }
     }
   }

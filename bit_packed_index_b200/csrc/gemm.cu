@@ -42,14 +42,15 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int kATile = BM * BK * 2;             // 16 KB
+constexpr int BM = 128, BN = 256, BK = 64;       // one MMA: M = 128, N = 256, K = 16
+constexpr int kATile = BM * BK * 2;             // 16 KB per 128-row A sub-tile
 constexpr int kBTile = BN * BK * 2;             // 32 KB
-constexpr int kStageBytes = kATile + kBTile;    // 48 KB
+// A CTA covers MSUB (1 or 2) A sub-tiles of 128 rows that share each B tile:
+// two sub-tiles halve the weight-tile bytes (and, fused, the gathers) per FLOP.
+__host__ __device__ constexpr int stage_bytes(int msub) { return msub * kATile + kBTile; }
 constexpr int kThreads = 384;                   // 12 warps
 constexpr int kProducerThread0 = 128;           // warps 4..11 produce B tiles
 constexpr int kProducers = 256;
-constexpr uint32_t kTmemCols = 256;
 constexpr int kCtrlBytes = 3072;                // barriers, flags, scale/bias staging
 constexpr long long kWaitBudget = 4000000000LL; // SM clocks (about 2 s)
 constexpr int kMaxStages = 8;
@@ -203,7 +204,7 @@ __device__ __forceinline__ void produce_row_generic(const Layer& L, const BookVi
   }
 }
 
-template <int MODE, int B1, int B2>
+template <int MODE, int B1, int B2, int MSUB>
 __global__ void __launch_bounds__(kThreads, 1)
     vq_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b, GemmArgs g) {
@@ -211,9 +212,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = align1024(smem_raw);
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem);
   uint8_t* stages = smem + kCtrlBytes + (1024 - kCtrlBytes % 1024) % 1024;
-  uint16_t* books = reinterpret_cast<uint16_t*>(stages + g.stages * kStageBytes);
+  constexpr int kStage = stage_bytes(MSUB);
+  uint16_t* books = reinterpret_cast<uint16_t*>(stages + g.stages * kStage);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
+  constexpr uint32_t kTmemCols = 256 * MSUB;      // one 256-column fp32 accumulator per sub-tile
+  const int m0 = blockIdx.x * BM * MSUB, n0 = blockIdx.y * BN;
   const Layer& L = g.L;
   volatile int* abort_flag = &ctrl->abort_flag;
 
@@ -272,10 +275,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = kt % g.stages;
         const uint32_t ph = (kt / g.stages) & 1;
         if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, kWaitBudget)) break;
-        uint8_t* a = stages + s * kStageBytes;
-        mbar_arrive_expect_tx(&ctrl->full[s], MODE == kStaged ? kATile + kBTile : kATile);
-        tma_load_2d(a, &tmap_a, &ctrl->full[s], kt * BK, m0);
-        if (MODE == kStaged) tma_load_2d(a + kATile, &tmap_b, &ctrl->full[s], kt * BK, n0);
+        uint8_t* a = stages + s * kStage;
+        mbar_arrive_expect_tx(&ctrl->full[s], MODE == kStaged ? kStage : MSUB * kATile);
+#pragma unroll
+        for (int sub = 0; sub < MSUB; ++sub)
+          tma_load_2d(a + sub * kATile, &tmap_a, &ctrl->full[s], kt * BK, m0 + sub * BM);
+        if (MODE == kStaged) tma_load_2d(a + MSUB * kATile, &tmap_b, &ctrl->full[s], kt * BK, n0);
         issued = kt + 1;
       }
       if (*abort_flag) {   // let loads already in flight land before the block exits
@@ -292,12 +297,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (kt / g.stages) & 1;
         if (!bounded_wait(&ctrl->full[s], ph, abort_flag, g.status, kWaitBudget)) break;
         tc_fence_after();
-        const uint32_t a = smem_addr(stages + s * kStageBytes);
-        const uint32_t b = a + kATile;
+        const uint32_t a = smem_addr(stages + s * kStage);
+        const uint32_t b = a + MSUB * kATile;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk)
-          umma_f16(tmem, sw128_kmajor_desc(a + kk * 32), sw128_kmajor_desc(b + kk * 32), idesc,
-                   (kt | kk) != 0);
+#pragma unroll
+          for (int sub = 0; sub < MSUB; ++sub)
+            umma_f16(tmem + sub * 256, sw128_kmajor_desc(a + sub * kATile + kk * 32),
+                     sw128_kmajor_desc(b + kk * 32), idesc, (kt | kk) != 0);
         umma_commit(&ctrl->empty[s]);
       }
       umma_commit(&ctrl->acc_full);
@@ -309,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = kt % g.stages;
         const uint32_t ph = (kt / g.stages) & 1;
         if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, kWaitBudget)) break;
-        uint8_t* btile = stages + s * kStageBytes + kATile;
+        uint8_t* btile = stages + s * kStage + MSUB * kATile;
         if constexpr (B1 > 0) produce_row_d8<B1, B2>(L, bv, n0 + r, kt, btile, r);
         else if (L.nb == 2) produce_row_generic<2>(L, bv, n0 + r, kt, btile, r);
         else produce_row_generic<1>(L, bv, n0 + r, kt, btile, r);
@@ -317,16 +324,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&ctrl->full[s]);
       }
     }
-    if (warp < 8) {                                    // epilogue: warps 4..7 = TMEM lane quarters
+    if (warp < 4 + 4 * MSUB) {                         // epilogue: warp & 3 = TMEM lane quarter
       const int q = warp & 3;
+      const int sub = (warp - 4) >> 2;                 // which 128-row sub-tile
       if (bounded_wait(&ctrl->acc_full, 0, abort_flag, g.status, kWaitBudget)) {
         tc_fence_after();
-        const int row = m0 + q * 32 + lane;
-        const float rs = (MODE == kFused && row < g.m) ? g.rowsum[row] : 0.0f;
+        const int row = m0 + sub * BM + q * 32 + lane;
+        const float rs = (MODE == kFused && L.bias && row < g.m) ? g.rowsum[row] : 0.0f;
         const size_t es = g.yt == VQ_FP32 ? 4 : 2;
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t acc[32];
-          tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c * 32, acc);
+          tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + sub * 256 + c * 32, acc);
           tmem_wait_ld();
           const int nb = n0 + c * 32;
           if (row >= g.m || nb >= L.n) continue;
@@ -368,25 +376,46 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// x -> fp16 copy [m][kp] (zeros past kin) and fp32 row sums of the fp16 values.
-__global__ void gemm_prep(const uint16_t* __restrict__ x, int x_fp16, int m, int kin, int64_t ldx,
-                          uint16_t* __restrict__ x16, int kp, float* __restrict__ rowsum,
-                          int* __restrict__ status) {
-  if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
+// x -> fp16 copy [m][kp] (zeros past kin): one 8-element chunk per thread,
+// 16-byte loads and stores when x rows are 16-byte aligned.
+__global__ void gemm_convert(const uint16_t* __restrict__ x, int x_fp16, int m, int kin,
+                             int64_t ldx, int vec, uint16_t* __restrict__ x16, int kp) {
+  const int cpr = kp / 8;                                   // chunks per row
+  const int64_t total = static_cast<int64_t>(m) * cpr;
+  for (int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; q < total;
+       q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = q / cpr;
+    const int k = static_cast<int>(q - row * cpr) * 8;
+    const uint16_t* xr = x + row * ldx;
+    float v[8];
+    if (vec && k + 8 <= kin) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(xr + k));
+      const uint16_t* h = reinterpret_cast<const uint16_t*>(&u);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = x_fp16 ? h2f(h[i]) : bf2f(h[i]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = (k + i < kin) ? (x_fp16 ? h2f(xr[k + i]) : bf2f(xr[k + i])) : 0.0f;
+    }
+    uint32_t p[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      p[i] = f2h(v[2 * i]) | (static_cast<uint32_t>(f2h(v[2 * i + 1])) << 16);
+    *reinterpret_cast<uint4*>(x16 + row * kp + k) = make_uint4(p[0], p[1], p[2], p[3]);
+  }
+}
+
+// fp32 row sums of the fp16 operand rows a[m][lda] (first kin columns): the
+// bias term of the fused epilogue.  One warp per row.
+__global__ void gemm_rowsum(const uint16_t* __restrict__ a, int m, int kin, int64_t lda,
+                            float* __restrict__ rowsum) {
   const int warps = blockDim.x >> 5;
   const int row = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= m) return;
-  const uint16_t* xr = x + static_cast<int64_t>(row) * ldx;
-  uint16_t* outr = x16 + static_cast<int64_t>(row) * kp;
+  const uint16_t* r = a + static_cast<int64_t>(row) * lda;
   float s = 0.0f;
-  for (int k = lane; k < kp; k += 32) {
-    float v = 0.0f;
-    if (k < kin) v = x_fp16 ? h2f(xr[k]) : bf2f(xr[k]);
-    const uint16_t h = f2h(v);
-    outr[k] = h;
-    s += h2f(h);
-  }
+  for (int k = lane; k < kin; k += 32) s += h2f(r[k]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
   if (lane == 0) rowsum[row] = s;
@@ -428,36 +457,45 @@ size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 struct GemmLayout {
   int mode;
   int kp;
+  bool copy_x;       // bf16 activations (or misaligned fp16) need an fp16 copy
   size_t off_rowsum, off_x16, off_w, total;
 };
+
+bool fused_fast_path(const Layer& L) {
+  if (L.d != 8) return false;
+  const int b1 = L.b[0], b2 = L.nb == 2 ? L.b[1] : 0;
+  return (b1 == 16 && (b2 == 0 || b2 == 8)) || (b1 == 12 && b2 == 8) || (b1 == 8 && b2 == 8);
+}
 
 int choose_mode(const Layer& L, int m) {
   const char* env = std::getenv("VQ_GEMM_MODE");
   if (env && std::strcmp(env, "fused") == 0) return kFused;
   if (env && std::strcmp(env, "staged") == 0) return kStaged;
-  // The staged form gathers each centroid once; the fused form once per 128
-  // rows of x.  Prefer it once the gathers of the fused form would outweigh
-  // writing and re-reading W_hat.
+  // The staged form gathers each centroid once; the fused form once per
+  // 128-256 rows of x.  Fused only where its producers have a vectorised
+  // path and the gathers stay cheap: shared-memory books, or few rows.
   bool l2_book = false;
   for (int i = 0; i < L.nb; ++i) l2_book |= L.b[i] > 12;
+  if (!fused_fast_path(L)) return kStaged;
   return (l2_book && m > 256) || m >= 2048 ? kStaged : kFused;
 }
 
-GemmLayout layout_for(const Layer& L, int m) {
+GemmLayout layout_for(const Layer& L, int m, bool x_fp16) {
   GemmLayout g;
   g.mode = choose_mode(L, m);
   g.kp = (L.kin + 7) / 8 * 8;
+  g.copy_x = !x_fp16;   // fp16 activations are read in place (16-byte aligned, ldx % 8 == 0)
   g.off_rowsum = 256;
   g.off_x16 = g.off_rowsum + round256(static_cast<size_t>(m) * 4);
-  g.off_w = g.off_x16 + round256(static_cast<size_t>(m) * g.kp * 2);
+  g.off_w = g.off_x16 + (g.copy_x ? round256(static_cast<size_t>(m) * g.kp * 2) : 0);
   g.total = g.off_w + (g.mode == kStaged ? round256(static_cast<size_t>(L.n) * g.kp * 2) : 0);
   return g;
 }
 
-template <int MODE, int B1, int B2>
+template <int MODE, int B1, int B2, int MSUB>
 cudaError_t launch_kernel(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g,
                           size_t smem, dim3 grid, cudaStream_t stream) {
-  auto k = vq_gemm_kernel<MODE, B1, B2>;
+  auto k = vq_gemm_kernel<MODE, B1, B2, MSUB>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   count_launch();
@@ -465,16 +503,33 @@ cudaError_t launch_kernel(const CUtensorMap& ma, const CUtensorMap& mb, const Ge
   return cudaGetLastError();
 }
 
+template <int MSUB>
+cudaError_t dispatch(const Layer& L, int mode, const CUtensorMap& ma, const CUtensorMap& mb,
+                     const GemmArgs& g, size_t smem, dim3 grid, cudaStream_t stream) {
+  if (mode == kStaged) return launch_kernel<kStaged, 0, 0, MSUB>(ma, mb, g, smem, grid, stream);
+  if (L.d == 8 && L.nb == 1 && L.b[0] == 16)
+    return launch_kernel<kFused, 16, 0, MSUB>(ma, mb, g, smem, grid, stream);
+  if (L.d == 8 && L.nb == 2 && L.b[0] == 16 && L.b[1] == 8)
+    return launch_kernel<kFused, 16, 8, MSUB>(ma, mb, g, smem, grid, stream);
+  if (L.d == 8 && L.nb == 2 && L.b[0] == 12 && L.b[1] == 8)
+    return launch_kernel<kFused, 12, 8, MSUB>(ma, mb, g, smem, grid, stream);
+  if (L.d == 8 && L.nb == 2 && L.b[0] == 8 && L.b[1] == 8)
+    return launch_kernel<kFused, 8, 8, MSUB>(ma, mb, g, smem, grid, stream);
+  return launch_kernel<kFused, 0, 0, MSUB>(ma, mb, g, smem, grid, stream);
+}
+
 }  // namespace
 
-size_t gemm_workspace_bytes(const Layer& L, int m, bool) { return layout_for(L, m).total; }
+size_t gemm_workspace_bytes(const Layer& L, int m, bool x_fp16) {
+  return layout_for(L, m, x_fp16).total;
+}
 
 vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t ldx, void* y,
                       vq_dtype yt, int64_t ldy, void* ws, size_t ws_bytes, cudaStream_t stream) {
   const size_t es = yt == VQ_FP32 ? 4 : 2;
   if (L.kin == 0)
     return cuda_status(cudaMemset2DAsync(y, ldy * es, 0, static_cast<size_t>(L.n) * es, m, stream));
-  const GemmLayout lay = layout_for(L, m);
+  const GemmLayout lay = layout_for(L, m, x_fp16);
   if (ws_bytes < lay.total) return VQ_ERR_WORKSPACE;
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   int* status = reinterpret_cast<int*>(w8);
@@ -483,19 +538,36 @@ vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t
   uint16_t* what = reinterpret_cast<uint16_t*>(w8 + lay.off_w);
 
   {
-    const int warps = 8;
-    count_launch();
-    gemm_prep<<<(m + warps - 1) / warps, warps * 32, 0, stream>>>(
-        static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, m, L.kin, ldx, x16, lay.kp, rowsum, status);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), stream);
     if (e != cudaSuccess) return cuda_status(e);
+    if (lay.copy_x) {
+      const int vec = aligned(x, 16) && ldx % 8 == 0;
+      const int64_t chunks = static_cast<int64_t>(m) * (lay.kp / 8);
+      const int blocks = static_cast<int>(std::min<int64_t>((chunks + 255) / 256, 16 * device_sm_count()));
+      count_launch();
+      gemm_convert<<<blocks, 256, 0, stream>>>(static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, m,
+                                              L.kin, ldx, vec, x16, lay.kp);
+      if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+    }
+    if (lay.mode == kFused && L.bias != nullptr) {   // row sums feed the fused bias term only
+      const int warps = 8;
+      count_launch();
+      gemm_rowsum<<<(m + warps - 1) / warps, warps * 32, 0, stream>>>(
+          lay.copy_x ? x16 : static_cast<const uint16_t*>(x), m, L.kin,
+          lay.copy_x ? lay.kp : ldx, rowsum);
+      if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+    }
   }
   if (lay.mode == kStaged) {
     vq_status st = launch_dequant(L, what, lay.kp, stream);
     if (st != VQ_OK) return st;
   }
   CUtensorMap ma, mb;
-  if (!make_map(&ma, x16, L.kin, m, lay.kp, BM)) return VQ_ERR_CUDA;
+  if (lay.copy_x) {
+    if (!make_map(&ma, x16, L.kin, m, lay.kp, BM)) return VQ_ERR_CUDA;
+  } else {
+    if (!make_map(&ma, x, L.kin, m, ldx, BM)) return VQ_ERR_CUDA;
+  }
   if (lay.mode == kStaged) {
     if (!make_map(&mb, what, L.kin, L.n, lay.kp, BN)) return VQ_ERR_CUDA;
   } else {
@@ -514,10 +586,15 @@ vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t
   g.smem_mask = 0;
   g.book_bytes = 0;
   const int optin = device_smem_optin();
+  // Two 128-row sub-tiles per CTA when that still gives about one tile per SM.
+  const int sms = device_sm_count();
+  const int tiles2 = ((m + 2 * BM - 1) / (2 * BM)) * ((L.n + BN - 1) / BN);
+  const int msub = tiles2 * 5 >= sms * 4 ? 2 : 1;
+  const int kStageBytes = stage_bytes(msub);
   const size_t fixed = 1024 + 3072;   // alignment slack + control block
   if (lay.mode == kFused) {
     // Stage the books that fit next to at least three pipeline stages.
-    const size_t budget = static_cast<size_t>(optin) - fixed - 3 * kStageBytes;
+    const size_t budget = static_cast<size_t>(optin) - fixed - 2 * kStageBytes;
     int mask = 0;
     size_t used = 0;
     for (int i = 0; i < L.nb; ++i) {
@@ -530,23 +607,9 @@ vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t
   g.stages = static_cast<int>(std::min<size_t>(kMaxStages, (optin - fixed - g.book_bytes) / kStageBytes));
   g.stages = std::min(g.stages, 4);
   const size_t smem = fixed + static_cast<size_t>(g.stages) * kStageBytes + g.book_bytes;
-  dim3 grid((m + BM - 1) / BM, (L.n + BN - 1) / BN);
-
-  cudaError_t e;
-  if (lay.mode == kStaged) {
-    e = launch_kernel<kStaged, 0, 0>(ma, mb, g, smem, grid, stream);
-  } else if (L.d == 8 && L.nb == 1 && L.b[0] == 16) {
-    e = launch_kernel<kFused, 16, 0>(ma, mb, g, smem, grid, stream);
-  } else if (L.d == 8 && L.nb == 2 && L.b[0] == 16 && L.b[1] == 8) {
-    e = launch_kernel<kFused, 16, 8>(ma, mb, g, smem, grid, stream);
-  } else if (L.d == 8 && L.nb == 2 && L.b[0] == 12 && L.b[1] == 8) {
-    e = launch_kernel<kFused, 12, 8>(ma, mb, g, smem, grid, stream);
-  } else if (L.d == 8 && L.nb == 2 && L.b[0] == 8 && L.b[1] == 8) {
-    e = launch_kernel<kFused, 8, 8>(ma, mb, g, smem, grid, stream);
-  } else {
-    e = launch_kernel<kFused, 0, 0>(ma, mb, g, smem, grid, stream);
-  }
-  return cuda_status(e);
+  dim3 grid((m + BM * msub - 1) / (BM * msub), (L.n + BN - 1) / BN);
+  return cuda_status(msub == 2 ? dispatch<2>(L, lay.mode, ma, mb, g, smem, grid, stream)
+                               : dispatch<1>(L, lay.mode, ma, mb, g, smem, grid, stream));
 }
 
 }  // namespace vqk

@@ -122,8 +122,8 @@ __device__ __forceinline__ float warp_sum1(float v) {
 
 template <int D, int B1, int B2, bool SM1, bool SM2>
 __global__ void __launch_bounds__(kThreads1, 1) gemv1_kernel(
-    Layer L, const uint16_t* __restrict__ x, int x_fp16, int chunks_per_split, int smem_mask,
-    int book_bytes, void* __restrict__ y, vq_dtype yt, float* __restrict__ ws) {
+    Layer L, const uint16_t* __restrict__ x, int x_fp16, int chunks_per_split, int rpb,
+    int smem_mask, int book_bytes, void* __restrict__ y, vq_dtype yt, float* __restrict__ ws) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr bool NB2 = B2 > 0;
@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv1_kernel(
   const int split = blockIdx.y;
   const int c0 = split * chunks_per_split;
   const int nck = min(chunks_per_split, nchunks_total - c0);
-  float* part = reinterpret_cast<float*>(smem + book_bytes);   // [kRows1][nck]
+  float* part = reinterpret_cast<float*>(smem + book_bytes);   // [rpb][nck]
   float* xsum_s = part + kRows1 * chunks_per_split;
 
   // Sum of x over this split's columns.
@@ -163,16 +163,16 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv1_kernel(
   }
   __syncthreads();
 
-  const int nrb = (L.n + kRows1 - 1) / kRows1;
+  const int nrb = (L.n + rpb - 1) / rpb;
   // Work items: (chunk, pair of rows) in chunk-major order; each warp takes a
   // contiguous range, so it stays on one chunk (one load of x) almost always.
-  constexpr int kPairs = kRows1 / kR;
+  const int kPairs = rpb / kR;
   const int items = nck * kPairs;
   const int per_warp = (items + kWarps1 - 1) / kWarps1;
   const int it_begin = warp * per_warp;
   const int it_end = min(items, it_begin + per_warp);
   for (int rb = blockIdx.x; rb < nrb; rb += gridDim.x) {
-    const int o0 = rb * kRows1;
+    const int o0 = rb * rpb;
     int cur_chunk = -1;
     float xr[kG][D];
     bool lane_live = false;
@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv1_kernel(
       }
     }
     __syncthreads();
-    for (int rl = tid; rl < kRows1; rl += kThreads1) {
+    for (int rl = tid; rl < rpb; rl += kThreads1) {
       const int o = o0 + rl;
       if (o >= L.n) continue;
       float dot = 0.0f;
@@ -288,7 +288,7 @@ cudaError_t launch1(const Layer& L, const GemvPlan& p, const void* x, bool xf, v
   dim3 grid(p.grid_x, p.nsplit);
   count_launch();
   k<<<grid, kThreads1, p.smem, stream>>>(L, static_cast<const uint16_t*>(x), xf ? 1 : 0, p.vps / kChunk,
-                                         p.books_in_smem, p.book_bytes, y, yt,
+                                         p.rpb, p.books_in_smem, p.book_bytes, y, yt,
                                          p.nsplit > 1 ? ws : nullptr);
   return cudaGetLastError();
 }
@@ -319,23 +319,29 @@ void plan_gemv1(const Layer& L, GemvPlan* p) {
     }
   }
   const int nchunks = (L.nvec + kChunk - 1) / kChunk;
-  const int nrb = (L.n + kRows1 - 1) / kRows1;
-  const int sms = device_sm_count();
-  // Split the input dimension only when there are too few row blocks.
+  // One block per SM (the kernel is register-heavy).  Split the input
+  // dimension only when there are too few 128-row blocks to fill the SMs.
+  const int slots = device_sm_count();
   int nsplit = 1;
-  while (nsplit < nchunks && nrb * nsplit < sms) nsplit *= 2;
+  while (nsplit < nchunks && ((L.n + kRows1 - 1) / kRows1) * nsplit < slots) nsplit *= 2;
   nsplit = std::min(nsplit, nchunks);
   const int cps = (nchunks + nsplit - 1) / nsplit;
   nsplit = (nchunks + cps - 1) / cps;
+  // Rows per block: every block of a split handles the same number of row
+  // blocks (`rounds`), each at most 128 rows, so no SM idles in a last wave.
+  const int grid_x = std::max(1, slots / nsplit);
+  const int rounds = std::max(1, (L.n + grid_x * kRows1 - 1) / (grid_x * kRows1));
+  int rpb = (L.n + grid_x * rounds - 1) / (grid_x * rounds);
+  rpb = std::min(kRows1, std::max(kR, (rpb + kR - 1) / kR * kR));
+  const int nrb = (L.n + rpb - 1) / rpb;
   p->bt = 1;
   p->nsplit = nsplit;
   p->vps = cps * kChunk;
-  p->rpb = kRows1;
+  p->rpb = rpb;
   p->books_in_smem = mask;
   p->book_bytes = static_cast<int>(books);
   p->smem = static_cast<int>(books + sizeof(float) * (kRows1 * cps + 4));
-  const int per_sm = std::max(1, std::min(2, static_cast<int>((200 * 1024) / (p->smem + 1024))));
-  p->grid_x = std::max(1, std::min(nrb, (sms * per_sm + nsplit - 1) / nsplit));
+  p->grid_x = std::max(1, std::min(nrb, grid_x));
   p->ws_bytes = nsplit > 1 ? static_cast<size_t>(nsplit) * L.n * sizeof(float) : 0;
   p->fast = 1;
 }

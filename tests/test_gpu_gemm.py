@@ -118,6 +118,25 @@ def test_gemm_both_modes_on_prefill_shape(monkeypatch):
         assert_close(y[:, torch.from_numpy(cols).cuda()].double().cpu().numpy(), ref, "float32")
 
 
+@pytest.mark.parametrize("spec,m,mode", [
+    (LayerSpec(30000, 520, 8, (12, 8), (0.02, 0.005)), 700, "fused"),
+    (LayerSpec(30000, 520, 8, (16,), (0.02,)), 1000, "staged"),
+    (LayerSpec(30000, 6 * 90 + 4, 6, (12, 4), (0.02, 0.005)), 515, "staged"),
+])
+def test_gemm_two_subtile_blocks(monkeypatch, spec, m, mode):
+    """Wide layers make each CTA cover 256 rows of x (two accumulators sharing
+    every weight tile); ragged M and K on both weight-tile sources."""
+    monkeypatch.setenv("VQ_GEMM_MODE", mode)
+    data = synth.make_layer(spec, seed=m)
+    kin = spec.in_features
+    ld = (kin + 7) // 8 * 8
+    x = synth.make_x(m + 1, m, kin, outlier_frac=0.01, ld=ld)
+    cols = sample_rows(spec.out_features, 64, m + 2)
+    ref = oracle.linear(data, x[:, :kin], cols)
+    y = _run(_vq().Layer.from_synth(data), _x_dev(x)[:, :kin], torch.float32, kin)
+    assert_close(y[:, torch.from_numpy(cols).cuda()].double().cpu().numpy(), ref, "float32")
+
+
 def test_gemm_degenerate_and_errors():
     vq = _vq()
     spec = LayerSpec(40, 0, 8, (4,), (0.02,))
