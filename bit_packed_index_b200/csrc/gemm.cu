@@ -42,7 +42,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128, BN = 256, BK = 64;       // one MMA: M = 128, N = 256, K = 16
+constexpr int BM = 128, BN = 256, BK = 64;       // one MMA: M = 128, N <= 256, K = 16
 constexpr int kATile = BM * BK * 2;             // 16 KB per 128-row A sub-tile
 constexpr int kBTile = BN * BK * 2;             // 32 KB
 // A CTA covers MSUB (1 or 2) A sub-tiles of 128 rows that share each B tile:
@@ -64,6 +64,8 @@ struct GemmArgs {
   int stages;
   int smem_mask;
   int book_bytes;
+  int bn;                 // tile width along N (multiple of 32, <= BN)
+  uint32_t idesc;         // tcgen05 instruction descriptor for M = 128, N = bn
   const float* rowsum;
   void* y;
   vq_dtype yt;
@@ -216,7 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint16_t* books = reinterpret_cast<uint16_t*>(stages + g.stages * kStage);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr uint32_t kTmemCols = 256 * MSUB;      // one 256-column fp32 accumulator per sub-tile
-  const int m0 = blockIdx.x * BM * MSUB, n0 = blockIdx.y * BN;
+  const int bn = g.bn;
+  const int m0 = blockIdx.x * BM * MSUB, n0 = blockIdx.y * bn;
   const Layer& L = g.L;
   volatile int* abort_flag = &ctrl->abort_flag;
 
@@ -276,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (kt / g.stages) & 1;
         if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, kWaitBudget)) break;
         uint8_t* a = stages + s * kStage;
-        mbar_arrive_expect_tx(&ctrl->full[s], MODE == kStaged ? kStage : MSUB * kATile);
+        mbar_arrive_expect_tx(&ctrl->full[s], MODE == kStaged ? MSUB * kATile + bn * BK * 2 : MSUB * kATile);
 #pragma unroll
         for (int sub = 0; sub < MSUB; ++sub)
           tma_load_2d(a + sub * kATile, &tmap_a, &ctrl->full[s], kt * BK, m0 + sub * BM);
@@ -291,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {                                   // MMA issuer
-      constexpr uint32_t idesc = f16_idesc(BM, BN);
+      const uint32_t idesc = g.idesc;
       for (int kt = 0; kt < g.num_kt; ++kt) {
         const int s = kt % g.stages;
         const uint32_t ph = (kt / g.stages) & 1;
@@ -317,9 +320,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (kt / g.stages) & 1;
         if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, kWaitBudget)) break;
         uint8_t* btile = stages + s * kStage + MSUB * kATile;
-        if constexpr (B1 > 0) produce_row_d8<B1, B2>(L, bv, n0 + r, kt, btile, r);
-        else if (L.nb == 2) produce_row_generic<2>(L, bv, n0 + r, kt, btile, r);
-        else produce_row_generic<1>(L, bv, n0 + r, kt, btile, r);
+        if (r < bn) {                                  // rows past the tile width stay idle
+          if constexpr (B1 > 0) produce_row_d8<B1, B2>(L, bv, n0 + r, kt, btile, r);
+          else if (L.nb == 2) produce_row_generic<2>(L, bv, n0 + r, kt, btile, r);
+          else produce_row_generic<1>(L, bv, n0 + r, kt, btile, r);
+        }
         fence_proxy_async_smem();
         mbar_arrive(&ctrl->full[s]);
       }
@@ -332,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = m0 + sub * BM + q * 32 + lane;
         const float rs = (MODE == kFused && L.bias && row < g.m) ? g.rowsum[row] : 0.0f;
         const size_t es = g.yt == VQ_FP32 ? 4 : 2;
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < bn / 32; ++c) {
           uint32_t acc[32];
           tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + sub * 256 + c * 32, acc);
           tmem_wait_ld();
@@ -503,6 +508,23 @@ cudaError_t launch_kernel(const CUtensorMap& ma, const CUtensorMap& mb, const Ge
   return cudaGetLastError();
 }
 
+// Tile shape: two 128-row sub-tiles per CTA when that still gives about one
+// tile per SM; then the N width (a multiple of 32, 128..256) that wastes the
+// least of the last wave: cost ~ waves * (width + 64), the 64 standing for
+// the activation bytes every tile loads whatever its width.
+void choose_tiles(int m, int n, int sms, int* msub, int* bn) {
+  const int tiles2 = ((m + 2 * BM - 1) / (2 * BM)) * ((n + BN - 1) / BN);
+  *msub = tiles2 * 5 >= sms * 4 ? 2 : 1;
+  const int mt = (m + BM * *msub - 1) / (BM * *msub);
+  long best = -1;
+  for (int w = BN; w >= 128; w -= 32) {
+    const long tiles = static_cast<long>(mt) * ((n + w - 1) / w);
+    const long waves = (tiles + sms - 1) / sms;
+    const long cost = waves * (w + 64);
+    if (best < 0 || cost < best) { best = cost; *bn = w; }
+  }
+}
+
 template <int MSUB>
 cudaError_t dispatch(const Layer& L, int mode, const CUtensorMap& ma, const CUtensorMap& mb,
                      const GemmArgs& g, size_t smem, dim3 grid, cudaStream_t stream) {
@@ -562,6 +584,8 @@ vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t
     vq_status st = launch_dequant(L, what, lay.kp, stream);
     if (st != VQ_OK) return st;
   }
+  int msub = 1, bn = BN;
+  choose_tiles(m, L.n, device_sm_count(), &msub, &bn);
   CUtensorMap ma, mb;
   if (lay.copy_x) {
     if (!make_map(&ma, x16, L.kin, m, lay.kp, BM)) return VQ_ERR_CUDA;
@@ -569,7 +593,7 @@ vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t
     if (!make_map(&ma, x, L.kin, m, ldx, BM)) return VQ_ERR_CUDA;
   }
   if (lay.mode == kStaged) {
-    if (!make_map(&mb, what, L.kin, L.n, lay.kp, BN)) return VQ_ERR_CUDA;
+    if (!make_map(&mb, what, L.kin, L.n, lay.kp, bn)) return VQ_ERR_CUDA;
   } else {
     mb = ma;
   }
@@ -586,10 +610,6 @@ vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t
   g.smem_mask = 0;
   g.book_bytes = 0;
   const int optin = device_smem_optin();
-  // Two 128-row sub-tiles per CTA when that still gives about one tile per SM.
-  const int sms = device_sm_count();
-  const int tiles2 = ((m + 2 * BM - 1) / (2 * BM)) * ((L.n + BN - 1) / BN);
-  const int msub = tiles2 * 5 >= sms * 4 ? 2 : 1;
   const int kStageBytes = stage_bytes(msub);
   const size_t fixed = 1024 + 3072;   // alignment slack + control block
   if (lay.mode == kFused) {
@@ -607,7 +627,9 @@ vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t
   g.stages = static_cast<int>(std::min<size_t>(kMaxStages, (optin - fixed - g.book_bytes) / kStageBytes));
   g.stages = std::min(g.stages, 4);
   const size_t smem = fixed + static_cast<size_t>(g.stages) * kStageBytes + g.book_bytes;
-  dim3 grid((m + BM * msub - 1) / (BM * msub), (L.n + BN - 1) / BN);
+  g.bn = bn;
+  g.idesc = f16_idesc(BM, bn);
+  dim3 grid((m + BM * msub - 1) / (BM * msub), (L.n + bn - 1) / bn);
   return cuda_status(msub == 2 ? dispatch<2>(L, lay.mode, ma, mb, g, smem, grid, stream)
                                : dispatch<1>(L, lay.mode, ma, mb, g, smem, grid, stream));
 }
