@@ -141,20 +141,22 @@ __device__ __forceinline__ uint4 zero_tail8(uint4 v, int valid) {   // keep `val
   return v;
 }
 
-// Fused B-tile row (d = 8, compile-time index widths; B2 = 0: one book).
+// Fused B-tile rows at d = 8 with compile-time index widths (B2 = 0: one
+// book), split in three steps so a producer can keep the next stage's index
+// loads and centroid gathers in flight while it waits for a free stage:
+// the 8 index fields of row n for K-step kt, the 8 centroid rows (fp16 sum of
+// both books), and the swizzled 16-byte stores into the tile.
 template <int B1, int B2>
-__device__ __forceinline__ void produce_row_d8(const Layer& L, const BookView (&bv)[2], int n,
-                                               int kt, uint8_t* btile, int r) {
-  if (n >= L.n) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(btile + sw128_off(r, c)) = make_uint4(0, 0, 0, 0);
-    return;
-  }
+__device__ __forceinline__ void d8_fields(const Layer& L, int n, int kt, uint32_t (&f1)[8],
+                                          uint32_t (&f2)[8]) {
   const int j0 = kt * 8;
-  uint32_t f1[8], f2[8];
   fields8<B1>(L.idx[0] + static_cast<int64_t>(n) * L.rw[0], L.rw[0], j0, f1);
   if constexpr (B2 > 0) fields8<B2>(L.idx[1] + static_cast<int64_t>(n) * L.rw[1], L.rw[1], j0, f2);
-  uint4 c[8];
+}
+
+template <int B2>
+__device__ __forceinline__ void d8_gather(const BookView (&bv)[2], const uint32_t (&f1)[8],
+                                          const uint32_t (&f2)[8], uint4 (&c)[8]) {
 #pragma unroll
   for (int v = 0; v < 8; ++v) c[v] = *reinterpret_cast<const uint4*>(bv[0].base + static_cast<size_t>(f1[v]) * 8);
   if constexpr (B2 > 0) {
@@ -162,10 +164,14 @@ __device__ __forceinline__ void produce_row_d8(const Layer& L, const BookView (&
     for (int v = 0; v < 8; ++v)
       c[v] = hadd8(c[v], *reinterpret_cast<const uint4*>(bv[1].base + static_cast<size_t>(f2[v]) * 8));
   }
+}
+
+__device__ __forceinline__ void d8_store(const Layer& L, bool live, int kt, const uint4 (&c)[8],
+                                         uint8_t* btile, int r) {
   const int k0 = kt * BK;
 #pragma unroll
   for (int v = 0; v < 8; ++v) {
-    const int valid = L.kin - (k0 + 8 * v);
+    const int valid = live ? L.kin - (k0 + 8 * v) : 0;
     uint4 x = c[v];
     if (valid < 8) x = zero_tail8(x, valid < 0 ? 0 : valid);
     *reinterpret_cast<uint4*>(btile + sw128_off(r, v)) = x;
@@ -313,7 +319,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(&ctrl->acc_full);
     }
   } else if (warp >= 4) {
-    if (MODE == kFused) {                              // B-tile producers
+    if (MODE == kFused && B1 > 0) {                    // B-tile producers, d = 8 fast path
+      // Software pipeline: while waiting for stage kt to be free, the index
+      // loads of kt+2 and the centroid gathers of kt+1 are in flight.
+      const int r = threadIdx.x - kProducerThread0;
+      const int n = n0 + r;
+      const bool live = r < bn && n < L.n;
+      uint32_t fa[8], fb[8], ga[8], gb[8];
+      uint4 cur[8], nxt[8];
+#pragma unroll
+      for (int v = 0; v < 8; ++v) { fa[v] = fb[v] = ga[v] = gb[v] = 0u; }
+      if (live && g.num_kt > 0) d8_fields<B1, B2>(L, n, 0, fa, fb);
+      if (live && g.num_kt > 0) d8_gather<B2>(bv, fa, fb, nxt);
+      if (live && g.num_kt > 1) d8_fields<B1, B2>(L, n, 1, ga, gb);
+      for (int kt = 0; kt < g.num_kt; ++kt) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) cur[v] = nxt[v];
+        if (live && kt + 1 < g.num_kt) {
+          d8_gather<B2>(bv, ga, gb, nxt);
+          if (kt + 2 < g.num_kt) d8_fields<B1, B2>(L, n, kt + 2, ga, gb);
+        }
+        const int s = kt % g.stages;
+        const uint32_t ph = (kt / g.stages) & 1;
+        if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, kWaitBudget)) break;
+        if (r < bn) d8_store(L, live, kt, cur, stages + s * kStage + MSUB * kATile, r);
+        fence_proxy_async_smem();
+        mbar_arrive(&ctrl->full[s]);
+      }
+    } else if (MODE == kFused) {                       // B-tile producers, any d <= 8
       const int r = threadIdx.x - kProducerThread0;
       for (int kt = 0; kt < g.num_kt; ++kt) {
         const int s = kt % g.stages;
@@ -321,8 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, kWaitBudget)) break;
         uint8_t* btile = stages + s * kStage + MSUB * kATile;
         if (r < bn) {                                  // rows past the tile width stay idle
-          if constexpr (B1 > 0) produce_row_d8<B1, B2>(L, bv, n0 + r, kt, btile, r);
-          else if (L.nb == 2) produce_row_generic<2>(L, bv, n0 + r, kt, btile, r);
+          if (L.nb == 2) produce_row_generic<2>(L, bv, n0 + r, kt, btile, r);
           else produce_row_generic<1>(L, bv, n0 + r, kt, btile, r);
         }
         fence_proxy_async_smem();

@@ -209,6 +209,10 @@ vq_status plan_gemv(const Layer& L, int batch, GemvPlan* p) {
     plan_gemv1(L, p);
     if (p->smem <= device_smem_optin()) return VQ_OK;
   }
+  if (gemvb_supported(L, batch)) {
+    plan_gemvb(L, batch, p);
+    if (p->smem <= device_smem_optin()) return VQ_OK;
+  }
   p->fast = 0;
   int bt = 1;
   while (bt < batch) bt <<= 1;
@@ -251,8 +255,10 @@ vq_status launch_gemv(const Layer& L, const GemvPlan& p, const void* x, bool x_f
   }
   const int D = (L.d == 8) ? 8 : (L.d == 6 ? 6 : 0);
   cudaError_t e;
-  if (p.fast) {
+  if (p.fast == 1) {
     e = launch_gemv1(L, p, x, x_fp16, y, yt, ws, stream);
+  } else if (p.fast == 2) {
+    e = launch_gemvb(L, p, x, x_fp16, batch, ldx, y, yt, ldy, ws, stream);
   } else if (L.nb == 1) {
     e = D == 8 ? launch_d<8, 1>(L, p, x, x_fp16, batch, ldx, y, yt, ldy, ws, stream)
       : D == 6 ? launch_d<6, 1>(L, p, x, x_fp16, batch, ldx, y, yt, ldy, ws, stream)

@@ -59,10 +59,15 @@ struct GemvPlan {
   int books_in_smem;  // bit m set: book m staged in shared memory
   int book_bytes;     // shared memory taken by the staged books
   size_t ws_bytes;
-  int fast = 0;       // 1: the single-row kernel of gemv1.cu
+  int fast = 0;       // 1: single-row kernel (gemv1.cu), 2: batched kernel (gemvb.cu)
 };
 vq_status plan_gemv(const Layer& L, int batch, GemvPlan* plan);
 bool gemv1_supported(const Layer& L);
+bool gemvb_supported(const Layer& L, int batch);
+void plan_gemvb(const Layer& L, int batch, GemvPlan* plan);
+cudaError_t launch_gemvb(const Layer& L, const GemvPlan& plan, const void* x, bool x_fp16, int batch,
+                         int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy, float* ws,
+                         cudaStream_t stream);
 void plan_gemv1(const Layer& L, GemvPlan* plan);
 cudaError_t launch_gemv1(const Layer& L, const GemvPlan& plan, const void* x, bool x_fp16, void* y,
                          vq_dtype y_dtype, float* ws, cudaStream_t stream);

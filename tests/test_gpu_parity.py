@@ -126,7 +126,7 @@ def test_gemv_output_types_and_fp16_input(out_dtype):
     assert np.array_equal(yb.view(torch.int16).cpu().numpy().view(np.uint16), oracle.f32_to_bf16(y32))
 
 
-# Single-row (batch 1) kernel: every supported (d, index widths) pair, ragged
+# Specialised kernels: every supported (d, index widths) pair, ragged
 # rows and columns, partial 256-vector chunks, and narrow layers that take the
 # split along the input dimension.
 FAST_SPECS = [
@@ -144,12 +144,14 @@ FAST_SPECS = [
 
 
 @pytest.mark.parametrize("i", range(len(FAST_SPECS)))
-def test_gemv_single_row_kernel(i):
+@pytest.mark.parametrize("batch", [1, 2, 3, 5, 16])
+def test_gemv_specialised_kernels(i, batch):
+    """Single-row (batch 1) and batched (2..16) kernels."""
     spec = FAST_SPECS[i]
     data = synth.make_layer(spec, seed=1300 + i, pad_garbage=True)
     layer = _dev_layer(data)
     for fp16 in (False, True):
-        x = synth.make_x(90 + i, 1, spec.in_features, outlier_frac=0.01, as_fp16=fp16)
+        x = synth.make_x(90 + i, batch, spec.in_features, outlier_frac=0.01, as_fp16=fp16)
         ref = oracle.linear(data, x, x_is_fp16=fp16)
         y = _vq().gemv(layer, _x_dev(x, fp16), out_dtype=torch.float32)
         assert_close(_f64(y), ref, "float32")

@@ -42,7 +42,7 @@ def test_noalloc_matches_workspace_version_twice(spec, batch):
 
 def test_noalloc_rejects_layers_beyond_the_scratch():
     from bit_packed_index_b200 import vq
-    spec = LayerSpec(53248, 6 * 2731, 6, (12, 4), (0.02, 0.005))
+    spec = LayerSpec(28672, 8192, 8, (16,), (0.02,))       # split K at batch 16: ~11 MB
     data = synth.make_layer(spec, seed=4244)
     layer = vq.Layer.from_synth(data)
     assert vq.gemv_workspace_size(layer, 16) > vq.NOALLOC_SCRATCH_BYTES
