@@ -8,8 +8,8 @@ input generators in ``synth``.
 The arithmetic lives in ``vq_oracle.c`` (plain C, built here with gcc into
 ``liboracle.so``); this module marshals numpy arrays for it.  What each
 routine computes, and the page passage it follows, is documented in the C
-file.  Functions pinned by the not-gpu tests: the conversions, unpack/pack,
-dequant, matmul/linear and the encoders.
+file.  Functions pinned by the not-gpu tests: the conversions, unpack/pack
+(row order and tiled order), dequant, matmul/linear and the encoders.
 """
 from __future__ import annotations
 
@@ -62,6 +62,8 @@ def _load():
                 "vqo_f32_to_bf16_array": [P, P, I64], "vqo_bf16_to_f32_array": [P, P, I64],
                 "vqo_unpack": [P, I64, I64, I32, I64, P],
                 "vqo_pack": [P, I64, I64, I32, I64, P],
+                "vqo_unpack_tile4": [P, I64, I64, I32, I64, P],
+                "vqo_pack_tile4": [P, I64, I64, I32, I64, P],
                 "vqo_dequant": [P, P, I64],
                 "vqo_dequant_rows": [P, P, I64, P, I64],
                 "vqo_matmul": [I64, I64, I64, P, I32, I64, P, I64, P, I64],
@@ -135,6 +137,32 @@ def pack(idx: np.ndarray, b: int, row_words: Optional[int] = None) -> np.ndarray
         row_words = -(-(nvec * b) // 128) * 4
     out = np.empty((n, row_words), np.uint32)
     _check(_load().vqo_pack(_p(idx), n, nvec, b, row_words, _p(out)), "pack")
+    return out
+
+
+def tile4_words(n_rows: int, b: int) -> int:
+    """Smallest 16-byte-padded tile of the tiled order: n_rows records of 4 fields."""
+    return -(-(n_rows * 4 * b) // 128) * 4
+
+
+def unpack_tile4(words: np.ndarray, b: int, n_rows: int, nvec: int) -> np.ndarray:
+    """Indices [n_rows][nvec] from a tiled stream [ceil(nvec/4)][tile_words]."""
+    words = np.ascontiguousarray(words, np.uint32)
+    tile_words = words.shape[1]
+    out = np.empty((n_rows, nvec), np.uint32)
+    _check(_load().vqo_unpack_tile4(_p(words), n_rows, tile_words, b, nvec, _p(out)),
+           "unpack_tile4")
+    return out
+
+
+def pack_tile4(idx: np.ndarray, b: int, tile_words: Optional[int] = None) -> np.ndarray:
+    """The tiled stream [ceil(nvec/4)][tile_words] of idx [N][nvec] (zero padding)."""
+    idx = np.ascontiguousarray(idx, np.uint32)
+    n, nvec = idx.shape
+    if tile_words is None:
+        tile_words = tile4_words(n, b)
+    out = np.empty((-(-nvec // 4), tile_words), np.uint32)
+    _check(_load().vqo_pack_tile4(_p(idx), n, nvec, b, tile_words, _p(out)), "pack_tile4")
     return out
 
 

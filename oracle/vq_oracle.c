@@ -12,7 +12,8 @@
  *
  *  - fp16 / bf16 <-> fp32 conversions from the IEEE 754 definitions
  *    (round to nearest, ties to even; subnormals kept; overflow to infinity).
- *  - unpack / pack of b-bit index fields, one bit at a time.
+ *  - unpack / pack of b-bit index fields, one bit at a time, in the row
+ *    order and in the tiled order (four vectors per tile, rows consecutive).
  *  - dequantisation: w_hat = C1[i1] (+ C2[i2]), times the row scale, plus the
  *    row bias, each an fp32 operation rounded to nearest-even, in that order,
  *    then rounded once to fp16.  Follows "VPTQ Guide: Extreme 2-Bit Vector
@@ -197,6 +198,43 @@ int vqo_pack(const uint32_t* idx, int64_t n, int64_t nvec, int b, int64_t row_wo
             for (int t = 0; t < b; ++t) {
                 int64_t p = j * (int64_t)b + t;
                 row[p >> 5] |= ((v >> t) & 1u) << (p & 31);
+            }
+        }
+    }
+    return 0;
+}
+
+/* The tiled arrangement of the same fields ("tile4", this library's second
+ * storage order; the pages fix only the field width).  A book's stream is a
+ * sequence of tiles tile_words words apart; tile t covers vectors 4t..4t+3.
+ * Inside a tile the rows follow one another, row o contributing one record of
+ * four b-bit fields: those of vectors 4t, 4t+1, 4t+2, 4t+3, in that order.
+ * So field (o, j) occupies bits [(4*o + j%4)*b, +b) of tile j/4, numbered as
+ * in the row stream.  Fields of vectors >= nvec (the tail of the last tile)
+ * are written as zero and never read. */
+static int64_t tile4_count(int64_t nvec) { return (nvec + 3) / 4; }
+
+int vqo_unpack_tile4(const uint32_t* words, int64_t n, int64_t tile_words, int b, int64_t nvec,
+                     uint32_t* idx) {
+    if (b < 1 || b > 32 || n * 4 * (int64_t)b > tile_words * 32) return 1;
+    for (int64_t o = 0; o < n; ++o)
+        for (int64_t j = 0; j < nvec; ++j)
+            idx[o * nvec + j] = field(words + (j / 4) * tile_words, b, 4 * o + j % 4);
+    return 0;
+}
+
+int vqo_pack_tile4(const uint32_t* idx, int64_t n, int64_t nvec, int b, int64_t tile_words,
+                   uint32_t* words) {
+    if (b < 1 || b > 32 || n * 4 * (int64_t)b > tile_words * 32) return 1;
+    memset(words, 0, (size_t)(tile4_count(nvec) * tile_words) * sizeof(uint32_t));
+    for (int64_t o = 0; o < n; ++o) {
+        for (int64_t j = 0; j < nvec; ++j) {
+            uint32_t v = idx[o * nvec + j];
+            if (b < 32 && (v >> b) != 0) return 2;
+            uint32_t* tile = words + (j / 4) * tile_words;
+            for (int t = 0; t < b; ++t) {
+                int64_t p = (4 * o + j % 4) * (int64_t)b + t;
+                tile[p >> 5] |= ((v >> t) & 1u) << (p & 31);
             }
         }
     }

@@ -114,6 +114,47 @@ def test_pack_rejects_wide_fields():
         oracle.pack(np.array([[8]], np.uint32), 3)
 
 
+def test_golden_tile4_layout():
+    with open(os.path.join(GOLDEN, "index_stream_tile4.txt")) as fh:
+        rows = [ln for ln in fh if ln.strip() and not ln.startswith("#")]
+    assert len(rows) == 2
+    for ln in rows:
+        b, n, nvec, fields, tiles = ln.split("|")
+        b, n, nvec = int(b), int(n), int(nvec)
+        fields = np.array([int(v) for v in fields.split()], np.uint32).reshape(n, nvec)
+        words = np.array([[int(v, 16) for v in t.split()] for t in tiles.split("/")], np.uint32)
+        assert np.array_equal(oracle.pack_tile4(fields, b), words)
+        assert np.array_equal(oracle.unpack_tile4(words, b, n, nvec), fields)
+
+
+@pytest.mark.parametrize("b", [1, 3, 4, 7, 8, 12, 16])
+def test_tile4_order_holds_the_same_fields(b):
+    """Both storage orders carry the same indices: unpacking either gives the
+    matrix that was packed, for ragged nvec and padded tiles."""
+    rng = np.random.default_rng(300 + b)
+    for n, nvec in ((1, 1), (5, 7), (33, 4), (17, 13)):
+        idx = rng.integers(0, 1 << b, size=(n, nvec), dtype=np.uint64).astype(np.uint32)
+        tw = oracle.tile4_words(n, b) + 4 * int(rng.integers(0, 2))
+        tiles = oracle.pack_tile4(idx, b, tw)
+        assert tiles.shape == (-(-nvec // 4), tw)
+        assert np.array_equal(oracle.unpack_tile4(tiles, b, n, nvec), idx)
+        assert np.array_equal(oracle.unpack(oracle.pack(idx, b), b, nvec), idx)
+        # every bit past the last record of a tile, and every field of a
+        # vector >= nvec, is zero
+        bits = np.unpackbits(tiles.view(np.uint8), axis=1, bitorder="little")
+        assert not bits[:, n * 4 * b:].any()
+        if nvec % 4:
+            rec = bits[-1, : n * 4 * b].reshape(n, 4, b)
+            assert not rec[:, nvec % 4:, :].any()
+
+
+def test_tile4_rejects_wide_fields_and_short_tiles():
+    with pytest.raises(ValueError):
+        oracle.pack_tile4(np.array([[8]], np.uint32), 3)
+    with pytest.raises(ValueError):
+        oracle.pack_tile4(np.zeros((40, 4), np.uint32), 16, tile_words=4)
+
+
 # -- dequantisation -----------------------------------------------------------
 
 ONE = np.float16(1.0).view(np.uint16)
