@@ -138,6 +138,7 @@ cudaError_t launch_dq(const Layer& L, uint16_t* w, int64_t ldw, int smem_mask, s
 
 vq_status launch_dequant(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream) {
   if (L.n == 0 || L.kin == 0) return VQ_OK;
+  if (L.layout == VQ_IDX_TILE4) return launch_dequant_tile4(L, w, ldw, stream);
   int smem_mask = 0;
   const size_t smem = stage_plan(L, std::min<size_t>(kDqSmemBooks, device_smem_optin()), &smem_mask);
   const int vec_store = aligned(w, 16) && (ldw % 8 == 0);

@@ -505,6 +505,9 @@ bool fused_fast_path(const Layer& L) {
 }
 
 int choose_mode(const Layer& L, int m) {
+  // The fused producers read row-order records; a tiled layer is dequantised
+  // by its own kernel into the workspace.
+  if (L.layout == VQ_IDX_TILE4) return kStaged;
   const char* env = std::getenv("VQ_GEMM_MODE");
   if (env && std::strcmp(env, "fused") == 0) return kFused;
   if (env && std::strcmp(env, "staged") == 0) return kStaged;

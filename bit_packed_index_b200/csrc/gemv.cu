@@ -204,7 +204,11 @@ cudaError_t launch_d(const Layer& L, const GemvPlan& p, const void* x, bool xf, 
 
 }  // namespace
 
-vq_status plan_gemv(const Layer& L, int batch, GemvPlan* p) {
+vq_status plan_gemv(const Layer& L, int batch, GemvPlan* p, size_t ws_cap) {
+  if (L.layout == VQ_IDX_TILE4) {
+    plan_gemv_tile4(L, batch, ws_cap, p);
+    return VQ_OK;
+  }
   if (batch == 1 && gemv1_supported(L)) {
     plan_gemv1(L, p);
     if (p->smem <= device_smem_optin()) return VQ_OK;
@@ -255,7 +259,9 @@ vq_status launch_gemv(const Layer& L, const GemvPlan& p, const void* x, bool x_f
   }
   const int D = (L.d == 8) ? 8 : (L.d == 6 ? 6 : 0);
   cudaError_t e;
-  if (p.fast == 1) {
+  if (p.fast >= 3) {
+    return cuda_status(launch_gemv_tile4(L, p, x, x_fp16, batch, ldx, y, yt, ldy, ws, stream));
+  } else if (p.fast == 1) {
     e = launch_gemv1(L, p, x, x_fp16, y, yt, ws, stream);
   } else if (p.fast == 2) {
     e = launch_gemvb(L, p, x, x_fp16, batch, ldx, y, yt, ldy, ws, stream);

@@ -14,8 +14,9 @@
 // on a device shares it.  Host code cannot use the variable's name as a device
 // address: the library looks the address up with cudaGetSymbolAddress on the
 // first call made on each device (with that device current) and caches it.
-// The split-K kernels write every partial sum before the finalize pass reads
-// it, so nothing in the array has to start at zero and leftover contents from
+// Plans that can shrink their scratch (the tiled lookup-table kernel runs on
+// fewer blocks) are sized to the array.  The split-K kernels write every
+// partial sum before the finalize pass reads it, so nothing in the array has to start at zero and leftover contents from
 // an earlier call are harmless.  Two calls whose kernels overlap on the GPU
 // (different streams, same device) race on the array.
 #include <mutex>
@@ -58,7 +59,7 @@ extern "C" vq_status vq_gemv_noalloc(const vq_layer_desc* layer, const void* x, 
                                      int32_t batch, int64_t ldx, void* y, vq_dtype y_dtype,
                                      int64_t ldy, void* stream) {
   size_t need = 0;
-  vq_status st = vq_gemv_workspace_size(layer, batch, &need);
+  vq_status st = gemv_workspace_bytes(layer, batch, kScratchBytes, &need);
   if (st != VQ_OK) return st;
   if (need > kScratchBytes) return VQ_ERR_WORKSPACE;
   void* ws = nullptr;
@@ -67,5 +68,6 @@ extern "C" vq_status vq_gemv_noalloc(const vq_layer_desc* layer, const void* x, 
     ws = scratch_for_current_device(&e);
     if (!ws) return cuda_status(e);
   }
-  return vq_gemv(layer, x, x_dtype, batch, ldx, y, y_dtype, ldy, ws, need, stream);
+  return gemv_run(layer, x, x_dtype, batch, ldx, y, y_dtype, ldy, ws, need, kScratchBytes,
+                  static_cast<cudaStream_t>(stream));
 }

@@ -1,7 +1,8 @@
 // sm100.cuh -- thin inline-PTX wrappers for the Blackwell (sm_100a) pieces the
-// prefill GEMM uses: mbarriers (with bounded waits), TMA tile loads, tensor
-// memory allocation, tcgen05 MMA / commit / load, and the shared-memory
-// matrix descriptor for 128-byte-swizzled K-major tiles.
+// prefill GEMM and the decode lookup-table GEMV use: mbarriers (with bounded
+// waits), TMA tile loads, tensor memory allocation, tcgen05 MMA / commit /
+// load / store, and the shared-memory matrix descriptor for 128-byte-swizzled
+// K-major tiles.
 //
 // No wait here can spin forever: bounded_wait() gives up after a clock budget,
 // raises the block's abort flag and records VQ_ERR_TIMEOUT in a global status
@@ -145,6 +146,29 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// 8 consecutive fp32 columns of one TMEM lane per thread, and the store back.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+                   taddr),
+               "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+               "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+               "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // Shared-memory matrix descriptor: K-major operand in the 128-byte swizzle

@@ -1,0 +1,517 @@
+// tile4.cu -- kernels for the tiled index order (VQ_IDX_TILE4, include/vq.h):
+// the repack from row order, W_hat from a tiled layer, a plain tiled GEMV for
+// any batch, and the decode lookup-table GEMV (batch 1) that the order exists
+// for.
+//
+// The lookup-table GEMV ("Vector Quantization for LLM Weights in Production",
+// section "2. Lookup Table (LUT) Overhead vs. Bit-Shifting": codebook lookups
+// feeding the accumulation; "VPTQ Guide", section "Step 3": y = x . W_hat^T)
+// reorders the sum y[o] = sum_j <x_j, C[i(o, j)]> around the codebook instead
+// of around the rows.  For a group of four vectors j and a quarter ("slice")
+// of the 2^16 centroids k it forms T[k][j] = <x_j, C[k]> once -- a 16 x 8 x 8
+// tensor-core product per 16 centroids -- stores T in shared memory as fp16,
+// and then every row adds the four entries its indices select.  A row's four
+// indices sit side by side in the tiled order, and consecutive rows follow one
+// another, so each thread reads one 8-byte record per row and a warp reads 256
+// contiguous bytes.  Each (group, slice) pair is one task; a block owns every
+// row of the layer for the tasks it runs, and keeps its per-row sums in tensor
+// memory (TMEM) across tasks.  A second kernel adds the per-block sums and
+// applies scale and bias.
+#include <algorithm>
+
+#include "codebook.cuh"
+#include "sm100.cuh"
+
+namespace vqk {
+namespace {
+
+// ---------------------------------------------------------------------------
+// Repack: row order -> tiled order.  One thread per output word; the word's 32
+// bits collect every field that overlaps them.  Works for any field width.
+// ---------------------------------------------------------------------------
+__global__ void repack_tile4_kernel(const uint32_t* __restrict__ src, int64_t src_rw, int b, int n,
+                                    int nvec, uint32_t* __restrict__ dst, int64_t tw) {
+  const int ntile = (nvec + 3) / 4;
+  const int64_t total = static_cast<int64_t>(ntile) * tw;
+  const int64_t nbits = static_cast<int64_t>(n) * 4 * b;   // record bits per tile
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = i / tw;
+    const int64_t bit0 = (i - t * tw) * 32;
+    uint32_t out = 0;
+    if (bit0 < nbits) {
+      const int64_t q0 = bit0 / b;
+      const int64_t q1 = min((nbits - 1) / b, (bit0 + 31) / b);
+      for (int64_t q = q0; q <= q1; ++q) {          // field q = record q/4, slot q%4
+        const int64_t o = q >> 2;
+        const int64_t j = t * 4 + (q & 3);
+        if (j >= nvec) continue;
+        const uint32_t v = load_field(src + o * src_rw, j * b, b);
+        const int64_t pos = q * b - bit0;            // in (-b, 32)
+        out |= pos >= 0 ? (v << pos) : (v >> (-pos));
+      }
+    }
+    dst[i] = out;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// W_hat from a tiled layer: one thread per (tile, row), writing the row's four
+// vectors.  The fp32 operations and their order are those of vq_dequant's
+// row-order kernel (centroid sum, times scale, plus bias, one fp16 rounding).
+// ---------------------------------------------------------------------------
+template <int D, int NB>
+__global__ void dequant_tile4_kernel(Layer L, uint16_t* __restrict__ w, int64_t ldw) {
+  const int ntile = (L.nvec + 3) / 4;
+  const int64_t total = static_cast<int64_t>(ntile) * L.n;
+  const int d = D > 0 ? D : L.d;
+  const bool has_s = L.scale != nullptr, has_t = L.bias != nullptr;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = i / L.n, o = i - t * L.n;
+    const float s = has_s ? h2f(L.scale[o]) : 1.0f;
+    const float tb = has_t ? h2f(L.bias[o]) : 0.0f;
+    const uint32_t* tile0 = L.idx[0] + t * L.rw[0];
+    const uint32_t* tile1 = L.idx[1] + t * L.rw[1];
+    uint16_t* wrow = w + o * ldw;
+#pragma unroll 1
+    for (int jj = 0; jj < 4; ++jj) {
+      const int64_t j = t * 4 + jj;
+      if (j >= L.nvec) break;
+      float c[kMaxVecDim];
+      load_centroid<D>(BookView{L.book[0], d}, load_field(tile0, (o * 4 + jj) * L.b[0], L.b[0]), d, c);
+      if constexpr (NB == 2) {
+        float c2[kMaxVecDim];
+        load_centroid<D>(BookView{L.book[1], d}, load_field(tile1, (o * 4 + jj) * L.b[1], L.b[1]), d, c2);
+#pragma unroll
+        for (int e = 0; e < kMaxVecDim; ++e)
+          if (e < d) c[e] = __fadd_rn(c[e], c2[e]);
+      }
+      const int64_t k0 = j * d;
+#pragma unroll
+      for (int e = 0; e < kMaxVecDim; ++e) {
+        if (e < d && k0 + e < L.kin) {
+          float v = c[e];
+          if (has_s) v = __fmul_rn(v, s);
+          if (has_t) v = __fadd_rn(v, tb);
+          wrow[k0 + e] = f2h(v);
+        }
+      }
+    }
+  }
+}
+
+template <int D, int NB>
+cudaError_t launch_dq4(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream) {
+  const int64_t total = static_cast<int64_t>((L.nvec + 3) / 4) * L.n;
+  const int grid = static_cast<int>(std::min<int64_t>((total + 255) / 256, 16LL * device_sm_count()));
+  count_launch();
+  dequant_tile4_kernel<D, NB><<<grid, 256, 0, stream>>>(L, w, ldw);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+vq_status launch_repack_tile4(const Layer& L, uint32_t* const dst[2], const int64_t tw[2],
+                              cudaStream_t stream) {
+  for (int m = 0; m < L.nb; ++m) {
+    const int64_t total = static_cast<int64_t>((L.nvec + 3) / 4) * tw[m];
+    const int grid = static_cast<int>(std::min<int64_t>((total + 255) / 256, 16LL * device_sm_count()));
+    count_launch();
+    repack_tile4_kernel<<<grid, 256, 0, stream>>>(L.idx[m], L.rw[m], L.b[m], L.n, L.nvec, dst[m], tw[m]);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  return VQ_OK;
+}
+
+vq_status launch_dequant_tile4(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream) {
+  if (L.n == 0 || L.kin == 0) return VQ_OK;
+  cudaError_t e;
+  if (L.nb == 1)
+    e = L.d == 8 ? launch_dq4<8, 1>(L, w, ldw, stream)
+      : L.d == 6 ? launch_dq4<6, 1>(L, w, ldw, stream) : launch_dq4<0, 1>(L, w, ldw, stream);
+  else
+    e = L.d == 8 ? launch_dq4<8, 2>(L, w, ldw, stream)
+      : L.d == 6 ? launch_dq4<6, 2>(L, w, ldw, stream) : launch_dq4<0, 2>(L, w, ldw, stream);
+  return cuda_status(e);
+}
+
+
+namespace {
+
+__device__ __forceinline__ float x_at(const uint16_t* __restrict__ x, int x_fp16, int64_t i) {
+  const uint16_t u = __ldg(x + i);
+  return x_fp16 ? h2f(u) : bf2f(u);
+}
+
+// ---------------------------------------------------------------------------
+// Plain tiled GEMV, any batch (1..16), any d and book count: one thread per
+// output row walks the row's records tile by tile, gathers the centroids and
+// accumulates x . c in fp32 for every batch row.  Consecutive threads read
+// consecutive records, and all lanes of a warp read the same x element.
+// ---------------------------------------------------------------------------
+template <int NB>
+__global__ void __launch_bounds__(256) gemv_tile4_kernel(Layer L, const uint16_t* __restrict__ x,
+                                                         int x_fp16, int batch, int64_t ldx,
+                                                         void* __restrict__ y, vq_dtype yt,
+                                                         int64_t ldy) {
+  __shared__ float red[8];
+  __shared__ float xsum[kMaxBatch];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int b = 0; b < batch; ++b) {          // sum_k x[b][k] for the bias term, fixed order
+    float v = 0.0f;
+    for (int k = threadIdx.x; k < L.kin; k += blockDim.x) v += x_at(x, x_fp16, b * ldx + k);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float t = 0.0f;
+      for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t += red[i];
+      xsum[b] = t;
+    }
+    __syncthreads();
+  }
+  const int d = L.d;
+  const int ntile = (L.nvec + 3) / 4;
+  for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < L.n;
+       o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float acc[kMaxBatch];
+#pragma unroll
+    for (int b = 0; b < kMaxBatch; ++b) acc[b] = 0.0f;
+    for (int t = 0; t < ntile; ++t) {
+      const uint32_t* tile0 = L.idx[0] + t * L.rw[0];
+      const uint32_t* tile1 = L.idx[1] + t * L.rw[1];
+      for (int jj = 0; jj < 4; ++jj) {
+        const int j = t * 4 + jj;
+        if (j >= L.nvec) break;
+        float c[kMaxVecDim];
+        load_centroid<0>(BookView{L.book[0], d}, load_field(tile0, (o * 4 + jj) * L.b[0], L.b[0]), d, c);
+        if constexpr (NB == 2) {
+          float c2[kMaxVecDim];
+          load_centroid<0>(BookView{L.book[1], d}, load_field(tile1, (o * 4 + jj) * L.b[1], L.b[1]), d, c2);
+#pragma unroll
+          for (int e = 0; e < kMaxVecDim; ++e) c[e] += c2[e];
+        }
+        const int64_t k0 = static_cast<int64_t>(j) * d;
+        for (int e = 0; e < d; ++e) {
+          if (k0 + e >= L.kin) break;
+#pragma unroll
+          for (int b = 0; b < kMaxBatch; ++b)
+            if (b < batch) acc[b] = fmaf(x_at(x, x_fp16, b * ldx + k0 + e), c[e], acc[b]);
+        }
+      }
+    }
+    const float sc = L.scale ? h2f(L.scale[o]) : 1.0f;
+    const float tb = L.bias ? h2f(L.bias[o]) : 0.0f;
+#pragma unroll
+    for (int b = 0; b < kMaxBatch; ++b)
+      if (b < batch) store_out(y, yt, b * ldy + o, sc * acc[b] + tb * xsum[b]);
+  }
+}
+
+}  // namespace
+
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Decode lookup-table GEMV (batch 1; one book; d = 8; 16-bit indices).
+// ---------------------------------------------------------------------------
+constexpr int kLutThreads = 1024;
+constexpr int kLutLog2S = 14;                       // a slice holds 2^14 centroids
+constexpr int kLutS = 1 << kLutLog2S;
+constexpr int kLutSlices = 65536 / kLutS;           // 4 slices of the 2^16 book
+constexpr int kLutSmem = kLutS * 4 * 2;             // T[S][4] in fp16: 128 KB
+constexpr int kLutPD = 8;                           // 16-centroid tiles per load batch
+
+__device__ __forceinline__ uint32_t ldg_stream32(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint2 ldg_stream64(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+
+// RB8 batches of 8 rows per thread: a block covers N <= 8 * RB8 * 1024 rows;
+// thread (warp w, lane l) keeps its row sums in TMEM lane 32*(w%4)+l, columns
+// (w/4)*8*RB8 .. +8*RB8 (warps may only touch their own quarter of the lanes).
+template <int RB8>
+__global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const uint16_t* __restrict__ x,
+                                                                  int x_fp16, float* __restrict__ part,
+                                                                  float* __restrict__ xpart) {
+  constexpr int CPW = 8 * RB8;                      // TMEM columns per group of 4 warps
+  constexpr int TCOLS = 8 * CPW;                    // 64 .. 512, a power of two
+  constexpr int TILES_PER_WARP = kLutS / 16 / (kLutThreads / 32);
+  constexpr int NBATCH = TILES_PER_WARP / kLutPD;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint16_t* lut = reinterpret_cast<uint16_t*>(smem);   // T[k - slice base][4 vectors]
+  __shared__ uint32_t s_tmem;
+  __shared__ float s_scale;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n = L.n, kin = L.kin;
+  const int ntasks = ((L.nvec + 3) / 4) * kLutSlices;
+
+  if (warp == 0) {
+    sm100::tmem_alloc(&s_tmem, TCOLS);
+    sm100::tmem_relinquish();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tbase = s_tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) +
+                         static_cast<uint32_t>((warp >> 2) * CPW);
+  {
+    float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int b = 0; b < RB8; ++b) sm100::tmem_st8(tbase + 8 * b, z);
+    sm100::tmem_wait_st();
+  }
+  float xs_acc = 0.0f;   // warp 0: sum of x, one group per slice-0 task
+
+  for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
+    const int g = task / kLutSlices, s = task - g * kLutSlices;
+    // B operand of m16n8k8: x'[vector 4g + lane/4][components 2t, 2t+1], columns
+    // 4..7 zero.  x' = x * 2^-e with ||x'_j||_1 < 1 for all four vectors, so
+    // |T| <= max |c| and no product overflows fp16; 2^e is applied per row.
+    uint32_t bfrag;
+    {
+      const int jj = lane >> 2, t = lane & 3;
+      const int64_t k = (static_cast<int64_t>(g) * 4 + jj) * 8 + 2 * t;
+      float a = 0.0f, b = 0.0f;
+      if (jj < 4) {
+        if (k < kin) a = x_at(x, x_fp16, k);
+        if (k + 1 < kin) b = x_at(x, x_fp16, k + 1);
+      }
+      float l1 = fabsf(a) + fabsf(b);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      float mx = l1;
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      int e = 0;
+      if (mx > 0.0f && mx < INFINITY) frexpf(mx, &e);
+      const __half2 h = __floats2half2_rn(ldexpf(a, -e), ldexpf(b, -e));
+      bfrag = *reinterpret_cast<const uint32_t*>(&h);
+      if (tid == 0) s_scale = ldexpf(1.0f, e);
+      if (warp == 0 && s == 0) {
+        float v = a + b;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        xs_acc += v;
+      }
+    }
+    // Phase A: T for this slice.  Warp w builds tiles [32w, 32w+32) of 16
+    // centroids; each tile's A operand is read straight from the codebook
+    // (lane: centroid lane/4 (+8), components 2t, 2t+1), two batches in flight.
+    {
+      const uint16_t* bslice = L.book[0] + static_cast<size_t>(s) * kLutS * 8;
+      const int t0w = warp * TILES_PER_WARP;
+      uint32_t afr[2][kLutPD][2];
+#pragma unroll
+      for (int p = 0; p < kLutPD; ++p) {
+        const uint16_t* c0 = bslice + ((t0w + p) * 16 + (lane >> 2)) * 8 + 2 * (lane & 3);
+        afr[0][p][0] = ldg_stream32(c0);
+        afr[0][p][1] = ldg_stream32(c0 + 64);
+      }
+#pragma unroll
+      for (int bt = 0; bt < NBATCH; ++bt) {
+        const int cur = bt & 1;
+        if (bt + 1 < NBATCH) {
+#pragma unroll
+          for (int p = 0; p < kLutPD; ++p) {
+            const uint16_t* c0 = bslice + ((t0w + (bt + 1) * kLutPD + p) * 16 + (lane >> 2)) * 8 + 2 * (lane & 3);
+            afr[cur ^ 1][p][0] = ldg_stream32(c0);
+            afr[cur ^ 1][p][1] = ldg_stream32(c0 + 64);
+          }
+        }
+#pragma unroll
+        for (int p = 0; p < kLutPD; ++p) {
+          float d0, d1, d2, d3;
+          asm volatile(
+              "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
+              "{%7, %8, %9, %10};"
+              : "=f"(d0), "=f"(d1), "=f"(d2), "=f"(d3)
+              : "r"(afr[cur][p][0]), "r"(afr[cur][p][1]), "r"(bfrag), "f"(0.0f), "f"(0.0f), "f"(0.0f),
+                "f"(0.0f));
+          if ((lane & 3) < 2) {                     // columns 0..3 are the four vectors
+            const int kl = (t0w + bt * kLutPD + p) * 16 + (lane >> 2);
+            *reinterpret_cast<__half2*>(lut + kl * 4 + 2 * (lane & 3)) = __floats2half2_rn(d0, d1);
+            *reinterpret_cast<__half2*>(lut + (kl + 8) * 4 + 2 * (lane & 3)) = __floats2half2_rn(d2, d3);
+          }
+        }
+      }
+    }
+    __syncthreads();   // T complete
+    // Phase B: every row adds the T entries its four indices select from this
+    // slice; the records come straight from global memory, two batches of 8
+    // rows in flight, and the running sums live in TMEM.
+    {
+      const float sc = s_scale;
+      const uint2* trow = reinterpret_cast<const uint2*>(L.idx[0] + static_cast<int64_t>(g) * L.rw[0]);
+      uint2 w[2][8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int o = r * kLutThreads + tid;
+        w[0][r] = o < n ? ldg_stream64(trow + o) : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int b = 0; b < RB8; ++b) {
+        const int cur = b & 1;
+        if (b + 1 < RB8) {
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            const int o = ((b + 1) * 8 + r) * kLutThreads + tid;
+            w[cur ^ 1][r] = o < n ? ldg_stream64(trow + o) : make_uint2(0u, 0u);
+          }
+        }
+        float acc[8];
+        sm100::tmem_ld8(tbase + 8 * b, acc);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          float v[4];
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            const uint32_t k = ((jj < 2 ? w[cur][r].x : w[cur][r].y) >> (16 * (jj & 1))) & 0xFFFFu;
+            v[jj] = 0.0f;
+            if ((k >> kLutLog2S) == static_cast<uint32_t>(s)) v[jj] = h2f(lut[(k & (kLutS - 1)) * 4 + jj]);
+          }
+          acc[r] = fmaf((v[0] + v[1]) + (v[2] + v[3]), sc, acc[r]);
+        }
+        sm100::tmem_st8(tbase + 8 * b, acc);
+      }
+      sm100::tmem_wait_st();
+    }
+    __syncthreads();   // all lookups done before the next task rewrites T
+  }
+
+#pragma unroll
+  for (int b = 0; b < RB8; ++b) {
+    float acc[8];
+    sm100::tmem_ld8(tbase + 8 * b, acc);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int o = (b * 8 + r) * kLutThreads + tid;
+      if (o < n) part[static_cast<int64_t>(blockIdx.x) * n + o] = acc[r];
+    }
+  }
+  if (tid == 0) xpart[blockIdx.x] = xs_acc;
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  if (warp == 0) sm100::tmem_dealloc(s_tmem, TCOLS);
+}
+
+// y[o] = s[o] * sum_b part[b][o] + t[o] * sum_b xpart[b], in a fixed order.
+// 32 rows per block: lane = row, the 8 warps stride the per-block sums.
+__global__ void __launch_bounds__(256) gemv_lut_finalize(const float* __restrict__ part,
+                                                         const float* __restrict__ xpart, int nparts,
+                                                         int n, const uint16_t* __restrict__ scale,
+                                                         const uint16_t* __restrict__ bias,
+                                                         void* __restrict__ y, vq_dtype yt) {
+  __shared__ float red[8][33];
+  __shared__ float s_xsum;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int o = blockIdx.x * 32 + lane;
+  if (warp == 0) {
+    float v = 0.0f;
+    if (bias)
+      for (int i = lane; i < nparts; i += 32) v += xpart[i];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if (lane == 0) s_xsum = v;
+  }
+  float s4[4] = {0.f, 0.f, 0.f, 0.f};
+  if (o < n) {
+    int b = warp;
+    for (; b + 24 < nparts; b += 32)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) s4[u] += part[static_cast<int64_t>(b + 8 * u) * n + o];
+    for (; b < nparts; b += 8) s4[0] += part[static_cast<int64_t>(b) * n + o];
+  }
+  red[warp][lane] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+  __syncthreads();
+  if (warp == 0 && o < n) {
+    float t = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += red[w][lane];
+    const float sc = scale ? h2f(scale[o]) : 1.0f;
+    const float tb = bias ? h2f(bias[o]) : 0.0f;
+    store_out(y, yt, o, sc * t + tb * s_xsum);
+  }
+}
+
+template <int RB8>
+cudaError_t launch_lut(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, void* y,
+                       vq_dtype yt, float* ws, cudaStream_t stream) {
+  auto k = gemv_lut_kernel<RB8>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutSmem);
+  if (e != cudaSuccess) return e;
+  float* part = ws;
+  float* xpart = ws + static_cast<int64_t>(p.grid_x) * L.n;
+  count_launch();
+  k<<<p.grid_x, kLutThreads, kLutSmem, stream>>>(L, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, part, xpart);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  count_launch();
+  gemv_lut_finalize<<<(L.n + 31) / 32, 256, 0, stream>>>(part, xpart, p.grid_x, L.n, L.scale, L.bias, y, yt);
+  return cudaGetLastError();
+}
+
+bool lut_supported(const Layer& L) {
+  return L.layout == VQ_IDX_TILE4 && L.nb == 1 && L.d == 8 && L.b[0] == 16 && L.n >= 1 &&
+         L.n <= 8 * 8 * kLutThreads && L.nvec >= 1 && device_smem_optin() >= kLutSmem + 1024;
+}
+
+}  // namespace
+
+void plan_gemv_tile4(const Layer& L, int batch, size_t ws_cap, GemvPlan* p) {
+  *p = GemvPlan{};
+  p->nsplit = 1;
+  if (batch == 1 && lut_supported(L)) {
+    const int ntasks = ((L.nvec + 3) / 4) * kLutSlices;
+    const size_t per_block = (static_cast<size_t>(L.n) + 1) * sizeof(float);
+    int grid = std::min(device_sm_count(), ntasks);
+    if (ws_cap / per_block < static_cast<size_t>(grid)) grid = static_cast<int>(ws_cap / per_block);
+    if (grid >= 1) {
+      int rb8 = 1;
+      while (static_cast<int64_t>(rb8) * 8 * kLutThreads < L.n) rb8 <<= 1;
+      p->fast = 3;
+      p->grid_x = grid;
+      p->bt = rb8;
+      p->smem = kLutSmem;
+      p->ws_bytes = per_block * grid;
+      return;
+    }
+  }
+  p->fast = 4;
+  p->bt = batch;
+  p->grid_x = std::max(1, std::min((L.n + 255) / 256, 8 * device_sm_count()));
+  p->ws_bytes = 0;
+}
+
+cudaError_t launch_gemv_tile4(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16,
+                              int batch, int64_t ldx, void* y, vq_dtype yt, int64_t ldy, float* ws,
+                              cudaStream_t stream) {
+  if (p.fast == 3) {
+    switch (p.bt) {
+      case 1: return launch_lut<1>(L, p, x, x_fp16, y, yt, ws, stream);
+      case 2: return launch_lut<2>(L, p, x, x_fp16, y, yt, ws, stream);
+      case 4: return launch_lut<4>(L, p, x, x_fp16, y, yt, ws, stream);
+      default: return launch_lut<8>(L, p, x, x_fp16, y, yt, ws, stream);
+    }
+  }
+  count_launch();
+  if (L.nb == 1)
+    gemv_tile4_kernel<1><<<p.grid_x, 256, 0, stream>>>(L, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0,
+                                                        batch, ldx, y, yt, ldy);
+  else
+    gemv_tile4_kernel<2><<<p.grid_x, 256, 0, stream>>>(L, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0,
+                                                        batch, ldx, y, yt, ldy);
+  return cudaGetLastError();
+}
+
+}  // namespace vqk

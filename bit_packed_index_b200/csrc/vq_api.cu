@@ -7,7 +7,7 @@
 
 #include "vq_internal.cuh"
 
-static_assert(sizeof(vq_layer_desc) == 88, "vq_layer_desc layout is part of the ABI");
+static_assert(sizeof(vq_layer_desc) == 96, "vq_layer_desc layout is part of the ABI");
 
 namespace vqk {
 namespace {
@@ -60,7 +60,10 @@ vq_status check_layer(const vq_layer_desc* desc, Layer* out) {
   if (D.out_features < 0 || D.in_features < 0) return VQ_ERR_INVALID_ARG;
   if (D.vec_dim < 1 || D.vec_dim > kMaxVecDim) return VQ_ERR_INVALID_ARG;
   if (D.n_books < 1 || D.n_books > 2) return VQ_ERR_INVALID_ARG;
+  if ((D.idx_layout != VQ_IDX_ROWS && D.idx_layout != VQ_IDX_TILE4) || D.reserved != 0)
+    return VQ_ERR_INVALID_ARG;
   Layer L{};
+  L.layout = D.idx_layout;
   L.n = D.out_features;
   L.kin = D.in_features;
   L.d = D.vec_dim;
@@ -69,7 +72,9 @@ vq_status check_layer(const vq_layer_desc* desc, Layer* out) {
   for (int m = 0; m < L.nb; ++m) {
     const int b = D.log2k[m];
     if (b < 1 || b > 16) return VQ_ERR_INVALID_ARG;
-    const int64_t need = (static_cast<int64_t>(L.nvec) * b + 127) / 128 * 4;
+    const int64_t need = L.layout == VQ_IDX_ROWS
+                             ? (static_cast<int64_t>(L.nvec) * b + 127) / 128 * 4
+                             : (static_cast<int64_t>(L.n) * 4 * b + 127) / 128 * 4;
     const int64_t rw = D.idx_row_words[m];
     if (rw < need || rw % 4 != 0) return VQ_ERR_INVALID_ARG;
     if (L.n > 0 && L.nvec > 0) {
@@ -94,6 +99,46 @@ vq_status check_layer(const vq_layer_desc* desc, Layer* out) {
   return VQ_OK;
 }
 
+vq_status gemv_workspace_bytes(const vq_layer_desc* layer, int32_t batch, size_t cap,
+                               size_t* bytes) {
+  if (!bytes) return VQ_ERR_INVALID_ARG;
+  Layer L;
+  vq_status st = check_layer(layer, &L);
+  if (st != VQ_OK) return st;
+  if (batch < 0) return VQ_ERR_INVALID_ARG;
+  if (batch > kMaxBatch) return VQ_ERR_UNSUPPORTED;
+  *bytes = 0;
+  if (batch == 0 || L.n == 0) return VQ_OK;
+  GemvPlan p;
+  st = plan_gemv(L, batch, &p, cap);
+  if (st != VQ_OK) return st;
+  *bytes = p.ws_bytes;
+  return VQ_OK;
+}
+
+vq_status gemv_run(const vq_layer_desc* layer, const void* x, vq_dtype x_dtype, int32_t batch,
+                   int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy, void* workspace,
+                   size_t workspace_bytes, size_t cap, cudaStream_t stream) {
+  Layer L;
+  vq_status st = check_layer(layer, &L);
+  if (st != VQ_OK) return st;
+  if (batch < 0 || !dtype_ok_in(x_dtype) || !dtype_ok_out(y_dtype)) return VQ_ERR_INVALID_ARG;
+  if (batch > kMaxBatch) return VQ_ERR_UNSUPPORTED;
+  if (ldx < L.kin || ldy < L.n) return VQ_ERR_INVALID_ARG;
+  if (batch == 0 || L.n == 0) return VQ_OK;
+  if (!y || (!x && L.kin > 0)) return VQ_ERR_INVALID_ARG;
+  if (!aligned(x, 2) || !aligned(y, dtype_size(y_dtype))) return VQ_ERR_ALIGNMENT;
+  GemvPlan p;
+  st = plan_gemv(L, batch, &p, cap);
+  if (st != VQ_OK) return st;
+  if (p.ws_bytes > 0) {
+    if (!workspace || workspace_bytes < p.ws_bytes) return VQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return VQ_ERR_ALIGNMENT;
+  }
+  return launch_gemv(L, p, x, x_dtype == VQ_FP16, batch, ldx, y, y_dtype, ldy,
+                     static_cast<float*>(workspace), stream);
+}
+
 }  // namespace vqk
 
 using namespace vqk;
@@ -111,43 +156,33 @@ vq_status vq_dequant(const vq_layer_desc* layer, uint16_t* w_hat, int64_t ldw, v
   return launch_dequant(L, w_hat, ldw, static_cast<cudaStream_t>(stream));
 }
 
-vq_status vq_gemv_workspace_size(const vq_layer_desc* layer, int32_t batch, size_t* bytes) {
-  if (!bytes) return VQ_ERR_INVALID_ARG;
+vq_status vq_repack_tile4(const vq_layer_desc* src, uint32_t* const dst[2],
+                          const int64_t dst_tile_words[2], void* stream) {
   Layer L;
-  vq_status st = check_layer(layer, &L);
+  vq_status st = check_layer(src, &L);
   if (st != VQ_OK) return st;
-  if (batch < 0) return VQ_ERR_INVALID_ARG;
-  if (batch > kMaxBatch) return VQ_ERR_UNSUPPORTED;
-  *bytes = 0;
-  if (batch == 0 || L.n == 0) return VQ_OK;
-  GemvPlan p;
-  st = plan_gemv(L, batch, &p);
-  if (st != VQ_OK) return st;
-  *bytes = p.ws_bytes;
-  return VQ_OK;
+  if (L.layout != VQ_IDX_ROWS || !dst || !dst_tile_words) return VQ_ERR_INVALID_ARG;
+  for (int m = 0; m < L.nb; ++m) {
+    const int64_t need = (static_cast<int64_t>(L.n) * 4 * L.b[m] + 127) / 128 * 4;
+    if (dst_tile_words[m] < need || dst_tile_words[m] % 4 != 0) return VQ_ERR_INVALID_ARG;
+    if (L.n > 0 && L.nvec > 0) {
+      if (!dst[m]) return VQ_ERR_INVALID_ARG;
+      if (!aligned(dst[m], 16)) return VQ_ERR_ALIGNMENT;
+    }
+  }
+  if (L.n == 0 || L.nvec == 0) return VQ_OK;
+  return launch_repack_tile4(L, dst, dst_tile_words, static_cast<cudaStream_t>(stream));
+}
+
+vq_status vq_gemv_workspace_size(const vq_layer_desc* layer, int32_t batch, size_t* bytes) {
+  return gemv_workspace_bytes(layer, batch, ~static_cast<size_t>(0), bytes);
 }
 
 vq_status vq_gemv(const vq_layer_desc* layer, const void* x, vq_dtype x_dtype, int32_t batch,
                   int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy, void* workspace,
                   size_t workspace_bytes, void* stream) {
-  Layer L;
-  vq_status st = check_layer(layer, &L);
-  if (st != VQ_OK) return st;
-  if (batch < 0 || !dtype_ok_in(x_dtype) || !dtype_ok_out(y_dtype)) return VQ_ERR_INVALID_ARG;
-  if (batch > kMaxBatch) return VQ_ERR_UNSUPPORTED;
-  if (ldx < L.kin || ldy < L.n) return VQ_ERR_INVALID_ARG;
-  if (batch == 0 || L.n == 0) return VQ_OK;
-  if (!y || (!x && L.kin > 0)) return VQ_ERR_INVALID_ARG;
-  if (!aligned(x, 2) || !aligned(y, dtype_size(y_dtype))) return VQ_ERR_ALIGNMENT;
-  GemvPlan p;
-  st = plan_gemv(L, batch, &p);
-  if (st != VQ_OK) return st;
-  if (p.ws_bytes > 0) {
-    if (!workspace || workspace_bytes < p.ws_bytes) return VQ_ERR_WORKSPACE;
-    if (!aligned(workspace, 256)) return VQ_ERR_ALIGNMENT;
-  }
-  return launch_gemv(L, p, x, x_dtype == VQ_FP16, batch, ldx, y, y_dtype, ldy,
-                     static_cast<float*>(workspace), static_cast<cudaStream_t>(stream));
+  return gemv_run(layer, x, x_dtype, batch, ldx, y, y_dtype, ldy, workspace, workspace_bytes,
+                  ~static_cast<size_t>(0), static_cast<cudaStream_t>(stream));
 }
 
 vq_status vq_gemm_workspace_size(const vq_layer_desc* layer, int32_t m, vq_dtype x_dtype,

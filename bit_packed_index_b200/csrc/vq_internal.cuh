@@ -26,17 +26,24 @@ struct Layer {
   int nb;           // number of codebooks (1 or 2)
   int nvec;         // ceil(kin / d)
   int b[2];         // index width per book
-  int64_t rw[2];    // stream row stride, 32-bit words
+  int64_t rw[2];    // stream row (row order) or tile (tiled order) stride, 32-bit words
   const uint32_t* idx[2];
   const uint16_t* book[2];
   const uint16_t* scale;  // may be null
   const uint16_t* bias;   // may be null
+  int layout;             // VQ_IDX_ROWS or VQ_IDX_TILE4
 };
 
 // ---------------------------------------------------------------------------
 // Host helpers (vq_api.cu).
 // ---------------------------------------------------------------------------
 vq_status check_layer(const vq_layer_desc* desc, Layer* out);
+// The GEMV entry points, with the largest workspace the caller can give
+// (vq_gemv: unlimited; vq_gemv_noalloc: its fixed scratch array).
+vq_status gemv_workspace_bytes(const vq_layer_desc* layer, int32_t batch, size_t cap, size_t* bytes);
+vq_status gemv_run(const vq_layer_desc* layer, const void* x, vq_dtype x_dtype, int32_t batch,
+                   int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy, void* workspace,
+                   size_t workspace_bytes, size_t cap, cudaStream_t stream);
 vq_status cuda_status(cudaError_t e);  // records e, returns VQ_ERR_CUDA (or VQ_OK)
 void count_launch(int n = 1);          // adds to the process-wide kernel launch counter
 int device_sm_count();
@@ -49,6 +56,11 @@ __host__ __device__ inline bool aligned(const void* p, size_t a) { return (reint
 // ---------------------------------------------------------------------------
 vq_status launch_dequant(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream);
 
+// Tiled index order (tile4.cu).
+vq_status launch_repack_tile4(const Layer& src, uint32_t* const dst[2], const int64_t tile_words[2],
+                              cudaStream_t stream);
+vq_status launch_dequant_tile4(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream);
+
 struct GemvPlan {
   int bt;        // batch tile (power of two >= batch)
   int nsplit;    // K splits
@@ -59,9 +71,16 @@ struct GemvPlan {
   int books_in_smem;  // bit m set: book m staged in shared memory
   int book_bytes;     // shared memory taken by the staged books
   size_t ws_bytes;
-  int fast = 0;       // 1: single-row kernel (gemv1.cu), 2: batched kernel (gemvb.cu)
+  int fast = 0;       // 1: single-row kernel (gemv1.cu), 2: batched kernel (gemvb.cu),
+                      // 3: lookup-table kernel, 4: plain tiled kernel (tile4.cu)
 };
-vq_status plan_gemv(const Layer& L, int batch, GemvPlan* plan);
+// ws_cap: largest workspace the caller can provide (plans that need more
+// either shrink, for the tiled kernels, or are reported by their ws_bytes).
+vq_status plan_gemv(const Layer& L, int batch, GemvPlan* plan, size_t ws_cap = ~static_cast<size_t>(0));
+void plan_gemv_tile4(const Layer& L, int batch, size_t ws_cap, GemvPlan* plan);
+cudaError_t launch_gemv_tile4(const Layer& L, const GemvPlan& plan, const void* x, bool x_fp16,
+                              int batch, int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy,
+                              float* ws, cudaStream_t stream);
 bool gemv1_supported(const Layer& L);
 bool gemvb_supported(const Layer& L, int batch);
 void plan_gemvb(const Layer& L, int batch, GemvPlan* plan);

@@ -4,9 +4,10 @@ Every computation runs in the CUDA kernels behind the C ABI; this module only
 turns torch tensors into pointers, sizes and the current CUDA stream.  There
 is no fallback: if ``libvq.so`` is missing or fails to load, every call raises.
 
-Names follow the C ABI: ``dequant``, ``gemv``, ``gemm``, plus the workspace
-size queries.  A ``Layer`` holds the device tensors of one quantised layer
-(packed index streams, fp16 codebooks, optional fp16 scale and bias).
+Names follow the C ABI: ``dequant``, ``gemv``, ``gemm``, ``repack_tile4``,
+plus the workspace size queries.  A ``Layer`` holds the device tensors of one
+quantised layer (packed index streams in row order or in the tiled order,
+fp16 codebooks, optional fp16 scale and bias).
 """
 from __future__ import annotations
 
@@ -26,6 +27,8 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "vq.h")
 VQ_OK, VQ_ERR_INVALID_ARG, VQ_ERR_UNSUPPORTED, VQ_ERR_ALIGNMENT = 0, 1, 2, 3
 VQ_ERR_WORKSPACE, VQ_ERR_CUDA, VQ_ERR_TIMEOUT = 4, 5, 6
 VQ_BF16, VQ_FP16, VQ_FP32 = 0, 1, 2
+VQ_IDX_ROWS, VQ_IDX_TILE4 = 0, 1
+_LAYOUT = {"rows": VQ_IDX_ROWS, "tile4": VQ_IDX_TILE4}
 
 _DTYPE = {torch.bfloat16: VQ_BF16, torch.float16: VQ_FP16, torch.float32: VQ_FP32}
 
@@ -44,6 +47,7 @@ class _Desc(C.Structure):
         ("vec_dim", C.c_int32), ("n_books", C.c_int32), ("log2k", C.c_int32 * 2),
         ("idx", C.c_void_p * 2), ("idx_row_words", C.c_int64 * 2),
         ("codebook", C.c_void_p * 2), ("scale", C.c_void_p), ("bias", C.c_void_p),
+        ("idx_layout", C.c_int32), ("reserved", C.c_int32),
     ]
 
 
@@ -74,8 +78,9 @@ def lib():
             L.vq_gemv_noalloc.argtypes = [P, P, C.c_int, I32, I64, P, C.c_int, I64, P]
             L.vq_gemm_workspace_size.argtypes = [P, I32, C.c_int, C.POINTER(SZ)]
             L.vq_gemm.argtypes = [P, P, C.c_int, I32, I64, P, C.c_int, I64, P, SZ, P]
+            L.vq_repack_tile4.argtypes = [P, C.POINTER(P), C.POINTER(I64), P]
             for fn in ("vq_dequant", "vq_gemv_workspace_size", "vq_gemv", "vq_gemv_noalloc",
-                       "vq_gemm_workspace_size", "vq_gemm"):
+                       "vq_gemm_workspace_size", "vq_gemm", "vq_repack_tile4"):
                 getattr(L, fn).restype = C.c_int
             L.vq_status_string.argtypes = [C.c_int]
             L.vq_status_string.restype = C.c_char_p
@@ -108,10 +113,12 @@ class Layer:
     in_features: int
     vec_dim: int
     log2k: List[int]
-    idx: List[torch.Tensor]            # int32 views of uint32 words [N][row_words]
+    idx: List[torch.Tensor]            # int32 views of uint32 words: [N][row_words] in row
+                                       # order, [ceil(nvec/4)][tile_words] tiled
     codebooks: List[torch.Tensor]      # float16 [K][d]
     scale: Optional[torch.Tensor] = None   # float16 [N]
     bias: Optional[torch.Tensor] = None    # float16 [N]
+    layout: str = "rows"               # "rows" or "tile4"
     _desc: Optional[_Desc] = field(default=None, repr=False)
 
     @property
@@ -134,6 +141,7 @@ class Layer:
                 d.codebook[m] = self.codebooks[m].data_ptr()
             d.scale = None if self.scale is None else self.scale.data_ptr()
             d.bias = None if self.bias is None else self.bias.data_ptr()
+            d.idx_layout = _LAYOUT[self.layout]
             self._desc = d
         return self._desc
 
@@ -159,16 +167,46 @@ class Layer:
                    halves(scale), halves(bias))
 
     @classmethod
-    def from_synth(cls, data, device="cuda") -> "Layer":
+    def from_synth(cls, data, device="cuda", layout: str = "rows") -> "Layer":
+        """From generated host data (row-order streams); layout="tile4" converts
+        them on the device with vq_repack_tile4."""
         s = data.spec
-        return cls.from_host(s.out_features, s.in_features, s.d, s.log2k, data.idx_words,
-                             data.codebooks, data.scale, data.bias, device)
+        layer = cls.from_host(s.out_features, s.in_features, s.d, s.log2k, data.idx_words,
+                              data.codebooks, data.scale, data.bias, device)
+        if layout == "tile4":
+            layer = repack_tile4(layer)
+        elif layout != "rows":
+            raise ValueError(f"unknown index layout {layout!r}")
+        return layer
 
     def nbytes(self) -> int:
         n = sum(t.numel() * t.element_size() for t in self.idx + self.codebooks)
         for t in (self.scale, self.bias):
             n += 0 if t is None else t.numel() * 2
         return n
+
+
+def tile4_words(out_features: int, log2k: int) -> int:
+    """Smallest tile stride (32-bit words) of the tiled order: N records of 4 fields."""
+    return -(-(out_features * 4 * log2k) // 128) * 4
+
+
+def repack_tile4(layer: Layer, tile_words: Optional[Sequence[int]] = None) -> Layer:
+    """The same layer with its index streams in the tiled order (vq_repack_tile4);
+    codebooks, scale and bias are shared with ``layer``."""
+    if layer.layout != "rows":
+        raise ValueError("repack_tile4 needs a row-order layer")
+    nvec = -(-layer.in_features // layer.vec_dim)
+    ntile = -(-nvec // 4)
+    tw = [tile4_words(layer.out_features, b) if tile_words is None else int(tile_words[m])
+          for m, b in enumerate(layer.log2k)]
+    dst = [torch.empty((ntile, w), dtype=torch.int32, device=layer.device) for w in tw]
+    ptrs = (C.c_void_p * 2)(*([t.data_ptr() for t in dst] + [0] * (2 - len(dst))))
+    words = (C.c_int64 * 2)(*(tw + [0] * (2 - len(tw))))
+    _check("vq_repack_tile4", lib().vq_repack_tile4(C.byref(layer.desc()), ptrs, words,
+                                                    C.c_void_p(_stream(layer.device))))
+    return Layer(layer.out_features, layer.in_features, layer.vec_dim, list(layer.log2k), dst,
+                 layer.codebooks, layer.scale, layer.bias, layout="tile4")
 
 
 def dequant(layer: Layer, out: Optional[torch.Tensor] = None) -> torch.Tensor:

@@ -39,6 +39,19 @@
  * ceil(nvec*b / 128) * 4.  Bits past nvec*b in a row are ignored.  Indices are
  * unsigned and K = 2^b exactly, so every index is inside its codebook.
  *
+ * A second storage order, VQ_IDX_TILE4 (also this library's), holds the same
+ * fields tiled by four vectors: a book's stream is ceil(nvec/4) tiles,
+ * idx_row_words 32-bit words apart; tile t covers vectors 4t..4t+3, and inside
+ * it the rows follow one another, row o contributing one 4b-bit record with
+ * the fields of vectors 4t, 4t+1, 4t+2, 4t+3 in that order.  Field (o, j)
+ * thus occupies bits [(4*o + j%4)*b, +b) of tile j/4, numbered as above.
+ * Tiles start 16-byte aligned: idx_row_words is a multiple of 4 and at least
+ * ceil(N*4*b / 128) * 4.  Fields of vectors >= nvec are ignored.  It costs
+ * the same bits per weight; the decode lookup-table kernel (vq_gemv, batch 1)
+ * needs it, because one tile row puts four consecutive vectors of a row next
+ * to those of the following rows.  vq_repack_tile4 converts a row-order
+ * layer.
+ *
  * Conventions for every call
  * --------------------------
  * - Pointers named "device" must be CUDA device (or managed) memory visible
@@ -63,7 +76,7 @@
 extern "C" {
 #endif
 
-#define VQ_ABI_VERSION 1
+#define VQ_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define VQ_API __attribute__((visibility("default")))
@@ -81,6 +94,11 @@ typedef enum vq_status {
     VQ_ERR_TIMEOUT = 6        /* reserved: a bounded device-side wait gave up   */
 } vq_status;
 
+typedef enum vq_idx_layout {
+    VQ_IDX_ROWS = 0,          /* one stream row per output row (default)        */
+    VQ_IDX_TILE4 = 1          /* tiles of four vectors, rows consecutive inside */
+} vq_idx_layout;
+
 typedef enum vq_dtype {
     VQ_BF16 = 0,
     VQ_FP16 = 1,
@@ -94,13 +112,16 @@ typedef enum vq_dtype {
  *   vec_dim        d, 1..16
  *   n_books        1 or 2 (main codebook plus optional residual/additive one)
  *   log2k[m]       b_m, 1..16; K_m = 2^b_m
- *   idx[m]         packed stream of book m, [N][idx_row_words[m]] uint32,
- *                  16-byte aligned
- *   idx_row_words[m]  row stride in 32-bit words, a multiple of 4,
- *                  >= ceil(nvec*b_m / 128) * 4
+ *   idx[m]         packed stream of book m, 16-byte aligned: [N][idx_row_words[m]]
+ *                  uint32 in row order, [ceil(nvec/4)][idx_row_words[m]] tiled
+ *   idx_row_words[m]  stride between stream rows (row order) or tiles (tiled
+ *                  order) in 32-bit words, a multiple of 4, >= ceil(nvec*b_m /
+ *                  128) * 4 in row order, >= ceil(N*4*b_m / 128) * 4 tiled
  *   codebook[m]    fp16 [K_m][d] row-major, 16-byte aligned, finite values
  *   scale          fp16 [N], or NULL for no scale
  *   bias           fp16 [N], or NULL for no bias
+ *   idx_layout     VQ_IDX_ROWS or VQ_IDX_TILE4 (a zero-filled struct means rows)
+ *   reserved       must be 0
  * Entries for m >= n_books are ignored.
  */
 typedef struct vq_layer_desc {
@@ -114,6 +135,8 @@ typedef struct vq_layer_desc {
     const uint16_t* codebook[2];
     const uint16_t* scale;
     const uint16_t* bias;
+    int32_t idx_layout;
+    int32_t reserved;
 } vq_layer_desc;
 
 /*
@@ -125,6 +148,22 @@ typedef struct vq_layer_desc {
  * VQ_ERR_ALIGNMENT (misaligned idx/codebook), VQ_ERR_CUDA.
  */
 VQ_API vq_status vq_dequant(const vq_layer_desc* layer, uint16_t* w_hat, int64_t ldw, void* stream);
+
+/*
+ * vq_repack_tile4 -- write the index streams of a row-order layer in the
+ * tiled order (VQ_IDX_TILE4), on the device.  src->idx_layout must be
+ * VQ_IDX_ROWS.  For each book m < src->n_books, dst[m] (device, 16-byte
+ * aligned, caller-owned, not overlapping src->idx[m]) receives
+ * ceil(nvec/4) * dst_tile_words[m] words, every one of them written: fields,
+ * then zero padding (also for vectors >= nvec).  dst_tile_words[m] follows the
+ * tiled-order rule above.  A layer description that points idx[] at dst[],
+ * with idx_row_words = dst_tile_words and idx_layout = VQ_IDX_TILE4, then
+ * describes the same weights.
+ * Errors: VQ_ERR_INVALID_ARG (bad layer or tile stride, NULL dst with data,
+ * src already tiled), VQ_ERR_ALIGNMENT, VQ_ERR_CUDA.
+ */
+VQ_API vq_status vq_repack_tile4(const vq_layer_desc* src, uint32_t* const dst[2],
+                                 const int64_t dst_tile_words[2], void* stream);
 
 /*
  * vq_gemv_workspace_size -- bytes of device workspace vq_gemv needs for this
@@ -147,6 +186,15 @@ VQ_API vq_status vq_gemv_workspace_size(const vq_layer_desc* layer, int32_t batc
  * Scale and bias are applied as y = s[o] * sum_k x[k] (C1+C2)[o][k]
  * + t[o] * sum_k x[k], equal to the definition up to the fp16 rounding of
  * W_hat (well inside a 2e-3 normwise relative error).
+ * Tiled layers (VQ_IDX_TILE4) with batch 1, one book, vec_dim 8, 16-bit
+ * indices and N <= 65536 run the lookup-table kernel: per group of four
+ * vectors it forms the dot products of x with every centroid (fp32 products
+ * of fp16 operands on the tensor cores, each group of x scaled by a power of
+ * two so that no product can overflow fp16), rounds them to fp16, and sums the
+ * entries the indices select.  That rounding adds about 2^-12 relative error
+ * per term, inside the same tolerance as long as the codebook's values are
+ * normal fp16 numbers (|c| >= 2^-14).  Other tiled layers use a plain tiled
+ * kernel.
  * Errors: VQ_ERR_INVALID_ARG, VQ_ERR_UNSUPPORTED (batch > 16), VQ_ERR_ALIGNMENT
  * (x or y not aligned to its element size), VQ_ERR_WORKSPACE, VQ_ERR_CUDA.
  */
@@ -189,8 +237,11 @@ VQ_API vq_status vq_gemm_workspace_size(const vq_layer_desc* layer, int32_t m, v
 /*
  * vq_gemm -- prefill product y[i][o] = sum_k x[i][k] * W_hat[o][k] for
  * i < m, on the tcgen05 tensor cores (fp16 x fp16 products, fp32 accumulation
- * in tensor memory); W_hat tiles are produced on chip from the index streams
- * and never written to global memory.  The pages call prefill the
+ * in tensor memory).  W_hat tiles are either produced on chip from the index
+ * streams (fused form: W_hat never reaches global memory) or written once into
+ * the workspace by the vq_dequant kernel and streamed in by TMA (staged form);
+ * the call picks the form from the codebook sizes and m, and tiled layers
+ * (VQ_IDX_TILE4) always take the staged form.  The pages call prefill the
  * compute-bound regime where lookups compete with the matrix multiply
  * ("Vector Quantization for LLM Weights in Production", section "1. Prefill
  * vs. Decode Bottlenecks", and the "GEMV / Tensor Core Dot Products" stage of
