@@ -407,12 +407,17 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
 }
 
 // y[o] = s[o] * sum_b part[b][o] + t[o] * sum_b xpart[b], in a fixed order.
-// 32 rows per block: lane = row, the 8 warps stride the per-block sums.
-__global__ void __launch_bounds__(256) gemv_lut_finalize(const float* __restrict__ part,
-                                                         const float* __restrict__ xpart, int nparts,
-                                                         int n, const uint16_t* __restrict__ scale,
-                                                         const uint16_t* __restrict__ bias,
-                                                         void* __restrict__ y, vq_dtype yt) {
+// 32 rows per block: lane = row, the 8 warps stride the per-block sums with
+// every load of a thread in flight at once.  The reduction is bound by load
+// latency, so the block is capped at 32 registers per thread: 8 blocks per SM
+// and one wave for the 70B layers (896 blocks).
+constexpr int kFinU = 20;
+
+__global__ void __launch_bounds__(256, 8) gemv_lut_finalize(const float* __restrict__ part,
+                                                            const float* __restrict__ xpart, int nparts,
+                                                            int n, const uint16_t* __restrict__ scale,
+                                                            const uint16_t* __restrict__ bias,
+                                                            void* __restrict__ y, vq_dtype yt) {
   __shared__ float red[8][33];
   __shared__ float s_xsum;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -425,15 +430,21 @@ __global__ void __launch_bounds__(256) gemv_lut_finalize(const float* __restrict
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
     if (lane == 0) s_xsum = v;
   }
-  float s4[4] = {0.f, 0.f, 0.f, 0.f};
+  float acc = 0.0f;
   if (o < n) {
-    int b = warp;
-    for (; b + 24 < nparts; b += 32)
+    const float* col = part + o;
+    for (int b0 = warp; b0 < nparts; b0 += 8 * kFinU) {
+      float v[kFinU];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) s4[u] += part[static_cast<int64_t>(b + 8 * u) * n + o];
-    for (; b < nparts; b += 8) s4[0] += part[static_cast<int64_t>(b) * n + o];
+      for (int u = 0; u < kFinU; ++u) {
+        const int b = b0 + 8 * u;
+        v[u] = b < nparts ? col[static_cast<int64_t>(b) * n] : 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < kFinU; ++u) acc += v[u];
+    }
   }
-  red[warp][lane] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+  red[warp][lane] = acc;
   __syncthreads();
   if (warp == 0 && o < n) {
     float t = 0.0f;

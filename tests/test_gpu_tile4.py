@@ -139,12 +139,14 @@ def test_lut_gemv(i):
     spec = LUT_SPECS[i]
     data = synth.make_layer(spec, seed=2400 + i)
     layer = _oracle_tiled_layer(data)
-    assert vq.gemv_workspace_size(layer, 1) > 0            # the lookup-table plan
+    nws = vq.gemv_workspace_size(layer, 1)
+    assert nws > 0                                          # the lookup-table plan
+    ws = torch.full((nws,), 0x55, dtype=torch.uint8, device="cuda")   # stale contents are fine
     for fp16 in (False, True):
         x = synth.make_x(2450 + i, 1, spec.in_features, outlier_frac=0.01, as_fp16=fp16)
         ref = oracle.linear(data, x, x_is_fp16=fp16)
         for od in (torch.float32, torch.bfloat16, torch.float16):
-            y = vq.gemv(layer, _x_dev(x, fp16), out_dtype=od)
+            y = vq.gemv(layer, _x_dev(x, fp16), out_dtype=od, workspace=ws)
             assert_close(_f64(y), ref, str(od).split(".")[-1])
 
 
