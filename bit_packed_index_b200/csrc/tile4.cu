@@ -7,13 +7,14 @@
 // section "2. Lookup Table (LUT) Overhead vs. Bit-Shifting": codebook lookups
 // feeding the accumulation; "VPTQ Guide", section "Step 3": y = x . W_hat^T)
 // reorders the sum y[o] = sum_j <x_j, C[i(o, j)]> around the codebook instead
-// of around the rows.  For a group of four vectors j and a quarter ("slice")
-// of the 2^16 centroids k it forms T[k][j] = <x_j, C[k]> once -- a 16 x 8 x 8
-// tensor-core product per 16 centroids -- stores T in shared memory as fp16,
-// and then every row adds the four entries its indices select.  A row's four
-// indices sit side by side in the tiled order, and consecutive rows follow one
-// another, so each thread reads one 8-byte record per row and a warp reads 256
-// contiguous bytes.  Each (group, slice) pair is one task; a block owns every
+// of around the rows.  For a group of four vectors j (one tile) and a slice
+// of the 2^16 centroids k (24576, 24576, then 16384) it forms
+// T[k][j] = <x_j, C[k]> once -- a 16 x 8 x 8 tensor-core product per 16
+// centroids -- stores T in shared memory as fp16, and then every row adds the
+// entries its four indices select.  A row's indices sit side by side in the
+// tiled order and consecutive rows follow one another, so each thread reads
+// one 8-byte record per row and a warp reads 256 contiguous bytes.  Each
+// (group, slice) is one task; a block owns every
 // row of the layer for the tasks it runs, and keeps its per-row sums in tensor
 // memory (TMEM) across tasks.  A second kernel adds the per-block sums and
 // applies scale and bias.
@@ -220,10 +221,10 @@ namespace {
 // Decode lookup-table GEMV (batch 1; one book; d = 8; 16-bit indices).
 // ---------------------------------------------------------------------------
 constexpr int kLutThreads = 1024;
-constexpr int kLutLog2S = 14;                       // a slice holds 2^14 centroids
-constexpr int kLutS = 1 << kLutLog2S;
-constexpr int kLutSlices = 65536 / kLutS;           // 4 slices of the 2^16 book
-constexpr int kLutSmem = kLutS * 4 * 2;             // T[S][4] in fp16: 128 KB
+constexpr int kLutNJ = 4;                           // vectors per task: one tile
+constexpr int kLutS = 24576;                        // centroids per slice (the last: 16384)
+constexpr int kLutSlices = (65536 + kLutS - 1) / kLutS;   // 3 slices of the 2^16 book
+constexpr int kLutSmem = kLutS * kLutNJ * 2;        // T[S][4] in fp16: 192 KB
 constexpr int kLutPD = 8;                           // 16-centroid tiles per load batch
 
 __device__ __forceinline__ uint32_t ldg_stream32(const void* p) {
@@ -246,15 +247,17 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
                                                                   float* __restrict__ xpart) {
   constexpr int CPW = 8 * RB8;                      // TMEM columns per group of 4 warps
   constexpr int TCOLS = 8 * CPW;                    // 64 .. 512, a power of two
-  constexpr int TILES_PER_WARP = kLutS / 16 / (kLutThreads / 32);
-  constexpr int NBATCH = TILES_PER_WARP / kLutPD;
+  constexpr int NBATCH = kLutS / 16 / (kLutThreads / 32) / kLutPD;   // batches, full slice
+  static_assert(kLutS % (16 * (kLutThreads / 32) * kLutPD) == 0 &&
+                (65536 % kLutS) % (16 * (kLutThreads / 32) * kLutPD) == 0,
+                "every slice splits into whole load batches per warp");
   extern __shared__ __align__(128) uint8_t smem[];
-  uint16_t* lut = reinterpret_cast<uint16_t*>(smem);   // T[k - slice base][4 vectors]
+  uint16_t* lut = reinterpret_cast<uint16_t*>(smem);   // T[k - slice base][kLutNJ vectors]
   __shared__ uint32_t s_tmem;
   __shared__ float s_scale;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = L.n, kin = L.kin;
-  const int ntasks = ((L.nvec + 3) / 4) * kLutSlices;
+  const int ntasks = ((L.nvec + kLutNJ - 1) / kLutNJ) * kLutSlices;
 
   if (warp == 0) {
     sm100::tmem_alloc(&s_tmem, TCOLS);
@@ -275,15 +278,16 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
 
   for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
     const int g = task / kLutSlices, s = task - g * kLutSlices;
-    // B operand of m16n8k8: x'[vector 4g + lane/4][components 2t, 2t+1], columns
-    // 4..7 zero.  x' = x * 2^-e with ||x'_j||_1 < 1 for all four vectors, so
-    // |T| <= max |c| and no product overflows fp16; 2^e is applied per row.
+    // B operand of m16n8k8: x'[vector kLutNJ*g + lane/4][components 2t, 2t+1],
+    // other columns zero.  x' = x * 2^-e with ||x'_j||_1 < 1 for the task's
+    // vectors, so |T| <= max |c| and no product overflows fp16; 2^e is
+    // applied per row.
     uint32_t bfrag;
     {
       const int jj = lane >> 2, t = lane & 3;
-      const int64_t k = (static_cast<int64_t>(g) * 4 + jj) * 8 + 2 * t;
+      const int64_t k = (static_cast<int64_t>(g) * kLutNJ + jj) * 8 + 2 * t;
       float a = 0.0f, b = 0.0f;
-      if (jj < 4) {
+      if (jj < kLutNJ) {
         if (k < kin) a = x_at(x, x_fp16, k);
         if (k + 1 < kin) b = x_at(x, x_fp16, k + 1);
       }
@@ -305,12 +309,16 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
         xs_acc += v;
       }
     }
-    // Phase A: T for this slice.  Warp w builds tiles [32w, 32w+32) of 16
-    // centroids; each tile's A operand is read straight from the codebook
-    // (lane: centroid lane/4 (+8), components 2t, 2t+1), two batches in flight.
+    // Phase A: T for this slice.  Warp w builds its share of the slice's
+    // 16-centroid tiles; each tile's A operand is read straight from the
+    // codebook (lane: centroid lane/4 (+8), components 2t, 2t+1), two load
+    // batches in flight.
     {
       const uint16_t* bslice = L.book[0] + static_cast<size_t>(s) * kLutS * 8;
-      const int t0w = warp * TILES_PER_WARP;
+      const int slice_n = min(kLutS, 65536 - s * kLutS);
+      const int tpw = slice_n / 16 / (kLutThreads / 32);        // tiles per warp
+      const int nb = tpw / kLutPD;                                // load batches
+      const int t0w = warp * tpw;
       uint32_t afr[2][kLutPD][2];
 #pragma unroll
       for (int p = 0; p < kLutPD; ++p) {
@@ -320,8 +328,9 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
       }
 #pragma unroll
       for (int bt = 0; bt < NBATCH; ++bt) {
+        if (bt >= nb) break;                        // uniform: the slice's own size
         const int cur = bt & 1;
-        if (bt + 1 < NBATCH) {
+        if (bt + 1 < nb) {
 #pragma unroll
           for (int p = 0; p < kLutPD; ++p) {
             const uint16_t* c0 = bslice + ((t0w + (bt + 1) * kLutPD + p) * 16 + (lane >> 2)) * 8 + 2 * (lane & 3);
@@ -338,10 +347,10 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
               : "=f"(d0), "=f"(d1), "=f"(d2), "=f"(d3)
               : "r"(afr[cur][p][0]), "r"(afr[cur][p][1]), "r"(bfrag), "f"(0.0f), "f"(0.0f), "f"(0.0f),
                 "f"(0.0f));
-          if ((lane & 3) < 2) {                     // columns 0..3 are the four vectors
+          if ((lane & 3) < kLutNJ / 2) {            // columns 0..kLutNJ-1 are the vectors
             const int kl = (t0w + bt * kLutPD + p) * 16 + (lane >> 2);
-            *reinterpret_cast<__half2*>(lut + kl * 4 + 2 * (lane & 3)) = __floats2half2_rn(d0, d1);
-            *reinterpret_cast<__half2*>(lut + (kl + 8) * 4 + 2 * (lane & 3)) = __floats2half2_rn(d2, d3);
+            *reinterpret_cast<__half2*>(lut + kl * kLutNJ + 2 * (lane & 3)) = __floats2half2_rn(d0, d1);
+            *reinterpret_cast<__half2*>(lut + (kl + 8) * kLutNJ + 2 * (lane & 3)) = __floats2half2_rn(d2, d3);
           }
         }
       }
@@ -373,12 +382,13 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
         sm100::tmem_ld8(tbase + 8 * b, acc);
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
-          float v[4];
+          float v[kLutNJ];
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
+          for (int jj = 0; jj < kLutNJ; ++jj) {
             const uint32_t k = ((jj < 2 ? w[cur][r].x : w[cur][r].y) >> (16 * (jj & 1))) & 0xFFFFu;
             v[jj] = 0.0f;
-            if ((k >> kLutLog2S) == static_cast<uint32_t>(s)) v[jj] = h2f(lut[(k & (kLutS - 1)) * 4 + jj]);
+            const uint32_t t = k - static_cast<uint32_t>(s * kLutS);   // wraps when below
+            if (t < static_cast<uint32_t>(kLutS)) v[jj] = h2f(lut[t * kLutNJ + jj]);
           }
           acc[r] = fmaf((v[0] + v[1]) + (v[2] + v[3]), sc, acc[r]);
         }
