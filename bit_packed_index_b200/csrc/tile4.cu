@@ -416,6 +416,180 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
   if (warp == 0) sm100::tmem_dealloc(s_tmem, TCOLS);
 }
 
+// ---------------------------------------------------------------------------
+// Lookup-table GEMV for small books (batch 1; d = 6 or 8; one or two books of
+// at most 2^12 centroids each).  The whole table of a group of four vectors
+// fits in shared memory -- T_m[k][4] for each book, at most 64 KB -- so a task
+// is one group, each index is looked up exactly once and there is no slice
+// test.  Records of 4 fields are 4*b_m bits wide and read with a bit-exact
+// funnel (consecutive rows share words, so the loads go through L1).  The
+// rest is the 2^16 kernel's structure: tensor-core table products, row sums in
+// TMEM, per-block sums added by gemv_lut_finalize.
+// ---------------------------------------------------------------------------
+constexpr int kLutSmallMaxTiles = 8;                 // 16-centroid tiles per warp: K <= 4096
+
+// The 4*b-bit record of row o in a tiled stream (b <= 12: at most 48 bits,
+// spread over up to three words; only words holding record bits are read).
+__device__ __forceinline__ uint64_t load_record(const uint32_t* __restrict__ tile, int64_t o, int b) {
+  const int64_t p = o * 4 * b;
+  const uint32_t* w = tile + (p >> 5);
+  const int sh = static_cast<int>(p & 31);
+  const int nbits = 4 * b;
+  const uint64_t lo = __ldg(w);
+  const uint64_t mid = (sh + nbits > 32) ? __ldg(w + 1) : 0u;
+  uint64_t r = ((mid << 32) | lo) >> sh;
+  if (sh + nbits > 64) r |= static_cast<uint64_t>(__ldg(w + 2)) << (64 - sh);
+  return r;
+}
+
+// Table of one book for the task's four vectors: T[k][4] = <x'_j, C[k]>.
+template <int D>
+__device__ __forceinline__ void build_small_table(const uint16_t* __restrict__ book, int K, uint32_t bfrag,
+                                                  uint16_t* __restrict__ tab, int warp, int lane) {
+  const int tiles = (K + 15) / 16;
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t a[kLutSmallMaxTiles][2];
+#pragma unroll
+  for (int i = 0; i < kLutSmallMaxTiles; ++i) {
+    const int tile = warp + 32 * i;
+    const int r0 = tile * 16 + g, r1 = r0 + 8;
+    const bool cok = 2 * t < D;                       // d = 6: components 6, 7 are zero
+    a[i][0] = (tile < tiles && r0 < K && cok) ? __ldg(reinterpret_cast<const uint32_t*>(book + r0 * D + 2 * t)) : 0u;
+    a[i][1] = (tile < tiles && r1 < K && cok) ? __ldg(reinterpret_cast<const uint32_t*>(book + r1 * D + 2 * t)) : 0u;
+  }
+#pragma unroll
+  for (int i = 0; i < kLutSmallMaxTiles; ++i) {
+    const int tile = warp + 32 * i;
+    if (tile >= tiles) break;                          // uniform per warp
+    float d0, d1, d2, d3;
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
+        "{%7, %8, %9, %10};"
+        : "=f"(d0), "=f"(d1), "=f"(d2), "=f"(d3)
+        : "r"(a[i][0]), "r"(a[i][1]), "r"(bfrag), "f"(0.0f), "f"(0.0f), "f"(0.0f), "f"(0.0f));
+    const int r0 = tile * 16 + g;
+    if (t < 2) {
+      if (r0 < K) *reinterpret_cast<__half2*>(tab + r0 * 4 + 2 * t) = __floats2half2_rn(d0, d1);
+      if (r0 + 8 < K) *reinterpret_cast<__half2*>(tab + (r0 + 8) * 4 + 2 * t) = __floats2half2_rn(d2, d3);
+    }
+  }
+}
+
+template <int RB8, int D, int NB>
+__global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_small_kernel(Layer L, const uint16_t* __restrict__ x,
+                                                                        int x_fp16, float* __restrict__ part,
+                                                                        float* __restrict__ xpart) {
+  constexpr int CPW = 8 * RB8;
+  constexpr int TCOLS = 8 * CPW;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int K1 = 1 << L.b[0], K2 = NB == 2 ? (1 << L.b[1]) : 0;
+  uint16_t* tab1 = reinterpret_cast<uint16_t*>(smem);   // T1[K1][4]
+  uint16_t* tab2 = tab1 + K1 * 4;                        // T2[K2][4]
+  __shared__ uint32_t s_tmem;
+  __shared__ float s_scale;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n = L.n, kin = L.kin;
+  const int ntasks = (L.nvec + 3) / 4;
+
+  if (warp == 0) {
+    sm100::tmem_alloc(&s_tmem, TCOLS);
+    sm100::tmem_relinquish();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tbase = s_tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) +
+                         static_cast<uint32_t>((warp >> 2) * CPW);
+  {
+    float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int b = 0; b < RB8; ++b) sm100::tmem_st8(tbase + 8 * b, z);
+    sm100::tmem_wait_st();
+  }
+  float xs_acc = 0.0f;
+
+  for (int g = blockIdx.x; g < ntasks; g += gridDim.x) {
+    uint32_t bfrag;
+    {
+      const int jj = lane >> 2, t = lane & 3;
+      const int64_t k = (static_cast<int64_t>(g) * 4 + jj) * D + 2 * t;
+      float a = 0.0f, b = 0.0f;
+      if (jj < 4 && 2 * t < D) {
+        if (k < kin) a = x_at(x, x_fp16, k);
+        if (k + 1 < kin) b = x_at(x, x_fp16, k + 1);
+      }
+      float l1 = fabsf(a) + fabsf(b);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      float mx = l1;
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      int e = 0;
+      if (mx > 0.0f && mx < INFINITY) frexpf(mx, &e);
+      const __half2 h = __floats2half2_rn(ldexpf(a, -e), ldexpf(b, -e));
+      bfrag = *reinterpret_cast<const uint32_t*>(&h);
+      if (tid == 0) s_scale = ldexpf(1.0f, e);
+      if (warp == 0) {
+        float v = a + b;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        xs_acc += v;
+      }
+    }
+    build_small_table<D>(L.book[0], K1, bfrag, tab1, warp, lane);
+    if constexpr (NB == 2) build_small_table<D>(L.book[1], K2, bfrag, tab2, warp, lane);
+    __syncthreads();   // tables complete
+    {
+      const float sc = s_scale;
+      const uint32_t* tile1 = L.idx[0] + static_cast<int64_t>(g) * L.rw[0];
+      const uint32_t* tile2 = L.idx[1] + static_cast<int64_t>(g) * L.rw[1];
+      const int b1 = L.b[0], b2 = L.b[1];
+      const uint32_t m1 = (1u << b1) - 1u, m2 = (1u << b2) - 1u;
+#pragma unroll
+      for (int b = 0; b < RB8; ++b) {
+        float acc[8];
+        sm100::tmem_ld8(tbase + 8 * b, acc);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const int o = (b * 8 + r) * kLutThreads + tid;
+          if (o < n) {
+            const uint64_t rec1 = load_record(tile1, o, b1);
+            uint64_t rec2 = 0;
+            if constexpr (NB == 2) rec2 = load_record(tile2, o, b2);
+            float v = 0.0f;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              float u = h2f(tab1[(static_cast<uint32_t>(rec1 >> (jj * b1)) & m1) * 4 + jj]);
+              if constexpr (NB == 2) u += h2f(tab2[(static_cast<uint32_t>(rec2 >> (jj * b2)) & m2) * 4 + jj]);
+              v += u;
+            }
+            acc[r] = fmaf(v, sc, acc[r]);
+          }
+        }
+        sm100::tmem_st8(tbase + 8 * b, acc);
+      }
+      sm100::tmem_wait_st();
+    }
+    __syncthreads();   // all lookups done before the next task rewrites the tables
+  }
+
+#pragma unroll
+  for (int b = 0; b < RB8; ++b) {
+    float acc[8];
+    sm100::tmem_ld8(tbase + 8 * b, acc);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int o = (b * 8 + r) * kLutThreads + tid;
+      if (o < n) part[static_cast<int64_t>(blockIdx.x) * n + o] = acc[r];
+    }
+  }
+  if (tid == 0) xpart[blockIdx.x] = xs_acc;
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  if (warp == 0) sm100::tmem_dealloc(s_tmem, TCOLS);
+}
+
 // y[o] = s[o] * sum_b part[b][o] + t[o] * sum_b xpart[b], in a fixed order.
 // 32 rows per block: lane = row, the 8 warps stride the per-block sums with
 // every load of a thread in flight at once.  The reduction is bound by load
@@ -482,6 +656,44 @@ cudaError_t launch_lut(const Layer& L, const GemvPlan& p, const void* x, bool x_
   return cudaGetLastError();
 }
 
+template <int RB8, int D, int NB>
+cudaError_t launch_lut_small_t(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, float* ws,
+                               cudaStream_t stream) {
+  auto k = gemv_lut_small_kernel<RB8, D, NB>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
+  if (e != cudaSuccess) return e;
+  count_launch();
+  k<<<p.grid_x, kLutThreads, p.smem, stream>>>(L, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, ws,
+                                               ws + static_cast<int64_t>(p.grid_x) * L.n);
+  return cudaGetLastError();
+}
+
+template <int RB8>
+cudaError_t launch_lut_small(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, void* y,
+                             vq_dtype yt, float* ws, cudaStream_t stream) {
+  cudaError_t e;
+  if (L.d == 8) e = L.nb == 1 ? launch_lut_small_t<RB8, 8, 1>(L, p, x, x_fp16, ws, stream)
+                              : launch_lut_small_t<RB8, 8, 2>(L, p, x, x_fp16, ws, stream);
+  else e = L.nb == 1 ? launch_lut_small_t<RB8, 6, 1>(L, p, x, x_fp16, ws, stream)
+                     : launch_lut_small_t<RB8, 6, 2>(L, p, x, x_fp16, ws, stream);
+  if (e != cudaSuccess) return e;
+  count_launch();
+  gemv_lut_finalize<<<(L.n + 31) / 32, 256, 0, stream>>>(ws, ws + static_cast<int64_t>(p.grid_x) * L.n,
+                                                        p.grid_x, L.n, L.scale, L.bias, y, yt);
+  return cudaGetLastError();
+}
+
+size_t lut_small_smem(const Layer& L) {
+  const size_t k = (static_cast<size_t>(1) << L.b[0]) + (L.nb == 2 ? (static_cast<size_t>(1) << L.b[1]) : 0);
+  return k * 4 * 2;
+}
+
+bool lut_small_supported(const Layer& L) {
+  return L.layout == VQ_IDX_TILE4 && (L.d == 6 || L.d == 8) && L.b[0] <= 12 &&
+         (L.nb == 1 || L.b[1] <= 12) && L.n >= 1 && L.n <= 8 * 8 * kLutThreads && L.nvec >= 1 &&
+         lut_small_smem(L) + 1024 <= static_cast<size_t>(device_smem_optin());
+}
+
 bool lut_supported(const Layer& L) {
   return L.layout == VQ_IDX_TILE4 && L.nb == 1 && L.d == 8 && L.b[0] == 16 && L.n >= 1 &&
          L.n <= 8 * 8 * kLutThreads && L.nvec >= 1 && device_smem_optin() >= kLutSmem + 1024;
@@ -492,18 +704,19 @@ bool lut_supported(const Layer& L) {
 void plan_gemv_tile4(const Layer& L, int batch, size_t ws_cap, GemvPlan* p) {
   *p = GemvPlan{};
   p->nsplit = 1;
-  if (batch == 1 && lut_supported(L)) {
-    const int ntasks = ((L.nvec + 3) / 4) * kLutSlices;
+  const bool big = lut_supported(L), small = !big && lut_small_supported(L);
+  if (batch == 1 && (big || small)) {
+    const int ntasks = ((L.nvec + 3) / 4) * (big ? kLutSlices : 1);
     const size_t per_block = (static_cast<size_t>(L.n) + 1) * sizeof(float);
     int grid = std::min(device_sm_count(), ntasks);
     if (ws_cap / per_block < static_cast<size_t>(grid)) grid = static_cast<int>(ws_cap / per_block);
     if (grid >= 1) {
       int rb8 = 1;
       while (static_cast<int64_t>(rb8) * 8 * kLutThreads < L.n) rb8 <<= 1;
-      p->fast = 3;
+      p->fast = big ? 3 : 5;
       p->grid_x = grid;
       p->bt = rb8;
-      p->smem = kLutSmem;
+      p->smem = big ? kLutSmem : static_cast<int>(lut_small_smem(L));
       p->ws_bytes = per_block * grid;
       return;
     }
@@ -523,6 +736,14 @@ cudaError_t launch_gemv_tile4(const Layer& L, const GemvPlan& p, const void* x, 
       case 2: return launch_lut<2>(L, p, x, x_fp16, y, yt, ws, stream);
       case 4: return launch_lut<4>(L, p, x, x_fp16, y, yt, ws, stream);
       default: return launch_lut<8>(L, p, x, x_fp16, y, yt, ws, stream);
+    }
+  }
+  if (p.fast == 5) {
+    switch (p.bt) {
+      case 1: return launch_lut_small<1>(L, p, x, x_fp16, y, yt, ws, stream);
+      case 2: return launch_lut_small<2>(L, p, x, x_fp16, y, yt, ws, stream);
+      case 4: return launch_lut_small<4>(L, p, x, x_fp16, y, yt, ws, stream);
+      default: return launch_lut_small<8>(L, p, x, x_fp16, y, yt, ws, stream);
     }
   }
   count_launch();

@@ -72,7 +72,8 @@ struct GemvPlan {
   int book_bytes;     // shared memory taken by the staged books
   size_t ws_bytes;
   int fast = 0;       // 1: single-row kernel (gemv1.cu), 2: batched kernel (gemvb.cu),
-                      // 3: lookup-table kernel, 4: plain tiled kernel (tile4.cu)
+                      // 3: lookup-table kernel (2^16 book), 4: plain tiled kernel,
+                      // 5: lookup-table kernel for books of <= 2^12 entries (tile4.cu)
 };
 // ws_cap: largest workspace the caller can provide (plans that need more
 // either shrink, for the tiled kernels, or are reported by their ws_bytes).

@@ -83,15 +83,18 @@ def test_layout_field_validation_needs_no_device(lib):
 
 def test_tiled_workspace_sizes(lib):
     """Batch 1 on a lookup-table-eligible tiled layer needs per-block row sums;
-    other batches use the plain tiled kernel, which needs none."""
+    other batches and other layers use the plain tiled kernel, which needs none."""
     n = C.c_size_t(0)
     d = _tiled_desc(n=1000, kin=64)
     assert lib.vq_gemv_workspace_size(C.byref(d), 1, C.byref(n)) == vq.VQ_OK
     assert n.value > 0 and n.value % (1001 * 4) == 0
     assert lib.vq_gemv_workspace_size(C.byref(d), 3, C.byref(n)) == vq.VQ_OK
     assert n.value == 0
-    d.log2k[0] = 12                                                        # not a 16-bit book
+    d.log2k[0] = 12                                    # a 2^12 book: the small-book table plan
     d.idx_row_words[0] = vq.tile4_words(1000, 12)
+    assert lib.vq_gemv_workspace_size(C.byref(d), 1, C.byref(n)) == vq.VQ_OK
+    assert n.value > 0 and n.value % (1001 * 4) == 0
+    d.vec_dim, d.in_features = 16, 128                 # no table kernel for d = 16: plain kernel
     assert lib.vq_gemv_workspace_size(C.byref(d), 1, C.byref(n)) == vq.VQ_OK
     assert n.value == 0
 

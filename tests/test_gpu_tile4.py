@@ -5,10 +5,11 @@
 - layers whose tiled streams come from the oracle's packer (not from the
   library) give vq_dequant bit-exact and vq_gemv / vq_gemm within the bar, so
   the kernels read the documented order and not just whatever repack writes;
-- the lookup-table GEMV (batch 1, one 2^16-entry book, d = 8) is checked on
-  ragged shapes, every block-row size it compiles for, both activation types,
-  every output type, scale/bias present and absent, large and small
-  activation magnitudes, and the 70B decode shapes on sampled rows; the plain
+- the lookup-table GEMVs (batch 1: one 2^16-entry book at d = 8, sliced; or
+  books of up to 2^12 entries at d = 6 or 8, whole) are checked on ragged
+  shapes, every block-row size they compile for, both activation types, every
+  output type, scale/bias present and absent, large and small activation
+  magnitudes, and the 70B / 405B / 8B decode shapes on sampled rows; the plain
   tiled kernel on every other case."""
 import numpy as np
 import pytest
@@ -253,3 +254,46 @@ def test_70b_decode_layers_tiled(li):
     for b in (1, 4):
         y = vq.gemv(layer, _x_dev(x)[:b], out_dtype=torch.bfloat16)
         assert_close(_f64(y[:, rd]), ref[:b], "bfloat16")
+
+
+# Small-book lookup tables: d = 6 and 8, one and two books, books smaller than
+# one 16-centroid tile, odd field widths, ragged N / nvec / Kin.
+SMALL_LUT_SPECS = [
+    LayerSpec(777, 6 * 130 + 4, 6, (12, 4), (0.02, 0.005)),
+    LayerSpec(1000, 8 * 125, 8, (12, 8), (0.02, 0.005)),
+    LayerSpec(513, 8 * 61 + 3, 8, (12,), (0.02,), None, None),
+    LayerSpec(300, 6 * 77, 6, (9,), (0.02,), (0.5, 1.5), None),
+    LayerSpec(9000, 6 * 20 + 5, 6, (3, 5), (0.02, 0.005)),
+    LayerSpec(17000, 8 * 9, 8, (7, 11), (0.02, 0.005)),
+    LayerSpec(65536, 6 * 5, 6, (12, 4), (0.02, 0.005)),
+]
+
+
+@pytest.mark.parametrize("i", range(len(SMALL_LUT_SPECS)))
+def test_small_book_lut_gemv(i):
+    vq = _vq()
+    spec = SMALL_LUT_SPECS[i]
+    data = synth.make_layer(spec, seed=2900 + i)
+    layer = _oracle_tiled_layer(data)
+    assert vq.gemv_workspace_size(layer, 1) > 0            # a lookup-table plan
+    for fp16 in (False, True):
+        x = synth.make_x(2950 + i, 1, spec.in_features, outlier_frac=0.01, as_fp16=fp16)
+        ref = oracle.linear(data, x, x_is_fp16=fp16)
+        for od in (torch.float32, torch.bfloat16):
+            y = vq.gemv(layer, _x_dev(x, fp16), out_dtype=od)
+            assert_close(_f64(y), ref, str(od).split(".")[-1])
+
+
+@pytest.mark.parametrize("name,li", [("llama31_405b", 4), ("llama31_405b", 6), ("llama31_405b", 1),
+                                     ("llama3_8b_up", 0)])
+def test_small_book_decode_layers_tiled(name, li):
+    vq = _vq()
+    w = WORKLOADS[name]
+    spec, seed = w.layers[li]
+    data = synth.make_layer(spec, seed)
+    layer = vq.repack_tile4(vq.Layer.from_synth(data))
+    rows = sample_rows(spec.out_features, 192, seed + 3)
+    x = synth.make_x(w.x_seed + li, 1, spec.in_features, w.outlier_frac)
+    ref = oracle.linear(data, x, rows)
+    y = vq.gemv(layer, _x_dev(x), out_dtype=torch.bfloat16)
+    assert_close(_f64(y[:, torch.from_numpy(rows).cuda()]), ref, "bfloat16")
