@@ -545,26 +545,31 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_small_kernel(Layer L,
       const uint32_t* tile2 = L.idx[1] + static_cast<int64_t>(g) * L.rw[1];
       const int b1 = L.b[0], b2 = L.b[1];
       const uint32_t m1 = (1u << b1) - 1u, m2 = (1u << b2) - 1u;
-#pragma unroll
+#pragma unroll 1
       for (int b = 0; b < RB8; ++b) {
+        if (b * 8 * kLutThreads >= n) break;          // uniform: no row of this batch exists
+        // Every record of the batch is requested before any is used (rows past
+        // N read row N-1 and are never stored), so the loads overlap.
+        uint64_t rec1[8], rec2[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const int o = min((b * 8 + r) * kLutThreads + tid, n - 1);
+          rec1[r] = load_record(tile1, o, b1);
+          if constexpr (NB == 2) rec2[r] = load_record(tile2, o, b2);
+        }
         float acc[8];
         sm100::tmem_ld8(tbase + 8 * b, acc);
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
-          const int o = (b * 8 + r) * kLutThreads + tid;
-          if (o < n) {
-            const uint64_t rec1 = load_record(tile1, o, b1);
-            uint64_t rec2 = 0;
-            if constexpr (NB == 2) rec2 = load_record(tile2, o, b2);
-            float v = 0.0f;
+          if ((b * 8 + r) * kLutThreads >= n) break;  // uniform: no thread has this row
+          float v = 0.0f;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-              float u = h2f(tab1[(static_cast<uint32_t>(rec1 >> (jj * b1)) & m1) * 4 + jj]);
-              if constexpr (NB == 2) u += h2f(tab2[(static_cast<uint32_t>(rec2 >> (jj * b2)) & m2) * 4 + jj]);
-              v += u;
-            }
-            acc[r] = fmaf(v, sc, acc[r]);
+          for (int jj = 0; jj < 4; ++jj) {
+            float u = h2f(tab1[(static_cast<uint32_t>(rec1[r] >> (jj * b1)) & m1) * 4 + jj]);
+            if constexpr (NB == 2) u += h2f(tab2[(static_cast<uint32_t>(rec2[r] >> (jj * b2)) & m2) * 4 + jj]);
+            v += u;
           }
+          acc[r] = fmaf(v, sc, acc[r]);
         }
         sm100::tmem_st8(tbase + 8 * b, acc);
       }
@@ -580,6 +585,162 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_small_kernel(Layer L,
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int o = (b * 8 + r) * kLutThreads + tid;
+      if (o < n) part[static_cast<int64_t>(blockIdx.x) * n + o] = acc[r];
+    }
+  }
+  if (tid == 0) xpart[blockIdx.x] = xs_acc;
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  if (warp == 0) sm100::tmem_dealloc(s_tmem, TCOLS);
+}
+
+// Rows in pairs, for 12-bit main books (with no second book, or a 4- or
+// 8-bit one): two 48-bit records are exactly three words, so every field of
+// the pair sits at a fixed bit position and its table byte offset (index * 8)
+// takes one shift and one mask.  Same tables, same sums, same order of the
+// four lookups of a row as gemv_lut_small_kernel; a thread's batch is four
+// pairs (8 rows, 8 TMEM columns).
+template <int B, int Q, int NW>
+__device__ __forceinline__ uint32_t field_off(const uint32_t (&w)[NW]) {
+  constexpr int bit = Q * B, wi = bit >> 5, sh = bit & 31;
+  uint32_t v;
+  if constexpr (sh + B <= 32) {
+    v = w[wi] >> sh;
+  } else {
+    v = __funnelshift_r(w[wi], w[wi + 1], sh);
+  }
+  return (v & ((1u << B) - 1u)) << 3;
+}
+
+template <int B, int H, int NW>
+__device__ __forceinline__ float row_lookup(const uint32_t (&w)[NW], const uint8_t* tab) {
+  // fields 4H .. 4H+3 of the pair: the four vectors of row 2p + H
+  const float a = h2f(*reinterpret_cast<const uint16_t*>(tab + field_off<B, 4 * H + 0>(w) + 0));
+  const float b = h2f(*reinterpret_cast<const uint16_t*>(tab + field_off<B, 4 * H + 1>(w) + 2));
+  const float c = h2f(*reinterpret_cast<const uint16_t*>(tab + field_off<B, 4 * H + 2>(w) + 4));
+  const float d = h2f(*reinterpret_cast<const uint16_t*>(tab + field_off<B, 4 * H + 3>(w) + 6));
+  return (a + b) + (c + d);
+}
+
+template <int RB8, int D, int B2>
+__global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_pair_kernel(Layer L, const uint16_t* __restrict__ x,
+                                                                       int x_fp16, float* __restrict__ part,
+                                                                       float* __restrict__ xpart) {
+  constexpr int B1 = 12;
+  constexpr int NB = B2 > 0 ? 2 : 1;
+  constexpr int W2 = B2 == 8 ? 2 : 1;               // words per pair of book-2 records
+  constexpr int CPW = 8 * RB8;
+  constexpr int TCOLS = 8 * CPW;
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int K1 = 1 << B1, K2 = B2 > 0 ? (1 << B2) : 0;
+  uint16_t* tab1 = reinterpret_cast<uint16_t*>(smem);   // T1[K1][4]
+  uint16_t* tab2 = tab1 + K1 * 4;                        // T2[K2][4]
+  __shared__ uint32_t s_tmem;
+  __shared__ float s_scale;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n = L.n, kin = L.kin;
+  const int ntasks = (L.nvec + 3) / 4;
+  const int npairs = (n + 1) / 2;
+  const int64_t nw1 = (static_cast<int64_t>(n) * 4 * B1 + 31) / 32;   // words holding records
+  const int64_t nw2 = (static_cast<int64_t>(n) * 4 * (B2 > 0 ? B2 : 1) + 31) / 32;
+
+  if (warp == 0) {
+    sm100::tmem_alloc(&s_tmem, TCOLS);
+    sm100::tmem_relinquish();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tbase = s_tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) +
+                         static_cast<uint32_t>((warp >> 2) * CPW);
+  {
+    float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int b = 0; b < RB8; ++b) sm100::tmem_st8(tbase + 8 * b, z);
+    sm100::tmem_wait_st();
+  }
+  float xs_acc = 0.0f;
+
+  for (int g = blockIdx.x; g < ntasks; g += gridDim.x) {
+    uint32_t bfrag;
+    {
+      const int jj = lane >> 2, t = lane & 3;
+      const int64_t k = (static_cast<int64_t>(g) * 4 + jj) * D + 2 * t;
+      float a = 0.0f, b = 0.0f;
+      if (jj < 4 && 2 * t < D) {
+        if (k < kin) a = x_at(x, x_fp16, k);
+        if (k + 1 < kin) b = x_at(x, x_fp16, k + 1);
+      }
+      float l1 = fabsf(a) + fabsf(b);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      float mx = l1;
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      int e = 0;
+      if (mx > 0.0f && mx < INFINITY) frexpf(mx, &e);
+      const __half2 h = __floats2half2_rn(ldexpf(a, -e), ldexpf(b, -e));
+      bfrag = *reinterpret_cast<const uint32_t*>(&h);
+      if (tid == 0) s_scale = ldexpf(1.0f, e);
+      if (warp == 0) {
+        float v = a + b;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        xs_acc += v;
+      }
+    }
+    build_small_table<D>(L.book[0], K1, bfrag, tab1, warp, lane);
+    if constexpr (NB == 2) build_small_table<D>(L.book[1], K2, bfrag, tab2, warp, lane);
+    __syncthreads();   // tables complete
+    {
+      const float sc = s_scale;
+      const uint32_t* tile1 = L.idx[0] + static_cast<int64_t>(g) * L.rw[0];
+      const uint32_t* tile2 = L.idx[1] + static_cast<int64_t>(g) * L.rw[1];
+      const uint8_t* t1 = reinterpret_cast<const uint8_t*>(tab1);
+      const uint8_t* t2 = reinterpret_cast<const uint8_t*>(tab2);
+#pragma unroll 1
+      for (int b = 0; b < RB8; ++b) {
+        if (b * 8 * kLutThreads >= n) break;          // uniform: no row of this batch exists
+        uint32_t w1[4][3], w2[4][W2];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {                 // all loads of the batch first
+          const int64_t pi = static_cast<int64_t>(b * 4 + r) * kLutThreads + tid;
+#pragma unroll
+          for (int i = 0; i < 3; ++i) w1[r][i] = 3 * pi + i < nw1 ? __ldg(tile1 + 3 * pi + i) : 0u;
+          if constexpr (NB == 2) {
+#pragma unroll
+            for (int i = 0; i < W2; ++i) w2[r][i] = W2 * pi + i < nw2 ? __ldg(tile2 + W2 * pi + i) : 0u;
+          }
+        }
+        float acc[8];
+        sm100::tmem_ld8(tbase + 8 * b, acc);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          if ((b * 4 + r) * kLutThreads >= npairs) break;   // uniform: no thread has this pair
+          float va = row_lookup<B1, 0>(w1[r], t1);
+          float vb = row_lookup<B1, 1>(w1[r], t1);
+          if constexpr (NB == 2) {
+            va += row_lookup<B2, 0>(w2[r], t2);
+            vb += row_lookup<B2, 1>(w2[r], t2);
+          }
+          acc[2 * r] = fmaf(va, sc, acc[2 * r]);
+          acc[2 * r + 1] = fmaf(vb, sc, acc[2 * r + 1]);
+        }
+        sm100::tmem_st8(tbase + 8 * b, acc);
+      }
+      sm100::tmem_wait_st();
+    }
+    __syncthreads();   // all lookups done before the next task rewrites the tables
+  }
+
+#pragma unroll 1
+  for (int b = 0; b < RB8; ++b) {
+    float acc[8];
+    sm100::tmem_ld8(tbase + 8 * b, acc);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int64_t o = 2 * (static_cast<int64_t>(b * 4 + (r >> 1)) * kLutThreads + tid) + (r & 1);
       if (o < n) part[static_cast<int64_t>(blockIdx.x) * n + o] = acc[r];
     }
   }
@@ -668,14 +829,39 @@ cudaError_t launch_lut_small_t(const Layer& L, const GemvPlan& p, const void* x,
   return cudaGetLastError();
 }
 
+template <int RB8, int D, int B2>
+cudaError_t launch_lut_pair_t(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, float* ws,
+                              cudaStream_t stream) {
+  auto k = gemv_lut_pair_kernel<RB8, D, B2>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
+  if (e != cudaSuccess) return e;
+  count_launch();
+  k<<<p.grid_x, kLutThreads, p.smem, stream>>>(L, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, ws,
+                                               ws + static_cast<int64_t>(p.grid_x) * L.n);
+  return cudaGetLastError();
+}
+
 template <int RB8>
 cudaError_t launch_lut_small(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, void* y,
                              vq_dtype yt, float* ws, cudaStream_t stream) {
   cudaError_t e;
-  if (L.d == 8) e = L.nb == 1 ? launch_lut_small_t<RB8, 8, 1>(L, p, x, x_fp16, ws, stream)
-                              : launch_lut_small_t<RB8, 8, 2>(L, p, x, x_fp16, ws, stream);
-  else e = L.nb == 1 ? launch_lut_small_t<RB8, 6, 1>(L, p, x, x_fp16, ws, stream)
-                     : launch_lut_small_t<RB8, 6, 2>(L, p, x, x_fp16, ws, stream);
+  const int b2 = L.nb == 2 ? L.b[1] : 0;
+  if (L.b[0] == 12 && (b2 == 0 || b2 == 4 || b2 == 8)) {      // rows in pairs, fixed offsets
+    if (L.d == 8)
+      e = b2 == 0 ? launch_lut_pair_t<RB8, 8, 0>(L, p, x, x_fp16, ws, stream)
+        : b2 == 4 ? launch_lut_pair_t<RB8, 8, 4>(L, p, x, x_fp16, ws, stream)
+                  : launch_lut_pair_t<RB8, 8, 8>(L, p, x, x_fp16, ws, stream);
+    else
+      e = b2 == 0 ? launch_lut_pair_t<RB8, 6, 0>(L, p, x, x_fp16, ws, stream)
+        : b2 == 4 ? launch_lut_pair_t<RB8, 6, 4>(L, p, x, x_fp16, ws, stream)
+                  : launch_lut_pair_t<RB8, 6, 8>(L, p, x, x_fp16, ws, stream);
+  } else if (L.d == 8) {
+    e = L.nb == 1 ? launch_lut_small_t<RB8, 8, 1>(L, p, x, x_fp16, ws, stream)
+                  : launch_lut_small_t<RB8, 8, 2>(L, p, x, x_fp16, ws, stream);
+  } else {
+    e = L.nb == 1 ? launch_lut_small_t<RB8, 6, 1>(L, p, x, x_fp16, ws, stream)
+                  : launch_lut_small_t<RB8, 6, 2>(L, p, x, x_fp16, ws, stream);
+  }
   if (e != cudaSuccess) return e;
   count_launch();
   gemv_lut_finalize<<<(L.n + 31) / 32, 256, 0, stream>>>(ws, ws + static_cast<int64_t>(p.grid_x) * L.n,
