@@ -475,6 +475,47 @@ __device__ __forceinline__ void build_small_table(const uint16_t* __restrict__ b
   }
 }
 
+// The same table as fp32, one array per vector (T[j][k], K entries apart), for
+// the paired-row kernel: a lookup is one 4-byte load, and lanes that read the
+// same vector's array spread over all 32 banks.
+template <int D>
+__device__ __forceinline__ void build_small_table_f32(const uint16_t* __restrict__ book, int K, uint32_t bfrag,
+                                                      float* __restrict__ tab, int warp, int lane) {
+  const int tiles = (K + 15) / 16;
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t a[kLutSmallMaxTiles][2];
+#pragma unroll
+  for (int i = 0; i < kLutSmallMaxTiles; ++i) {
+    const int tile = warp + 32 * i;
+    const int r0 = tile * 16 + g, r1 = r0 + 8;
+    const bool cok = 2 * t < D;
+    a[i][0] = (tile < tiles && r0 < K && cok) ? __ldg(reinterpret_cast<const uint32_t*>(book + r0 * D + 2 * t)) : 0u;
+    a[i][1] = (tile < tiles && r1 < K && cok) ? __ldg(reinterpret_cast<const uint32_t*>(book + r1 * D + 2 * t)) : 0u;
+  }
+#pragma unroll
+  for (int i = 0; i < kLutSmallMaxTiles; ++i) {
+    const int tile = warp + 32 * i;
+    if (tile >= tiles) break;
+    float d0, d1, d2, d3;
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
+        "{%7, %8, %9, %10};"
+        : "=f"(d0), "=f"(d1), "=f"(d2), "=f"(d3)
+        : "r"(a[i][0]), "r"(a[i][1]), "r"(bfrag), "f"(0.0f), "f"(0.0f), "f"(0.0f), "f"(0.0f));
+    const int r0 = tile * 16 + g;
+    if (t < 2) {
+      if (r0 < K) {
+        tab[(2 * t) * K + r0] = d0;
+        tab[(2 * t + 1) * K + r0] = d1;
+      }
+      if (r0 + 8 < K) {
+        tab[(2 * t) * K + r0 + 8] = d2;
+        tab[(2 * t + 1) * K + r0 + 8] = d3;
+      }
+    }
+  }
+}
+
 template <int RB8, int D, int NB>
 __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_small_kernel(Layer L, const uint16_t* __restrict__ x,
                                                                         int x_fp16, float* __restrict__ part,
@@ -597,10 +638,10 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_small_kernel(Layer L,
 
 // Rows in pairs, for 12-bit main books (with no second book, or a 4- or
 // 8-bit one): two 48-bit records are exactly three words, so every field of
-// the pair sits at a fixed bit position and its table byte offset (index * 8)
-// takes one shift and one mask.  Same tables, same sums, same order of the
-// four lookups of a row as gemv_lut_small_kernel; a thread's batch is four
-// pairs (8 rows, 8 TMEM columns).
+// the pair sits at a fixed bit position and its table byte offset (index * 4)
+// takes one shift and one mask.  The tables are fp32, one array per vector
+// (build_small_table_f32); a thread's batch is four pairs (8 rows, 8 TMEM
+// columns).
 template <int B, int Q, int NW>
 __device__ __forceinline__ uint32_t field_off(const uint32_t (&w)[NW]) {
   constexpr int bit = Q * B, wi = bit >> 5, sh = bit & 31;
@@ -610,16 +651,18 @@ __device__ __forceinline__ uint32_t field_off(const uint32_t (&w)[NW]) {
   } else {
     v = __funnelshift_r(w[wi], w[wi + 1], sh);
   }
-  return (v & ((1u << B) - 1u)) << 3;
+  return (v & ((1u << B) - 1u)) << 2;
 }
 
 template <int B, int H, int NW>
 __device__ __forceinline__ float row_lookup(const uint32_t (&w)[NW], const uint8_t* tab) {
-  // fields 4H .. 4H+3 of the pair: the four vectors of row 2p + H
-  const float a = h2f(*reinterpret_cast<const uint16_t*>(tab + field_off<B, 4 * H + 0>(w) + 0));
-  const float b = h2f(*reinterpret_cast<const uint16_t*>(tab + field_off<B, 4 * H + 1>(w) + 2));
-  const float c = h2f(*reinterpret_cast<const uint16_t*>(tab + field_off<B, 4 * H + 2>(w) + 4));
-  const float d = h2f(*reinterpret_cast<const uint16_t*>(tab + field_off<B, 4 * H + 3>(w) + 6));
+  // fields 4H .. 4H+3 of the pair: the four vectors of row 2p + H, each in its
+  // own array of 2^B floats
+  constexpr int stride = 4 << B;
+  const float a = *reinterpret_cast<const float*>(tab + field_off<B, 4 * H + 0>(w));
+  const float b = *reinterpret_cast<const float*>(tab + field_off<B, 4 * H + 1>(w) + stride);
+  const float c = *reinterpret_cast<const float*>(tab + field_off<B, 4 * H + 2>(w) + 2 * stride);
+  const float d = *reinterpret_cast<const float*>(tab + field_off<B, 4 * H + 3>(w) + 3 * stride);
   return (a + b) + (c + d);
 }
 
@@ -634,8 +677,8 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_pair_kernel(Layer L, 
   constexpr int TCOLS = 8 * CPW;
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int K1 = 1 << B1, K2 = B2 > 0 ? (1 << B2) : 0;
-  uint16_t* tab1 = reinterpret_cast<uint16_t*>(smem);   // T1[K1][4]
-  uint16_t* tab2 = tab1 + K1 * 4;                        // T2[K2][4]
+  float* tab1 = reinterpret_cast<float*>(smem);          // T1[4][K1]
+  float* tab2 = tab1 + K1 * 4;                           // T2[4][K2]
   __shared__ uint32_t s_tmem;
   __shared__ float s_scale;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -690,8 +733,8 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_pair_kernel(Layer L, 
         xs_acc += v;
       }
     }
-    build_small_table<D>(L.book[0], K1, bfrag, tab1, warp, lane);
-    if constexpr (NB == 2) build_small_table<D>(L.book[1], K2, bfrag, tab2, warp, lane);
+    build_small_table_f32<D>(L.book[0], K1, bfrag, tab1, warp, lane);
+    if constexpr (NB == 2) build_small_table_f32<D>(L.book[1], K2, bfrag, tab2, warp, lane);
     __syncthreads();   // tables complete
     {
       const float sc = s_scale;
@@ -829,6 +872,11 @@ cudaError_t launch_lut_small_t(const Layer& L, const GemvPlan& p, const void* x,
   return cudaGetLastError();
 }
 
+bool lut_pair_path(const Layer& L) {
+  const int b2 = L.nb == 2 ? L.b[1] : 0;
+  return L.b[0] == 12 && (b2 == 0 || b2 == 4 || b2 == 8);
+}
+
 template <int RB8, int D, int B2>
 cudaError_t launch_lut_pair_t(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, float* ws,
                               cudaStream_t stream) {
@@ -846,7 +894,7 @@ cudaError_t launch_lut_small(const Layer& L, const GemvPlan& p, const void* x, b
                              vq_dtype yt, float* ws, cudaStream_t stream) {
   cudaError_t e;
   const int b2 = L.nb == 2 ? L.b[1] : 0;
-  if (L.b[0] == 12 && (b2 == 0 || b2 == 4 || b2 == 8)) {      // rows in pairs, fixed offsets
+  if (lut_pair_path(L)) {                                       // rows in pairs, fixed offsets
     if (L.d == 8)
       e = b2 == 0 ? launch_lut_pair_t<RB8, 8, 0>(L, p, x, x_fp16, ws, stream)
         : b2 == 4 ? launch_lut_pair_t<RB8, 8, 4>(L, p, x, x_fp16, ws, stream)
@@ -869,9 +917,11 @@ cudaError_t launch_lut_small(const Layer& L, const GemvPlan& p, const void* x, b
   return cudaGetLastError();
 }
 
+// Tables of the small-book kernels: fp16 [K][4] per book, or fp32 [4][K] on
+// the paired-row path.
 size_t lut_small_smem(const Layer& L) {
   const size_t k = (static_cast<size_t>(1) << L.b[0]) + (L.nb == 2 ? (static_cast<size_t>(1) << L.b[1]) : 0);
-  return k * 4 * 2;
+  return k * 4 * (lut_pair_path(L) ? 4 : 2);
 }
 
 bool lut_small_supported(const Layer& L) {
