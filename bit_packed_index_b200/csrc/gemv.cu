@@ -1,6 +1,7 @@
 // gemv.cu -- vq_gemv: decode-time y = x . W_hat^T for batch <= 16, fused
 // unpack -> centroid gather -> multiply-accumulate, W_hat never leaves
-// registers.
+// registers.  The general split-K kernel here reads either index order; the
+// batch-1 fast paths are gemv1.cu (row order) and tile4.cu (tiled order).
 //
 // The pages describe the kernel shape this follows ("VPTQ Guide: Extreme
 // 2-Bit Vector Quantization", section "Step 3: Fused Low-Bit VPTQ Linear
@@ -43,7 +44,9 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-template <int D, int NB, int BT>
+// TILED: the index streams are in the tiled order (VQ_IDX_TILE4): field
+// (o, j) is slot j % 4 of row o's record in tile j / 4.
+template <int D, int NB, int BT, bool TILED>
 __global__ void __launch_bounds__(kGvThreads) gemv_kernel(
     Layer L, const uint16_t* __restrict__ x, int x_fp16, int batch, int64_t ldx, int vps, int rpb,
     int smem_mask, int book_bytes, void* __restrict__ y, vq_dtype yt, int64_t ldy,
@@ -104,12 +107,21 @@ __global__ void __launch_bounds__(kGvThreads) gemv_kernel(
     for (int o = rb * rpb + warp * R; o < o_end; o += kGvWarps * R) {
       const uint32_t* row0[R];
       const uint32_t* row1[R];
+      int64_t orows[R];
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         const int64_t orow = min(o + r, o_end - 1);     // clamp: results of extra rows are dropped
+        orows[r] = orow;
         row0[r] = L.idx[0] + orow * L.rw[0];
         row1[r] = (NB == 2) ? L.idx[1] + orow * L.rw[NB - 1] : nullptr;
       }
+      // Field j of row r, book m, in either storage order.
+      auto field = [&](int m, int r, int64_t j) -> uint32_t {
+        if constexpr (TILED)
+          return load_field(L.idx[m] + (j >> 2) * L.rw[m], (orows[r] * 4 + (j & 3)) * L.b[m], L.b[m]);
+        else
+          return load_field(m == 0 ? row0[r] : row1[r], j * L.b[m], L.b[m]);
+      };
       float acc[R][BT];
 #pragma unroll
       for (int r = 0; r < R; ++r)
@@ -122,10 +134,10 @@ __global__ void __launch_bounds__(kGvThreads) gemv_kernel(
         float wv[R][DM];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          load_centroid<D>(bv[0], load_field(row0[r], j * L.b[0], L.b[0]), d, wv[r]);
+          load_centroid<D>(bv[0], field(0, r, j), d, wv[r]);
           if constexpr (NB == 2) {
             float c2[DM];
-            load_centroid<D>(bv[1], load_field(row1[r], j * L.b[1], L.b[1]), d, c2);
+            load_centroid<D>(bv[1], field(1, r, j), d, c2);
 #pragma unroll
             for (int e = 0; e < DM; ++e) wv[r][e] += c2[e];
           }
@@ -179,7 +191,7 @@ template <int D, int NB, int BT>
 cudaError_t launch_bt(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, int batch,
                       int64_t ldx, void* y, vq_dtype yt, int64_t ldy, float* ws,
                       cudaStream_t stream) {
-  auto k = gemv_kernel<D, NB, BT>;
+  auto k = L.layout == VQ_IDX_TILE4 ? gemv_kernel<D, NB, BT, true> : gemv_kernel<D, NB, BT, false>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.grid_x, p.nsplit);
@@ -206,17 +218,20 @@ cudaError_t launch_d(const Layer& L, const GemvPlan& p, const void* x, bool xf, 
 
 vq_status plan_gemv(const Layer& L, int batch, GemvPlan* p, size_t ws_cap) {
   if (L.layout == VQ_IDX_TILE4) {
-    plan_gemv_tile4(L, batch, ws_cap, p);
-    return VQ_OK;
+    // batch 1: the lookup-table kernels; everything else: the split-K gather
+    // kernel below, reading the tiled records
+    if (plan_gemv_lut(L, batch, ws_cap, p)) return VQ_OK;
+  } else {
+    if (batch == 1 && gemv1_supported(L)) {
+      plan_gemv1(L, p);
+      if (p->smem <= device_smem_optin()) return VQ_OK;
+    }
+    if (gemvb_supported(L, batch)) {
+      plan_gemvb(L, batch, p);
+      if (p->smem <= device_smem_optin()) return VQ_OK;
+    }
   }
-  if (batch == 1 && gemv1_supported(L)) {
-    plan_gemv1(L, p);
-    if (p->smem <= device_smem_optin()) return VQ_OK;
-  }
-  if (gemvb_supported(L, batch)) {
-    plan_gemvb(L, batch, p);
-    if (p->smem <= device_smem_optin()) return VQ_OK;
-  }
+  *p = GemvPlan{};
   p->fast = 0;
   int bt = 1;
   while (bt < batch) bt <<= 1;
@@ -260,7 +275,7 @@ vq_status launch_gemv(const Layer& L, const GemvPlan& p, const void* x, bool x_f
   const int D = (L.d == 8) ? 8 : (L.d == 6 ? 6 : 0);
   cudaError_t e;
   if (p.fast >= 3) {
-    return cuda_status(launch_gemv_tile4(L, p, x, x_fp16, batch, ldx, y, yt, ldy, ws, stream));
+    return cuda_status(launch_gemv_lut(L, p, x, x_fp16, y, yt, ws, stream));
   } else if (p.fast == 1) {
     e = launch_gemv1(L, p, x, x_fp16, y, yt, ws, stream);
   } else if (p.fast == 2) {

@@ -1,7 +1,7 @@
 // tile4.cu -- kernels for the tiled index order (VQ_IDX_TILE4, include/vq.h):
-// the repack from row order, W_hat from a tiled layer, a plain tiled GEMV for
-// any batch, and the decode lookup-table GEMV (batch 1) that the order exists
-// for.
+// the repack from row order, W_hat from a tiled layer, and the decode
+// lookup-table GEMVs (batch 1) that the order exists for.  Other batches and
+// layers run gemv.cu's split-K kernel, which reads either order.
 //
 // The lookup-table GEMV ("Vector Quantization for LLM Weights in Production",
 // section "2. Lookup Table (LUT) Overhead vs. Bit-Shifting": codebook lookups
@@ -144,72 +144,6 @@ namespace {
 __device__ __forceinline__ float x_at(const uint16_t* __restrict__ x, int x_fp16, int64_t i) {
   const uint16_t u = __ldg(x + i);
   return x_fp16 ? h2f(u) : bf2f(u);
-}
-
-// ---------------------------------------------------------------------------
-// Plain tiled GEMV, any batch (1..16), any d and book count: one thread per
-// output row walks the row's records tile by tile, gathers the centroids and
-// accumulates x . c in fp32 for every batch row.  Consecutive threads read
-// consecutive records, and all lanes of a warp read the same x element.
-// ---------------------------------------------------------------------------
-template <int NB>
-__global__ void __launch_bounds__(256) gemv_tile4_kernel(Layer L, const uint16_t* __restrict__ x,
-                                                         int x_fp16, int batch, int64_t ldx,
-                                                         void* __restrict__ y, vq_dtype yt,
-                                                         int64_t ldy) {
-  __shared__ float red[8];
-  __shared__ float xsum[kMaxBatch];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int b = 0; b < batch; ++b) {          // sum_k x[b][k] for the bias term, fixed order
-    float v = 0.0f;
-    for (int k = threadIdx.x; k < L.kin; k += blockDim.x) v += x_at(x, x_fp16, b * ldx + k);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float t = 0.0f;
-      for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t += red[i];
-      xsum[b] = t;
-    }
-    __syncthreads();
-  }
-  const int d = L.d;
-  const int ntile = (L.nvec + 3) / 4;
-  for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < L.n;
-       o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    float acc[kMaxBatch];
-#pragma unroll
-    for (int b = 0; b < kMaxBatch; ++b) acc[b] = 0.0f;
-    for (int t = 0; t < ntile; ++t) {
-      const uint32_t* tile0 = L.idx[0] + t * L.rw[0];
-      const uint32_t* tile1 = L.idx[1] + t * L.rw[1];
-      for (int jj = 0; jj < 4; ++jj) {
-        const int j = t * 4 + jj;
-        if (j >= L.nvec) break;
-        float c[kMaxVecDim];
-        load_centroid<0>(BookView{L.book[0], d}, load_field(tile0, (o * 4 + jj) * L.b[0], L.b[0]), d, c);
-        if constexpr (NB == 2) {
-          float c2[kMaxVecDim];
-          load_centroid<0>(BookView{L.book[1], d}, load_field(tile1, (o * 4 + jj) * L.b[1], L.b[1]), d, c2);
-#pragma unroll
-          for (int e = 0; e < kMaxVecDim; ++e) c[e] += c2[e];
-        }
-        const int64_t k0 = static_cast<int64_t>(j) * d;
-        for (int e = 0; e < d; ++e) {
-          if (k0 + e >= L.kin) break;
-#pragma unroll
-          for (int b = 0; b < kMaxBatch; ++b)
-            if (b < batch) acc[b] = fmaf(x_at(x, x_fp16, b * ldx + k0 + e), c[e], acc[b]);
-        }
-      }
-    }
-    const float sc = L.scale ? h2f(L.scale[o]) : 1.0f;
-    const float tb = L.bias ? h2f(L.bias[o]) : 0.0f;
-#pragma unroll
-    for (int b = 0; b < kMaxBatch; ++b)
-      if (b < batch) store_out(y, yt, b * ldy + o, sc * acc[b] + tb * xsum[b]);
-  }
 }
 
 }  // namespace
@@ -937,35 +871,28 @@ bool lut_supported(const Layer& L) {
 
 }  // namespace
 
-void plan_gemv_tile4(const Layer& L, int batch, size_t ws_cap, GemvPlan* p) {
+bool plan_gemv_lut(const Layer& L, int batch, size_t ws_cap, GemvPlan* p) {
+  const bool big = lut_supported(L), small = !big && lut_small_supported(L);
+  if (batch != 1 || !(big || small)) return false;
+  const int ntasks = ((L.nvec + 3) / 4) * (big ? kLutSlices : 1);
+  const size_t per_block = (static_cast<size_t>(L.n) + 1) * sizeof(float);
+  int grid = std::min(device_sm_count(), ntasks);
+  if (ws_cap / per_block < static_cast<size_t>(grid)) grid = static_cast<int>(ws_cap / per_block);
+  if (grid < 1) return false;
+  int rb8 = 1;
+  while (static_cast<int64_t>(rb8) * 8 * kLutThreads < L.n) rb8 <<= 1;
   *p = GemvPlan{};
   p->nsplit = 1;
-  const bool big = lut_supported(L), small = !big && lut_small_supported(L);
-  if (batch == 1 && (big || small)) {
-    const int ntasks = ((L.nvec + 3) / 4) * (big ? kLutSlices : 1);
-    const size_t per_block = (static_cast<size_t>(L.n) + 1) * sizeof(float);
-    int grid = std::min(device_sm_count(), ntasks);
-    if (ws_cap / per_block < static_cast<size_t>(grid)) grid = static_cast<int>(ws_cap / per_block);
-    if (grid >= 1) {
-      int rb8 = 1;
-      while (static_cast<int64_t>(rb8) * 8 * kLutThreads < L.n) rb8 <<= 1;
-      p->fast = big ? 3 : 5;
-      p->grid_x = grid;
-      p->bt = rb8;
-      p->smem = big ? kLutSmem : static_cast<int>(lut_small_smem(L));
-      p->ws_bytes = per_block * grid;
-      return;
-    }
-  }
-  p->fast = 4;
-  p->bt = batch;
-  p->grid_x = std::max(1, std::min((L.n + 255) / 256, 8 * device_sm_count()));
-  p->ws_bytes = 0;
+  p->fast = big ? 3 : 5;
+  p->grid_x = grid;
+  p->bt = rb8;
+  p->smem = big ? kLutSmem : static_cast<int>(lut_small_smem(L));
+  p->ws_bytes = per_block * grid;
+  return true;
 }
 
-cudaError_t launch_gemv_tile4(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16,
-                              int batch, int64_t ldx, void* y, vq_dtype yt, int64_t ldy, float* ws,
-                              cudaStream_t stream) {
+cudaError_t launch_gemv_lut(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, void* y,
+                            vq_dtype yt, float* ws, cudaStream_t stream) {
   if (p.fast == 3) {
     switch (p.bt) {
       case 1: return launch_lut<1>(L, p, x, x_fp16, y, yt, ws, stream);
@@ -974,22 +901,12 @@ cudaError_t launch_gemv_tile4(const Layer& L, const GemvPlan& p, const void* x, 
       default: return launch_lut<8>(L, p, x, x_fp16, y, yt, ws, stream);
     }
   }
-  if (p.fast == 5) {
-    switch (p.bt) {
-      case 1: return launch_lut_small<1>(L, p, x, x_fp16, y, yt, ws, stream);
-      case 2: return launch_lut_small<2>(L, p, x, x_fp16, y, yt, ws, stream);
-      case 4: return launch_lut_small<4>(L, p, x, x_fp16, y, yt, ws, stream);
-      default: return launch_lut_small<8>(L, p, x, x_fp16, y, yt, ws, stream);
-    }
+  switch (p.bt) {
+    case 1: return launch_lut_small<1>(L, p, x, x_fp16, y, yt, ws, stream);
+    case 2: return launch_lut_small<2>(L, p, x, x_fp16, y, yt, ws, stream);
+    case 4: return launch_lut_small<4>(L, p, x, x_fp16, y, yt, ws, stream);
+    default: return launch_lut_small<8>(L, p, x, x_fp16, y, yt, ws, stream);
   }
-  count_launch();
-  if (L.nb == 1)
-    gemv_tile4_kernel<1><<<p.grid_x, 256, 0, stream>>>(L, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0,
-                                                        batch, ldx, y, yt, ldy);
-  else
-    gemv_tile4_kernel<2><<<p.grid_x, 256, 0, stream>>>(L, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0,
-                                                        batch, ldx, y, yt, ldy);
-  return cudaGetLastError();
 }
 
 }  // namespace vqk

@@ -71,17 +71,18 @@ struct GemvPlan {
   int books_in_smem;  // bit m set: book m staged in shared memory
   int book_bytes;     // shared memory taken by the staged books
   size_t ws_bytes;
-  int fast = 0;       // 1: single-row kernel (gemv1.cu), 2: batched kernel (gemvb.cu),
-                      // 3: lookup-table kernel (2^16 book), 4: plain tiled kernel,
-                      // 5: lookup-table kernel for books of <= 2^12 entries (tile4.cu)
+  int fast = 0;       // 0: split-K gather kernel (gemv.cu, either index order),
+                      // 1: single-row kernel (gemv1.cu), 2: batched kernel (gemvb.cu),
+                      // 3: lookup-table kernel (2^16 book), 5: lookup-table kernel for
+                      // books of <= 2^12 entries (tile4.cu, tiled order, batch 1)
 };
 // ws_cap: largest workspace the caller can provide (plans that need more
 // either shrink, for the tiled kernels, or are reported by their ws_bytes).
 vq_status plan_gemv(const Layer& L, int batch, GemvPlan* plan, size_t ws_cap = ~static_cast<size_t>(0));
-void plan_gemv_tile4(const Layer& L, int batch, size_t ws_cap, GemvPlan* plan);
-cudaError_t launch_gemv_tile4(const Layer& L, const GemvPlan& plan, const void* x, bool x_fp16,
-                              int batch, int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy,
-                              float* ws, cudaStream_t stream);
+// Lookup-table plans (tiled order, batch 1); false when no table kernel applies.
+bool plan_gemv_lut(const Layer& L, int batch, size_t ws_cap, GemvPlan* plan);
+cudaError_t launch_gemv_lut(const Layer& L, const GemvPlan& plan, const void* x, bool x_fp16, void* y,
+                            vq_dtype y_dtype, float* ws, cudaStream_t stream);
 bool gemv1_supported(const Layer& L);
 bool gemvb_supported(const Layer& L, int batch);
 void plan_gemvb(const Layer& L, int batch, GemvPlan* plan);

@@ -193,8 +193,10 @@ VQ_API vq_status vq_gemv_workspace_size(const vq_layer_desc* layer, int32_t batc
  * two so that no product can overflow fp16), rounds them to fp16, and sums the
  * entries the indices select.  That rounding adds about 2^-12 relative error
  * per term, inside the same tolerance as long as the codebook's values are
- * normal fp16 numbers (|c| >= 2^-14).  Other tiled layers use a plain tiled
- * kernel.
+ * normal fp16 numbers (|c| >= 2^-14).  Books of up to 2^12 entries (one or
+ * two, d = 6 or 8) get a table kernel without slices.  Every other tiled case
+ * (batches above 1, other shapes) runs the split-K gather kernel, which reads
+ * either index order.
  * Errors: VQ_ERR_INVALID_ARG, VQ_ERR_UNSUPPORTED (batch > 16), VQ_ERR_ALIGNMENT
  * (x or y not aligned to its element size), VQ_ERR_WORKSPACE, VQ_ERR_CUDA.
  */

@@ -9,8 +9,8 @@
   books of up to 2^12 entries at d = 6 or 8, whole) are checked on ragged
   shapes, every block-row size they compile for, both activation types, every
   output type, scale/bias present and absent, large and small activation
-  magnitudes, and the 70B / 405B / 8B decode shapes on sampled rows; the plain
-  tiled kernel on every other case."""
+  magnitudes, and the 70B / 405B / 8B decode shapes on sampled rows; the
+  split-K gather kernel reading tiled records on every other case."""
 import numpy as np
 import pytest
 import torch
@@ -181,8 +181,9 @@ def test_lut_gemv_all_zero_input_and_single_outlier():
     assert_close(_f64(y), oracle.linear(data, x), "float32")
 
 
-# Plain tiled kernel: every other case (batches > 1, two books, other d and b).
-PLAIN_SPECS = [
+# Every other case (batches > 1, two books, other d and b): the split-K gather
+# kernel reading tiled records.
+SPLITK_SPECS = [
     LayerSpec(300, 8 * 300 + 5, 8, (16,), (0.02,)),
     LayerSpec(300, 8 * 300 + 5, 8, (16, 8), (0.02, 0.005)),
     LayerSpec(300, 6 * 600 + 4, 6, (12, 4), (0.02, 0.005)),
@@ -191,11 +192,11 @@ PLAIN_SPECS = [
 ]
 
 
-@pytest.mark.parametrize("i", range(len(PLAIN_SPECS)))
+@pytest.mark.parametrize("i", range(len(SPLITK_SPECS)))
 @pytest.mark.parametrize("batch", [1, 2, 5, 16])
-def test_plain_tiled_gemv(i, batch):
+def test_split_k_gemv_on_tiled_records(i, batch):
     vq = _vq()
-    spec = PLAIN_SPECS[i]
+    spec = SPLITK_SPECS[i]
     data = synth.make_layer(spec, seed=2600 + i)
     layer = _oracle_tiled_layer(data)
     x = synth.make_x(2650 + i, batch, spec.in_features, outlier_frac=0.01)
@@ -238,7 +239,7 @@ def test_noalloc_on_a_tiled_layer_shrinks_the_grid():
 @pytest.mark.parametrize("li", [0, 1, 2])
 def test_70b_decode_layers_tiled(li):
     """The 2-bpw 70B MLP layers in the tiled order: dequant bit-exact on sampled
-    rows; batch 1 (lookup table) and batch 4 (plain) on sampled rows."""
+    rows; batch 1 (lookup table) and batch 4 (split-K gather kernel) on sampled rows."""
     vq = _vq()
     w = WORKLOADS["llama3_70b_mlp"]
     spec, seed = w.layers[li]
