@@ -210,7 +210,22 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
   }
   float xs_acc = 0.0f;   // warp 0: sum of x, one group per slice-0 task
 
-  for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
+  // Work items: the tasks of the whole rounds, then the last partial round's
+  // tasks split by 8192-row batches over the blocks that would idle (each
+  // piece builds the task's table, then does its share of the lookups).
+  const int full = (ntasks / static_cast<int>(gridDim.x)) * static_cast<int>(gridDim.x);
+  const int tail = ntasks - full;
+  const int nbat = (n + 8 * kLutThreads - 1) / (8 * kLutThreads);
+  const int parts = tail > 0 ? max(1, min(nbat, static_cast<int>(gridDim.x) / tail)) : 1;
+  const int nitems = full + tail * parts;
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+    int task = item, b_lo = 0, b_hi = RB8;
+    if (item >= full) {
+      const int q = item - full, part = q % parts;
+      task = full + q / parts;
+      b_lo = part * nbat / parts;
+      b_hi = (part + 1) * nbat / parts;
+    }
     const int g = task / kLutSlices, s = task - g * kLutSlices;
     // B operand of m16n8k8: x'[vector kLutNJ*g + lane/4][components 2t, 2t+1],
     // other columns zero.  x' = x * 2^-e with ||x'_j||_1 < 1 for the task's
@@ -236,7 +251,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
       const __half2 h = __floats2half2_rn(ldexpf(a, -e), ldexpf(b, -e));
       bfrag = *reinterpret_cast<const uint32_t*>(&h);
       if (tid == 0) s_scale = ldexpf(1.0f, e);
-      if (warp == 0 && s == 0) {
+      if (warp == 0 && s == 0 && b_lo == 0) {
         float v = a + b;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
@@ -312,6 +327,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
             w[cur ^ 1][r] = o < n ? ldg_stream64(trow + o) : make_uint2(0u, 0u);
           }
         }
+        if (b < b_lo || b >= b_hi) continue;         // uniform: another piece's rows
         float acc[8];
         sm100::tmem_ld8(tbase + 8 * b, acc);
 #pragma unroll
