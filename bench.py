@@ -462,11 +462,11 @@ def run_profile(args):
     import torch
     from bit_packed_index_b200 import vq
     dev = torch.device("cuda", 0)
-    if args.profile in ("gemv", "lut", "dequant"):
-        w = WORKLOADS[DECODE]
-        spec, seed = w.layers[0]
+    if args.profile in ("gemv", "lut", "lut_small", "dequant"):
+        w = WORKLOADS[DECODE if args.profile != "lut_small" else "llama31_405b"]
+        spec, seed = w.layers[0 if args.profile != "lut_small" else 4]
         layer = vq.Layer.from_synth(synth.make_layer(spec, seed), dev,
-                                    layout="tile4" if args.profile == "lut" else "rows")
+                                    layout="tile4" if args.profile.startswith("lut") else "rows")
         x = torch.from_numpy(synth.make_x(w.x_seed, BATCH, spec.in_features, w.outlier_frac)
                              .view(np.int16)).to(dev).view(torch.bfloat16)
         out = (torch.empty((spec.out_features, spec.in_features), dtype=torch.float16, device=dev)
@@ -501,9 +501,10 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["gemv", "lut", "gemm", "dequant"],
+    ap.add_argument("--profile", choices=["gemv", "lut", "lut_small", "gemm", "dequant"],
                     help="run a few untimed launches of one call on its workload (for ncu): "
-                         "gemv / lut = gate_proj in row / tiled order")
+                         "gemv / lut = 70B gate_proj in row / tiled order, lut_small = 405B "
+                         "gate_proj in tiled order")
     ap.add_argument("--profile-launches", type=int, default=3)
     args = ap.parse_args(argv)
     if args.profile:
