@@ -57,57 +57,123 @@ __global__ void repack_tile4_kernel(const uint32_t* __restrict__ src, int64_t sr
 }
 
 // ---------------------------------------------------------------------------
-// W_hat from a tiled layer: one thread per (tile, row), writing the row's four
-// vectors.  The fp32 operations and their order are those of vq_dequant's
-// row-order kernel (centroid sum, times scale, plus bias, one fp16 rounding).
+// W_hat from a tiled layer.  Work unit = (row, tile): the row's four vectors
+// of that tile.  Four consecutive threads take four consecutive tiles of one
+// row, so a warp writes 8 rows x 256 contiguous bytes (d = 8) and reads 8
+// consecutive records from each of 4 tiles.  Books that fit are staged in
+// shared memory as in vq_dequant's row-order kernel.  The fp32 operations and
+// their order are that kernel's (centroid sum, times scale, plus bias, one
+// fp16 rounding).
 // ---------------------------------------------------------------------------
 template <int D, int NB>
-__global__ void dequant_tile4_kernel(Layer L, uint16_t* __restrict__ w, int64_t ldw) {
+__global__ void dequant_tile4_kernel(Layer L, uint16_t* __restrict__ w, int64_t ldw, int vec_store,
+                                     int smem_mask) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  BookView bv[2];
+  {
+    size_t off = 0;
+#pragma unroll
+    for (int m = 0; m < NB; ++m) {
+      if (smem_mask & (1 << m)) {
+        const int pad = L.d <= 8 ? 8 : 16;
+        uint16_t* dst = reinterpret_cast<uint16_t*>(smem + off);
+        stage_book(dst, L.book[m], 1 << L.b[m], L.d, pad);
+        bv[m] = {dst, pad};
+        off += (static_cast<size_t>(1) << L.b[m]) * pad * sizeof(uint16_t);
+      } else {
+        bv[m] = {L.book[m], L.d};
+      }
+    }
+    if (smem_mask) __syncthreads();
+  }
   const int ntile = (L.nvec + 3) / 4;
-  const int64_t total = static_cast<int64_t>(ntile) * L.n;
+  const int ntb = (ntile + 3) / 4;                        // groups of four tiles
+  const int64_t total = static_cast<int64_t>(ntb) * L.n * 4;
   const int d = D > 0 ? D : L.d;
   const bool has_s = L.scale != nullptr, has_t = L.bias != nullptr;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t t = i / L.n, o = i - t * L.n;
+    const int64_t rest = i >> 2;
+    const int64_t tb = rest / L.n, o = rest - tb * L.n;
+    const int64_t t = tb * 4 + (i & 3);
+    if (t >= ntile) continue;
     const float s = has_s ? h2f(L.scale[o]) : 1.0f;
-    const float tb = has_t ? h2f(L.bias[o]) : 0.0f;
+    const float tbias = has_t ? h2f(L.bias[o]) : 0.0f;
     const uint32_t* tile0 = L.idx[0] + t * L.rw[0];
     const uint32_t* tile1 = L.idx[1] + t * L.rw[1];
     uint16_t* wrow = w + o * ldw;
-#pragma unroll 1
+    // The record's four fields and their centroids first (all gathers in
+    // flight), then the arithmetic and the stores.
+    uint32_t f0[4], f1[4];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      f0[jj] = load_field(tile0, (o * 4 + jj) * L.b[0], L.b[0]);
+      if constexpr (NB == 2) f1[jj] = load_field(tile1, (o * 4 + jj) * L.b[1], L.b[1]);
+    }
+    constexpr int DM = D > 0 ? D : kMaxVecDim;
+    float c[4][DM];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      load_centroid<D>(bv[0], f0[jj], d, c[jj]);
+      if constexpr (NB == 2) {
+        float c2[DM];
+        load_centroid<D>(bv[1], f1[jj], d, c2);
+#pragma unroll
+        for (int e = 0; e < DM; ++e)
+          if (e < d) c[jj][e] = __fadd_rn(c[jj][e], c2[e]);
+      }
+    }
+#pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
       const int64_t j = t * 4 + jj;
       if (j >= L.nvec) break;
-      float c[kMaxVecDim];
-      load_centroid<D>(BookView{L.book[0], d}, load_field(tile0, (o * 4 + jj) * L.b[0], L.b[0]), d, c);
-      if constexpr (NB == 2) {
-        float c2[kMaxVecDim];
-        load_centroid<D>(BookView{L.book[1], d}, load_field(tile1, (o * 4 + jj) * L.b[1], L.b[1]), d, c2);
-#pragma unroll
-        for (int e = 0; e < kMaxVecDim; ++e)
-          if (e < d) c[e] = __fadd_rn(c[e], c2[e]);
-      }
       const int64_t k0 = j * d;
+      uint16_t h[DM];
 #pragma unroll
-      for (int e = 0; e < kMaxVecDim; ++e) {
-        if (e < d && k0 + e < L.kin) {
-          float v = c[e];
+      for (int e = 0; e < DM; ++e) {
+        if (e < d) {
+          float v = c[jj][e];
           if (has_s) v = __fmul_rn(v, s);
-          if (has_t) v = __fadd_rn(v, tb);
-          wrow[k0 + e] = f2h(v);
+          if (has_t) v = __fadd_rn(v, tbias);
+          h[e] = f2h(v);
         }
+      }
+      if (D == 8 && vec_store == 2 && k0 + 8 <= L.kin) {      // one 16-byte store
+        *reinterpret_cast<uint4*>(wrow + k0) =
+            make_uint4(h[0] | (static_cast<uint32_t>(h[1]) << 16), h[2] | (static_cast<uint32_t>(h[3]) << 16),
+                       h[4] | (static_cast<uint32_t>(h[5]) << 16), h[6] | (static_cast<uint32_t>(h[7]) << 16));
+      } else if (D == 6 && vec_store >= 1 && k0 + 6 <= L.kin) {  // three 4-byte stores
+#pragma unroll
+        for (int e = 0; e < 6; e += 2)
+          *reinterpret_cast<uint32_t*>(wrow + k0 + e) = h[e] | (static_cast<uint32_t>(h[e + 1]) << 16);
+      } else {
+#pragma unroll
+        for (int e = 0; e < DM; ++e)
+          if (e < d && k0 + e < L.kin) wrow[k0 + e] = h[e];
       }
     }
   }
 }
 
+constexpr size_t kDq4SmemBooks = 96 * 1024;   // stage books up to this size
+
 template <int D, int NB>
 cudaError_t launch_dq4(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream) {
-  const int64_t total = static_cast<int64_t>((L.nvec + 3) / 4) * L.n;
-  const int grid = static_cast<int>(std::min<int64_t>((total + 255) / 256, 16LL * device_sm_count()));
+  int smem_mask = 0;
+  const size_t smem = stage_plan(L, std::min<size_t>(kDq4SmemBooks, device_smem_optin()), &smem_mask);
+  auto k = dequant_tile4_kernel<D, NB>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  const int per_sm = smem ? std::max(1, std::min(8, static_cast<int>((228 * 1024) / (smem + 1024)))) : 8;
+  const int64_t total = static_cast<int64_t>((((L.nvec + 3) / 4) + 3) / 4) * L.n * 4;
+  const int grid = static_cast<int>(std::min<int64_t>((total + 255) / 256,
+                                                      static_cast<int64_t>(device_sm_count()) * per_sm));
+  // 2: 16-byte rows of 8 halves aligned; 1: 4-byte pairs aligned (rows of even length)
+  const int vec_store = (aligned(w, 16) && ldw % 8 == 0) ? 2 : (aligned(w, 4) && ldw % 2 == 0) ? 1 : 0;
   count_launch();
-  dequant_tile4_kernel<D, NB><<<grid, 256, 0, stream>>>(L, w, ldw);
+  k<<<grid, 256, smem, stream>>>(L, w, ldw, vec_store, smem_mask);
   return cudaGetLastError();
 }
 

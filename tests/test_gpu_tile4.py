@@ -41,14 +41,32 @@ def _f64(t: torch.Tensor) -> np.ndarray:
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def _oracle_tiled_layer(data, extra_words=0):
-    """A device layer whose tiled streams the oracle packed (never the library)."""
+def _garbage(tiles, b, n, nvec, seed):
+    """Random bits wherever the format says bits are ignored: fields of vectors
+    >= nvec in the last tile, and every bit past the N records of a tile."""
+    rng = np.random.default_rng(seed)
+    bits = np.unpackbits(tiles.view(np.uint8), axis=1, bitorder="little")
+    bits[:, n * 4 * b:] = rng.integers(0, 2, size=bits[:, n * 4 * b:].shape, dtype=np.uint8)
+    if nvec % 4:
+        rec = bits[-1, : n * 4 * b].reshape(n, 4, b)
+        rec[:, nvec % 4:, :] = rng.integers(0, 2, size=rec[:, nvec % 4:, :].shape, dtype=np.uint8)
+        bits[-1, : n * 4 * b] = rec.reshape(-1)
+    return np.packbits(bits, axis=1, bitorder="little").view(np.uint32).reshape(tiles.shape)
+
+
+def _oracle_tiled_layer(data, extra_words=0, garbage=False):
+    """A device layer whose tiled streams the oracle packed (never the library);
+    with ``garbage`` every ignored bit is random."""
     vq = _vq()
     s = data.spec
     tiles = []
     for m, b in enumerate(s.log2k):
         idx = oracle.unpack(data.idx_words[m], b, s.nvec)
-        tiles.append(oracle.pack_tile4(idx, b, oracle.tile4_words(s.out_features, b) + extra_words))
+        t = oracle.pack_tile4(idx, b, oracle.tile4_words(s.out_features, b) + extra_words)
+        if garbage:
+            t = _garbage(t, b, s.out_features, s.nvec, seed=77 + m)
+            assert np.array_equal(oracle.unpack_tile4(t, b, s.out_features, s.nvec), idx)
+        tiles.append(t)
     layer = vq.Layer.from_host(s.out_features, s.in_features, s.d, s.log2k, tiles,
                                data.codebooks, data.scale, data.bias)
     layer.layout = "tile4"
@@ -298,3 +316,27 @@ def test_small_book_decode_layers_tiled(name, li):
     ref = oracle.linear(data, x, rows)
     y = vq.gemv(layer, _x_dev(x), out_dtype=torch.bfloat16)
     assert_close(_f64(y[:, torch.from_numpy(rows).cuda()]), ref, "bfloat16")
+
+
+GARBAGE_SPECS = [
+    LayerSpec(1001, 8 * 33 + 3, 8, (16,), (0.02,)),            # 2^16 table kernel
+    LayerSpec(777, 6 * 31 + 4, 6, (12, 4), (0.02, 0.005)),     # paired small-book kernel
+    LayerSpec(301, 7 * 13 + 2, 7, (9, 3), (0.02, 0.005)),      # split-K kernel
+]
+
+
+@pytest.mark.parametrize("i", range(len(GARBAGE_SPECS)))
+def test_ignored_bits_are_ignored(i):
+    """Random bits in every bit the tiled format ignores change nothing: dequant
+    stays bit-exact and the products stay within the bar, at batch 1 and 3."""
+    vq = _vq()
+    spec = GARBAGE_SPECS[i]
+    data = synth.make_layer(spec, seed=3000 + i)
+    layer = _oracle_tiled_layer(data, extra_words=4, garbage=True)
+    w = vq.dequant(layer)
+    torch.cuda.synchronize()
+    assert np.array_equal(_w_bits(w), oracle.dequant(data))
+    for batch in (1, 3):
+        x = synth.make_x(3050 + i, batch, spec.in_features, outlier_frac=0.01)
+        y = vq.gemv(layer, _x_dev(x), out_dtype=torch.float32)
+        assert_close(_f64(y), oracle.linear(data, x), "float32")
