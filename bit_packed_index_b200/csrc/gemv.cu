@@ -275,7 +275,7 @@ vq_status launch_gemv(const Layer& L, const GemvPlan& p, const void* x, bool x_f
   const int D = (L.d == 8) ? 8 : (L.d == 6 ? 6 : 0);
   cudaError_t e;
   if (p.fast >= 3) {
-    return cuda_status(launch_gemv_lut(L, p, x, x_fp16, y, yt, ws, stream));
+    return cuda_status(launch_gemv_lut(L, p, x, x_fp16, batch, ldx, y, yt, ldy, ws, stream));
   } else if (p.fast == 1) {
     e = launch_gemv1(L, p, x, x_fp16, y, yt, ws, stream);
   } else if (p.fast == 2) {

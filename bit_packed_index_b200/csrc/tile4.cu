@@ -19,6 +19,7 @@
 // memory (TMEM) across tasks.  A second kernel adds the per-block sums and
 // applies scale and bias.
 #include <algorithm>
+#include <cstdlib>
 
 #include "codebook.cuh"
 #include "sm100.cuh"
@@ -953,9 +954,26 @@ bool lut_supported(const Layer& L) {
 
 }  // namespace
 
+cudaError_t launch_gemv_lut_row(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, void* y,
+                                vq_dtype yt, float* ws, cudaStream_t stream);
+// Measured crossovers against the split-K kernel on tiled layers (B200): a
+// 2^16 book pays up to batch 2 (70B gate: 187 against 352 us at B = 2, 276
+// against 263 at B = 3); books of <= 2^12 entries up to batch 8 and beyond
+// (405B q at B = 8: 484 against 872 us).
+constexpr int kLutMaxBatchBig = 2;
+constexpr int kLutMaxBatchSmall = 8;
+
+// Largest batch served by running the batch-1 table kernel once per row of x
+// (each run reads the index streams again); larger batches take the split-K
+// gather kernel.  Environment override for measurements: VQ_LUT_MAX_BATCH.
+int lut_batch_limit(const Layer& L, bool big) {
+  if (const char* env = std::getenv("VQ_LUT_MAX_BATCH")) return std::atoi(env);
+  return big ? kLutMaxBatchBig : kLutMaxBatchSmall;
+}
+
 bool plan_gemv_lut(const Layer& L, int batch, size_t ws_cap, GemvPlan* p) {
   const bool big = lut_supported(L), small = !big && lut_small_supported(L);
-  if (batch != 1 || !(big || small)) return false;
+  if (!(big || small) || batch < 1 || batch > lut_batch_limit(L, big)) return false;
   const int ntasks = ((L.nvec + 3) / 4) * (big ? kLutSlices : 1);
   const size_t per_block = (static_cast<size_t>(L.n) + 1) * sizeof(float);
   int grid = std::min(device_sm_count(), ntasks);
@@ -973,8 +991,21 @@ bool plan_gemv_lut(const Layer& L, int batch, size_t ws_cap, GemvPlan* p) {
   return true;
 }
 
-cudaError_t launch_gemv_lut(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, void* y,
-                            vq_dtype yt, float* ws, cudaStream_t stream) {
+cudaError_t launch_gemv_lut(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, int batch,
+                            int64_t ldx, void* y, vq_dtype yt, int64_t ldy, float* ws, cudaStream_t stream) {
+  // One batch-1 table pass per row of x, in stream order (the workspace is
+  // reused by each pass).
+  const size_t ysz = yt == VQ_FP32 ? 4 : 2;
+  for (int b = 0; b < batch; ++b) {
+    cudaError_t e = launch_gemv_lut_row(L, p, static_cast<const uint16_t*>(x) + b * ldx, x_fp16,
+                                        static_cast<char*>(y) + b * ldy * ysz, yt, ws, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_gemv_lut_row(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, void* y,
+                                vq_dtype yt, float* ws, cudaStream_t stream) {
   if (p.fast == 3) {
     switch (p.bt) {
       case 1: return launch_lut<1>(L, p, x, x_fp16, y, yt, ws, stream);

@@ -79,10 +79,12 @@ struct GemvPlan {
 // ws_cap: largest workspace the caller can provide (plans that need more
 // either shrink, for the tiled kernels, or are reported by their ws_bytes).
 vq_status plan_gemv(const Layer& L, int batch, GemvPlan* plan, size_t ws_cap = ~static_cast<size_t>(0));
-// Lookup-table plans (tiled order, batch 1); false when no table kernel applies.
+// Lookup-table plans (tiled order; a batch runs one table pass per row of x,
+// up to a per-layer limit); false when no table kernel applies.
 bool plan_gemv_lut(const Layer& L, int batch, size_t ws_cap, GemvPlan* plan);
-cudaError_t launch_gemv_lut(const Layer& L, const GemvPlan& plan, const void* x, bool x_fp16, void* y,
-                            vq_dtype y_dtype, float* ws, cudaStream_t stream);
+cudaError_t launch_gemv_lut(const Layer& L, const GemvPlan& plan, const void* x, bool x_fp16, int batch,
+                            int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy, float* ws,
+                            cudaStream_t stream);
 bool gemv1_supported(const Layer& L);
 bool gemvb_supported(const Layer& L, int batch);
 void plan_gemvb(const Layer& L, int batch, GemvPlan* plan);

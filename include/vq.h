@@ -194,9 +194,11 @@ VQ_API vq_status vq_gemv_workspace_size(const vq_layer_desc* layer, int32_t batc
  * entries the indices select.  That rounding adds about 2^-12 relative error
  * per term, inside the same tolerance as long as the codebook's values are
  * normal fp16 numbers (|c| >= 2^-14).  Books of up to 2^12 entries (one or
- * two, d = 6 or 8) get a table kernel without slices.  Every other tiled case
- * (batches above 1, other shapes) runs the split-K gather kernel, which reads
- * either index order.
+ * two, d = 6 or 8) get a table kernel without slices.  Batches of 2 (2^16
+ * book) or up to 8 (small books) run one table pass per row of x.  Every
+ * other tiled case runs the split-K gather kernel, which reads either index
+ * order.  The environment variable VQ_LUT_MAX_BATCH overrides those batch
+ * limits (0 turns the table kernels off), for measurements.
  * Errors: VQ_ERR_INVALID_ARG, VQ_ERR_UNSUPPORTED (batch > 16), VQ_ERR_ALIGNMENT
  * (x or y not aligned to its element size), VQ_ERR_WORKSPACE, VQ_ERR_CUDA.
  */

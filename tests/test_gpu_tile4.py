@@ -199,8 +199,9 @@ def test_lut_gemv_all_zero_input_and_single_outlier():
     assert_close(_f64(y), oracle.linear(data, x), "float32")
 
 
-# Every other case (batches > 1, two books, other d and b): the split-K gather
-# kernel reading tiled records.
+# Batches 1..16 on tiled layers: small batches of table-eligible layers run one
+# table pass per row of x, everything else the split-K gather kernel reading
+# tiled records.
 SPLITK_SPECS = [
     LayerSpec(300, 8 * 300 + 5, 8, (16,), (0.02,)),
     LayerSpec(300, 8 * 300 + 5, 8, (16, 8), (0.02, 0.005)),
@@ -212,7 +213,7 @@ SPLITK_SPECS = [
 
 @pytest.mark.parametrize("i", range(len(SPLITK_SPECS)))
 @pytest.mark.parametrize("batch", [1, 2, 5, 16])
-def test_split_k_gemv_on_tiled_records(i, batch):
+def test_tiled_gemv_batches(i, batch):
     vq = _vq()
     spec = SPLITK_SPECS[i]
     data = synth.make_layer(spec, seed=2600 + i)
@@ -340,3 +341,23 @@ def test_ignored_bits_are_ignored(i):
         x = synth.make_x(3050 + i, batch, spec.in_features, outlier_frac=0.01)
         y = vq.gemv(layer, _x_dev(x), out_dtype=torch.float32)
         assert_close(_f64(y), oracle.linear(data, x), "float32")
+
+
+def test_table_batch_limit_override(monkeypatch):
+    """VQ_LUT_MAX_BATCH moves a batch between the per-row table passes (a
+    workspace of per-block row sums) and the split-K kernel (split partials);
+    both give the same products within the bar."""
+    vq = _vq()
+    spec = LayerSpec(2000, 6 * 100 + 2, 6, (12, 4), (0.02, 0.005))
+    data = synth.make_layer(spec, seed=3100)
+    layer = _oracle_tiled_layer(data)
+    x = synth.make_x(3101, 5, spec.in_features, outlier_frac=0.01)
+    ref = oracle.linear(data, x)
+    sizes = {}
+    for limit in ("0", "16"):
+        monkeypatch.setenv("VQ_LUT_MAX_BATCH", limit)
+        sizes[limit] = vq.gemv_workspace_size(layer, 5)
+        y = vq.gemv(layer, _x_dev(x), out_dtype=torch.float32)
+        assert_close(_f64(y), ref, "float32")
+    assert sizes["16"] % ((spec.out_features + 1) * 4) == 0
+    assert sizes["0"] != sizes["16"]
