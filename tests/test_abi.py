@@ -113,3 +113,18 @@ def test_repack_argument_checks_need_no_device(lib):
     assert lib.vq_repack_tile4(C.byref(src), dst, tw, None) == vq.VQ_ERR_INVALID_ARG  # no dst
     dst[0] = 0x30008
     assert lib.vq_repack_tile4(C.byref(src), dst, tw, None) == vq.VQ_ERR_ALIGNMENT
+
+
+def test_table_batch_limit_needs_no_device(lib, monkeypatch):
+    """Small batches of a 2^16-book tiled layer plan the per-row table passes
+    (per-block row sums) up to batch 2, then the split-K kernel; the
+    VQ_LUT_MAX_BATCH override moves that limit."""
+    n = C.c_size_t(0)
+    d = _tiled_desc(n=1000, kin=64 * 8)
+    table = lambda v: v > 0 and v % (1001 * 4) == 0
+    for batch, want in ((1, True), (2, True), (3, False)):
+        assert lib.vq_gemv_workspace_size(C.byref(d), batch, C.byref(n)) == vq.VQ_OK
+        assert table(n.value) == want, (batch, n.value)
+    monkeypatch.setenv("VQ_LUT_MAX_BATCH", "0")
+    assert lib.vq_gemv_workspace_size(C.byref(d), 1, C.byref(n)) == vq.VQ_OK
+    assert not table(n.value)
