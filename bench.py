@@ -394,6 +394,7 @@ def run_gpu(args):
            "ms_per_step": e2e_ms / args.steps}
 
     gemm = run_gemm(dev, peaks, peak_src, vq)
+    decode_405b = run_decode_405b(dev, peaks, peak_src, vq)
 
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -408,6 +409,7 @@ def run_gpu(args):
         "gpu_launches": int(launches),
         "clocks": clocks.summary(),
         "gemm": gemm,
+        "decode_405b_gate": decode_405b,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gbs, rows, dt, cores = oracle_rate(10.0, w.layers, xs_host)
@@ -454,6 +456,38 @@ def run_gemm(dev, peaks, peak_src, vq):
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"],
                          "peak_source": peak_src + " (bf16 burst; fp16 nominal rate is the same)"}}
+
+
+def run_decode_405b(dev, peaks, peak_src, vq):
+    """Beside the headline: the Llama-3.1-405B gate_proj (53248 x 16384, d = 6,
+    K = 2^12 + 2^4, 2.67 bpw) at batch 1 in the tiled order, where the
+    small-book lookup-table kernel runs; L2 flushed between timed calls."""
+    import torch
+    w = WORKLOADS["llama31_405b"]
+    spec, seed = w.layers[4]
+    layer = vq.Layer.from_synth(synth.make_layer(spec, seed), dev, layout="tile4")
+    x = torch.from_numpy(synth.make_x(w.x_seed + 4, 1, spec.in_features).view(np.int16)).to(dev)
+    x = x.view(torch.bfloat16)
+    y = torch.empty((1, spec.out_features), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(256, vq.gemv_workspace_size(layer, 1)), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        vq.gemv(layer, x, out=y, workspace=ws)
+    times = []
+    for _ in range(20):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        vq.gemv(layer, x, out=y, workspace=ws)
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    gbs = alg_bytes(spec, 1) / (ms * 1e-3) / 1e9
+    return {"workload": "llama31_405b gate_proj 53248x16384, d=6, K=2^12 + residual K=2^4 (2.67 bpw), "
+                        "B=1, tiled index order (small-book lookup-table kernel)",
+            "us": ms * 1e3, "achieved_gbs": gbs, "frac_of_measured_hbm": gbs / peaks["hbm_gbs"],
+            "algorithmic_bytes": alg_bytes(spec, 1), "peak_source": peak_src}
 
 
 def run_profile(args):
