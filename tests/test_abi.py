@@ -83,7 +83,8 @@ def test_layout_field_validation_needs_no_device(lib):
 
 def test_tiled_workspace_sizes(lib):
     """Batch 1 on a lookup-table-eligible tiled layer needs per-block row sums;
-    other batches and other layers use the plain tiled kernel, which needs none."""
+    batch 3 of a 2^16 book and layers no table kernel takes use the split-K
+    gather kernel, which for this narrow layer runs one split (no workspace)."""
     n = C.c_size_t(0)
     d = _tiled_desc(n=1000, kin=64)
     assert lib.vq_gemv_workspace_size(C.byref(d), 1, C.byref(n)) == vq.VQ_OK
@@ -94,7 +95,7 @@ def test_tiled_workspace_sizes(lib):
     d.idx_row_words[0] = vq.tile4_words(1000, 12)
     assert lib.vq_gemv_workspace_size(C.byref(d), 1, C.byref(n)) == vq.VQ_OK
     assert n.value > 0 and n.value % (1001 * 4) == 0
-    d.vec_dim, d.in_features = 16, 128                 # no table kernel for d = 16: plain kernel
+    d.vec_dim, d.in_features = 16, 128                 # no table kernel for d = 16: split-K
     assert lib.vq_gemv_workspace_size(C.byref(d), 1, C.byref(n)) == vq.VQ_OK
     assert n.value == 0
 
