@@ -361,3 +361,18 @@ def test_table_batch_limit_override(monkeypatch):
         assert_close(_f64(y), ref, "float32")
     assert sizes["16"] % ((spec.out_features + 1) * 4) == 0
     assert sizes["0"] != sizes["16"]
+
+
+def test_tiled_small_batch_strided_x_and_y():
+    """The per-row table passes honour the row strides of x and y."""
+    vq = _vq()
+    for i, spec in enumerate([LayerSpec(700, 8 * 60, 8, (16,), (0.02,)),
+                              LayerSpec(500, 6 * 70 + 2, 6, (12, 4), (0.02, 0.005))]):
+        data = synth.make_layer(spec, seed=3200 + i)
+        layer = _oracle_tiled_layer(data)
+        x = synth.make_x(3210 + i, 2, spec.in_features, outlier_frac=0.01, ld=spec.in_features + 40)
+        ref = oracle.linear(data, x[:, :spec.in_features])
+        ybuf = torch.zeros((2, spec.out_features + 24), dtype=torch.float32, device="cuda")
+        vq.gemv(layer, _x_dev(x)[:, :spec.in_features], out=ybuf[:, :spec.out_features])
+        assert_close(_f64(ybuf[:, :spec.out_features]), ref, "float32")
+        assert (ybuf[:, spec.out_features:] == 0).all()
