@@ -226,7 +226,7 @@ constexpr int kLutNJ = 4;                           // vectors per task: one til
 constexpr int kLutS = 24576;                        // centroids per slice (the last: 16384)
 constexpr int kLutSlices = (65536 + kLutS - 1) / kLutS;   // 3 slices of the 2^16 book
 constexpr int kLutSmem = kLutS * kLutNJ * 2;        // T[S][4] in fp16: 192 KB
-constexpr int kLutPD = 8;                           // 16-centroid tiles per load batch
+constexpr int kLutPD = 4;                           // 32-centroid tiles per load batch
 
 __device__ __forceinline__ uint32_t ldg_stream32(const void* p) {
   uint32_t v;
@@ -239,6 +239,72 @@ __device__ __forceinline__ uint2 ldg_stream64(const void* p) {
   return v;
 }
 
+// The table products of a 2^16 book run as m16n8k16 with two centroids per A
+// row: row r of a 32-centroid tile is centroids 2r and 2r+1 (16 consecutive
+// halves), B column n < 4 holds x'_n against the even centroid and n >= 4
+// x'_(n-4) against the odd one, so all eight output columns are table entries
+// and every lane stores.  Any permutation of k serves if A and B share it: lane
+// (n = lane/4, t = lane%4) takes k = {2t, 2t+1} and {2t+8, 2t+9} from the four
+// consecutive halves 4t..4t+3 of its row, one 8-byte load.  Those halves are
+// components 4(t%2)..+3 of the even (t < 2) or odd (t >= 2) centroid, so the
+// lane's B pair is x' of vector n%4 at those components when t/2 == n/4, zero
+// otherwise.  x' = x * 2^-e with ||x'_j||_1 < 1 for the group's four vectors,
+// so no product overflows fp16; the return value is 2^e.  *xpart gets the
+// lane's share of the group's sum of x (each element counted once per warp).
+__device__ __forceinline__ float lut_pair_bfrag(const uint16_t* __restrict__ x, int x_fp16, int kin, int g,
+                                                int lane, uint32_t (&bf)[2], float* xpart) {
+  const int n = lane >> 2, t = lane & 3;
+  const int64_t k0 = (static_cast<int64_t>(g) * kLutNJ + (n & 3)) * 8 + 4 * (t & 1);
+  float v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = k0 + i < kin ? x_at(x, x_fp16, k0 + i) : 0.0f;
+  float l1 = (fabsf(v[0]) + fabsf(v[1])) + (fabsf(v[2]) + fabsf(v[3]));
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);       // the vector's other half
+  float mx = l1;
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  int e = 0;
+  if (mx > 0.0f && mx < INFINITY) frexpf(mx, &e);
+  const bool on = (t >> 1) == (n >> 2);
+  const __half2 h0 = on ? __floats2half2_rn(ldexpf(v[0], -e), ldexpf(v[1], -e)) : __floats2half2_rn(0.f, 0.f);
+  const __half2 h1 = on ? __floats2half2_rn(ldexpf(v[2], -e), ldexpf(v[3], -e)) : __floats2half2_rn(0.f, 0.f);
+  bf[0] = *reinterpret_cast<const uint32_t*>(&h0);
+  bf[1] = *reinterpret_cast<const uint32_t*>(&h1);
+  *xpart = (n < 4 && t < 2) ? (v[0] + v[1]) + (v[2] + v[3]) : 0.0f;
+  return ldexpf(1.0f, e);
+}
+
+// One 32-centroid tile: D = A x B (fp32), A = afr (rows g and g+8 of the
+// tile, each an 8-byte load), then the eight table entries of this lane in
+// fp16.  Lane (n, t) owns T[32*tile + 2n + t/2][2(t%2), +1] and the same for
+// row n+8; a warp's two stores are 128 contiguous bytes each.
+__device__ __forceinline__ void lut_pair_mma_store(const uint32_t (&afr)[4], const uint32_t (&bf)[2],
+                                                   uint16_t* __restrict__ lut, int tile, int lane) {
+  float d0, d1, d2, d3;
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%10, %11, %12, %13};"
+      : "=f"(d0), "=f"(d1), "=f"(d2), "=f"(d3)
+      : "r"(afr[0]), "r"(afr[1]), "r"(afr[2]), "r"(afr[3]), "r"(bf[0]), "r"(bf[1]), "f"(0.0f), "f"(0.0f),
+        "f"(0.0f), "f"(0.0f));
+  uint16_t* p = lut + tile * 32 * kLutNJ + 2 * lane;   // = T[32 tile + 2n + t/2][2(t%2)]
+  *reinterpret_cast<__half2*>(p) = __floats2half2_rn(d0, d1);
+  *reinterpret_cast<__half2*>(p + 16 * kLutNJ) = __floats2half2_rn(d2, d3);
+}
+
+// A operand of one 32-centroid tile read from the book (rows n and n+8 of
+// the tile: centroids 32 tile + 2n, +1 and 32 tile + 2n + 16, +17).
+__device__ __forceinline__ void lut_pair_afr(const uint16_t* __restrict__ bslice, int tile, int lane,
+                                             uint32_t (&afr)[4]) {
+  const uint16_t* c = bslice + tile * 32 * 8 + 4 * lane;
+  const uint2 r0 = ldg_stream64(c);
+  const uint2 r1 = ldg_stream64(c + 16 * 8);
+  afr[0] = r0.x;   // row n,   k = 2t, 2t+1
+  afr[1] = r1.x;   // row n+8, k = 2t, 2t+1
+  afr[2] = r0.y;   // row n,   k = 2t+8, 2t+9
+  afr[3] = r1.y;   // row n+8, k = 2t+8, 2t+9
+}
+
 // RB8 batches of 8 rows per thread: a block covers N <= 8 * RB8 * 1024 rows;
 // thread (warp w, lane l) keeps its row sums in TMEM lane 32*(w%4)+l, columns
 // (w/4)*8*RB8 .. +8*RB8 (warps may only touch their own quarter of the lanes).
@@ -248,9 +314,9 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
                                                                   float* __restrict__ xpart) {
   constexpr int CPW = 8 * RB8;                      // TMEM columns per group of 4 warps
   constexpr int TCOLS = 8 * CPW;                    // 64 .. 512, a power of two
-  constexpr int NBATCH = kLutS / 16 / (kLutThreads / 32) / kLutPD;   // batches, full slice
-  static_assert(kLutS % (16 * (kLutThreads / 32) * kLutPD) == 0 &&
-                (65536 % kLutS) % (16 * (kLutThreads / 32) * kLutPD) == 0,
+  constexpr int NBATCH = kLutS / 32 / (kLutThreads / 32) / kLutPD;   // batches, full slice
+  static_assert(kLutS % (32 * (kLutThreads / 32) * kLutPD) == 0 &&
+                (65536 % kLutS) % (32 * (kLutThreads / 32) * kLutPD) == 0,
                 "every slice splits into whole load batches per warp");
   extern __shared__ __align__(128) uint8_t smem[];
   uint16_t* lut = reinterpret_cast<uint16_t*>(smem);   // T[k - slice base][kLutNJ vectors]
@@ -294,81 +360,39 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
       b_hi = (part + 1) * nbat / parts;
     }
     const int g = task / kLutSlices, s = task - g * kLutSlices;
-    // B operand of m16n8k8: x'[vector kLutNJ*g + lane/4][components 2t, 2t+1],
-    // other columns zero.  x' = x * 2^-e with ||x'_j||_1 < 1 for the task's
-    // vectors, so |T| <= max |c| and no product overflows fp16; 2^e is
-    // applied per row.
-    uint32_t bfrag;
+    uint32_t bfrag[2];
     {
-      const int jj = lane >> 2, t = lane & 3;
-      const int64_t k = (static_cast<int64_t>(g) * kLutNJ + jj) * 8 + 2 * t;
-      float a = 0.0f, b = 0.0f;
-      if (jj < kLutNJ) {
-        if (k < kin) a = x_at(x, x_fp16, k);
-        if (k + 1 < kin) b = x_at(x, x_fp16, k + 1);
-      }
-      float l1 = fabsf(a) + fabsf(b);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-      float mx = l1;
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      int e = 0;
-      if (mx > 0.0f && mx < INFINITY) frexpf(mx, &e);
-      const __half2 h = __floats2half2_rn(ldexpf(a, -e), ldexpf(b, -e));
-      bfrag = *reinterpret_cast<const uint32_t*>(&h);
-      if (tid == 0) s_scale = ldexpf(1.0f, e);
+      float xp;
+      const float sc = lut_pair_bfrag(x, x_fp16, kin, g, lane, bfrag, &xp);
+      if (tid == 0) s_scale = sc;
       if (warp == 0 && s == 0 && b_lo == 0) {
-        float v = a + b;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        xs_acc += v;
+        for (int off = 16; off > 0; off >>= 1) xp += __shfl_xor_sync(0xffffffffu, xp, off);
+        xs_acc += xp;
       }
     }
     // Phase A: T for this slice.  Warp w builds its share of the slice's
-    // 16-centroid tiles; each tile's A operand is read straight from the
-    // codebook (lane: centroid lane/4 (+8), components 2t, 2t+1), two load
-    // batches in flight.
+    // 32-centroid tiles, the A operands read straight from the codebook, two
+    // load batches in flight.
     {
       const uint16_t* bslice = L.book[0] + static_cast<size_t>(s) * kLutS * 8;
       const int slice_n = min(kLutS, 65536 - s * kLutS);
-      const int tpw = slice_n / 16 / (kLutThreads / 32);        // tiles per warp
+      const int tpw = slice_n / 32 / (kLutThreads / 32);        // tiles per warp
       const int nb = tpw / kLutPD;                                // load batches
       const int t0w = warp * tpw;
-      uint32_t afr[2][kLutPD][2];
+      uint32_t afr[2][kLutPD][4];
 #pragma unroll
-      for (int p = 0; p < kLutPD; ++p) {
-        const uint16_t* c0 = bslice + ((t0w + p) * 16 + (lane >> 2)) * 8 + 2 * (lane & 3);
-        afr[0][p][0] = ldg_stream32(c0);
-        afr[0][p][1] = ldg_stream32(c0 + 64);
-      }
+      for (int p = 0; p < kLutPD; ++p) lut_pair_afr(bslice, t0w + p, lane, afr[0][p]);
 #pragma unroll
       for (int bt = 0; bt < NBATCH; ++bt) {
         if (bt >= nb) break;                        // uniform: the slice's own size
         const int cur = bt & 1;
         if (bt + 1 < nb) {
 #pragma unroll
-          for (int p = 0; p < kLutPD; ++p) {
-            const uint16_t* c0 = bslice + ((t0w + (bt + 1) * kLutPD + p) * 16 + (lane >> 2)) * 8 + 2 * (lane & 3);
-            afr[cur ^ 1][p][0] = ldg_stream32(c0);
-            afr[cur ^ 1][p][1] = ldg_stream32(c0 + 64);
-          }
+          for (int p = 0; p < kLutPD; ++p) lut_pair_afr(bslice, t0w + (bt + 1) * kLutPD + p, lane, afr[cur ^ 1][p]);
         }
 #pragma unroll
-        for (int p = 0; p < kLutPD; ++p) {
-          float d0, d1, d2, d3;
-          asm volatile(
-              "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
-              "{%7, %8, %9, %10};"
-              : "=f"(d0), "=f"(d1), "=f"(d2), "=f"(d3)
-              : "r"(afr[cur][p][0]), "r"(afr[cur][p][1]), "r"(bfrag), "f"(0.0f), "f"(0.0f), "f"(0.0f),
-                "f"(0.0f));
-          if ((lane & 3) < kLutNJ / 2) {            // columns 0..kLutNJ-1 are the vectors
-            const int kl = (t0w + bt * kLutPD + p) * 16 + (lane >> 2);
-            *reinterpret_cast<__half2*>(lut + kl * kLutNJ + 2 * (lane & 3)) = __floats2half2_rn(d0, d1);
-            *reinterpret_cast<__half2*>(lut + (kl + 8) * kLutNJ + 2 * (lane & 3)) = __floats2half2_rn(d2, d3);
-          }
-        }
+        for (int p = 0; p < kLutPD; ++p) lut_pair_mma_store(afr[cur][p], bfrag, lut, t0w + bt * kLutPD + p, lane);
       }
     }
     __syncthreads();   // T complete
