@@ -254,24 +254,34 @@ __device__ __forceinline__ uint2 ldg_stream64(const void* p) {
 __device__ __forceinline__ float lut_pair_bfrag(const uint16_t* __restrict__ x, int x_fp16, int kin, int g,
                                                 int lane, uint32_t (&bf)[2], float* xpart) {
   const int n = lane >> 2, t = lane & 3;
-  const int64_t k0 = (static_cast<int64_t>(g) * kLutNJ + (n & 3)) * 8 + 4 * (t & 1);
+  const int k0 = (g * kLutNJ + (n & 3)) * 8 + 4 * (t & 1);
   float v[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) v[i] = k0 + i < kin ? x_at(x, x_fp16, k0 + i) : 0.0f;
+  for (int i = 0; i < 4; ++i) {
+    const uint16_t u = k0 + i < kin ? __ldg(x + k0 + i) : static_cast<uint16_t>(0);
+    v[i] = x_fp16 ? h2f(u) : bf2f(u);
+  }
   float l1 = (fabsf(v[0]) + fabsf(v[1])) + (fabsf(v[2]) + fabsf(v[3]));
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);       // the vector's other half
   float mx = l1;
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  // e: the exponent with mx = m * 2^e, 0.5 <= m < 1, read from the bits
+  // (-126 for a subnormal mx, which only makes x' smaller); 0 when mx is
+  // zero or not finite.  2^-e is applied as two factors 2^-(e/2) and
+  // 2^-(e - e/2), each a normal float for every e in [-126, 128], so x' is
+  // the exactly scaled x (or rounds to zero only where fp16 would anyway).
   int e = 0;
-  if (mx > 0.0f && mx < INFINITY) frexpf(mx, &e);
+  if (mx > 0.0f && mx < INFINITY) e = static_cast<int>(__float_as_uint(mx) >> 23) - 126;
+  const float f1 = __uint_as_float(static_cast<uint32_t>(127 - e / 2) << 23);
+  const float f2 = __uint_as_float(static_cast<uint32_t>(127 - (e - e / 2)) << 23);
   const bool on = (t >> 1) == (n >> 2);
-  const __half2 h0 = on ? __floats2half2_rn(ldexpf(v[0], -e), ldexpf(v[1], -e)) : __floats2half2_rn(0.f, 0.f);
-  const __half2 h1 = on ? __floats2half2_rn(ldexpf(v[2], -e), ldexpf(v[3], -e)) : __floats2half2_rn(0.f, 0.f);
+  const __half2 h0 = __floats2half2_rn(on ? v[0] * f1 * f2 : 0.0f, on ? v[1] * f1 * f2 : 0.0f);
+  const __half2 h1 = __floats2half2_rn(on ? v[2] * f1 * f2 : 0.0f, on ? v[3] * f1 * f2 : 0.0f);
   bf[0] = *reinterpret_cast<const uint32_t*>(&h0);
   bf[1] = *reinterpret_cast<const uint32_t*>(&h1);
   *xpart = (n < 4 && t < 2) ? (v[0] + v[1]) + (v[2] + v[3]) : 0.0f;
-  return ldexpf(1.0f, e);
+  return __uint_as_float(static_cast<uint32_t>(127 + e) << 23);   // 2^e (inf for e = 128)
 }
 
 // One 32-centroid tile: D = A x B (fp32), A = afr (rows g and g+8 of the
@@ -360,6 +370,26 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
       b_hi = (part + 1) * nbat / parts;
     }
     const int g = task / kLutSlices, s = task - g * kLutSlices;
+    // The next item's index tile row, pulled into L2 while this one runs.
+    {
+      const int nx = item + static_cast<int>(gridDim.x);
+      if (nx < nitems) {
+        const int ntask = nx < full ? nx : full + (nx - full) / parts;
+        const char* row = reinterpret_cast<const char*>(L.idx[0] + static_cast<int64_t>(ntask / kLutSlices) * L.rw[0]);
+        for (int l = tid; l < (n * 8 + 127) / 128; l += kLutThreads)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(row + static_cast<int64_t>(l) * 128));
+      }
+    }
+    // Phase A operands of the first load batch go out before the activations
+    // are read, so the two latencies overlap.
+    const uint16_t* bslice = L.book[0] + static_cast<size_t>(s) * kLutS * 8;
+    const int slice_n = min(kLutS, 65536 - s * kLutS);
+    const int tpw = slice_n / 32 / (kLutThreads / 32);        // tiles per warp
+    const int nb = tpw / kLutPD;                                // load batches
+    const int t0w = warp * tpw;
+    uint32_t afr[2][kLutPD][4];
+#pragma unroll
+    for (int p = 0; p < kLutPD; ++p) lut_pair_afr(bslice, t0w + p, lane, afr[0][p]);
     uint32_t bfrag[2];
     {
       float xp;
@@ -375,14 +405,6 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
     // 32-centroid tiles, the A operands read straight from the codebook, two
     // load batches in flight.
     {
-      const uint16_t* bslice = L.book[0] + static_cast<size_t>(s) * kLutS * 8;
-      const int slice_n = min(kLutS, 65536 - s * kLutS);
-      const int tpw = slice_n / 32 / (kLutThreads / 32);        // tiles per warp
-      const int nb = tpw / kLutPD;                                // load batches
-      const int t0w = warp * tpw;
-      uint32_t afr[2][kLutPD][4];
-#pragma unroll
-      for (int p = 0; p < kLutPD; ++p) lut_pair_afr(bslice, t0w + p, lane, afr[0][p]);
 #pragma unroll
       for (int bt = 0; bt < NBATCH; ++bt) {
         if (bt >= nb) break;                        // uniform: the slice's own size
