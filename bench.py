@@ -60,6 +60,11 @@ BATCH = 1
 # whose batch-1 kernel measured faster on that shape (the tiled table kernel
 # on all three: 89 / 89 / 140 us against 150 / 150 / 161 in row order).
 LAYOUTS = ("tile4", "tile4", "tile4")
+# Encoder workload (vq_encode): a 4096 x 4096 fp16 weight matrix ~ N(0, 0.02)
+# against one K = 2^16, d = 8 codebook ~ N(0, 0.02) (2.0 bpw).
+ENCODE_SHAPE = (4096, 4096, 8, [16])
+ENCODE_STD = [0.02]
+ENCODE_SEED = 11
 
 
 def kernel_sources_sha(files) -> str:
@@ -495,7 +500,15 @@ def run_profile(args):
     import torch
     from bit_packed_index_b200 import vq
     dev = torch.device("cuda", 0)
-    if args.profile in ("gemv", "lut", "lut_down", "lut_small", "dequant"):
+    if args.profile == "encode":
+        n, kin, d, log2k = ENCODE_SHAPE
+        w, books = synth.make_encode_input(n, kin, d, log2k, ENCODE_STD, seed=ENCODE_SEED)
+        W = torch.from_numpy(w.view(np.int16)).to(dev).view(torch.float16)
+        B = [torch.from_numpy(b.view(np.int16)).to(dev).view(torch.float16) for b in books]
+        ws = torch.empty(vq.encode_workspace_size(n, kin, log2k, d), dtype=torch.uint8, device=dev)
+        for _ in range(args.profile_launches):
+            vq.encode(W, B, log2k, d, workspace=ws)
+    elif args.profile in ("gemv", "lut", "lut_down", "lut_small", "dequant"):
         w = WORKLOADS[DECODE if args.profile != "lut_small" else "llama31_405b"]
         spec, seed = w.layers[{"lut_small": 4, "lut_down": 2}.get(args.profile, 0)]
         layer = vq.Layer.from_synth(synth.make_layer(spec, seed), dev,
@@ -534,10 +547,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["gemv", "lut", "lut_down", "lut_small", "gemm", "dequant"],
+    ap.add_argument("--profile", choices=["gemv", "lut", "lut_down", "lut_small", "gemm", "dequant",
+                                          "encode"],
                     help="run a few untimed launches of one call on its workload (for ncu): "
                          "gemv / lut = 70B gate_proj in row / tiled order, lut_down = 70B "
-                         "down_proj in tiled order, lut_small = 405B gate_proj in tiled order")
+                         "down_proj in tiled order, lut_small = 405B gate_proj in tiled order, "
+                         "encode = the encoder on its bench workload")
     ap.add_argument("--profile-launches", type=int, default=3)
     args = ap.parse_args(argv)
     if args.profile:

@@ -1,0 +1,694 @@
+// encode.cu -- the nearest-centroid encoder (vq_encode in include/vq.h):
+// idx[o][j] = argmin_k ||v - C[k]||^2 for every vector of a weight matrix,
+// ties to the lowest k, equal to the exact (fp64) definition; with two books
+// the second stage encodes the residual of the first (greedy cascade).
+// Follows "VPTQ Guide: Extreme 2-Bit Vector Quantization", section "The
+// Information-Theoretic Superiority of Vector Quantization" (q = argmin) and
+// section "2. Multi-Stage Residual Vector Quantization (RVQ)".
+//
+// Design:
+//  * ||v - c||^2 = ||v||^2 + (||c||^2 - 2<v, c>), and only the bracket depends
+//    on c.  The bracket is one dot product of length d + 2 <= 16: A row =
+//    [v~, 1, 1, 0...], B row = [-2 c~, hi, lo, 0...] with hi + lo = ||c~||^2
+//    split into two fp16 values, so a single tcgen05 MMA (M = 128 vectors,
+//    N = 256 centroids, K = 16, fp16 x fp16 -> fp32 in tensor memory) gives the
+//    whole bracket for 32768 pairs.  v~ and c~ are v and c times one power of
+//    two per book, chosen so that max ||c~||^2 lies in [2^8, 2^10): the
+//    argmin does not change and every operand stays well inside fp16.
+//  * The prepared book ([-2c~, hi, lo] rows, 32 bytes per centroid) is laid
+//    out in global memory exactly as the 128-byte-swizzled K-major operand the
+//    MMA reads -- four centroids of different 256-row groups share a 128-byte
+//    row -- so 1024 centroids arrive with one 32 KB bulk copy and the four
+//    MMAs of that block address it with a 32-byte column offset.
+//  * Sixteen epilogue warps read the accumulators (two TMEM buffers of 256
+//    columns, so the MMA of the next tile overlaps) and keep, per vector and
+//    column quarter, the smallest value, its column and the second smallest:
+//    a 32-column chunk costs 31 min operations and one compare, and only a
+//    chunk that holds a new minimum is scanned again.
+//  * A vector whose second smallest value exceeds the smallest by more than
+//    twice a bound on the arithmetic error (fp32 accumulation, the hi/lo
+//    split, fp16 rounding of a residual) has the exact argmin in hand.  Every
+//    other vector -- near-ties, partial last vectors, values fp16 cannot hold
+//    -- is decided by an fp64 pass over the whole book that repeats the
+//    definition operation by operation, so the output equals the definition.
+//  * Every mbarrier wait is bounded; a wait that runs out of budget raises
+//    the block's abort flag, records VQ_ERR_TIMEOUT in the workspace's status
+//    word and lets every warp fall through to the teardown.
+#include <climits>
+#include <cmath>
+
+#include "sm100.cuh"
+#include "vq_internal.cuh"
+
+namespace vqk {
+namespace {
+
+using namespace sm100;
+
+constexpr int kEncM = 128;                          // vectors per block (MMA M)
+constexpr int kEncN = 256;                          // centroids per MMA (N)
+constexpr int kEncBlockK = 1024;                    // centroids per staged block: 4 MMAs
+constexpr int kEncBlockBytes = kEncBlockK / 4 * 128;   // 256 rows x 128 B = 32 KB
+constexpr int kEncStages = 3;
+constexpr int kEncEpiWarps = 16;                    // 4 lane quarters x 4 column quarters
+constexpr int kEncThreads = (4 + kEncEpiWarps) * 32;
+constexpr int kEncATile = kEncM * 128;              // 16 KB: rows of 128 B, first 32 B used
+constexpr long long kEncWaitBudget = 4000000000LL;  // SM clocks (about 2 s)
+constexpr float kEncPadNorm = 30000.0f;             // hi = lo of padding centroids
+constexpr int kEncMaxD = 14;                        // d + 2 <= 16
+constexpr int kEncExactThreads = 256;
+
+struct EncCtrl {
+  uint64_t full[kEncStages];
+  uint64_t empty[kEncStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint32_t tmem_base;
+  int abort_flag;
+  float eps[kEncM];              // error bound of each vector's bracket values
+  int flag[kEncM];               // 0: decide here, 1: exact pass, 2: no vector
+  float best[4][kEncM];          // per column quarter: smallest value,
+  float second[4][kEncM];        //   second smallest,
+  int arg[4][kEncM];             //   column of the smallest
+};
+
+// Workspace control words (first 256 bytes).
+struct EncWsCtrl {
+  int status;
+  int list_count[2];             // vectors left to the exact pass, per stage
+  unsigned cmax_bits[2];         // max_k ||C_m[k]||^2 (fp32 bits; non-negative)
+};
+
+__device__ __forceinline__ uint8_t* enc_align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Byte offset of 16-byte chunk c of row r in a 128-byte-swizzled operand.
+__device__ __forceinline__ uint32_t enc_sw128(int r, int c) {
+  return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+// Power-of-two exponent s with cmax * 4^s in [2^8, 2^10) (s = 0 for a zero or
+// non-finite cmax; a subnormal cmax is treated as 2^-127).
+__device__ __forceinline__ int enc_scale_exp(float cmax) {
+  if (!(cmax > 0.0f) || !(cmax < INFINITY)) return 0;
+  const int e = static_cast<int>((__float_as_uint(cmax) >> 23) & 0xffu) - 127;
+  return (9 - e) >> 1;                               // floor((9 - e) / 2)
+}
+__device__ __forceinline__ float enc_pow2(int s) {  // 2^s, s in [-126, 127]
+  return __uint_as_float(static_cast<uint32_t>(127 + s) << 23);
+}
+
+// Plain bulk copy global -> shared (no multicast), completing on bar.
+__device__ __forceinline__ void enc_bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Book preparation.
+// ---------------------------------------------------------------------------
+__global__ void enc_book_norm_kernel(const uint16_t* __restrict__ book, int K, int d,
+                                     unsigned* __restrict__ cmax_bits) {
+  float m = 0.0f;
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < K; k += gridDim.x * blockDim.x) {
+    float s = 0.0f;
+    for (int e = 0; e < d; ++e) {
+      const float c = h2f(book[static_cast<int64_t>(k) * d + e]);
+      s = fmaf(c, c, s);
+    }
+    m = fmaxf(m, s);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((threadIdx.x & 31) == 0) atomicMax(cmax_bits, __float_as_uint(m));   // m >= 0: bits order as values
+}
+
+// Prepared book: centroid k = 1024 q + 256 sl + r sits in block q (32 KB),
+// row r, 16-half column slot sl, 128-byte swizzled; halves [-2 c~ (d), hi,
+// lo, 0...], c~ = fp16(c * 2^s), hi + lo = ||c~||^2.  Centroids k >= K (the
+// padding up to a whole block) get hi = lo = kEncPadNorm and zero c~.
+__global__ void enc_book_prep_kernel(const uint16_t* __restrict__ book, int K, int d, int kp,
+                                     const unsigned* __restrict__ cmax_bits, uint8_t* __restrict__ bprep) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= kp) return;
+  const float f = enc_pow2(enc_scale_exp(__uint_as_float(*cmax_bits)));
+  uint16_t h[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) h[i] = 0;
+  if (k < K) {
+    float nrm = 0.0f;
+    for (int e = 0; e < d; ++e) {
+      const float c = h2f(f2h(h2f(book[static_cast<int64_t>(k) * d + e]) * f));
+      h[e] = f2h(-2.0f * c);
+      nrm = __fadd_rn(nrm, __fmul_rn(c, c));
+    }
+    const uint16_t hi = f2h(nrm);
+    h[d] = hi;
+    h[d + 1] = f2h(nrm - h2f(hi));
+  } else {
+    h[d] = f2h(kEncPadNorm);
+    h[d + 1] = f2h(kEncPadNorm);
+  }
+  const int q = k / kEncBlockK, rem = k % kEncBlockK, sl = rem / kEncN, r = rem % kEncN;
+  uint8_t* base = bprep + static_cast<size_t>(q) * kEncBlockBytes;
+  uint4 c0, c1;
+  c0.x = h[0] | (static_cast<uint32_t>(h[1]) << 16);
+  c0.y = h[2] | (static_cast<uint32_t>(h[3]) << 16);
+  c0.z = h[4] | (static_cast<uint32_t>(h[5]) << 16);
+  c0.w = h[6] | (static_cast<uint32_t>(h[7]) << 16);
+  c1.x = h[8] | (static_cast<uint32_t>(h[9]) << 16);
+  c1.y = h[10] | (static_cast<uint32_t>(h[11]) << 16);
+  c1.z = h[12] | (static_cast<uint32_t>(h[13]) << 16);
+  c1.w = h[14] | (static_cast<uint32_t>(h[15]) << 16);
+  *reinterpret_cast<uint4*>(base + enc_sw128(r, 2 * sl)) = c0;
+  *reinterpret_cast<uint4*>(base + enc_sw128(r, 2 * sl + 1)) = c1;
+}
+
+// ---------------------------------------------------------------------------
+// The tensor-core pass.
+// ---------------------------------------------------------------------------
+struct EncArgs {
+  const uint16_t* w;
+  int64_t ldw;
+  int n, kin, d, nfull, nvec;    // nfull = kin / d whole vectors per row
+  int64_t nv_full;               // n * nfull
+  const uint8_t* bprep;
+  int kp, K;                     // padded and real book size
+  const unsigned* cmax_bits;
+  const uint16_t* book1;         // second stage: v = w - C_1[idx1] (else null)
+  const uint32_t* idx1;
+  uint32_t* idx_out;             // [n][nvec]
+  int* list;                     // vector ids o * nvec + j left to the exact pass
+  int* list_count;
+  int* status;
+};
+
+// One 32-column chunk of bracket values for centroids k0 .. k0+31: running
+// smallest value, its centroid and the second smallest value.
+__device__ __forceinline__ void enc_chunk(const uint32_t (&r)[32], int k0, float& best, float& second,
+                                          int& arg) {
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    m[i] = fminf(fminf(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1])),
+                 fminf(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
+  const float mn = fminf(fminf(fminf(m[0], m[1]), fminf(m[2], m[3])), fminf(fminf(m[4], m[5]), fminf(m[6], m[7])));
+  if (mn < best) {                 // rare after the first chunks: find the column and the runner-up
+    int pos = 0;
+    bool found = false;
+    float s2 = INFINITY;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float v = __uint_as_float(r[i]);
+      if (!found && v == mn) {
+        pos = i;
+        found = true;
+      } else {
+        s2 = fminf(s2, v);
+      }
+    }
+    second = fminf(best, s2);
+    best = mn;
+    arg = k0 + pos;
+  } else {
+    second = fminf(second, mn);
+  }
+}
+
+__global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
+  extern __shared__ __align__(1024) uint8_t enc_smem[];
+  EncCtrl* ctrl = reinterpret_cast<EncCtrl*>(enc_smem);
+  uint8_t* atile = enc_align1024(enc_smem + sizeof(EncCtrl));
+  uint8_t* stages = atile + kEncATile;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &ctrl->abort_flag;
+  const int64_t v0 = static_cast<int64_t>(blockIdx.x) * kEncM;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kEncStages; ++s) {
+      mbar_init(&ctrl->full[s], 1);
+      mbar_init(&ctrl->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctrl->acc_full[b], 1);
+      mbar_init(&ctrl->acc_empty[b], kEncEpiWarps);
+    }
+    ctrl->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctrl->tmem_base, 512);
+    tmem_relinquish();
+  }
+
+  // A operand: row t = [v~ (d halves), 1, 1, 0...] of vector v0 + t, and the
+  // vector's error bound.  With s the book's exponent and v~ = fp16(v 2^s),
+  // the MMA returns D(k) = sum_e v~_e (-2 c~_ke) + hi_k + lo_k, and
+  //   |D(k) - (||c_k||^2 - 2<v, c_k>) 4^s|
+  //     <= 2^-18 (||v~||^2 + 2 C + 1)      fp32 accumulation, hi/lo split
+  //      + 2^-22 ||v~||_1 (1 + sqrt C)     fp16 rounding of tiny c~ components
+  //      + 2 delta (sqrt C + 1)            v~ against v 2^s (delta: its L1 error)
+  // with C = max_k ||c~_k||^2 < 2^10; the terms are loose by design.
+  if (threadIdx.x < kEncM) {
+    const int t = threadIdx.x;
+    const int64_t gv = v0 + t;
+    const float cmax = __uint_as_float(*a.cmax_bits);
+    const int se = enc_scale_exp(cmax);
+    const float f = enc_pow2(se);
+    uint16_t h[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) h[i] = 0;
+    float eps = 0.0f;
+    int flag = 2;
+    if (gv < a.nv_full) {
+      flag = 0;
+      const int o = static_cast<int>(gv / a.nfull), j = static_cast<int>(gv % a.nfull);
+      const uint16_t* wr = a.w + static_cast<int64_t>(o) * a.ldw + static_cast<int64_t>(j) * a.d;
+      const uint16_t* c1 = a.book1 ? a.book1 + static_cast<int64_t>(a.idx1[static_cast<int64_t>(o) * a.nvec + j]) * a.d
+                                   : nullptr;
+      float n2 = 0.0f, l1 = 0.0f, dl = 0.0f;
+      for (int e = 0; e < a.d; ++e) {
+        float v = h2f(wr[e]);
+        if (c1) v = __fsub_rn(v, h2f(c1[e]));
+        const float vs = v * f;                      // exact: a power-of-two scale in range
+        const uint16_t hv = f2h(vs);
+        const float vt = h2f(hv);
+        if (!(fabsf(vt) <= 65504.0f)) flag = 1;      // overflow or NaN: exact pass
+        h[e] = hv;
+        n2 = fmaf(vt, vt, n2);
+        l1 += fabsf(vt);
+        dl += fabsf(vt - vs) + fabsf(vs) * 0x1p-22f + 0x1p-24f;
+      }
+      h[a.d] = 0x3C00u;                              // 1.0 (times hi)
+      h[a.d + 1] = 0x3C00u;                          // 1.0 (times lo)
+      const float cs = cmax * f * f;
+      const float rc = sqrtf(cs);
+      eps = 0x1p-18f * (n2 + 2.0f * cs + 1.0f) + 0x1p-22f * l1 * (1.0f + rc) + 2.0f * dl * (rc + 1.0f);
+      if (!(eps < INFINITY)) flag = 1;
+    }
+    ctrl->eps[t] = eps;
+    ctrl->flag[t] = flag;
+    uint4 c0, c1v;
+    c0.x = h[0] | (static_cast<uint32_t>(h[1]) << 16);
+    c0.y = h[2] | (static_cast<uint32_t>(h[3]) << 16);
+    c0.z = h[4] | (static_cast<uint32_t>(h[5]) << 16);
+    c0.w = h[6] | (static_cast<uint32_t>(h[7]) << 16);
+    c1v.x = h[8] | (static_cast<uint32_t>(h[9]) << 16);
+    c1v.y = h[10] | (static_cast<uint32_t>(h[11]) << 16);
+    c1v.z = h[12] | (static_cast<uint32_t>(h[13]) << 16);
+    c1v.w = h[14] | (static_cast<uint32_t>(h[15]) << 16);
+    *reinterpret_cast<uint4*>(atile + enc_sw128(t, 0)) = c0;
+    *reinterpret_cast<uint4*>(atile + enc_sw128(t, 1)) = c1v;
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+  const int nq = a.kp / kEncBlockK;
+  const int ntiles = nq * 4;
+
+  if (warp == 0) {
+    if (lane == 0) {                                   // staged-book loader
+      int issued = 0;
+      for (int q = 0; q < nq; ++q) {
+        const int s = q % kEncStages;
+        const uint32_t ph = (q / kEncStages) & 1;
+        if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, a.status, kEncWaitBudget)) break;
+        mbar_arrive_expect_tx(&ctrl->full[s], kEncBlockBytes);
+        enc_bulk_load(stages + s * kEncBlockBytes, a.bprep + static_cast<size_t>(q) * kEncBlockBytes,
+                      kEncBlockBytes, &ctrl->full[s]);
+        issued = q + 1;
+      }
+      if (*abort_flag) {   // let copies already in flight land before the block exits
+        for (int q = max(0, issued - kEncStages); q < issued; ++q)
+          bounded_wait(&ctrl->full[q % kEncStages], (q / kEncStages) & 1, abort_flag, nullptr,
+                       kEncWaitBudget / 8);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {                                   // MMA issuer
+      const uint32_t idesc = f16_idesc(kEncM, kEncN);
+      const uint64_t adesc = sw128_kmajor_desc(smem_addr(atile));
+      for (int t = 0; t < ntiles; ++t) {
+        const int q = t >> 2, sl = t & 3, s = q % kEncStages;
+        if (sl == 0 && !bounded_wait(&ctrl->full[s], (q / kEncStages) & 1, abort_flag, a.status, kEncWaitBudget))
+          break;
+        const int ab = t & 1;
+        if (!bounded_wait(&ctrl->acc_empty[ab], ((t >> 1) & 1) ^ 1, abort_flag, a.status, kEncWaitBudget)) break;
+        tc_fence_after();
+        const uint32_t b = smem_addr(stages + s * kEncBlockBytes) + sl * 32;
+        umma_f16(tmem + ab * kEncN, adesc, sw128_kmajor_desc(b), idesc, 0);
+        umma_commit(&ctrl->acc_full[ab]);
+        if (sl == 3) umma_commit(&ctrl->empty[s]);
+      }
+    }
+  } else if (warp >= 4) {                              // epilogue
+    const int lq = warp & 3, cq = (warp - 4) >> 2;
+    const int row = lq * 32 + lane;
+    float best = INFINITY, second = INFINITY;
+    int arg = 0;
+    for (int t = 0; t < ntiles; ++t) {
+      const int ab = t & 1;
+      if (!bounded_wait(&ctrl->acc_full[ab], (t >> 1) & 1, abort_flag, a.status, kEncWaitBudget)) break;
+      tc_fence_after();
+      uint32_t r0[32], r1[32];
+      const uint32_t ta = tmem + (static_cast<uint32_t>(lq * 32) << 16) + ab * kEncN + cq * 64;
+      tmem_ld32(ta, r0);
+      tmem_ld32(ta + 32, r1);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctrl->acc_empty[ab]);
+      const int k0 = (t >> 2) * kEncBlockK + (t & 3) * kEncN + cq * 64;
+      enc_chunk(r0, k0, best, second, arg);
+      enc_chunk(r1, k0 + 32, best, second, arg);
+    }
+    ctrl->best[cq][row] = best;
+    ctrl->second[cq][row] = second;
+    ctrl->arg[cq][row] = arg;
+  }
+  tc_fence_before();
+  __syncthreads();
+
+  // Merge the four column quarters (in column order) and decide.
+  if (threadIdx.x < kEncM && !*abort_flag) {
+    const int t = threadIdx.x;
+    const int flag = ctrl->flag[t];
+    if (flag != 2) {
+      float b = ctrl->best[0][t], s2 = ctrl->second[0][t];
+      int k = ctrl->arg[0][t];
+#pragma unroll
+      for (int q = 1; q < 4; ++q) {
+        const float bq = ctrl->best[q][t];
+        if (bq < b) {
+          s2 = fminf(b, ctrl->second[q][t]);
+          b = bq;
+          k = ctrl->arg[q][t];
+        } else {
+          s2 = fminf(s2, bq);
+        }
+      }
+      const int64_t gv = v0 + t;
+      const int o = static_cast<int>(gv / a.nfull), j = static_cast<int>(gv % a.nfull);
+      const int64_t vid = static_cast<int64_t>(o) * a.nvec + j;
+      if (flag == 0 && k < a.K && s2 - b > 2.0f * ctrl->eps[t]) {
+        a.idx_out[vid] = static_cast<uint32_t>(k);
+      } else {
+        const int pos = atomicAdd(a.list_count, 1);
+        a.list[pos] = static_cast<int>(vid);
+      }
+    }
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The exact pass: the definition, operation by operation, in fp64.
+// ---------------------------------------------------------------------------
+struct EncExactArgs {
+  const uint16_t* w;
+  int64_t ldw;
+  int n, kin, d, nvec;
+  const uint16_t* book;
+  int K;
+  const uint16_t* book1;         // second stage: v = w - C_1[idx1] in fp64 (else null)
+  const uint32_t* idx1;
+  uint32_t* idx_out;
+  const int* list;
+  const int* list_count;
+  int partial_rows;              // n when the last vector of every row is partial, else 0
+};
+
+// Work items: the listed vectors, then the partial last vector of every row.
+// A block scans the whole book for one vector: dist(k) = sum_e (v_e - c_e)^2
+// with every difference, square and sum rounded once in fp64, e ascending;
+// the smallest dist wins, ties to the lowest k; a NaN distance never wins and
+// a vector with no finite distance gets index 0.
+__global__ void __launch_bounds__(kEncExactThreads) enc_exact_kernel(EncExactArgs a) {
+  __shared__ double sv[kEncMaxD];
+  __shared__ double rd[kEncExactThreads / 32];
+  __shared__ int rk[kEncExactThreads / 32];
+  const int nlist = *a.list_count;
+  const int nitems = nlist + a.partial_rows;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+    int o, j;
+    if (item < nlist) {
+      const int vid = a.list[item];
+      o = vid / a.nvec;
+      j = vid % a.nvec;
+    } else {
+      o = item - nlist;
+      j = a.nvec - 1;
+    }
+    const int dv = min(a.d, a.kin - j * a.d);
+    if (threadIdx.x < dv) {
+      const int e = threadIdx.x;
+      double v = static_cast<double>(h2f(a.w[static_cast<int64_t>(o) * a.ldw + static_cast<int64_t>(j) * a.d + e]));
+      if (a.book1) {
+        const int64_t i1 = a.idx1[static_cast<int64_t>(o) * a.nvec + j];
+        v = __dsub_rn(v, static_cast<double>(h2f(a.book1[i1 * a.d + e])));
+      }
+      sv[e] = v;
+    }
+    __syncthreads();
+    double best = INFINITY;
+    int arg = INT_MAX;
+    for (int k = threadIdx.x; k < a.K; k += kEncExactThreads) {
+      const uint16_t* c = a.book + static_cast<int64_t>(k) * a.d;
+      double dist = 0.0;
+      for (int e = 0; e < dv; ++e) {
+        const double t = __dsub_rn(sv[e], static_cast<double>(h2f(c[e])));
+        dist = __dadd_rn(dist, __dmul_rn(t, t));
+      }
+      if (dist < best) {           // k ascends per thread: the first minimum
+        best = dist;
+        arg = k;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const double ob = __shfl_xor_sync(0xffffffffu, best, off);
+      const int ok = __shfl_xor_sync(0xffffffffu, arg, off);
+      if (ob < best || (ob == best && ok < arg)) {
+        best = ob;
+        arg = ok;
+      }
+    }
+    if (lane == 0) {
+      rd[warp] = best;
+      rk[warp] = arg;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int w2 = 1; w2 < kEncExactThreads / 32; ++w2)
+        if (rd[w2] < best || (rd[w2] == best && rk[w2] < arg)) {
+          best = rd[w2];
+          arg = rk[w2];
+        }
+      a.idx_out[static_cast<int64_t>(o) * a.nvec + j] = arg == INT_MAX ? 0u : static_cast<uint32_t>(arg);
+    }
+    __syncthreads();               // sv, rd, rk are rewritten by the next item
+  }
+}
+
+// Row o's stream word t: the fields j whose bits [j b, j b + b) overlap
+// [32 t, 32 t + 32), LSB first; zero past the last field.
+__global__ void enc_pack_kernel(const uint32_t* __restrict__ idx, int n, int nvec, int b,
+                                uint32_t* __restrict__ out, int64_t rw) {
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (gid >= static_cast<int64_t>(n) * rw) return;
+  const int64_t o = gid / rw, t = gid % rw;
+  const int64_t bit0 = t * 32;
+  const uint32_t mask = b >= 32 ? 0xffffffffu : ((1u << b) - 1u);
+  uint32_t word = 0;
+  for (int64_t j = bit0 / b; j < nvec && j * b < bit0 + 32; ++j) {
+    const uint32_t f = idx[o * nvec + j] & mask;
+    const int64_t p = j * b - bit0;
+    word |= p >= 0 ? (f << p) : (f >> (-p));
+  }
+  out[o * rw + t] = word;
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+static_assert(sizeof(vq_encode_desc) == 88, "vq_encode_desc layout");
+
+struct EncPlan {
+  int n, kin, d, nb, nvec, nfull;
+  int b[2], K[2], kp[2];
+  int64_t nv_full;
+  size_t off_bprep[2], off_idx[2], off_list, total;
+};
+
+size_t enc_round256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Sizes and strides always; pointers only when `ptrs` (the size query takes
+// a description whose buffers do not exist yet).
+vq_status enc_check(const vq_encode_desc* e, EncPlan* p, bool ptrs) {
+  if (!e) return VQ_ERR_INVALID_ARG;
+  if (e->out_features < 0 || e->in_features < 0 || e->vec_dim < 1 || e->vec_dim > kEncMaxD ||
+      e->n_books < 1 || e->n_books > 2)
+    return VQ_ERR_INVALID_ARG;
+  p->n = e->out_features;
+  p->kin = e->in_features;
+  p->d = e->vec_dim;
+  p->nb = e->n_books;
+  p->nvec = (p->kin + p->d - 1) / p->d;
+  p->nfull = p->kin / p->d;
+  p->nv_full = static_cast<int64_t>(p->n) * p->nfull;
+  if (static_cast<int64_t>(p->n) * p->nvec >= (int64_t{1} << 31)) return VQ_ERR_UNSUPPORTED;
+  const bool data = ptrs && p->n > 0 && p->nvec > 0;
+  if (e->ldw < p->kin) return VQ_ERR_INVALID_ARG;
+  if (data && !e->w) return VQ_ERR_INVALID_ARG;
+  if (data && !aligned(e->w, 2)) return VQ_ERR_ALIGNMENT;
+  size_t off = 256;
+  for (int m = 0; m < p->nb; ++m) {
+    if (e->log2k[m] < 1 || e->log2k[m] > 16) return VQ_ERR_INVALID_ARG;
+    p->b[m] = e->log2k[m];
+    p->K[m] = 1 << p->b[m];
+    p->kp[m] = (p->K[m] + kEncBlockK - 1) / kEncBlockK * kEncBlockK;
+    const int64_t need = (static_cast<int64_t>(p->nvec) * p->b[m] + 127) / 128 * 4;
+    if (e->idx_row_words[m] < need || e->idx_row_words[m] % 4 != 0) return VQ_ERR_INVALID_ARG;
+    if (data) {
+      if (!e->codebook[m] || !e->idx[m]) return VQ_ERR_INVALID_ARG;
+      if (!aligned(e->codebook[m], 2)) return VQ_ERR_ALIGNMENT;
+      if (!aligned(e->idx[m], 16)) return VQ_ERR_ALIGNMENT;
+    }
+    p->off_bprep[m] = off;
+    off = enc_round256(off + static_cast<size_t>(p->kp[m]) * 32);
+  }
+  const size_t nv = static_cast<size_t>(p->n) * p->nvec;
+  for (int m = 0; m < p->nb; ++m) {
+    p->off_idx[m] = off;
+    off = enc_round256(off + nv * 4);
+  }
+  p->off_list = off;
+  off = enc_round256(off + nv * 4);
+  p->total = (p->n > 0 && p->nvec > 0) ? off : 0;
+  return VQ_OK;
+}
+
+}  // namespace
+}  // namespace vqk
+
+using namespace vqk;
+
+extern "C" {
+
+vq_status vq_encode_workspace_size(const vq_encode_desc* desc, size_t* bytes) {
+  if (!bytes) return VQ_ERR_INVALID_ARG;
+  EncPlan p;
+  vq_status st = enc_check(desc, &p, false);
+  if (st != VQ_OK) return st;
+  *bytes = p.total;
+  return VQ_OK;
+}
+
+vq_status vq_encode(const vq_encode_desc* desc, void* workspace, size_t workspace_bytes, void* stream_) {
+  EncPlan p;
+  vq_status st = enc_check(desc, &p, true);
+  if (st != VQ_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (p.n == 0) return VQ_OK;
+  if (p.nvec == 0) {                 // empty rows: the streams hold only padding
+    for (int m = 0; m < p.nb; ++m) {
+      if (desc->idx_row_words[m] == 0) continue;
+      if (!desc->idx[m]) return VQ_ERR_INVALID_ARG;
+      cudaError_t e = cudaMemset2DAsync(desc->idx[m], desc->idx_row_words[m] * 4, 0,
+                                        desc->idx_row_words[m] * 4, p.n, stream);
+      if (e != cudaSuccess) return cuda_status(e);
+    }
+    return VQ_OK;
+  }
+  if (!workspace || workspace_bytes < p.total) return VQ_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return VQ_ERR_ALIGNMENT;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  EncWsCtrl* wc = reinterpret_cast<EncWsCtrl*>(ws);
+  cudaError_t e = cudaMemsetAsync(ws, 0, 256, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+
+  for (int m = 0; m < p.nb; ++m) {
+    count_launch();
+    enc_book_norm_kernel<<<std::min(256, (p.K[m] + 255) / 256), 256, 0, stream>>>(
+        desc->codebook[m], p.K[m], p.d, &wc->cmax_bits[m]);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+    count_launch();
+    enc_book_prep_kernel<<<(p.kp[m] + 255) / 256, 256, 0, stream>>>(
+        desc->codebook[m], p.K[m], p.d, p.kp[m], &wc->cmax_bits[m], ws + p.off_bprep[m]);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+  }
+
+  const int smem = static_cast<int>(sizeof(EncCtrl)) + 1024 + kEncATile + kEncStages * kEncBlockBytes;
+  e = cudaFuncSetAttribute(enc_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return cuda_status(e);
+  int* list = reinterpret_cast<int*>(ws + p.off_list);
+  for (int m = 0; m < p.nb; ++m) {
+    uint32_t* idx_out = reinterpret_cast<uint32_t*>(ws + p.off_idx[m]);
+    const uint32_t* idx1 = m == 1 ? reinterpret_cast<const uint32_t*>(ws + p.off_idx[0]) : nullptr;
+    const uint16_t* book1 = m == 1 ? desc->codebook[0] : nullptr;
+    if (p.nv_full > 0) {
+      EncArgs a;
+      a.w = desc->w;
+      a.ldw = desc->ldw;
+      a.n = p.n;
+      a.kin = p.kin;
+      a.d = p.d;
+      a.nfull = p.nfull;
+      a.nvec = p.nvec;
+      a.nv_full = p.nv_full;
+      a.bprep = ws + p.off_bprep[m];
+      a.kp = p.kp[m];
+      a.K = p.K[m];
+      a.cmax_bits = &wc->cmax_bits[m];
+      a.book1 = book1;
+      a.idx1 = idx1;
+      a.idx_out = idx_out;
+      a.list = list;
+      a.list_count = &wc->list_count[m];
+      a.status = &wc->status;
+      const int64_t grid = (p.nv_full + kEncM - 1) / kEncM;
+      count_launch();
+      enc_tc_kernel<<<static_cast<unsigned>(grid), kEncThreads, smem, stream>>>(a);
+      if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+    }
+    EncExactArgs x;
+    x.w = desc->w;
+    x.ldw = desc->ldw;
+    x.n = p.n;
+    x.kin = p.kin;
+    x.d = p.d;
+    x.nvec = p.nvec;
+    x.book = desc->codebook[m];
+    x.K = p.K[m];
+    x.book1 = book1;
+    x.idx1 = idx1;
+    x.idx_out = idx_out;
+    x.list = list;
+    x.list_count = &wc->list_count[m];
+    x.partial_rows = p.nfull < p.nvec ? p.n : 0;
+    count_launch();
+    enc_exact_kernel<<<4 * device_sm_count(), kEncExactThreads, 0, stream>>>(x);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+  }
+  for (int m = 0; m < p.nb; ++m) {
+    const int64_t words = static_cast<int64_t>(p.n) * desc->idx_row_words[m];
+    count_launch();
+    enc_pack_kernel<<<static_cast<unsigned>((words + 255) / 256), 256, 0, stream>>>(
+        reinterpret_cast<const uint32_t*>(ws + p.off_idx[m]), p.n, p.nvec, p.b[m], desc->idx[m],
+        desc->idx_row_words[m]);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+  }
+  return VQ_OK;
+}
+
+}  // extern "C"

@@ -5,7 +5,7 @@ turns torch tensors into pointers, sizes and the current CUDA stream.  There
 is no fallback: if ``libvq.so`` is missing or fails to load, every call raises.
 
 Names follow the C ABI: ``dequant``, ``gemv``, ``gemm``, ``repack_tile4``,
-plus the workspace size queries.  A ``Layer`` holds the device tensors of one
+``encode``, plus the workspace size queries.  A ``Layer`` holds the device tensors of one
 quantised layer (packed index streams in row order or in the tiled order,
 fp16 codebooks, optional fp16 scale and bias).
 """
@@ -51,6 +51,16 @@ class _Desc(C.Structure):
     ]
 
 
+class _EncDesc(C.Structure):
+    _fields_ = [
+        ("out_features", C.c_int32), ("in_features", C.c_int32),
+        ("vec_dim", C.c_int32), ("n_books", C.c_int32), ("log2k", C.c_int32 * 2),
+        ("w", C.c_void_p), ("ldw", C.c_int64),
+        ("codebook", C.c_void_p * 2),
+        ("idx", C.c_void_p * 2), ("idx_row_words", C.c_int64 * 2),
+    ]
+
+
 _lock = threading.Lock()
 _lib = None
 
@@ -79,8 +89,11 @@ def lib():
             L.vq_gemm_workspace_size.argtypes = [P, I32, C.c_int, C.POINTER(SZ)]
             L.vq_gemm.argtypes = [P, P, C.c_int, I32, I64, P, C.c_int, I64, P, SZ, P]
             L.vq_repack_tile4.argtypes = [P, C.POINTER(P), C.POINTER(I64), P]
+            L.vq_encode_workspace_size.argtypes = [P, C.POINTER(SZ)]
+            L.vq_encode.argtypes = [P, P, SZ, P]
             for fn in ("vq_dequant", "vq_gemv_workspace_size", "vq_gemv", "vq_gemv_noalloc",
-                       "vq_gemm_workspace_size", "vq_gemm", "vq_repack_tile4"):
+                       "vq_gemm_workspace_size", "vq_gemm", "vq_repack_tile4",
+                       "vq_encode_workspace_size", "vq_encode"):
                 getattr(L, fn).restype = C.c_int
             L.vq_status_string.argtypes = [C.c_int]
             L.vq_status_string.restype = C.c_char_p
@@ -295,6 +308,59 @@ def gemm(layer: Layer, x: torch.Tensor, out_dtype=torch.bfloat16,
                                     _ptr(out), _DTYPE[out.dtype], ldy, _ptr(ws), ws_bytes,
                                     C.c_void_p(_stream(layer.device))))
     return out
+
+
+def row_words(in_features: int, vec_dim: int, log2k: int) -> int:
+    """Smallest row stride (32-bit words) of a row-order stream."""
+    nvec = -(-in_features // vec_dim)
+    return -(-(nvec * log2k) // 128) * 4
+
+
+def _encode_desc(w: torch.Tensor, codebooks, log2k, vec_dim: int, idx) -> _EncDesc:
+    d = _EncDesc()
+    d.out_features, d.in_features = w.shape[0], w.shape[1]
+    d.vec_dim, d.n_books = vec_dim, len(log2k)
+    d.w = w.data_ptr() if w.numel() else None
+    d.ldw = w.stride(0) if w.shape[0] > 1 else max(w.shape[1], 1)   # ldw >= Kin
+    for m, b in enumerate(log2k):
+        d.log2k[m] = b
+        d.codebook[m] = codebooks[m].data_ptr()
+        d.idx[m] = idx[m].data_ptr() if idx[m].numel() else None
+        d.idx_row_words[m] = idx[m].shape[1]
+    return d
+
+
+def encode_workspace_size(out_features: int, in_features: int, log2k: Sequence[int],
+                          vec_dim: int) -> int:
+    d = _EncDesc()
+    d.out_features, d.in_features, d.vec_dim, d.n_books = out_features, in_features, vec_dim, len(log2k)
+    d.ldw = max(in_features, 1)
+    for m, b in enumerate(log2k):
+        d.log2k[m] = int(b)
+        d.idx_row_words[m] = row_words(in_features, vec_dim, int(b))
+    n = C.c_size_t(0)
+    _check("vq_encode_workspace_size", lib().vq_encode_workspace_size(C.byref(d), C.byref(n)))
+    return n.value
+
+
+def encode(w: torch.Tensor, codebooks: Sequence[torch.Tensor], log2k: Sequence[int], vec_dim: int,
+           workspace: Optional[torch.Tensor] = None) -> Layer:
+    """Nearest-centroid encoding of W (float16 [N][Kin] on the device) against
+    one book, or two as a greedy residual cascade (vq_encode): a row-order
+    Layer holding the packed streams and the given codebooks (no scale or
+    bias)."""
+    if w.dtype != torch.float16 or w.dim() != 2 or (w.shape[0] > 1 and w.stride(1) != 1):
+        raise ValueError("w must be a row-major float16 matrix")
+    log2k = [int(b) for b in log2k]
+    books = [c.contiguous() for c in codebooks[:len(log2k)]]
+    idx = [torch.empty((w.shape[0], row_words(w.shape[1], vec_dim, b)), dtype=torch.int32,
+                       device=w.device) for b in log2k]
+    d = _encode_desc(w, books, log2k, vec_dim, idx)
+    n = C.c_size_t(0)
+    _check("vq_encode_workspace_size", lib().vq_encode_workspace_size(C.byref(d), C.byref(n)))
+    ws, ws_bytes = _workspace(n.value, w.device, workspace)
+    _check("vq_encode", lib().vq_encode(C.byref(d), _ptr(ws), ws_bytes, C.c_void_p(_stream(w.device))))
+    return Layer(w.shape[0], w.shape[1], vec_dim, log2k, idx, books)
 
 
 def kernel_launches() -> int:

@@ -76,7 +76,7 @@
 extern "C" {
 #endif
 
-#define VQ_ABI_VERSION 2
+#define VQ_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define VQ_API __attribute__((visibility("default")))
@@ -263,6 +263,69 @@ VQ_API vq_status vq_gemm_workspace_size(const vq_layer_desc* layer, int32_t m, v
 VQ_API vq_status vq_gemm(const vq_layer_desc* layer, const void* x, vq_dtype x_dtype, int32_t m,
                   int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy, void* workspace,
                   size_t workspace_bytes, void* stream);
+
+/*
+ * Nearest-centroid encoder: the step that produces the index streams.
+ *
+ * Vector j of output row o is v = W[o][j*d .. j*d+d) (the same orientation as
+ * the layer format); the last vector of a row keeps only its in_features -
+ * j*d valid components when in_features is not a multiple of d, and the
+ * distance below then runs over those components only.  For book 1,
+ *     idx_1[o][j] = argmin_k sum_e (v_e - C_1[k][e])^2,
+ * ties to the lowest k, the distance taken exactly as in fp64 (each
+ * difference, square and running sum rounded once, components in order).
+ * With two books the second index encodes the residual of the first (the
+ * greedy cascade): v_e - C_1[idx_1][e], formed in fp64, against C_2.
+ * Follows "VPTQ Guide: Extreme 2-Bit Vector Quantization", section "The
+ * Information-Theoretic Superiority of Vector Quantization" (q = argmin_k
+ * ||w - c_k||^2) and section "2. Multi-Stage Residual Vector Quantization
+ * (RVQ)" (the second stage quantises what the first leaves).
+ *
+ * Method: the tensor cores evaluate ||c||^2 - 2<v, c> for 128 vectors x 256
+ * centroids per tcgen05 MMA (fp16 operands scaled by one power of two per
+ * book, fp32 accumulation in tensor memory) and the epilogue keeps each
+ * vector's two smallest values.  Where the gap between them exceeds twice a
+ * bound on the arithmetic error, the smallest is the exact argmin; every
+ * other vector (and every partial last vector) is decided by an fp64 pass
+ * over the whole book.  The result therefore equals the exact definition.
+ *
+ *   out_features, in_features   N, Kin >= 0
+ *   vec_dim        d, 1..14
+ *   n_books        1 or 2;  log2k[m] in 1..16
+ *   w, ldw         device fp16 [N][ldw], ldw >= Kin, finite values
+ *   codebook[m]    device fp16 [K_m][d], finite values
+ *   idx[m], idx_row_words[m]   device output streams in row order (the layer
+ *                  format above): 16-byte aligned, idx_row_words[m] a multiple
+ *                  of 4 and >= ceil(nvec*b_m/128)*4; every word of the N rows
+ *                  is written (fields, then zero padding)
+ */
+typedef struct vq_encode_desc {
+    int32_t out_features;
+    int32_t in_features;
+    int32_t vec_dim;
+    int32_t n_books;
+    int32_t log2k[2];
+    const uint16_t* w;
+    int64_t ldw;
+    const uint16_t* codebook[2];
+    uint32_t* idx[2];
+    int64_t idx_row_words[2];
+} vq_encode_desc;
+
+/* Bytes of device workspace vq_encode needs (host-only, launches nothing;
+ * only the sizes and strides of desc are read). */
+VQ_API vq_status vq_encode_workspace_size(const vq_encode_desc* desc, size_t* bytes);
+
+/*
+ * vq_encode -- run the encoder above on `stream`.  workspace: device,
+ * 256-byte aligned, at least vq_encode_workspace_size() bytes; its first
+ * 32-bit word is a status word (VQ_OK, or VQ_ERR_TIMEOUT if a bounded
+ * device-side wait gave up), readable after the stream completes.
+ * Errors: VQ_ERR_INVALID_ARG (sizes, NULL pointers with data, short strides),
+ * VQ_ERR_ALIGNMENT, VQ_ERR_WORKSPACE, VQ_ERR_CUDA.
+ */
+VQ_API vq_status vq_encode(const vq_encode_desc* desc, void* workspace, size_t workspace_bytes,
+                           void* stream);
 
 /* Static description of a status code (never NULL). */
 VQ_API const char* vq_status_string(vq_status status);

@@ -174,6 +174,18 @@ def make_x(seed: int, rows: int, in_features: int, outlier_frac: float = 0.0,
 # "Configuration Sizing Matrix across Model Architectures").
 # --------------------------------------------------------------------------
 
+def make_encode_input(out_features: int, in_features: int, d: int, log2k: Sequence[int],
+                      book_std: Sequence[float], seed: int, w_std: float = 0.02):
+    """Inputs of the nearest-centroid encoder: fp16 bits of a weight matrix
+    W [N][Kin] ~ N(0, w_std) and of one codebook [K_m][d] ~ N(0, std_m) per
+    entry of log2k (unique rows).  Draw order: books, then W."""
+    rng = np.random.default_rng(seed)
+    books = [_draw_book(rng, 1 << b, d, s) for b, s in zip(log2k, book_std)]
+    w = to_f16_bits(rng.standard_normal((out_features, in_features), dtype=np.float32)
+                    * np.float32(w_std)).reshape(out_features, in_features)
+    return w, books
+
+
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str

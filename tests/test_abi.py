@@ -18,14 +18,15 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(names) == {"vq_dequant", "vq_repack_tile4", "vq_gemv_workspace_size", "vq_gemv",
                           "vq_gemv_noalloc", "vq_gemm_workspace_size", "vq_gemm",
                           "vq_status_string", "vq_last_cuda_error", "vq_abi_version",
-                          "vq_kernel_launches"}
+                          "vq_kernel_launches", "vq_encode_workspace_size", "vq_encode"}
     for n in names:
         assert hasattr(lib, n), n
 
 
 def test_host_only_calls(lib):
-    assert lib.vq_abi_version() == 2
+    assert lib.vq_abi_version() == 3
     assert C.sizeof(vq._Desc) == 96       # static_assert'ed in the library
+    assert C.sizeof(vq._EncDesc) == 88
     assert vq.kernel_launches() == 0          # nothing launched in this process
     for s in range(7):
         assert lib.vq_status_string(s)
@@ -129,3 +130,38 @@ def test_table_batch_limit_needs_no_device(lib, monkeypatch):
     monkeypatch.setenv("VQ_LUT_MAX_BATCH", "0")
     assert lib.vq_gemv_workspace_size(C.byref(d), 1, C.byref(n)) == vq.VQ_OK
     assert not table(n.value)
+
+
+def test_encode_workspace_and_validation_need_no_device(lib):
+    """vq_encode_workspace_size: control words + each prepared book (K padded to
+    1024, 32 bytes per centroid) + unpacked indices per book + the exact-pass
+    list, each rounded up to 256 bytes; malformed descriptions are rejected
+    before any CUDA call."""
+    r256 = lambda x: -(-x // 256) * 256
+    n, kin, d = 300, 8 * 100 + 5, 8
+    nvec = -(-kin // d)
+    got = vq.encode_workspace_size(n, kin, [16, 4], d)
+    want = 256 + r256(65536 * 32) + r256(1024 * 32) + 3 * r256(n * nvec * 4)
+    assert got == want
+    assert vq.encode_workspace_size(0, kin, [16], d) == 0
+    assert vq.encode_workspace_size(n, 0, [16], d) == 0
+    e = vq._EncDesc()
+    e.out_features, e.in_features, e.vec_dim, e.n_books = 4, 16, 8, 1
+    e.log2k[0] = 8
+    e.ldw = 16
+    e.idx_row_words[0] = 4
+    n_ = C.c_size_t(0)
+    assert lib.vq_encode_workspace_size(C.byref(e), C.byref(n_)) == vq.VQ_OK
+    for field, bad in (("vec_dim", 15), ("vec_dim", 0), ("n_books", 3), ("ldw", 15)):
+        old = getattr(e, field)
+        setattr(e, field, bad)
+        assert lib.vq_encode_workspace_size(C.byref(e), C.byref(n_)) == vq.VQ_ERR_INVALID_ARG, field
+        setattr(e, field, old)
+    e.log2k[0] = 17
+    assert lib.vq_encode_workspace_size(C.byref(e), C.byref(n_)) == vq.VQ_ERR_INVALID_ARG
+    e.log2k[0] = 8
+    e.idx_row_words[0] = 2                       # short and not a multiple of 4
+    assert lib.vq_encode_workspace_size(C.byref(e), C.byref(n_)) == vq.VQ_ERR_INVALID_ARG
+    e.idx_row_words[0] = 4
+    # vq_encode itself: NULL buffers with data are rejected before any launch
+    assert lib.vq_encode(C.byref(e), None, 0, None) == vq.VQ_ERR_INVALID_ARG
