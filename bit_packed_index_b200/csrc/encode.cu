@@ -67,9 +67,11 @@ struct EncCtrl {
   int abort_flag;
   float eps[kEncM];              // error bound of each vector's bracket values
   int flag[kEncM];               // 0: decide here, 1: exact pass, 2: no vector
-  float best[4][kEncM];          // per column quarter: smallest value,
-  float second[4][kEncM];        //   second smallest,
-  int arg[4][kEncM];             //   column of the smallest
+  float best[4][kEncM];          // per column quarter: smallest bracket value,
+  float second[4][kEncM];        //   smallest chunk minimum of the other chunks,
+  int chunk[4][kEncM];           //   first centroid of the chunk holding the smallest
+  double v[kEncM][kEncMaxD];     // the vectors, exactly (fp64)
+  double vnorm[kEncM];           // ||v||^2 (fp64)
 };
 
 // Workspace control words (first 256 bytes).
@@ -168,6 +170,12 @@ __global__ void enc_book_prep_kernel(const uint16_t* __restrict__ book, int K, i
   *reinterpret_cast<uint4*>(base + enc_sw128(r, 2 * sl + 1)) = c1;
 }
 
+// The book in fp64 (exact), for the exact distances.
+__global__ void enc_book64_kernel(const uint16_t* __restrict__ book, int64_t count, double* __restrict__ out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < count) out[i] = static_cast<double>(h2f(book[i]));
+}
+
 // ---------------------------------------------------------------------------
 // The tensor-core pass.
 // ---------------------------------------------------------------------------
@@ -179,6 +187,7 @@ struct EncArgs {
   const uint8_t* bprep;
   int kp, K;                     // padded and real book size
   const unsigned* cmax_bits;
+  const double* book64;          // the book in fp64 [K][d]
   const uint16_t* book1;         // second stage: v = w - C_1[idx1] (else null)
   const uint32_t* idx1;
   uint32_t* idx_out;             // [n][nvec]
@@ -187,36 +196,41 @@ struct EncArgs {
   int* status;
 };
 
-// One 32-column chunk of bracket values for centroids k0 .. k0+31: running
-// smallest value, its centroid and the second smallest value.
-__device__ __forceinline__ void enc_chunk(const uint32_t (&r)[32], int k0, float& best, float& second,
-                                          int& arg) {
-  float m[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    m[i] = fminf(fminf(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1])),
-                 fminf(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
-  const float mn = fminf(fminf(fminf(m[0], m[1]), fminf(m[2], m[3])), fminf(fminf(m[4], m[5]), fminf(m[6], m[7])));
-  if (mn < best) {                 // rare after the first chunks: find the column and the runner-up
-    int pos = 0;
-    bool found = false;
-    float s2 = INFINITY;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float v = __uint_as_float(r[i]);
-      if (!found && v == mn) {
-        pos = i;
-        found = true;
-      } else {
-        s2 = fminf(s2, v);
-      }
-    }
-    second = fminf(best, s2);
-    best = mn;
-    arg = k0 + pos;
-  } else {
-    second = fminf(second, mn);
+// sum_e (v_e - c_e)^2 with each difference, square and sum rounded once in
+// fp64, e ascending: the distance of the definition.
+__device__ __forceinline__ double enc_dist64(const double* v, const double* c, int d) {
+  double dist = 0.0;
+  for (int e = 0; e < d; ++e) {
+    const double t = __dsub_rn(v[e], c[e]);
+    dist = __dadd_rn(dist, __dmul_rn(t, t));
   }
+  return dist;
+}
+
+// One 32-column chunk of bracket values for centroids k0 .. k0+31: the
+// running smallest value, the first centroid of the chunk that holds it, and
+// the smallest chunk minimum among all other chunks.  Which column of the
+// best chunk holds the minimum is settled later, exactly.
+__device__ __forceinline__ float enc_min3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ void enc_chunk(const uint32_t (&r)[32], int k0, float& best, float& second,
+                                          int& chunk) {
+  float m[12];
+#pragma unroll
+  for (int i = 0; i < 10; ++i)
+    m[i] = enc_min3(__uint_as_float(r[3 * i]), __uint_as_float(r[3 * i + 1]), __uint_as_float(r[3 * i + 2]));
+  m[10] = __uint_as_float(r[30]);
+  m[11] = __uint_as_float(r[31]);
+  const float mn = fminf(enc_min3(enc_min3(m[0], m[1], m[2]), enc_min3(m[3], m[4], m[5]), enc_min3(m[6], m[7], m[8])),
+                         enc_min3(m[9], m[10], m[11]));
+  const bool p = mn < best;
+  second = p ? best : fminf(second, mn);
+  best = p ? mn : best;
+  chunk = p ? k0 : chunk;
 }
 
 __global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
@@ -271,7 +285,12 @@ __global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
       const uint16_t* c1 = a.book1 ? a.book1 + static_cast<int64_t>(a.idx1[static_cast<int64_t>(o) * a.nvec + j]) * a.d
                                    : nullptr;
       float n2 = 0.0f, l1 = 0.0f, dl = 0.0f;
+      double vn = 0.0;
       for (int e = 0; e < a.d; ++e) {
+        double ve = static_cast<double>(h2f(wr[e]));
+        if (c1) ve = __dsub_rn(ve, static_cast<double>(h2f(c1[e])));
+        ctrl->v[t][e] = ve;
+        vn = __dadd_rn(vn, __dmul_rn(ve, ve));
         float v = h2f(wr[e]);
         if (c1) v = __fsub_rn(v, h2f(c1[e]));
         const float vs = v * f;                      // exact: a power-of-two scale in range
@@ -283,6 +302,7 @@ __global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
         l1 += fabsf(vt);
         dl += fabsf(vt - vs) + fabsf(vs) * 0x1p-22f + 0x1p-24f;
       }
+      ctrl->vnorm[t] = vn;
       h[a.d] = 0x3C00u;                              // 1.0 (times hi)
       h[a.d + 1] = 0x3C00u;                          // 1.0 (times lo)
       const float cs = cmax * f * f;
@@ -351,7 +371,7 @@ __global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
     const int lq = warp & 3, cq = (warp - 4) >> 2;
     const int row = lq * 32 + lane;
     float best = INFINITY, second = INFINITY;
-    int arg = 0;
+    int chunk = 0;
     for (int t = 0; t < ntiles; ++t) {
       const int ab = t & 1;
       if (!bounded_wait(&ctrl->acc_full[ab], (t >> 1) & 1, abort_flag, a.status, kEncWaitBudget)) break;
@@ -365,40 +385,87 @@ __global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctrl->acc_empty[ab]);
       const int k0 = (t >> 2) * kEncBlockK + (t & 3) * kEncN + cq * 64;
-      enc_chunk(r0, k0, best, second, arg);
-      enc_chunk(r1, k0 + 32, best, second, arg);
+      enc_chunk(r0, k0, best, second, chunk);
+      enc_chunk(r1, k0 + 32, best, second, chunk);
     }
     ctrl->best[cq][row] = best;
     ctrl->second[cq][row] = second;
-    ctrl->arg[cq][row] = arg;
+    ctrl->chunk[cq][row] = chunk;
   }
   tc_fence_before();
   __syncthreads();
 
-  // Merge the four column quarters (in column order) and decide.
-  if (threadIdx.x < kEncM && !*abort_flag) {
+  // Merge the four column quarters: the best chunk overall and the smallest
+  // value outside it (quarter order breaks ties; a tie leaves no margin).
+  const bool live = !*abort_flag;
+  if (threadIdx.x < kEncM && live && ctrl->flag[threadIdx.x] == 0) {
+    const int t = threadIdx.x;
+    float b = ctrl->best[0][t], s2 = ctrl->second[0][t];
+    int c0 = ctrl->chunk[0][t];
+#pragma unroll
+    for (int q = 1; q < 4; ++q) {
+      const float bq = ctrl->best[q][t];
+      if (bq < b) {
+        s2 = fminf(fminf(s2, b), ctrl->second[q][t]);
+        b = bq;
+        c0 = ctrl->chunk[q][t];
+      } else {
+        s2 = fminf(fminf(s2, bq), ctrl->second[q][t]);
+      }
+    }
+    ctrl->second[0][t] = s2;
+    ctrl->chunk[0][t] = c0;
+  }
+  __syncthreads();
+  // The 32 centroids of each vector's best chunk, exactly (fp64, the
+  // definition's operation order); the staged-book buffers hold the results.
+  double* ex = reinterpret_cast<double*>(stages);       // [kEncM][32]
+  if (live) {
+    for (int p = threadIdx.x; p < kEncM * 32; p += kEncThreads) {
+      const int t = p >> 5, c = p & 31;
+      double e = INFINITY;
+      if (ctrl->flag[t] == 0) {
+        const int k = ctrl->chunk[0][t] + c;
+        if (k < a.K) e = enc_dist64(ctrl->v[t], a.book64 + static_cast<int64_t>(k) * a.d, a.d);
+      }
+      ex[p] = e;
+    }
+  }
+  __syncthreads();
+  // Decide: if every centroid outside the chunk is provably farther than the
+  // chunk's exact minimum, that minimum (lowest k on ties) is the answer.
+  //   outside:  D(k) >= second  =>  exact bracket >= second - eps
+  //   inside:   exact bracket of the best = (dist - ||v||^2) 4^s
+  if (threadIdx.x < kEncM && live) {
     const int t = threadIdx.x;
     const int flag = ctrl->flag[t];
     if (flag != 2) {
-      float b = ctrl->best[0][t], s2 = ctrl->second[0][t];
-      int k = ctrl->arg[0][t];
-#pragma unroll
-      for (int q = 1; q < 4; ++q) {
-        const float bq = ctrl->best[q][t];
-        if (bq < b) {
-          s2 = fminf(b, ctrl->second[q][t]);
-          b = bq;
-          k = ctrl->arg[q][t];
-        } else {
-          s2 = fminf(s2, bq);
-        }
-      }
       const int64_t gv = v0 + t;
       const int o = static_cast<int>(gv / a.nfull), j = static_cast<int>(gv % a.nfull);
       const int64_t vid = static_cast<int64_t>(o) * a.nvec + j;
-      if (flag == 0 && k < a.K && s2 - b > 2.0f * ctrl->eps[t]) {
-        a.idx_out[vid] = static_cast<uint32_t>(k);
-      } else {
+      bool done = false;
+      if (flag == 0) {
+        double emin = INFINITY;
+        int kmin = -1;
+        for (int c = 0; c < 32; ++c) {
+          const double e = ex[t * 32 + c];
+          if (e < emin) {
+            emin = e;
+            kmin = ctrl->chunk[0][t] + c;
+          }
+        }
+        if (kmin >= 0) {
+          const int se2 = 2 * enc_scale_exp(__uint_as_float(*a.cmax_bits));   // 4^s as a double
+          const double s4 = __longlong_as_double(static_cast<long long>(1023 + se2) << 52);
+          const double dex = (emin - ctrl->vnorm[t]) * s4;
+          const double slack = 0x1p-40 * (fabs(emin) + ctrl->vnorm[t]) * s4;
+          if (static_cast<double>(ctrl->second[0][t]) - dex > static_cast<double>(ctrl->eps[t]) + slack) {
+            a.idx_out[vid] = static_cast<uint32_t>(kmin);
+            done = true;
+          }
+        }
+      }
+      if (!done) {
         const int pos = atomicAdd(a.list_count, 1);
         a.list[pos] = static_cast<int>(vid);
       }
@@ -417,7 +484,7 @@ struct EncExactArgs {
   const uint16_t* w;
   int64_t ldw;
   int n, kin, d, nvec;
-  const uint16_t* book;
+  const double* book64;          // the book in fp64 [K][d]
   int K;
   const uint16_t* book1;         // second stage: v = w - C_1[idx1] in fp64 (else null)
   const uint32_t* idx1;
@@ -428,50 +495,71 @@ struct EncExactArgs {
 };
 
 // Work items: the listed vectors, then the partial last vector of every row.
-// A block scans the whole book for one vector: dist(k) = sum_e (v_e - c_e)^2
-// with every difference, square and sum rounded once in fp64, e ascending;
-// the smallest dist wins, ties to the lowest k; a NaN distance never wins and
-// a vector with no finite distance gets index 0.
+// A block takes eight items, one per warp, and streams the book through
+// shared memory in tiles of 512 fp64 centroids (stored component-major, so a
+// warp's loads are consecutive) that all eight warps scan, the lanes of a
+// warp striding over the tile.  dist(k) = sum_e (v_e - c_e)^2 with
+// every difference, square and sum rounded once in fp64, e ascending; the
+// smallest dist wins, ties to the lowest k; a NaN distance never wins and a
+// vector with no finite distance gets index 0.
+constexpr int kEncExactTile = 512;
+
 __global__ void __launch_bounds__(kEncExactThreads) enc_exact_kernel(EncExactArgs a) {
-  __shared__ double sv[kEncMaxD];
-  __shared__ double rd[kEncExactThreads / 32];
-  __shared__ int rk[kEncExactThreads / 32];
+  constexpr int NW = kEncExactThreads / 32;
+  extern __shared__ double tile[];                 // [d][kEncExactTile]
   const int nlist = *a.list_count;
   const int nitems = nlist + a.partial_rows;
+  const int ngroups = (nitems + NW - 1) / NW;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
-    int o, j;
-    if (item < nlist) {
-      const int vid = a.list[item];
-      o = vid / a.nvec;
-      j = vid % a.nvec;
-    } else {
-      o = item - nlist;
-      j = a.nvec - 1;
-    }
-    const int dv = min(a.d, a.kin - j * a.d);
-    if (threadIdx.x < dv) {
-      const int e = threadIdx.x;
-      double v = static_cast<double>(h2f(a.w[static_cast<int64_t>(o) * a.ldw + static_cast<int64_t>(j) * a.d + e]));
-      if (a.book1) {
-        const int64_t i1 = a.idx1[static_cast<int64_t>(o) * a.nvec + j];
-        v = __dsub_rn(v, static_cast<double>(h2f(a.book1[i1 * a.d + e])));
+  for (int grp = blockIdx.x; grp < ngroups; grp += gridDim.x) {
+    const int item = grp * NW + warp;
+    const bool has = item < nitems;
+    int o = 0, j = 0;
+    if (has) {
+      if (item < nlist) {
+        const int vid = a.list[item];
+        o = vid / a.nvec;
+        j = vid % a.nvec;
+      } else {
+        o = item - nlist;
+        j = a.nvec - 1;
       }
-      sv[e] = v;
     }
-    __syncthreads();
+    const int dv = has ? min(a.d, a.kin - j * a.d) : 0;
+    const int64_t vid = static_cast<int64_t>(o) * a.nvec + j;
+    double v[kEncMaxD];
+#pragma unroll
+    for (int e = 0; e < kEncMaxD; ++e) {
+      v[e] = 0.0;
+      if (e < dv) {
+        v[e] = static_cast<double>(h2f(a.w[static_cast<int64_t>(o) * a.ldw + static_cast<int64_t>(j) * a.d + e]));
+        if (a.book1)
+          v[e] = __dsub_rn(v[e], static_cast<double>(h2f(a.book1[static_cast<int64_t>(a.idx1[vid]) * a.d + e])));
+      }
+    }
     double best = INFINITY;
     int arg = INT_MAX;
-    for (int k = threadIdx.x; k < a.K; k += kEncExactThreads) {
-      const uint16_t* c = a.book + static_cast<int64_t>(k) * a.d;
-      double dist = 0.0;
-      for (int e = 0; e < dv; ++e) {
-        const double t = __dsub_rn(sv[e], static_cast<double>(h2f(c[e])));
-        dist = __dadd_rn(dist, __dmul_rn(t, t));
-      }
-      if (dist < best) {           // k ascends per thread: the first minimum
-        best = dist;
-        arg = k;
+    for (int k0 = 0; k0 < a.K; k0 += kEncExactTile) {
+      const int nk = min(kEncExactTile, a.K - k0);
+      __syncthreads();                             // the previous tile is consumed
+      for (int i = threadIdx.x; i < nk * a.d; i += kEncExactThreads)   // transposed: tile[e][kk]
+        tile[(i % a.d) * kEncExactTile + i / a.d] = a.book64[static_cast<int64_t>(k0) * a.d + i];
+      __syncthreads();
+      if (has) {
+        for (int kk = lane; kk < nk; kk += 32) {
+          double dist = 0.0;
+#pragma unroll
+          for (int e = 0; e < kEncMaxD; ++e) {
+            if (e < dv) {
+              const double t = __dsub_rn(v[e], tile[e * kEncExactTile + kk]);
+              dist = __dadd_rn(dist, __dmul_rn(t, t));
+            }
+          }
+          if (dist < best) {       // k ascends per lane: the first minimum
+            best = dist;
+            arg = k0 + kk;
+          }
+        }
       }
     }
 #pragma unroll
@@ -483,20 +571,7 @@ __global__ void __launch_bounds__(kEncExactThreads) enc_exact_kernel(EncExactArg
         arg = ok;
       }
     }
-    if (lane == 0) {
-      rd[warp] = best;
-      rk[warp] = arg;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      for (int w2 = 1; w2 < kEncExactThreads / 32; ++w2)
-        if (rd[w2] < best || (rd[w2] == best && rk[w2] < arg)) {
-          best = rd[w2];
-          arg = rk[w2];
-        }
-      a.idx_out[static_cast<int64_t>(o) * a.nvec + j] = arg == INT_MAX ? 0u : static_cast<uint32_t>(arg);
-    }
-    __syncthreads();               // sv, rd, rk are rewritten by the next item
+    if (has && lane == 0) a.idx_out[vid] = arg == INT_MAX ? 0u : static_cast<uint32_t>(arg);
   }
 }
 
@@ -527,7 +602,7 @@ struct EncPlan {
   int n, kin, d, nb, nvec, nfull;
   int b[2], K[2], kp[2];
   int64_t nv_full;
-  size_t off_bprep[2], off_idx[2], off_list, total;
+  size_t off_bprep[2], off_book64[2], off_idx[2], off_list, total;
 };
 
 size_t enc_round256(size_t x) { return (x + 255) / 256 * 256; }
@@ -566,6 +641,8 @@ vq_status enc_check(const vq_encode_desc* e, EncPlan* p, bool ptrs) {
     }
     p->off_bprep[m] = off;
     off = enc_round256(off + static_cast<size_t>(p->kp[m]) * 32);
+    p->off_book64[m] = off;
+    off = enc_round256(off + static_cast<size_t>(p->K[m]) * p->d * 8);
   }
   const size_t nv = static_cast<size_t>(p->n) * p->nvec;
   for (int m = 0; m < p->nb; ++m) {
@@ -626,6 +703,11 @@ vq_status vq_encode(const vq_encode_desc* desc, void* workspace, size_t workspac
     enc_book_prep_kernel<<<(p.kp[m] + 255) / 256, 256, 0, stream>>>(
         desc->codebook[m], p.K[m], p.d, p.kp[m], &wc->cmax_bits[m], ws + p.off_bprep[m]);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+    const int64_t cnt = static_cast<int64_t>(p.K[m]) * p.d;
+    count_launch();
+    enc_book64_kernel<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, stream>>>(
+        desc->codebook[m], cnt, reinterpret_cast<double*>(ws + p.off_book64[m]));
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   }
 
   const int smem = static_cast<int>(sizeof(EncCtrl)) + 1024 + kEncATile + kEncStages * kEncBlockBytes;
@@ -650,6 +732,7 @@ vq_status vq_encode(const vq_encode_desc* desc, void* workspace, size_t workspac
       a.kp = p.kp[m];
       a.K = p.K[m];
       a.cmax_bits = &wc->cmax_bits[m];
+      a.book64 = reinterpret_cast<const double*>(ws + p.off_book64[m]);
       a.book1 = book1;
       a.idx1 = idx1;
       a.idx_out = idx_out;
@@ -668,7 +751,7 @@ vq_status vq_encode(const vq_encode_desc* desc, void* workspace, size_t workspac
     x.kin = p.kin;
     x.d = p.d;
     x.nvec = p.nvec;
-    x.book = desc->codebook[m];
+    x.book64 = reinterpret_cast<const double*>(ws + p.off_book64[m]);
     x.K = p.K[m];
     x.book1 = book1;
     x.idx1 = idx1;
@@ -677,7 +760,13 @@ vq_status vq_encode(const vq_encode_desc* desc, void* workspace, size_t workspac
     x.list_count = &wc->list_count[m];
     x.partial_rows = p.nfull < p.nvec ? p.n : 0;
     count_launch();
-    enc_exact_kernel<<<4 * device_sm_count(), kEncExactThreads, 0, stream>>>(x);
+    const int xsmem = kEncExactTile * p.d * static_cast<int>(sizeof(double));
+    if (m == 0) {
+      e = cudaFuncSetAttribute(enc_exact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kEncExactTile * kEncMaxD * static_cast<int>(sizeof(double)));
+      if (e != cudaSuccess) return cuda_status(e);
+    }
+    enc_exact_kernel<<<2 * device_sm_count(), kEncExactThreads, xsmem, stream>>>(x);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   }
   for (int m = 0; m < p.nb; ++m) {

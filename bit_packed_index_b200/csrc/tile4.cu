@@ -228,11 +228,6 @@ constexpr int kLutSlices = (65536 + kLutS - 1) / kLutS;   // 3 slices of the 2^1
 constexpr int kLutSmem = kLutS * kLutNJ * 2;        // T[S][4] in fp16: 192 KB
 constexpr int kLutPD = 4;                           // 32-centroid tiles per load batch
 
-__device__ __forceinline__ uint32_t ldg_stream32(const void* p) {
-  uint32_t v;
-  asm volatile("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(v) : "l"(p));
-  return v;
-}
 __device__ __forceinline__ uint2 ldg_stream64(const void* p) {
   uint2 v;
   asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));

@@ -133,15 +133,17 @@ def test_table_batch_limit_needs_no_device(lib, monkeypatch):
 
 
 def test_encode_workspace_and_validation_need_no_device(lib):
-    """vq_encode_workspace_size: control words + each prepared book (K padded to
-    1024, 32 bytes per centroid) + unpacked indices per book + the exact-pass
-    list, each rounded up to 256 bytes; malformed descriptions are rejected
-    before any CUDA call."""
+    """vq_encode_workspace_size: control words + per book the prepared operand
+    (K padded to 1024, 32 bytes per centroid) and the fp64 copy (8 bytes per
+    component) + unpacked indices per book + the exact-pass list, each rounded
+    up to 256 bytes; malformed descriptions are rejected before any CUDA
+    call."""
     r256 = lambda x: -(-x // 256) * 256
     n, kin, d = 300, 8 * 100 + 5, 8
     nvec = -(-kin // d)
     got = vq.encode_workspace_size(n, kin, [16, 4], d)
-    want = 256 + r256(65536 * 32) + r256(1024 * 32) + 3 * r256(n * nvec * 4)
+    want = (256 + r256(65536 * 32) + r256(65536 * d * 8) + r256(1024 * 32) + r256(16 * d * 8)
+            + 3 * r256(n * nvec * 4))
     assert got == want
     assert vq.encode_workspace_size(0, kin, [16], d) == 0
     assert vq.encode_workspace_size(n, 0, [16], d) == 0
