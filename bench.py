@@ -19,6 +19,8 @@ e2e    = the same metric through the public Python API with the activations
          layer and copies y back.
 gemm   = the prefill GEMM (x [2048, 8192] bf16, 8192 x 8192 layer, K = 2^16
          + residual K = 2^8, 3.0 bpw) through vq_gemm, in TFLOP/s.
+encode = the nearest-centroid encoder (vq_encode) on a 4096 x 4096 matrix
+         against one K = 2^16, d = 8 book, in (vector, centroid) pairs/s.
 roofline, cpu_baseline, clocks and gpu_launches are described beside the
 keys they fill.  ``--impl reference`` times the CPU oracle on the same
 metric instead (a bounded sample of the same workload per step).
@@ -399,6 +401,8 @@ def run_gpu(args):
 
     gemm = run_gemm(dev, peaks, peak_src, vq)
     decode_405b = run_decode_405b(dev, peaks, peak_src, vq)
+    encode = run_encode(dev, peaks, peak_src, vq,
+                        with_oracle=rank == 0 and world == 1 and not args.no_cpu_baseline)
 
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -414,6 +418,7 @@ def run_gpu(args):
         "clocks": clocks.summary(),
         "gemm": gemm,
         "decode_405b_gate": decode_405b,
+        "encode": encode,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gbs, rows, dt, cores = oracle_rate(10.0, w.layers, xs_host)
@@ -492,6 +497,62 @@ def run_decode_405b(dev, peaks, peak_src, vq):
                         "B=1, tiled index order (small-book lookup-table kernel)",
             "us": ms * 1e3, "achieved_gbs": gbs, "frac_of_measured_hbm": gbs / peaks["hbm_gbs"],
             "algorithmic_bytes": alg_bytes(spec, 1), "peak_source": peak_src}
+
+
+def run_encode(dev, peaks, peak_src, vq, with_oracle: bool):
+    """Beside the headline: the nearest-centroid encoder (vq_encode) on a
+    4096 x 4096 fp16 matrix against one K = 2^16, d = 8 book (2M vectors x
+    65536 centroids), L2 flushed between timed calls; the oracle's brute force
+    on a sample of the same vectors for scale."""
+    import torch
+    n, kin, d, log2k = ENCODE_SHAPE
+    w, books = synth.make_encode_input(n, kin, d, log2k, ENCODE_STD, seed=ENCODE_SEED)
+    W = torch.from_numpy(w.view(np.int16)).to(dev).view(torch.float16)
+    B = [torch.from_numpy(b.view(np.int16)).to(dev).view(torch.float16) for b in books]
+    ws = torch.empty(vq.encode_workspace_size(n, kin, log2k, d), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        vq.encode(W, B, log2k, d, workspace=ws)
+    times = []
+    for _ in range(5):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        vq.encode(W, B, log2k, d, workspace=ws)
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    ctrl = ws[:16].view(torch.int32).cpu().numpy()
+    ms = statistics.median(times)
+    nv = n * (kin // d)
+    pairs = nv * sum(1 << b for b in log2k)
+    rate = pairs / (ms * 1e-3)
+    # ALU roofline: one minimum operation per (vector, centroid) pair at full
+    # issue on every SM sub-partition (148 SMs x 4 x 32 lanes x max SM clock).
+    alu_peak = 148 * 4 * 32 * 1.965e9
+    out = {"workload": f"encode {n}x{kin} fp16 W ~ N(0, {ENCODE_STD[0]}), d={d}, one K=2^{log2k[0]} book: "
+                       f"{nv} vectors x {1 << log2k[0]} centroids",
+           "ms": ms, "pairs_per_s": rate, "device_status": int(ctrl[0]),
+           "exact_pass_vectors": int(ctrl[1]), "exact_pass_share": int(ctrl[1]) / nv,
+           "roofline": {"bound": "alu", "achieved": rate, "peak": alu_peak, "unit": "pairs/s",
+                        "frac": rate / alu_peak,
+                        "peak_source": "derived: one ALU operation per pair at full issue, "
+                                       "148 SMs x 128 lanes x 1965 MHz"},
+           "tensor_tflops": 2.0 * d * pairs / (ms * 1e-3) / 1e12}
+    if not with_oracle:
+        return out
+    # CPU baseline: the oracle on a bounded sample of the same vectors (host cores)
+    import oracle
+    import time as _time
+    sample = 256
+    v = oracle.f16_to_f32(w[:sample * d // kin + 1]).astype(np.float64).reshape(-1, d)[:sample]
+    t0 = _time.perf_counter()
+    oracle.encode(v, books[0])
+    dt = _time.perf_counter() - t0
+    out["cpu_baseline"] = {"value": sample * (1 << log2k[0]) / dt, "unit": "pairs/s",
+                           "cores": oracle.num_threads(), "kind": "oracle",
+                           "sample": f"{sample} vectors x {1 << log2k[0]} centroids, {dt:.2f} s"}
+    return out
 
 
 def run_profile(args):
