@@ -310,11 +310,23 @@ __device__ __forceinline__ void lut_pair_afr(const uint16_t* __restrict__ bslice
   afr[3] = r1.y;   // row n+8, k = 2t+8, 2t+9
 }
 
-// RB8 batches of 8 rows per thread: a block covers N <= 8 * RB8 * 1024 rows;
-// thread (warp w, lane l) keeps its row sums in TMEM lane 32*(w%4)+l, columns
-// (w/4)*8*RB8 .. +8*RB8 (warps may only touch their own quarter of the lanes).
-template <int RB8>
-__global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const uint16_t* __restrict__ x,
+// One or more layers that share x (the projections of one block), run as one
+// task list.  Layer l's rows occupy the 8192-row batches l*LB .. l*LB+LB-1 of
+// the block's row sums, so a batch never mixes layers.
+constexpr int kLutMaxLayers = 4;
+struct LutSet {
+  Layer L[kLutMaxLayers];
+  int nl;
+  int row0[kLutMaxLayers + 1];   // first row of each layer in the partial sums; row0[nl] = rows
+};
+
+// RB8 batches of 8 rows per thread (all layers together): a block covers
+// 8 * RB8 * 1024 rows; thread (warp w, lane l) keeps its row sums in TMEM lane
+// 32*(w%4)+l, columns (w/4)*8*RB8 .. +8*RB8 (warps may only touch their own
+// quarter of the lanes).  Tasks: (group of four vectors, layer, slice), the
+// three slices of one layer and group consecutive.
+template <int RB8, int LB>
+__global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(LutSet S, const uint16_t* __restrict__ x,
                                                                   int x_fp16, float* __restrict__ part,
                                                                   float* __restrict__ xpart) {
   constexpr int CPW = 8 * RB8;                      // TMEM columns per group of 4 warps
@@ -328,8 +340,11 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
   __shared__ uint32_t s_tmem;
   __shared__ float s_scale;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int n = L.n, kin = L.kin;
-  const int ntasks = ((L.nvec + kLutNJ - 1) / kLutNJ) * kLutSlices;
+  constexpr bool MULTI = LB < RB8;                  // several layers, LB batches each
+  const int kin = S.L[0].kin;
+  const int nl = MULTI ? S.nl : 1;
+  const int ntot = S.row0[nl];                       // rows of the block's partial sums
+  const int ntasks = ((S.L[0].nvec + kLutNJ - 1) / kLutNJ) * nl * kLutSlices;
 
   if (warp == 0) {
     sm100::tmem_alloc(&s_tmem, TCOLS);
@@ -353,28 +368,28 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
   // piece builds the task's table, then does its share of the lookups).
   const int full = (ntasks / static_cast<int>(gridDim.x)) * static_cast<int>(gridDim.x);
   const int tail = ntasks - full;
-  const int nbat = (n + 8 * kLutThreads - 1) / (8 * kLutThreads);
-  const int parts = tail > 0 ? max(1, min(nbat, static_cast<int>(gridDim.x) / tail)) : 1;
+  int nbat_max = 1;
+  for (int l = 0; l < nl; ++l) nbat_max = max(nbat_max, (S.L[l].n + 8 * kLutThreads - 1) / (8 * kLutThreads));
+  const int parts = tail > 0 ? max(1, min(nbat_max, static_cast<int>(gridDim.x) / tail)) : 1;
   const int nitems = full + tail * parts;
   for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
-    int task = item, b_lo = 0, b_hi = RB8;
+    int task = item, part = 0, nparts = 1;
     if (item >= full) {
-      const int q = item - full, part = q % parts;
+      const int q = item - full;
+      part = q % parts;
+      nparts = parts;
       task = full + q / parts;
-      b_lo = part * nbat / parts;
-      b_hi = (part + 1) * nbat / parts;
     }
-    const int g = task / kLutSlices, s = task - g * kLutSlices;
-    // The next item's index tile row, pulled into L2 while this one runs.
-    {
-      const int nx = item + static_cast<int>(gridDim.x);
-      if (nx < nitems) {
-        const int ntask = nx < full ? nx : full + (nx - full) / parts;
-        const char* row = reinterpret_cast<const char*>(L.idx[0] + static_cast<int64_t>(ntask / kLutSlices) * L.rw[0]);
-        for (int l = tid; l < (n * 8 + 127) / 128; l += kLutThreads)
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(row + static_cast<int64_t>(l) * 128));
-      }
-    }
+    const int g = task / (nl * kLutSlices);
+    const int ls = task - g * nl * kLutSlices;
+    const int l = MULTI ? ls / kLutSlices : 0, s = ls - l * kLutSlices;
+    const Layer& L = S.L[l];
+    const int n = L.n;
+    // this layer's LB row-sum batches (rows past n unused)
+    const int bb0 = l * LB;
+    constexpr int nbat = LB;
+    const int nb_used = MULTI ? (n + 8 * kLutThreads - 1) / (8 * kLutThreads) : nbat_max;
+    const int b_lo = part * nb_used / nparts, b_hi = (part + 1) * nb_used / nparts;
     // Phase A operands of the first load batch go out before the activations
     // are read, so the two latencies overlap.
     const uint16_t* bslice = L.book[0] + static_cast<size_t>(s) * kLutS * 8;
@@ -390,7 +405,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
       float xp;
       const float sc = lut_pair_bfrag(x, x_fp16, kin, g, lane, bfrag, &xp);
       if (tid == 0) s_scale = sc;
-      if (warp == 0 && s == 0 && b_lo == 0) {
+      if (warp == 0 && s == 0 && l == 0 && part == 0) {   // each group of x once
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) xp += __shfl_xor_sync(0xffffffffu, xp, off);
         xs_acc += xp;
@@ -426,9 +441,10 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
         w[0][r] = o < n ? ldg_stream64(trow + o) : make_uint2(0u, 0u);
       }
 #pragma unroll
-      for (int b = 0; b < RB8; ++b) {
+      for (int b = 0; b < RB8; ++b) {               // b: this layer's batch
+        if (b >= nbat) break;                        // uniform
         const int cur = b & 1;
-        if (b + 1 < RB8) {
+        if (b + 1 < nbat) {
 #pragma unroll
           for (int r = 0; r < 8; ++r) {
             const int o = ((b + 1) * 8 + r) * kLutThreads + tid;
@@ -436,8 +452,9 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
           }
         }
         if (b < b_lo || b >= b_hi) continue;         // uniform: another piece's rows
+        const uint32_t tb = tbase + 8 * (bb0 + b);
         float acc[8];
-        sm100::tmem_ld8(tbase + 8 * b, acc);
+        sm100::tmem_ld8(tb, acc);
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
           float v[kLutNJ];
@@ -450,21 +467,26 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(Layer L, const
           }
           acc[r] = fmaf((v[0] + v[1]) + (v[2] + v[3]), sc, acc[r]);
         }
-        sm100::tmem_st8(tbase + 8 * b, acc);
+        sm100::tmem_st8(tb, acc);
       }
       sm100::tmem_wait_st();
     }
     __syncthreads();   // all lookups done before the next task rewrites T
   }
 
+  // Partial sums of every row of every layer, layers one after another.
+  for (int l = 0; l < nl; ++l) {
+    const int n = S.L[l].n;
+    float* dst = part + static_cast<int64_t>(blockIdx.x) * ntot + S.row0[l];
 #pragma unroll
-  for (int b = 0; b < RB8; ++b) {
-    float acc[8];
-    sm100::tmem_ld8(tbase + 8 * b, acc);
+    for (int b = 0; b < LB; ++b) {
+      float acc[8];
+      sm100::tmem_ld8(tbase + 8 * (l * LB + b), acc);
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int o = (b * 8 + r) * kLutThreads + tid;
-      if (o < n) part[static_cast<int64_t>(blockIdx.x) * n + o] = acc[r];
+      for (int r = 0; r < 8; ++r) {
+        const int o = (b * 8 + r) * kLutThreads + tid;
+        if (o < n) dst[o] = acc[r];
+      }
     }
   }
   if (tid == 0) xpart[blockIdx.x] = xs_acc;
@@ -859,63 +881,103 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_pair_kernel(Layer L, 
 // and one wave for the 70B layers (896 blocks).
 constexpr int kFinU = 20;
 
+// Outputs of a table launch: layer l's rows are rows row0[l] .. row0[l+1]-1
+// of the partial sums.
+struct LutOut {
+  int nl;
+  int row0[kLutMaxLayers + 1];
+  const uint16_t* scale[kLutMaxLayers];
+  const uint16_t* bias[kLutMaxLayers];
+  void* y[kLutMaxLayers];
+};
+
+LutOut lut_out_single(const Layer& L, void* y) {
+  LutOut o{};
+  o.nl = 1;
+  o.row0[0] = 0;
+  o.row0[1] = L.n;
+  o.scale[0] = L.scale;
+  o.bias[0] = L.bias;
+  o.y[0] = y;
+  return o;
+}
+
+// y_l[o] = s_l[o] * sum_b part[b][row0_l + o] + t_l[o] * sum_b xpart[b], the
+// partial sums added in a fixed order.
 __global__ void __launch_bounds__(256, 8) gemv_lut_finalize(const float* __restrict__ part,
                                                             const float* __restrict__ xpart, int nparts,
-                                                            int n, const uint16_t* __restrict__ scale,
-                                                            const uint16_t* __restrict__ bias,
-                                                            void* __restrict__ y, vq_dtype yt) {
+                                                            int ntot, LutOut out, vq_dtype yt) {
   __shared__ float red[8][33];
   __shared__ float s_xsum;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int o = blockIdx.x * 32 + lane;
+  const int v = blockIdx.x * 32 + lane;
   if (warp == 0) {
-    float v = 0.0f;
-    if (bias)
-      for (int i = lane; i < nparts; i += 32) v += xpart[i];
+    float t = 0.0f;
+    for (int i = lane; i < nparts; i += 32) t += xpart[i];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    if (lane == 0) s_xsum = v;
+    for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+    if (lane == 0) s_xsum = t;
   }
   float acc = 0.0f;
-  if (o < n) {
-    const float* col = part + o;
+  if (v < ntot) {
+    const float* col = part + v;
     for (int b0 = warp; b0 < nparts; b0 += 8 * kFinU) {
-      float v[kFinU];
+      float u[kFinU];
 #pragma unroll
-      for (int u = 0; u < kFinU; ++u) {
-        const int b = b0 + 8 * u;
-        v[u] = b < nparts ? col[static_cast<int64_t>(b) * n] : 0.0f;
+      for (int i = 0; i < kFinU; ++i) {
+        const int b = b0 + 8 * i;
+        u[i] = b < nparts ? col[static_cast<int64_t>(b) * ntot] : 0.0f;
       }
 #pragma unroll
-      for (int u = 0; u < kFinU; ++u) acc += v[u];
+      for (int i = 0; i < kFinU; ++i) acc += u[i];
     }
   }
   red[warp][lane] = acc;
   __syncthreads();
-  if (warp == 0 && o < n) {
+  if (warp == 0 && v < ntot) {
     float t = 0.0f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) t += red[w][lane];
-    const float sc = scale ? h2f(scale[o]) : 1.0f;
-    const float tb = bias ? h2f(bias[o]) : 0.0f;
-    store_out(y, yt, o, sc * t + tb * s_xsum);
+    int l = 0;
+    while (l + 1 < out.nl && v >= out.row0[l + 1]) ++l;
+    const int o = v - out.row0[l];
+    const float sc = out.scale[l] ? h2f(out.scale[l][o]) : 1.0f;
+    const float tb = out.bias[l] ? h2f(out.bias[l][o]) : 0.0f;
+    store_out(out.y[l], yt, o, sc * t + tb * s_xsum);
   }
+}
+
+// The layers of S share x; their partial sums take S.row0[S.nl] rows per block.
+template <int RB8, int LB>
+cudaError_t launch_lut_set(const LutSet& S, const LutOut& out, int grid, const void* x, bool x_fp16,
+                           vq_dtype yt, float* ws, cudaStream_t stream) {
+  auto k = gemv_lut_kernel<RB8, LB>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutSmem);
+  if (e != cudaSuccess) return e;
+  const int ntot = S.row0[S.nl];
+  float* part = ws;
+  float* xpart = ws + static_cast<int64_t>(grid) * ntot;
+  count_launch();
+  k<<<grid, kLutThreads, kLutSmem, stream>>>(S, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, part, xpart);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  count_launch();
+  gemv_lut_finalize<<<(ntot + 31) / 32, 256, 0, stream>>>(part, xpart, grid, ntot, out, yt);
+  return cudaGetLastError();
+}
+
+LutSet lut_set_single(const Layer& L) {
+  LutSet S{};
+  S.L[0] = L;
+  S.nl = 1;
+  S.row0[0] = 0;
+  S.row0[1] = L.n;
+  return S;
 }
 
 template <int RB8>
 cudaError_t launch_lut(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, void* y,
                        vq_dtype yt, float* ws, cudaStream_t stream) {
-  auto k = gemv_lut_kernel<RB8>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutSmem);
-  if (e != cudaSuccess) return e;
-  float* part = ws;
-  float* xpart = ws + static_cast<int64_t>(p.grid_x) * L.n;
-  count_launch();
-  k<<<p.grid_x, kLutThreads, kLutSmem, stream>>>(L, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, part, xpart);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  count_launch();
-  gemv_lut_finalize<<<(L.n + 31) / 32, 256, 0, stream>>>(part, xpart, p.grid_x, L.n, L.scale, L.bias, y, yt);
-  return cudaGetLastError();
+  return launch_lut_set<RB8, RB8>(lut_set_single(L), lut_out_single(L, y), p.grid_x, x, x_fp16, yt, ws, stream);
 }
 
 template <int RB8, int D, int NB>
@@ -971,7 +1033,7 @@ cudaError_t launch_lut_small(const Layer& L, const GemvPlan& p, const void* x, b
   if (e != cudaSuccess) return e;
   count_launch();
   gemv_lut_finalize<<<(L.n + 31) / 32, 256, 0, stream>>>(ws, ws + static_cast<int64_t>(p.grid_x) * L.n,
-                                                        p.grid_x, L.n, L.scale, L.bias, y, yt);
+                                                        p.grid_x, L.n, lut_out_single(L, y), yt);
   return cudaGetLastError();
 }
 
@@ -1030,6 +1092,52 @@ bool plan_gemv_lut(const Layer& L, int batch, size_t ws_cap, GemvPlan* p) {
   p->smem = big ? kLutSmem : static_cast<int>(lut_small_smem(L));
   p->ws_bytes = per_block * grid;
   return true;
+}
+
+// Several tiled 2^16-book layers that share x, at batch 1: one table launch
+// over all their tasks (one reduction launch) when 2..4 layers qualify and
+// their rows fit the block's row sums (8 batches of 8192).
+bool plan_gemv_lut_multi(const Layer* L, int nl, int batch, size_t ws_cap, LutMultiPlan* p) {
+  if (nl < 2 || nl > kLutMaxLayers || batch != 1) return false;
+  int lb = 1;
+  int64_t rows = 0;
+  for (int l = 0; l < nl; ++l) {
+    if (!lut_supported(L[l]) || L[l].kin != L[0].kin) return false;
+    while (static_cast<int64_t>(lb) * 8 * kLutThreads < L[l].n) lb <<= 1;
+    rows += L[l].n;
+  }
+  int rb8 = 1;
+  while (rb8 < nl * lb) rb8 <<= 1;
+  if (rb8 > 8) return false;
+  const int ntasks = ((L[0].nvec + kLutNJ - 1) / kLutNJ) * nl * kLutSlices;
+  const size_t per_block = (static_cast<size_t>(rows) + 1) * sizeof(float);
+  int grid = std::min(device_sm_count(), ntasks);
+  if (ws_cap / per_block < static_cast<size_t>(grid)) grid = static_cast<int>(ws_cap / per_block);
+  if (grid < 1) return false;
+  p->grid = grid;
+  p->rb8 = rb8;
+  p->lb = lb;
+  p->ws_bytes = per_block * grid;
+  return true;
+}
+
+cudaError_t launch_gemv_lut_multi(const Layer* L, int nl, const LutMultiPlan& p, const void* x, bool x_fp16,
+                                  void* const* y, vq_dtype yt, float* ws, cudaStream_t stream) {
+  LutSet S{};
+  LutOut out{};
+  S.nl = out.nl = nl;
+  for (int l = 0; l < nl; ++l) {
+    S.L[l] = L[l];
+    S.row0[l + 1] = out.row0[l + 1] = S.row0[l] + L[l].n;
+    out.scale[l] = L[l].scale;
+    out.bias[l] = L[l].bias;
+    out.y[l] = y[l];
+  }
+  if (p.rb8 == 2) return launch_lut_set<2, 1>(S, out, p.grid, x, x_fp16, yt, ws, stream);
+  if (p.rb8 == 4) return p.lb == 1 ? launch_lut_set<4, 1>(S, out, p.grid, x, x_fp16, yt, ws, stream)
+                                   : launch_lut_set<4, 2>(S, out, p.grid, x, x_fp16, yt, ws, stream);
+  return p.lb == 2 ? launch_lut_set<8, 2>(S, out, p.grid, x, x_fp16, yt, ws, stream)
+                   : launch_lut_set<8, 4>(S, out, p.grid, x, x_fp16, yt, ws, stream);
 }
 
 cudaError_t launch_gemv_lut(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, int batch,

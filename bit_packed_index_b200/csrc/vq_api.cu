@@ -1,6 +1,7 @@
 // vq_api.cu -- the extern "C" entry points of libvq (declared in include/vq.h):
 // argument validation on the host, then one launcher per call.  Nothing is
 // launched when an argument is rejected.
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <vector>
@@ -139,11 +140,91 @@ vq_status gemv_run(const vq_layer_desc* layer, const void* x, vq_dtype x_dtype, 
                      static_cast<float*>(workspace), stream);
 }
 
+// Layers sharing x: validated descriptions, the common checks of both entry points.
+constexpr int kMaxMultiLayers = 16;
+
+vq_status multi_check(const vq_layer_desc* const* layers, int32_t n_layers, int32_t batch, Layer* L) {
+  if (!layers || n_layers < 1 || n_layers > kMaxMultiLayers || batch < 0) return VQ_ERR_INVALID_ARG;
+  if (batch > kMaxBatch) return VQ_ERR_UNSUPPORTED;
+  for (int l = 0; l < n_layers; ++l) {
+    vq_status st = check_layer(layers[l], &L[l]);
+    if (st != VQ_OK) return st;
+    if (L[l].kin != L[0].kin) return VQ_ERR_INVALID_ARG;
+  }
+  return VQ_OK;
+}
+
+// Workspace of the fused launch when the layers qualify, else the largest
+// single-layer need (the layers then run one after another on the stream).
+vq_status multi_workspace(const Layer* L, const vq_layer_desc* const* layers, int n_layers, int32_t batch,
+                          bool* fused, LutMultiPlan* mp, size_t* bytes) {
+  *fused = batch == 1 && plan_gemv_lut_multi(L, n_layers, batch, ~static_cast<size_t>(0), mp);
+  if (*fused) {
+    *bytes = mp->ws_bytes;
+    return VQ_OK;
+  }
+  size_t need = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    size_t b = 0;
+    vq_status st = gemv_workspace_bytes(layers[l], batch, ~static_cast<size_t>(0), &b);
+    if (st != VQ_OK) return st;
+    need = std::max(need, b);
+  }
+  *bytes = need;
+  return VQ_OK;
+}
+
 }  // namespace vqk
 
 using namespace vqk;
 
 extern "C" {
+
+vq_status vq_gemv_multi_workspace_size(const vq_layer_desc* const* layers, int32_t n_layers, int32_t batch,
+                                       size_t* bytes) {
+  if (!bytes) return VQ_ERR_INVALID_ARG;
+  Layer L[kMaxMultiLayers];
+  vq_status st = multi_check(layers, n_layers, batch, L);
+  if (st != VQ_OK) return st;
+  bool fused;
+  LutMultiPlan mp;
+  return multi_workspace(L, layers, n_layers, batch, &fused, &mp, bytes);
+}
+
+vq_status vq_gemv_multi(const vq_layer_desc* const* layers, int32_t n_layers, const void* x, vq_dtype x_dtype,
+                        int32_t batch, int64_t ldx, void* const* y, vq_dtype y_dtype, const int64_t* ldy,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  Layer L[kMaxMultiLayers];
+  vq_status st = multi_check(layers, n_layers, batch, L);
+  if (st != VQ_OK) return st;
+  if (!y || !ldy || !dtype_ok_in(x_dtype) || !dtype_ok_out(y_dtype)) return VQ_ERR_INVALID_ARG;
+  if (ldx < L[0].kin) return VQ_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l)
+    if (ldy[l] < L[l].n) return VQ_ERR_INVALID_ARG;
+  bool fused;
+  LutMultiPlan mp;
+  size_t need = 0;
+  st = multi_workspace(L, layers, n_layers, batch, &fused, &mp, &need);
+  if (st != VQ_OK) return st;
+  if (!fused) {
+    for (int l = 0; l < n_layers; ++l) {
+      st = gemv_run(layers[l], x, x_dtype, batch, ldx, y[l], y_dtype, ldy[l], workspace, workspace_bytes,
+                    ~static_cast<size_t>(0), static_cast<cudaStream_t>(stream));
+      if (st != VQ_OK) return st;
+    }
+    return VQ_OK;
+  }
+  if (!x) return VQ_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l) {
+    if (!y[l]) return VQ_ERR_INVALID_ARG;
+    if (!aligned(y[l], dtype_size(y_dtype))) return VQ_ERR_ALIGNMENT;
+  }
+  if (!aligned(x, 2)) return VQ_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < need) return VQ_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return VQ_ERR_ALIGNMENT;
+  return cuda_status(launch_gemv_lut_multi(L, n_layers, mp, x, x_dtype == VQ_FP16, y, y_dtype,
+                                           static_cast<float*>(workspace), static_cast<cudaStream_t>(stream)));
+}
 
 vq_status vq_dequant(const vq_layer_desc* layer, uint16_t* w_hat, int64_t ldw, void* stream) {
   Layer L;

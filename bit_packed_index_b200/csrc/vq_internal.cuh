@@ -82,6 +82,16 @@ vq_status plan_gemv(const Layer& L, int batch, GemvPlan* plan, size_t ws_cap = ~
 // Lookup-table plans (tiled order; a batch runs one table pass per row of x,
 // up to a per-layer limit); false when no table kernel applies.
 bool plan_gemv_lut(const Layer& L, int batch, size_t ws_cap, GemvPlan* plan);
+// Layers sharing x in one table launch (tiled 2^16 books, batch 1).
+struct LutMultiPlan {
+  int grid;
+  int rb8;      // row-sum batches of all layers (power of two)
+  int lb;       // batches per layer (power of two)
+  size_t ws_bytes;
+};
+bool plan_gemv_lut_multi(const Layer* layers, int n_layers, int batch, size_t ws_cap, LutMultiPlan* plan);
+cudaError_t launch_gemv_lut_multi(const Layer* layers, int n_layers, const LutMultiPlan& plan, const void* x,
+                                  bool x_fp16, void* const* y, vq_dtype y_dtype, float* ws, cudaStream_t stream);
 cudaError_t launch_gemv_lut(const Layer& L, const GemvPlan& plan, const void* x, bool x_fp16, int batch,
                             int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy, float* ws,
                             cudaStream_t stream);

@@ -4,8 +4,8 @@ Every computation runs in the CUDA kernels behind the C ABI; this module only
 turns torch tensors into pointers, sizes and the current CUDA stream.  There
 is no fallback: if ``libvq.so`` is missing or fails to load, every call raises.
 
-Names follow the C ABI: ``dequant``, ``gemv``, ``gemm``, ``repack_tile4``,
-``encode``, plus the workspace size queries.  A ``Layer`` holds the device tensors of one
+Names follow the C ABI: ``dequant``, ``gemv``, ``gemv_multi``, ``gemm``,
+``repack_tile4``, ``encode``, plus the workspace size queries.  A ``Layer`` holds the device tensors of one
 quantised layer (packed index streams in row order or in the tiled order,
 fp16 codebooks, optional fp16 scale and bias).
 """
@@ -89,11 +89,14 @@ def lib():
             L.vq_gemm_workspace_size.argtypes = [P, I32, C.c_int, C.POINTER(SZ)]
             L.vq_gemm.argtypes = [P, P, C.c_int, I32, I64, P, C.c_int, I64, P, SZ, P]
             L.vq_repack_tile4.argtypes = [P, C.POINTER(P), C.POINTER(I64), P]
+            L.vq_gemv_multi_workspace_size.argtypes = [P, I32, I32, C.POINTER(SZ)]
+            L.vq_gemv_multi.argtypes = [P, I32, P, C.c_int, I32, I64, P, C.c_int, P, P, SZ, P]
             L.vq_encode_workspace_size.argtypes = [P, C.POINTER(SZ)]
             L.vq_encode.argtypes = [P, P, SZ, P]
             for fn in ("vq_dequant", "vq_gemv_workspace_size", "vq_gemv", "vq_gemv_noalloc",
                        "vq_gemm_workspace_size", "vq_gemm", "vq_repack_tile4",
-                       "vq_encode_workspace_size", "vq_encode"):
+                       "vq_encode_workspace_size", "vq_encode", "vq_gemv_multi_workspace_size",
+                       "vq_gemv_multi"):
                 getattr(L, fn).restype = C.c_int
             L.vq_status_string.argtypes = [C.c_int]
             L.vq_status_string.restype = C.c_char_p
@@ -308,6 +311,40 @@ def gemm(layer: Layer, x: torch.Tensor, out_dtype=torch.bfloat16,
                                     _ptr(out), _DTYPE[out.dtype], ldy, _ptr(ws), ws_bytes,
                                     C.c_void_p(_stream(layer.device))))
     return out
+
+
+def _desc_array(layers: Sequence[Layer]):
+    arr = (C.c_void_p * len(layers))(*[C.addressof(l.desc()) for l in layers])
+    return arr
+
+
+def gemv_multi_workspace_size(layers: Sequence[Layer], batch: int) -> int:
+    n = C.c_size_t(0)
+    _check("vq_gemv_multi_workspace_size",
+           lib().vq_gemv_multi_workspace_size(_desc_array(layers), len(layers), batch, C.byref(n)))
+    return n.value
+
+
+def gemv_multi(layers: Sequence[Layer], x: torch.Tensor, out_dtype=torch.bfloat16,
+               outs: Optional[Sequence[torch.Tensor]] = None,
+               workspace: Optional[torch.Tensor] = None) -> List[torch.Tensor]:
+    """y_l [B][N_l] = x [B][Kin] . W_hat_l^T for layers sharing x (vq_gemv_multi);
+    tiled 2^16-book layers at batch 1 run as one table launch."""
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    batch = x.shape[0]
+    dev = layers[0].device
+    if outs is None:
+        outs = [torch.empty((batch, l.out_features), dtype=out_dtype, device=dev) for l in layers]
+    ws, ws_bytes = _workspace(gemv_multi_workspace_size(layers, batch), dev, workspace)
+    ldx = x.stride(0) if batch > 1 else max(x.shape[1], layers[0].in_features)
+    ys = (C.c_void_p * len(layers))(*[o.data_ptr() for o in outs])
+    ldy = (C.c_int64 * len(layers))(*[o.stride(0) if batch > 1 else max(o.shape[1], l.out_features)
+                                      for o, l in zip(outs, layers)])
+    _check("vq_gemv_multi", lib().vq_gemv_multi(_desc_array(layers), len(layers), _ptr(x), _DTYPE[x.dtype],
+                                                batch, ldx, ys, _DTYPE[outs[0].dtype], ldy, _ptr(ws),
+                                                ws_bytes, C.c_void_p(_stream(dev))))
+    return list(outs)
 
 
 def row_words(in_features: int, vec_dim: int, log2k: int) -> int:

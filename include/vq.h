@@ -232,6 +232,25 @@ VQ_API vq_status vq_gemv_noalloc(const vq_layer_desc* layer, const void* x, vq_d
                                  int64_t ldy, void* stream);
 
 /*
+ * vq_gemv_multi -- y_l = x . W_hat_l^T for n_layers (1..16) layers that read
+ * the same x (the projections of one transformer block: gate and up, or q, k
+ * and v), with the same meaning, arguments and errors as n_layers calls of
+ * vq_gemv (y[l] and ldy[l] per layer).  At batch 1, two to four tiled layers
+ * with one 2^16-entry d = 8 book whose rows add up to at most 65536 in
+ * 8192-row batches run as one lookup-table launch over all their tasks and one
+ * reduction launch, which fills the machine better than separate calls
+ * ("VQ in Production", section "1. Prefill vs. Decode Bottlenecks": decode
+ * is a sequence of small, memory-bound products).  Every other case runs the
+ * layers one after another on the stream.
+ */
+VQ_API vq_status vq_gemv_multi_workspace_size(const vq_layer_desc* const* layers, int32_t n_layers,
+                                              int32_t batch, size_t* bytes);
+VQ_API vq_status vq_gemv_multi(const vq_layer_desc* const* layers, int32_t n_layers, const void* x,
+                               vq_dtype x_dtype, int32_t batch, int64_t ldx, void* const* y,
+                               vq_dtype y_dtype, const int64_t* ldy, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/*
  * vq_gemm_workspace_size -- bytes of device workspace vq_gemm needs for this
  * layer, row count m and activation type.  Host-only.
  */

@@ -18,7 +18,8 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(names) == {"vq_dequant", "vq_repack_tile4", "vq_gemv_workspace_size", "vq_gemv",
                           "vq_gemv_noalloc", "vq_gemm_workspace_size", "vq_gemm",
                           "vq_status_string", "vq_last_cuda_error", "vq_abi_version",
-                          "vq_kernel_launches", "vq_encode_workspace_size", "vq_encode"}
+                          "vq_kernel_launches", "vq_encode_workspace_size", "vq_encode",
+                          "vq_gemv_multi_workspace_size", "vq_gemv_multi"}
     for n in names:
         assert hasattr(lib, n), n
 

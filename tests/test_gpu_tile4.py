@@ -376,3 +376,49 @@ def test_tiled_small_batch_strided_x_and_y():
         vq.gemv(layer, _x_dev(x)[:, :spec.in_features], out=ybuf[:, :spec.out_features])
         assert_close(_f64(ybuf[:, :spec.out_features]), ref, "float32")
         assert (ybuf[:, spec.out_features:] == 0).all()
+
+
+# Layers that share x through vq_gemv_multi: tiled 2^16-book layers at batch
+# 1 run as one table launch (rows of all layers in one task list); any other
+# mix runs the layers one after another.
+MULTI_SETS = [
+    [LayerSpec(3000, 8 * 100 + 3, 8, (16,), (0.02,)), LayerSpec(777, 8 * 100 + 3, 8, (16,), (0.02,))],
+    [LayerSpec(8193, 8 * 40, 8, (16,), (0.02,), None, None), LayerSpec(300, 8 * 40, 8, (16,), (0.02,)),
+     LayerSpec(20000, 8 * 40, 8, (16,), (0.02,), (0.5, 1.5), None)],
+    [LayerSpec(5000, 8 * 33, 8, (16,), (0.02,)) for _ in range(4)],
+    # not fusable: a small-book layer in the set
+    [LayerSpec(3000, 8 * 64, 8, (16,), (0.02,)), LayerSpec(900, 8 * 64, 8, (12, 8), (0.02, 0.005))],
+]
+
+
+@pytest.mark.parametrize("i", range(len(MULTI_SETS)))
+@pytest.mark.parametrize("batch", [1, 3])
+def test_gemv_multi_matches_the_oracle(i, batch):
+    vq = _vq()
+    specs = MULTI_SETS[i]
+    datas = [synth.make_layer(s, seed=2900 + 10 * i + k) for k, s in enumerate(specs)]
+    layers = [_oracle_tiled_layer(d) for d in datas]
+    assert vq.gemv_multi_workspace_size(layers, batch) > 0
+    for fp16 in (False, True):
+        x = synth.make_x(2950 + i, batch, specs[0].in_features, outlier_frac=0.01, as_fp16=fp16)
+        for od in (torch.float32, torch.bfloat16):
+            ys = vq.gemv_multi(layers, _x_dev(x, fp16), out_dtype=od)
+            for y, d in zip(ys, datas):
+                assert_close(_f64(y), oracle.linear(d, x, x_is_fp16=fp16), str(od).split(".")[-1])
+
+
+def test_gemv_multi_70b_gate_up_sampled():
+    """The 70B gate/up pair (2 x 28672 rows = all eight row-sum batches) as one launch."""
+    vq = _vq()
+    w = WORKLOADS["llama3_70b_mlp"]
+    datas, layers = [], []
+    for li in (0, 1):
+        spec, seed = w.layers[li]
+        datas.append(synth.make_layer(spec, seed))
+        layers.append(vq.repack_tile4(vq.Layer.from_synth(datas[-1])))
+    x = synth.make_x(w.x_seed, 1, layers[0].in_features, w.outlier_frac)
+    rows = sample_rows(layers[0].out_features, 192, 2990)
+    rd = torch.from_numpy(rows).cuda()
+    ys = vq.gemv_multi(layers, _x_dev(x), out_dtype=torch.bfloat16)
+    for y, d in zip(ys, datas):
+        assert_close(_f64(y[:, rd]), oracle.linear(d, x, rows), "bfloat16")
