@@ -4,9 +4,10 @@
 Step = one decode pass of the Llama-3-70B-shaped MLP at 2.0 bits per weight:
 gate_proj and up_proj (28672 x 8192) and down_proj (8192 x 28672), d = 8, one
 K = 2^16 fp16 codebook, per-row fp16 scale and bias, batch B = 1, through
-vq_gemv.  All three layers are stored in the tiled index order (made by
-vq_repack_tile4 from the generated row-order streams, exactly 2.0 bits per
-weight like the row order) and run the lookup-table kernel.  Two copies of the three layers
+vq_gemv_multi (gate_proj and up_proj, which read the same x, in one launch)
+and vq_gemv (down_proj).  All three layers are stored in the tiled index
+order (made by vq_repack_tile4 from the generated row-order streams, exactly
+2.0 bits per weight like the row order) and run the lookup-table kernel.  Two copies of the three layers
 (352 MB of index streams) are used in turn, so every step reads its weights
 from HBM, not from the 126 MB L2.
 
@@ -15,8 +16,9 @@ value  = algorithmic bytes moved per step (packed indices + codebook + scale
          in GB/s; the timed region is bracketed by a barrier and a device
          synchronise on both sides and is the max over ranks.
 e2e    = the same metric through the public Python API with the activations
-         in pinned host memory: each step copies x to the device, runs the
-         layer and copies y back.
+         in pinned host memory: each step copies the three layers' x to the
+         device in one transfer, runs the layers and copies the three y back
+         in one transfer.
 gemm   = the prefill GEMM (x [2048, 8192] bf16, 8192 x 8192 layer, K = 2^16
          + residual K = 2^8, 3.0 bpw) through vq_gemm, in TFLOP/s.
 encode = the nearest-centroid encoder (vq_encode) on a 4096 x 4096 matrix
@@ -276,7 +278,7 @@ def decode_config():
                     "8192x28672; d=8, one K=2^16 fp16 codebook (2.0 bpw), fp16 scale/bias",
         "batch": BATCH, "layers": [s.name for s, _ in w.layers], "bpw": 2.0,
         "index_order": dict(zip([s.name for s, _ in w.layers], LAYOUTS)),
-        "x": "bf16 ~N(0,1), 0.1% outlier columns x20",
+        "x": "bf16 ~N(0,1), 0.1% outlier columns x20; gate_proj and up_proj read the same x",
         "l2": "inputs larger than L2: two copies of the three layers (352 MB of indices) used in turn",
         "parallelism": "replicas (each rank runs its own step; no collective on the data path)",
     }
@@ -305,30 +307,38 @@ def run_gpu(args):
             layers.append(vq.Layer.from_synth(synth.make_layer(spec, seed + 1000 * c + 17 * rank), dev,
                                               layout=lay))
         copies.append(layers)
-    xs_host = [synth.make_x(w.x_seed + i, BATCH, s.in_features, w.outlier_frac) for i, s in enumerate(specs)]
+    # gate_proj and up_proj read the same x (the block's input); down_proj its own.
+    xs_host = [synth.make_x(w.x_seed, BATCH, specs[0].in_features, w.outlier_frac),
+               synth.make_x(w.x_seed + 2, BATCH, specs[2].in_features, w.outlier_frac)]
     xs = [torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16) for x in xs_host]
     ys = [torch.empty((BATCH, s.out_features), dtype=torch.bfloat16, device=dev) for s in specs]
-    ws = []
-    for k in range(3):
-        need = max(vq.gemv_workspace_size(copies[c][k], BATCH) for c in range(2))
-        ws.append(torch.empty(max(need, 256), dtype=torch.uint8, device=dev))
+    need_gu = max(vq.gemv_multi_workspace_size(copies[c][:2], BATCH) for c in range(2))
+    need_d = max(vq.gemv_workspace_size(copies[c][2], BATCH) for c in range(2))
+    ws = [torch.empty(max(need_gu, 256), dtype=torch.uint8, device=dev),
+          torch.empty(max(need_d, 256), dtype=torch.uint8, device=dev)]
     step_bytes = sum(alg_bytes(s, BATCH) for s in specs)
 
+    def run_step(layers, x_gu, x_d, y_gu, y_d, events=None):
+        """gate_proj + up_proj as one vq_gemv_multi call, then down_proj."""
+        if events is not None:
+            events[0][0].record()
+        vq.gemv_multi(layers[:2], x_gu, outs=y_gu, workspace=ws[0])
+        if events is not None:
+            events[0][1].record()
+            events[1][0].record()
+        vq.gemv(layers[2], x_d, out=y_d, workspace=ws[1])
+        if events is not None:
+            events[1][1].record()
+
     def step(i, events=None):
-        layers = copies[i & 1]
-        for k in range(3):
-            if events is not None:
-                events[k][0].record()
-            vq.gemv(layers[k], xs[k], out=ys[k], workspace=ws[k])
-            if events is not None:
-                events[k][1].record()
+        run_step(copies[i & 1], xs[0], xs[1], ys[:2], ys[2], events)
 
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
 
     evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-            for _ in range(3)] for _ in range(args.steps)]
+            for _ in range(2)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     uuid = str(getattr(torch.cuda.get_device_properties(local), "uuid", "") or "")
     gpu_id = ("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or str(local))
@@ -348,39 +358,48 @@ def run_gpu(args):
     value = whole_job_value(step_bytes, args.steps, world, ms_total)
 
     # Live roofline of the dominant kernel, the lookup-table GEMV, on its
-    # gate_proj calls (the workload of the committed ncu capture): algorithmic
-    # bytes of one call / mean call time from CUDA events on the launching
-    # stream.  A call is the table kernel plus its per-block-sum reduction, so
-    # the figure slightly understates the kernel alone.
-    per_layer_ms = [statistics.mean(evs[i][k][0].elapsed_time(evs[i][k][1]) for i in range(args.steps))
-                    for k in range(3)]
-    gate_bytes = alg_bytes(specs[0], BATCH)
-    achieved = gate_bytes / (per_layer_ms[0] * 1e-3) / 1e9
+    # fused gate_proj + up_proj launches (the workload of the committed ncu
+    # capture): algorithmic bytes of one call / mean call time from CUDA
+    # events on the launching stream.  A call is the table kernel plus its
+    # per-block-sum reduction, so the figure slightly understates the kernel.
+    call_ms = [statistics.mean(evs[i][k][0].elapsed_time(evs[i][k][1]) for i in range(args.steps))
+               for k in range(2)]
+    gu_bytes = alg_bytes(specs[0], BATCH) + alg_bytes(specs[1], BATCH)
+    achieved = gu_bytes / (call_ms[0] * 1e-3) / 1e9
     rec = profiled_traffic("gemv_lut_kernel")
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"],
                 "traffic": rec["dram_bytes_per_launch"] if rec else None,
-                "algorithmic_bytes_per_launch": gate_bytes,
+                "algorithmic_bytes_per_launch": gu_bytes,
                 "kernel": "gemv_lut_kernel (+ gemv_lut_finalize)",
-                "launch": "gate_proj 28672x8192, B=1, tiled index order",
+                "launch": "gate_proj + up_proj (2 x 28672x8192) in one vq_gemv_multi launch, B=1, "
+                          "tiled index order",
                 "peak_source": peak_src + " (HBM copy, kernel timed alone)",
-                "per_layer_us": {s.name: ms * 1e3 for s, ms in zip(specs, per_layer_ms)},
+                "per_call_us": {"gate_proj+up_proj": call_ms[0] * 1e3, "down_proj": call_ms[1] * 1e3},
                 "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                 "row_order_gather_ceiling_us": 120.0,
                 "note": "not HBM-bound: the table kernel is bound by instruction issue and "
                         "shared-memory lookups (4 slice tests per index), the row-order kernel "
                         "by random 16-byte centroid gathers through L1/L2 (0.84/clk/SM)"}
 
-    # e2e through the public API with pinned host activations and outputs
-    xh = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in xs_host]
-    yh = [torch.empty((BATCH, s.out_features), dtype=torch.bfloat16).pin_memory() for s in specs]
+    # e2e through the public API with pinned host activations and outputs:
+    # each step copies all three layers' inputs to the device in one transfer,
+    # runs the layers, and copies all outputs back in one transfer.
+    xcat = np.concatenate([x.reshape(-1) for x in xs_host])
+    xh = torch.from_numpy(xcat.view(np.int16)).view(torch.bfloat16).pin_memory()
+    xd = torch.empty_like(xh, device=dev)
+    xoff = np.cumsum([0] + [x.size for x in xs_host])
+    xv = [xd[xoff[k]:xoff[k + 1]].view(BATCH, -1) for k in range(2)]
+    ycat = sum(BATCH * s.out_features for s in specs)
+    yh = torch.empty(ycat, dtype=torch.bfloat16).pin_memory()
+    yd = torch.empty(ycat, dtype=torch.bfloat16, device=dev)
+    yoff = np.cumsum([0] + [BATCH * s.out_features for s in specs])
+    yv = [yd[yoff[k]:yoff[k + 1]].view(BATCH, -1) for k in range(3)]
 
     def e2e_step(i):
-        layers = copies[i & 1]
-        for k in range(3):
-            xs[k].copy_(xh[k], non_blocking=True)
-            vq.gemv(layers[k], xs[k], out=ys[k], workspace=ws[k])
-            yh[k].copy_(ys[k], non_blocking=True)
+        xd.copy_(xh, non_blocking=True)
+        run_step(copies[i & 1], xv[0], xv[1], yv[:2], yv[2])
+        yh.copy_(yd, non_blocking=True)
 
     for i in range(args.warmup):
         e2e_step(i)
@@ -395,8 +414,8 @@ def run_gpu(args):
     barrier(dist_mod, dev)
     e2e_ms = reduce_max(a.elapsed_time(b), dist_mod, dev)
     e2e = {"value": whole_job_value(step_bytes, args.steps, world, e2e_ms), "unit": "GB/s",
-           "h2d_bytes_per_step": sum(x.numel() * 2 for x in xh),
-           "d2h_bytes_per_step": sum(y.numel() * 2 for y in yh),
+           "h2d_bytes_per_step": xh.numel() * 2,
+           "d2h_bytes_per_step": yh.numel() * 2,
            "ms_per_step": e2e_ms / args.steps}
 
     gemm = run_gemm(dev, peaks, peak_src, vq)
@@ -569,6 +588,15 @@ def run_profile(args):
         ws = torch.empty(vq.encode_workspace_size(n, kin, log2k, d), dtype=torch.uint8, device=dev)
         for _ in range(args.profile_launches):
             vq.encode(W, B, log2k, d, workspace=ws)
+    elif args.profile == "lut_gateup":
+        w = WORKLOADS[DECODE]
+        layers = [vq.Layer.from_synth(synth.make_layer(*w.layers[li]), dev, layout="tile4") for li in (0, 1)]
+        x = torch.from_numpy(synth.make_x(w.x_seed, BATCH, layers[0].in_features, w.outlier_frac)
+                             .view(np.int16)).to(dev).view(torch.bfloat16)
+        outs = [torch.empty((BATCH, l.out_features), dtype=torch.bfloat16, device=dev) for l in layers]
+        ws = torch.empty(vq.gemv_multi_workspace_size(layers, BATCH), dtype=torch.uint8, device=dev)
+        for _ in range(args.profile_launches):
+            vq.gemv_multi(layers, x, outs=outs, workspace=ws)
     elif args.profile in ("gemv", "lut", "lut_down", "lut_small", "dequant"):
         w = WORKLOADS[DECODE if args.profile != "lut_small" else "llama31_405b"]
         spec, seed = w.layers[{"lut_small": 4, "lut_down": 2}.get(args.profile, 0)]
@@ -608,10 +636,11 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["gemv", "lut", "lut_down", "lut_small", "gemm", "dequant",
-                                          "encode"],
+    ap.add_argument("--profile", choices=["gemv", "lut", "lut_gateup", "lut_down", "lut_small", "gemm",
+                                          "dequant", "encode"],
                     help="run a few untimed launches of one call on its workload (for ncu): "
-                         "gemv / lut = 70B gate_proj in row / tiled order, lut_down = 70B "
+                         "gemv / lut = 70B gate_proj in row / tiled order, lut_gateup = 70B "
+                         "gate_proj + up_proj in one vq_gemv_multi launch, lut_down = 70B "
                          "down_proj in tiled order, lut_small = 405B gate_proj in tiled order, "
                          "encode = the encoder on its bench workload")
     ap.add_argument("--profile-launches", type=int, default=3)
