@@ -746,10 +746,13 @@ __device__ __forceinline__ float row_lookup(const uint32_t (&w)[NW], const uint8
   return (a + b) + (c + d);
 }
 
-template <int RB8, int D, int B2>
-__global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_pair_kernel(Layer L, const uint16_t* __restrict__ x,
+// Layers of one set (S.nl of them, LB batches of 8192 rows each in the row
+// sums; one layer: LB = RB8) share x; a task is (group, layer).
+template <int RB8, int D, int B2, int LB>
+__global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_pair_kernel(LutSet S, const uint16_t* __restrict__ x,
                                                                        int x_fp16, float* __restrict__ part,
                                                                        float* __restrict__ xpart) {
+  constexpr bool MULTI = LB < RB8;
   constexpr int B1 = 12;
   constexpr int NB = B2 > 0 ? 2 : 1;
   constexpr int W2 = B2 == 8 ? 2 : 1;               // words per pair of book-2 records
@@ -762,11 +765,10 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_pair_kernel(Layer L, 
   __shared__ uint32_t s_tmem;
   __shared__ float s_scale;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int n = L.n, kin = L.kin;
-  const int ntasks = (L.nvec + 3) / 4;
-  const int npairs = (n + 1) / 2;
-  const int64_t nw1 = (static_cast<int64_t>(n) * 4 * B1 + 31) / 32;   // words holding records
-  const int64_t nw2 = (static_cast<int64_t>(n) * 4 * (B2 > 0 ? B2 : 1) + 31) / 32;
+  const int kin = S.L[0].kin;
+  const int nl = MULTI ? S.nl : 1;
+  const int ntot = S.row0[nl];
+  const int ntasks = ((S.L[0].nvec + 3) / 4) * nl;
 
   if (warp == 0) {
     sm100::tmem_alloc(&s_tmem, TCOLS);
@@ -785,7 +787,13 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_pair_kernel(Layer L, 
   }
   float xs_acc = 0.0f;
 
-  for (int g = blockIdx.x; g < ntasks; g += gridDim.x) {
+  for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
+    const int g = MULTI ? task / nl : task, l = MULTI ? task - g * nl : 0;
+    const Layer& L = S.L[l];
+    const int n = L.n;
+    const int npairs = (n + 1) / 2;
+    const int64_t nw1 = (static_cast<int64_t>(n) * 4 * B1 + 31) / 32;   // words holding records
+    const int64_t nw2 = (static_cast<int64_t>(n) * 4 * (B2 > 0 ? B2 : 1) + 31) / 32;
     uint32_t bfrag;
     {
       const int jj = lane >> 2, t = lane & 3;
@@ -806,7 +814,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_pair_kernel(Layer L, 
       const __half2 h = __floats2half2_rn(ldexpf(a, -e), ldexpf(b, -e));
       bfrag = *reinterpret_cast<const uint32_t*>(&h);
       if (tid == 0) s_scale = ldexpf(1.0f, e);
-      if (warp == 0) {
+      if (warp == 0 && l == 0) {                    // each group of x once
         float v = a + b;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
@@ -823,8 +831,9 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_pair_kernel(Layer L, 
       const uint8_t* t1 = reinterpret_cast<const uint8_t*>(tab1);
       const uint8_t* t2 = reinterpret_cast<const uint8_t*>(tab2);
 #pragma unroll 1
-      for (int b = 0; b < RB8; ++b) {
+      for (int b = 0; b < LB; ++b) {
         if (b * 8 * kLutThreads >= n) break;          // uniform: no row of this batch exists
+        const uint32_t tb = tbase + 8 * (l * LB + b);
         uint32_t w1[4][3], w2[4][W2];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {                 // all loads of the batch first
@@ -837,7 +846,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_pair_kernel(Layer L, 
           }
         }
         float acc[8];
-        sm100::tmem_ld8(tbase + 8 * b, acc);
+        sm100::tmem_ld8(tb, acc);
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           if ((b * 4 + r) * kLutThreads >= npairs) break;   // uniform: no thread has this pair
@@ -850,21 +859,25 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_pair_kernel(Layer L, 
           acc[2 * r] = fmaf(va, sc, acc[2 * r]);
           acc[2 * r + 1] = fmaf(vb, sc, acc[2 * r + 1]);
         }
-        sm100::tmem_st8(tbase + 8 * b, acc);
+        sm100::tmem_st8(tb, acc);
       }
       sm100::tmem_wait_st();
     }
     __syncthreads();   // all lookups done before the next task rewrites the tables
   }
 
+  for (int l = 0; l < nl; ++l) {
+    const int n = S.L[l].n;
+    float* dst = part + static_cast<int64_t>(blockIdx.x) * ntot + S.row0[l];
 #pragma unroll 1
-  for (int b = 0; b < RB8; ++b) {
-    float acc[8];
-    sm100::tmem_ld8(tbase + 8 * b, acc);
+    for (int b = 0; b < LB; ++b) {
+      float acc[8];
+      sm100::tmem_ld8(tbase + 8 * (l * LB + b), acc);
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int64_t o = 2 * (static_cast<int64_t>(b * 4 + (r >> 1)) * kLutThreads + tid) + (r & 1);
-      if (o < n) part[static_cast<int64_t>(blockIdx.x) * n + o] = acc[r];
+      for (int r = 0; r < 8; ++r) {
+        const int64_t o = 2 * (static_cast<int64_t>(b * 4 + (r >> 1)) * kLutThreads + tid) + (r & 1);
+        if (o < n) dst[o] = acc[r];
+      }
     }
   }
   if (tid == 0) xpart[blockIdx.x] = xs_acc;
@@ -997,16 +1010,22 @@ bool lut_pair_path(const Layer& L) {
   return L.b[0] == 12 && (b2 == 0 || b2 == 4 || b2 == 8);
 }
 
+template <int RB8, int D, int B2, int LB>
+cudaError_t launch_lut_pair_set(const LutSet& S, int grid, int smem, const void* x, bool x_fp16, float* ws,
+                                cudaStream_t stream) {
+  auto k = gemv_lut_pair_kernel<RB8, D, B2, LB>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  count_launch();
+  k<<<grid, kLutThreads, smem, stream>>>(S, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, ws,
+                                         ws + static_cast<int64_t>(grid) * S.row0[S.nl]);
+  return cudaGetLastError();
+}
+
 template <int RB8, int D, int B2>
 cudaError_t launch_lut_pair_t(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, float* ws,
                               cudaStream_t stream) {
-  auto k = gemv_lut_pair_kernel<RB8, D, B2>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
-  if (e != cudaSuccess) return e;
-  count_launch();
-  k<<<p.grid_x, kLutThreads, p.smem, stream>>>(L, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, ws,
-                                               ws + static_cast<int64_t>(p.grid_x) * L.n);
-  return cudaGetLastError();
+  return launch_lut_pair_set<RB8, D, B2, RB8>(lut_set_single(L), p.grid_x, p.smem, x, x_fp16, ws, stream);
 }
 
 template <int RB8>
@@ -1099,17 +1118,28 @@ bool plan_gemv_lut(const Layer& L, int batch, size_t ws_cap, GemvPlan* p) {
 // their rows fit the block's row sums (8 batches of 8192).
 bool plan_gemv_lut_multi(const Layer* L, int nl, int batch, size_t ws_cap, LutMultiPlan* p) {
   if (nl < 2 || nl > kLutMaxLayers || batch != 1) return false;
+  // All layers 2^16 books (the sliced kernel), or all on the paired-row path
+  // with the same vector length and books (d = 6 with 2^12 + 2^4, or d = 8
+  // with 2^12 + 2^8: the shapes of the 405B and 8B layers).
+  bool big = true, pair = true;
+  for (int l = 0; l < nl; ++l) {
+    if (L[l].kin != L[0].kin) return false;
+    big = big && lut_supported(L[l]);
+    pair = pair && lut_small_supported(L[l]) && lut_pair_path(L[l]) && L[l].nb == 2 && L[l].d == L[0].d &&
+           L[l].b[1] == L[0].b[1] && ((L[l].d == 6 && L[l].b[1] == 4) || (L[l].d == 8 && L[l].b[1] == 8));
+  }
+  if (!big && !pair) return false;
   int lb = 1;
   int64_t rows = 0;
   for (int l = 0; l < nl; ++l) {
-    if (!lut_supported(L[l]) || L[l].kin != L[0].kin) return false;
     while (static_cast<int64_t>(lb) * 8 * kLutThreads < L[l].n) lb <<= 1;
     rows += L[l].n;
   }
   int rb8 = 1;
   while (rb8 < nl * lb) rb8 <<= 1;
-  if (rb8 > 8) return false;
-  const int ntasks = ((L[0].nvec + kLutNJ - 1) / kLutNJ) * nl * kLutSlices;
+  if (pair) rb8 = std::max(rb8, 4);                  // the compiled paired-row shapes
+  if (rb8 > 8 || (pair && !((rb8 == 4 && lb <= 2) || (rb8 == 8 && lb == 2)))) return false;
+  const int ntasks = ((L[0].nvec + kLutNJ - 1) / kLutNJ) * nl * (big ? kLutSlices : 1);
   const size_t per_block = (static_cast<size_t>(rows) + 1) * sizeof(float);
   int grid = std::min(device_sm_count(), ntasks);
   if (ws_cap / per_block < static_cast<size_t>(grid)) grid = static_cast<int>(ws_cap / per_block);
@@ -1117,6 +1147,8 @@ bool plan_gemv_lut_multi(const Layer* L, int nl, int batch, size_t ws_cap, LutMu
   p->grid = grid;
   p->rb8 = rb8;
   p->lb = lb;
+  p->kind = big ? 0 : 1;
+  p->smem = big ? kLutSmem : static_cast<int>(lut_small_smem(L[0]));
   p->ws_bytes = per_block * grid;
   return true;
 }
@@ -1132,6 +1164,25 @@ cudaError_t launch_gemv_lut_multi(const Layer* L, int nl, const LutMultiPlan& p,
     out.scale[l] = L[l].scale;
     out.bias[l] = L[l].bias;
     out.y[l] = y[l];
+  }
+  if (p.kind == 1) {                                 // paired-row small-book kernel
+    const bool d6 = L[0].d == 6;
+    cudaError_t e;
+    if (p.rb8 == 8)
+      e = d6 ? launch_lut_pair_set<8, 6, 4, 2>(S, p.grid, p.smem, x, x_fp16, ws, stream)
+             : launch_lut_pair_set<8, 8, 8, 2>(S, p.grid, p.smem, x, x_fp16, ws, stream);
+    else if (p.lb == 2)
+      e = d6 ? launch_lut_pair_set<4, 6, 4, 2>(S, p.grid, p.smem, x, x_fp16, ws, stream)
+             : launch_lut_pair_set<4, 8, 8, 2>(S, p.grid, p.smem, x, x_fp16, ws, stream);
+    else
+      e = d6 ? launch_lut_pair_set<4, 6, 4, 1>(S, p.grid, p.smem, x, x_fp16, ws, stream)
+             : launch_lut_pair_set<4, 8, 8, 1>(S, p.grid, p.smem, x, x_fp16, ws, stream);
+    if (e != cudaSuccess) return e;
+    const int ntot = S.row0[nl];
+    count_launch();
+    gemv_lut_finalize<<<(ntot + 31) / 32, 256, 0, stream>>>(ws, ws + static_cast<int64_t>(p.grid) * ntot,
+                                                            p.grid, ntot, out, yt);
+    return cudaGetLastError();
   }
   if (p.rb8 == 2) return launch_lut_set<2, 1>(S, out, p.grid, x, x_fp16, yt, ws, stream);
   if (p.rb8 == 4) return p.lb == 1 ? launch_lut_set<4, 1>(S, out, p.grid, x, x_fp16, yt, ws, stream)

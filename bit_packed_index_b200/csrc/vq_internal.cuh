@@ -87,6 +87,8 @@ struct LutMultiPlan {
   int grid;
   int rb8;      // row-sum batches of all layers (power of two)
   int lb;       // batches per layer (power of two)
+  int kind;     // 0: 2^16-book kernel, 1: paired-row small-book kernel
+  int smem;     // dynamic shared memory of the table kernel
   size_t ws_bytes;
 };
 bool plan_gemv_lut_multi(const Layer* layers, int n_layers, int batch, size_t ws_cap, LutMultiPlan* plan);

@@ -236,9 +236,11 @@ VQ_API vq_status vq_gemv_noalloc(const vq_layer_desc* layer, const void* x, vq_d
  * the same x (the projections of one transformer block: gate and up, or q, k
  * and v), with the same meaning, arguments and errors as n_layers calls of
  * vq_gemv (y[l] and ldy[l] per layer).  At batch 1, two to four tiled layers
- * with one 2^16-entry d = 8 book whose rows add up to at most 65536 in
- * 8192-row batches run as one lookup-table launch over all their tasks and one
- * reduction launch, which fills the machine better than separate calls
+ * that all have one 2^16-entry d = 8 book, or all have a 2^12-entry main book
+ * with the same residual (d = 6 with 2^4, or d = 8 with 2^8), and whose rows
+ * fit eight 8192-row batches (a power of two per layer), run as one
+ * lookup-table launch over all their tasks and one reduction launch, which
+ * fills the machine better than separate calls
  * ("VQ in Production", section "1. Prefill vs. Decode Bottlenecks": decode
  * is a sequence of small, memory-bound products).  Every other case runs the
  * layers one after another on the stream.

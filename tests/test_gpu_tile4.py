@@ -388,6 +388,11 @@ MULTI_SETS = [
     [LayerSpec(5000, 8 * 33, 8, (16,), (0.02,)) for _ in range(4)],
     # not fusable: a small-book layer in the set
     [LayerSpec(3000, 8 * 64, 8, (16,), (0.02,)), LayerSpec(900, 8 * 64, 8, (12, 8), (0.02, 0.005))],
+    # paired-row small-book layers: q/k/v-like (d = 6, 2^12 + 2^4) and gate/up-like (d = 8, 2^12 + 2^8)
+    [LayerSpec(9000, 6 * 50 + 4, 6, (12, 4), (0.02, 0.005)), LayerSpec(1024, 6 * 50 + 4, 6, (12, 4), (0.02, 0.005)),
+     LayerSpec(1023, 6 * 50 + 4, 6, (12, 4), (0.02, 0.005))],
+    [LayerSpec(14336, 8 * 40, 8, (12, 8), (0.02, 0.005)), LayerSpec(14335, 8 * 40, 8, (12, 8), (0.02, 0.005))],
+    [LayerSpec(700, 6 * 30, 6, (12, 4), (0.02, 0.005)) for _ in range(4)],
 ]
 
 
@@ -421,4 +426,21 @@ def test_gemv_multi_70b_gate_up_sampled():
     rd = torch.from_numpy(rows).cuda()
     ys = vq.gemv_multi(layers, _x_dev(x), out_dtype=torch.bfloat16)
     for y, d in zip(ys, datas):
+        assert_close(_f64(y[:, rd]), oracle.linear(d, x, rows), "bfloat16")
+
+
+def test_gemv_multi_405b_qkv_sampled():
+    """The 405B q/k/v projections (16384 + 1024 + 1024 rows, d = 6) as one launch."""
+    vq = _vq()
+    w = WORKLOADS["llama31_405b"]
+    datas, layers = [], []
+    for li in (0, 1, 2):
+        spec, seed = w.layers[li]
+        datas.append(synth.make_layer(spec, seed))
+        layers.append(vq.repack_tile4(vq.Layer.from_synth(datas[-1])))
+    x = synth.make_x(w.x_seed, 1, layers[0].in_features, w.outlier_frac)
+    ys = vq.gemv_multi(layers, _x_dev(x), out_dtype=torch.bfloat16)
+    for k, (y, d) in enumerate(zip(ys, datas)):
+        rows = sample_rows(layers[k].out_features, 128, 2995 + k)
+        rd = torch.from_numpy(rows).cuda()
         assert_close(_f64(y[:, rd]), oracle.linear(d, x, rows), "bfloat16")
