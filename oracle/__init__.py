@@ -9,7 +9,8 @@ The arithmetic lives in ``vq_oracle.c`` (plain C, built here with gcc into
 ``liboracle.so``); this module marshals numpy arrays for it.  What each
 routine computes, and the page passage it follows, is documented in the C
 file.  Functions pinned by the not-gpu tests: the conversions, unpack/pack
-(row order and tiled order), dequant, matmul/linear and the encoders.
+(row order and tiled order), dequant, matmul/linear, the encoders and the
+randomized Hadamard transform.
 """
 from __future__ import annotations
 
@@ -71,12 +72,15 @@ def _load():
                 "vqo_encode": [P, I64, I32, P, I64, P],
                 "vqo_encode_residual": [P, I64, I32, P, I64, P, I64, P, P],
                 "vqo_encode_joint": [P, I64, I32, P, I64, P, I64, P, P],
+                "vqo_rht": [P, I64, I64, P, I32, P],
+                "vqo_rht_block": [I64],
                 "vqo_num_threads": [],
             }
             for name, args in sig.items():
                 fn = getattr(lib, name)
                 fn.argtypes = args
                 fn.restype = None if name.endswith("_array") else C.c_int
+            lib.vqo_rht_block.restype = C.c_int64
             _lib = lib
     return _lib
 
@@ -269,6 +273,22 @@ def encode_joint(v: np.ndarray, book1: np.ndarray, book2: np.ndarray):
     _check(_load().vqo_encode_joint(_p(v), nv, d, _p(b1), b1.shape[0], _p(b2), b2.shape[0],
                                     _p(i1), _p(i2)), "encode_joint")
     return i1, i2
+
+
+# -- randomized Hadamard transform (tests only) ----------------------------
+
+def rht_block(n: int) -> int:
+    return int(_load().vqo_rht_block(n))
+
+
+def rht(x: np.ndarray, signs: np.ndarray, inverse: bool = False) -> np.ndarray:
+    """Rows of x (fp64 [rows][n]) through the randomized Hadamard transform with
+    the sign bits `signs` (uint32 words, bit t set -> -1)."""
+    x = np.ascontiguousarray(np.atleast_2d(x), np.float64)
+    signs = np.ascontiguousarray(signs, np.uint32)
+    out = np.empty_like(x)
+    _check(_load().vqo_rht(_p(x), x.shape[0], x.shape[1], _p(signs), int(inverse), _p(out)), "rht")
+    return out
 
 
 def num_threads() -> int:

@@ -27,6 +27,8 @@
  *  - products y = x . W_hat^T accumulated in fp64 in ascending k order
  *    ("VPTQ Guide", section "Step 3: Fused Low-Bit VPTQ Linear Layer":
  *    forward computes y = x @ W^T with the dequantised weights).
+ *  - the randomized Hadamard transform of QuIP#-style incoherence processing
+ *    (plain O(n b) sums; section "Randomized Hadamard transform" below);
  *  - nearest-centroid encoding by brute force, ties to the lowest index
  *    ("VPTQ Guide", section "The Information-Theoretic Superiority of Vector
  *    Quantization": q = argmin_k ||w - c_k||^2; section "2. Multi-Stage
@@ -441,6 +443,60 @@ int vqo_encode_joint(const double* v, int64_t nv, int d, const uint16_t* book1, 
             }
         idx1[i] = (uint32_t)a1;
         idx2[i] = (uint32_t)a2;
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Randomized Hadamard transform (tests only).                             */
+/* ---------------------------------------------------------------------- */
+
+/* Incoherence processing: W~ = U W V^T and x~ = V x with U, V orthogonal
+ * randomized Walsh-Hadamard matrices, so y = W x = U^T (W~ x~) ("Vector
+ * Quantization for LLM Weights in Production", section "1. QuIP#:
+ * Incoherence Processing and Lattice Codebooks"; "Sub-4-Bit Quantization",
+ * section "QuIP#: Incoherence Processing": Hadamard plus random signs).
+ * Reading for lengths that are not powers of two: the transform of a row of
+ * length n is block diagonal, blocks of b = the largest power of two that
+ * divides n (at most 2^15), i.e. (I ⊗ H_b) diag(s) / sqrt(b).
+ *   forward:  out[k*b + i] = b^-1/2 * sum_j H_b[i][j] * s[k*b + j] * in[k*b + j]
+ *   inverse:  out[k*b + j] = s[k*b + j] * b^-1/2 * sum_i H_b[j][i] * in[k*b + i]
+ * with H_b[i][j] = (-1)^popcount(i & j) (Sylvester's construction) and
+ * s[t] = -1 where bit t of `signs` is set (LSB first in 32-bit words), +1
+ * otherwise.  Plain O(n b) sums in fp64, j (or i) ascending. */
+int64_t vqo_rht_block(int64_t n) {
+    if (n <= 0) return 0;
+    int64_t b = 1;
+    while (b < 32768 && n % (2 * b) == 0) b *= 2;
+    return b;
+}
+
+static double hadamard_entry(int64_t i, int64_t j) {
+    return (__builtin_popcountll((unsigned long long)(i & j)) & 1) ? -1.0 : 1.0;
+}
+
+static double sign_of(const uint32_t* signs, int64_t t) {
+    return (signs[t >> 5] >> (t & 31)) & 1u ? -1.0 : 1.0;
+}
+
+int vqo_rht(const double* in, int64_t rows, int64_t n, const uint32_t* signs, int inverse, double* out) {
+    if (rows < 0 || n < 0) return 1;
+    const int64_t b = vqo_rht_block(n);
+    const double scale = b > 0 ? 1.0 / sqrt((double)b) : 0.0;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const double* x = in + r * n;
+        double* y = out + r * n;
+        for (int64_t k0 = 0; k0 < n; k0 += b) {
+            for (int64_t i = 0; i < b; ++i) {
+                double acc = 0.0;
+                for (int64_t j = 0; j < b; ++j) {
+                    const double v = inverse ? x[k0 + j] : sign_of(signs, k0 + j) * x[k0 + j];
+                    acc += hadamard_entry(i, j) * v;
+                }
+                y[k0 + i] = inverse ? sign_of(signs, k0 + i) * (acc * scale) : acc * scale;
+            }
+        }
     }
     return 0;
 }

@@ -345,3 +345,62 @@ def test_two_book_encoders():
     r = v - c1[g1]
     dist = ((r[:, None, :] - c2[None]) ** 2).sum(-1)
     assert np.array_equal(g2, dist.argmin(1).astype(np.uint32))
+
+
+# -- randomized Hadamard transform ----------------------------------------------
+
+def _signs(n, seed):
+    rng = np.random.default_rng(seed)
+    bits = rng.integers(0, 2, size=n).astype(np.uint8)
+    words = np.packbits(np.concatenate([bits, np.zeros((-n) % 32, np.uint8)]), bitorder="little")
+    return words.view(np.uint32), np.where(bits == 1, -1.0, 1.0)
+
+
+def test_rht_hand_worked_example():
+    """H_4 = [[1,1,1,1],[1,-1,1,-1],[1,1,-1,-1],[1,-1,-1,1]] (Sylvester), signs
+    (+1, -1, +1, +1): x = (1, 2, 3, 4) -> H (1, -2, 3, 4) / 2 = (3, 1, -4, 2)."""
+    x = np.array([[1.0, 2.0, 3.0, 4.0]])
+    signs = np.array([0b0010], np.uint32)
+    assert np.array_equal(oracle.rht(x, signs), [[3.0, 1.0, -4.0, 2.0]])
+    assert np.array_equal(oracle.rht(x, np.zeros(1, np.uint32)), [[5.0, -1.0, -2.0, 0.0]])
+    # the inverse undoes it: signs applied after H
+    assert np.allclose(oracle.rht(np.array([[3.0, 1.0, -4.0, 2.0]]), signs, inverse=True), x, atol=1e-15)
+
+
+def test_rht_block_rule():
+    """Blocks: the largest power of two dividing n, at most 2^15."""
+    for n, b in [(1, 1), (7, 1), (12, 4), (6, 2), (8192, 8192), (28672, 4096), (53248, 4096),
+                 (16384, 16384), (1 << 20, 32768), (3 * 32768, 32768)]:
+        assert oracle.rht_block(n) == b, n
+
+
+@pytest.mark.parametrize("n", [8, 24, 96, 1024 + 512])
+def test_rht_matches_a_library_hadamard_and_is_orthogonal(n):
+    """Against scipy's Sylvester Hadamard matrix, block-diagonal with random
+    signs; forward then inverse returns x; norms are preserved."""
+    from scipy.linalg import hadamard, block_diag
+    words, s = _signs(n, 70 + n)
+    b = oracle.rht_block(n)
+    V = block_diag(*[hadamard(b)] * (n // b)) @ np.diag(s) / np.sqrt(b)
+    rng = np.random.default_rng(n)
+    x = rng.standard_normal((3, n))
+    y = oracle.rht(x, words)
+    assert np.allclose(y, x @ V.T, atol=1e-12)
+    assert np.allclose(oracle.rht(y, words, inverse=True), x, atol=1e-12)
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)
+    assert np.allclose(V @ V.T, np.eye(n), atol=1e-12)
+
+
+def test_rht_layer_identity():
+    """W x = U^T ((U W V^T) (V x)) for orthogonal U, V (the QuIP# identity)."""
+    rng = np.random.default_rng(5)
+    N, K = 48, 40                      # blocks of 16 and 8
+    W = rng.standard_normal((N, K))
+    x = rng.standard_normal(K)
+    su, _ = _signs(N, 6)
+    sv, _ = _signs(K, 7)
+    WVt = oracle.rht(W, sv)                              # rows: W V^T
+    Wt = oracle.rht(WVt.T.copy(), su).T                  # columns: U (W V^T)
+    xt = oracle.rht(x[None, :], sv)[0]                   # V x
+    y = oracle.rht((Wt @ xt)[None, :], su, inverse=True)[0]
+    assert np.allclose(y, W @ x, atol=1e-12)
