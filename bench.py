@@ -23,6 +23,8 @@ gemm   = the prefill GEMM (x [2048, 8192] bf16, 8192 x 8192 layer, K = 2^16
          + residual K = 2^8, 3.0 bpw) through vq_gemm, in TFLOP/s.
 encode = the nearest-centroid encoder (vq_encode) on a 4096 x 4096 matrix
          against one K = 2^16, d = 8 book, in (vector, centroid) pairs/s.
+rht_gate = the 70B gate_proj in the rotated basis (vq_gemv_rht) beside the
+         same layer through vq_gemv.
 roofline, cpu_baseline, clocks and gpu_launches are described beside the
 keys they fill.  ``--impl reference`` times the CPU oracle on the same
 metric instead (a bounded sample of the same workload per step).
@@ -69,6 +71,7 @@ LAYOUTS = ("tile4", "tile4", "tile4")
 ENCODE_SHAPE = (4096, 4096, 8, [16])
 ENCODE_STD = [0.02]
 ENCODE_SEED = 11
+RHT_SEED = 12           # sign bits of the rotated-basis measurement
 
 
 def kernel_sources_sha(files) -> str:
@@ -420,6 +423,7 @@ def run_gpu(args):
 
     gemm = run_gemm(dev, peaks, peak_src, vq)
     decode_405b = run_decode_405b(dev, peaks, peak_src, vq)
+    rht = run_rht(dev, vq)
     encode = run_encode(dev, peaks, peak_src, vq,
                         with_oracle=rank == 0 and world == 1 and not args.no_cpu_baseline)
 
@@ -437,6 +441,7 @@ def run_gpu(args):
         "clocks": clocks.summary(),
         "gemm": gemm,
         "decode_405b_gate": decode_405b,
+        "rht_gate": rht,
         "encode": encode,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -572,6 +577,48 @@ def run_encode(dev, peaks, peak_src, vq, with_oracle: bool):
                            "cores": oracle.num_threads(), "kind": "oracle",
                            "sample": f"{sample} vectors x {1 << log2k[0]} centroids, {dt:.2f} s"}
     return out
+
+
+def run_rht(dev, vq):
+    """Beside the headline: the 70B gate_proj (tiled) in the rotated basis of
+    QuIP#-style incoherence processing, y = U^T (W~ (V x)) through
+    vq_gemv_rht, against the same layer through vq_gemv; L2 flushed."""
+    import torch
+    w = WORKLOADS[DECODE]
+    spec, seed = w.layers[0]
+    layer = vq.Layer.from_synth(synth.make_layer(spec, seed), dev, layout="tile4")
+    x = torch.from_numpy(synth.make_x(w.x_seed, 1, spec.in_features, w.outlier_frac).view(np.int16)).to(dev)
+    x = x.view(torch.bfloat16)
+    rng = np.random.default_rng(RHT_SEED)
+    s_in = torch.from_numpy(rng.integers(0, 2**31, size=(spec.in_features + 31) // 32, dtype=np.int64)
+                            .astype(np.int32)).to(dev)
+    s_out = torch.from_numpy(rng.integers(0, 2**31, size=(spec.out_features + 31) // 32, dtype=np.int64)
+                             .astype(np.int32)).to(dev)
+    y = torch.empty((1, spec.out_features), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(256, vq.gemv_workspace_size(layer, 1)), dtype=torch.uint8, device=dev)
+    wr = torch.empty(vq.gemv_rht_workspace_size(layer, 1), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def med(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(20):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts) * 1e3
+
+    plain = med(lambda: vq.gemv(layer, x, out=y, workspace=ws))
+    rot = med(lambda: vq.gemv_rht(layer, s_in, s_out, x, out=y, workspace=wr))
+    return {"workload": "llama3_70b_mlp gate_proj 28672x8192, tiled, B=1, in the rotated basis "
+                        "(blocks of 8192 on x, 4096 on y)",
+            "us": rot, "us_without_rotation": plain, "rotation_overhead_us": rot - plain,
+            "achieved_gbs": alg_bytes(spec, 1) / (rot * 1e-6) / 1e9}
 
 
 def run_profile(args):

@@ -4,8 +4,9 @@ Every computation runs in the CUDA kernels behind the C ABI; this module only
 turns torch tensors into pointers, sizes and the current CUDA stream.  There
 is no fallback: if ``libvq.so`` is missing or fails to load, every call raises.
 
-Names follow the C ABI: ``dequant``, ``gemv``, ``gemv_multi``, ``gemm``,
-``repack_tile4``, ``encode``, plus the workspace size queries.  A ``Layer`` holds the device tensors of one
+Names follow the C ABI: ``dequant``, ``gemv``, ``gemv_multi``, ``gemv_rht``,
+``rht``, ``gemm``, ``repack_tile4``, ``encode``, plus the workspace size
+queries.  A ``Layer`` holds the device tensors of one
 quantised layer (packed index streams in row order or in the tiled order,
 fp16 codebooks, optional fp16 scale and bias).
 """
@@ -91,12 +92,15 @@ def lib():
             L.vq_repack_tile4.argtypes = [P, C.POINTER(P), C.POINTER(I64), P]
             L.vq_gemv_multi_workspace_size.argtypes = [P, I32, I32, C.POINTER(SZ)]
             L.vq_gemv_multi.argtypes = [P, I32, P, C.c_int, I32, I64, P, C.c_int, P, P, SZ, P]
+            L.vq_rht.argtypes = [P, C.c_int, I32, I32, I64, P, I32, P, C.c_int, I64, P]
+            L.vq_gemv_rht_workspace_size.argtypes = [P, I32, C.POINTER(SZ)]
+            L.vq_gemv_rht.argtypes = [P, P, P, P, C.c_int, I32, I64, P, C.c_int, I64, P, SZ, P]
             L.vq_encode_workspace_size.argtypes = [P, C.POINTER(SZ)]
             L.vq_encode.argtypes = [P, P, SZ, P]
             for fn in ("vq_dequant", "vq_gemv_workspace_size", "vq_gemv", "vq_gemv_noalloc",
                        "vq_gemm_workspace_size", "vq_gemm", "vq_repack_tile4",
                        "vq_encode_workspace_size", "vq_encode", "vq_gemv_multi_workspace_size",
-                       "vq_gemv_multi"):
+                       "vq_gemv_multi", "vq_rht", "vq_gemv_rht_workspace_size", "vq_gemv_rht"):
                 getattr(L, fn).restype = C.c_int
             L.vq_status_string.argtypes = [C.c_int]
             L.vq_status_string.restype = C.c_char_p
@@ -345,6 +349,47 @@ def gemv_multi(layers: Sequence[Layer], x: torch.Tensor, out_dtype=torch.bfloat1
                                                 batch, ldx, ys, _DTYPE[outs[0].dtype], ldy, _ptr(ws),
                                                 ws_bytes, C.c_void_p(_stream(dev))))
     return list(outs)
+
+
+def rht(x: torch.Tensor, signs: torch.Tensor, inverse: bool = False, out_dtype=None,
+        out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Randomized Hadamard transform of the rows of x (vq_rht); `signs` holds
+    the sign bits as int32 words (bit t set -> -1)."""
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    rows, n = x.shape
+    if out is None:
+        out = torch.empty((rows, n), dtype=out_dtype or x.dtype, device=x.device)
+    ld_in = x.stride(0) if rows > 1 else max(n, 1)
+    ld_out = out.stride(0) if rows > 1 else max(n, 1)
+    _check("vq_rht", lib().vq_rht(_ptr(x), _DTYPE[x.dtype], rows, n, ld_in, _ptr(signs), int(inverse),
+                                  _ptr(out), _DTYPE[out.dtype], ld_out, C.c_void_p(_stream(x.device))))
+    return out
+
+
+def gemv_rht_workspace_size(layer: Layer, batch: int) -> int:
+    n = C.c_size_t(0)
+    _check("vq_gemv_rht_workspace_size",
+           lib().vq_gemv_rht_workspace_size(C.byref(layer.desc()), batch, C.byref(n)))
+    return n.value
+
+
+def gemv_rht(layer: Layer, signs_in: torch.Tensor, signs_out: torch.Tensor, x: torch.Tensor,
+             out_dtype=torch.bfloat16, out: Optional[torch.Tensor] = None,
+             workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y = U^T (W~ (V x)) for a layer whose streams encode the rotated W~ (vq_gemv_rht)."""
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    batch = x.shape[0]
+    if out is None:
+        out = torch.empty((batch, layer.out_features), dtype=out_dtype, device=layer.device)
+    ws, ws_bytes = _workspace(gemv_rht_workspace_size(layer, batch), layer.device, workspace)
+    ldx = x.stride(0) if batch > 1 else max(x.shape[1], layer.in_features)
+    ldy = out.stride(0) if batch > 1 else max(out.shape[1], layer.out_features)
+    _check("vq_gemv_rht", lib().vq_gemv_rht(C.byref(layer.desc()), _ptr(signs_in), _ptr(signs_out), _ptr(x),
+                                            _DTYPE[x.dtype], batch, ldx, _ptr(out), _DTYPE[out.dtype], ldy,
+                                            _ptr(ws), ws_bytes, C.c_void_p(_stream(layer.device))))
+    return out
 
 
 def row_words(in_features: int, vec_dim: int, log2k: int) -> int:

@@ -348,6 +348,42 @@ VQ_API vq_status vq_encode_workspace_size(const vq_encode_desc* desc, size_t* by
 VQ_API vq_status vq_encode(const vq_encode_desc* desc, void* workspace, size_t workspace_bytes,
                            void* stream);
 
+/*
+ * Randomized Hadamard transform (QuIP#-style incoherence processing): a layer
+ * may be quantised in a rotated basis, W~ = U W V^T with U, V orthogonal
+ * randomized Walsh-Hadamard matrices, so that y = W x = U^T (W~ (V x))
+ * ("Vector Quantization for LLM Weights in Production", section "1. QuIP#:
+ * Incoherence Processing and Lattice Codebooks"; "Sub-4-Bit Quantization",
+ * section "QuIP#: Incoherence Processing": Hadamard plus random signs).
+ * A row of length n is transformed in blocks of b = the largest power of two
+ * dividing n (at most 2^15), i.e. by (I (x) H_b) diag(s) / sqrt(b):
+ *   forward:  out[k b + i] = b^-1/2 sum_j H_b[i][j] s[k b + j] in[k b + j]
+ *   inverse:  out[k b + j] = s[k b + j] b^-1/2 sum_i H_b[j][i] in[k b + i]
+ * H_b[i][j] = (-1)^popcount(i & j) (Sylvester), s[t] = -1 where bit t of
+ * `signs` is set (32-bit words, LSB first; ceil(n / 32) words), else +1.
+ * Arithmetic in fp32 (fast Walsh-Hadamard butterflies in shared memory).
+ */
+
+/* vq_rht -- transform `rows` (<= 65535) rows of length n: in [rows][ld_in] of
+ * in_dtype, out [rows][ld_out] of out_dtype (bf16, fp16 or fp32), device
+ * pointers, inverse = 0 for V, 1 for V^T.  in and out may not overlap.
+ * Errors: VQ_ERR_INVALID_ARG, VQ_ERR_UNSUPPORTED (rows > 65535),
+ * VQ_ERR_ALIGNMENT, VQ_ERR_CUDA. */
+VQ_API vq_status vq_rht(const void* in, vq_dtype in_dtype, int32_t rows, int32_t n, int64_t ld_in,
+                        const uint32_t* signs, int32_t inverse, void* out, vq_dtype out_dtype,
+                        int64_t ld_out, void* stream);
+
+/* vq_gemv_rht -- y = U^T (W~ (V x)) for a layer whose streams encode W~:
+ * V x with signs_in (in_features bits), the product as vq_gemv with x~ in
+ * fp16 and y~ in fp32, then U^T with signs_out (out_features bits).  Same
+ * arguments and errors as vq_gemv; the workspace (vq_gemv_rht_workspace_size,
+ * 256-byte aligned) also holds x~ and y~. */
+VQ_API vq_status vq_gemv_rht_workspace_size(const vq_layer_desc* layer, int32_t batch, size_t* bytes);
+VQ_API vq_status vq_gemv_rht(const vq_layer_desc* layer, const uint32_t* signs_in,
+                             const uint32_t* signs_out, const void* x, vq_dtype x_dtype,
+                             int32_t batch, int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
 /* Static description of a status code (never NULL). */
 VQ_API const char* vq_status_string(vq_status status);
 

@@ -19,7 +19,8 @@ def test_every_declared_symbol_is_exported(lib):
                           "vq_gemv_noalloc", "vq_gemm_workspace_size", "vq_gemm",
                           "vq_status_string", "vq_last_cuda_error", "vq_abi_version",
                           "vq_kernel_launches", "vq_encode_workspace_size", "vq_encode",
-                          "vq_gemv_multi_workspace_size", "vq_gemv_multi"}
+                          "vq_gemv_multi_workspace_size", "vq_gemv_multi", "vq_rht",
+                          "vq_gemv_rht_workspace_size", "vq_gemv_rht"}
     for n in names:
         assert hasattr(lib, n), n
 
