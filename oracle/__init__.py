@@ -9,8 +9,8 @@ The arithmetic lives in ``vq_oracle.c`` (plain C, built here with gcc into
 ``liboracle.so``); this module marshals numpy arrays for it.  What each
 routine computes, and the page passage it follows, is documented in the C
 file.  Functions pinned by the not-gpu tests: the conversions, unpack/pack
-(row order and tiled order), dequant, matmul/linear, the encoders and the
-randomized Hadamard transform.
+(row order and tiled order), dequant, matmul/linear, the encoders, the
+randomized Hadamard transform and the Hessian.
 """
 from __future__ import annotations
 
@@ -73,6 +73,7 @@ def _load():
                 "vqo_encode_residual": [P, I64, I32, P, I64, P, I64, P, P],
                 "vqo_encode_joint": [P, I64, I32, P, I64, P, I64, P, P],
                 "vqo_rht": [P, I64, I64, P, I32, P],
+                "vqo_hessian": [P, I32, I64, I64, I64, P],
                 "vqo_rht_block": [I64],
                 "vqo_num_threads": [],
             }
@@ -288,6 +289,18 @@ def rht(x: np.ndarray, signs: np.ndarray, inverse: bool = False) -> np.ndarray:
     signs = np.ascontiguousarray(signs, np.uint32)
     out = np.empty_like(x)
     _check(_load().vqo_rht(_p(x), x.shape[0], x.shape[1], _p(signs), int(inverse), _p(out)), "rht")
+    return out
+
+
+# -- Hessian collection (tests only) -----------------------------------------
+
+def hessian(x: np.ndarray, x_is_fp16: bool = False) -> np.ndarray:
+    """Normalised, damped Hessian (fp64 [d][d]) of activations x: bf16 (or fp16)
+    bits [n_tokens][d]."""
+    x = np.ascontiguousarray(x, np.uint16)
+    n, d = x.shape
+    out = np.empty((d, d), np.float64)
+    _check(_load().vqo_hessian(_p(x), int(x_is_fp16), n, d, d, _p(out)), "hessian")
     return out
 
 

@@ -27,6 +27,8 @@
  *  - products y = x . W_hat^T accumulated in fp64 in ascending k order
  *    ("VPTQ Guide", section "Step 3: Fused Low-Bit VPTQ Linear Layer":
  *    forward computes y = x @ W^T with the dequantised weights).
+ *  - the normalised, damped activation Hessian H = 2 X^T X / n + damping
+ *    (section "Hessian collection" below);
  *  - the randomized Hadamard transform of QuIP#-style incoherence processing
  *    (plain O(n b) sums; section "Randomized Hadamard transform" below);
  *  - nearest-centroid encoding by brute force, ties to the lowest index
@@ -498,6 +500,35 @@ int vqo_rht(const double* in, int64_t rows, int64_t n, const uint32_t* signs, in
             }
         }
     }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Hessian collection (tests only).                                        */
+/* ---------------------------------------------------------------------- */
+
+/* The normalised, damped activation Hessian of a layer's inputs ("VPTQ
+ * Guide", section "Step 1: Hessian Matrix Collection", and section "1.
+ * Second-Order Hessian-Weighted Optimization": H = 2 X X^T over the tokens):
+ *   H[i][j] = sum_t 2 x_t[i] x_t[j]        (fp64, tokens t ascending)
+ *   h = H / n_tokens;  damp = 0.01 * mean_i h[i][i];  h[i][i] += damp
+ * x: n_tokens rows of d values, bf16 (x_is_fp16 = 0) or fp16 bits, row
+ * stride ldx.  out: fp64 [d][d]. */
+int vqo_hessian(const uint16_t* x, int x_is_fp16, int64_t n_tokens, int64_t d, int64_t ldx, double* out) {
+    if (n_tokens < 1 || d < 0 || ldx < d) return 1;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < d; ++i) {
+        for (int64_t j = 0; j < d; ++j) {
+            double acc = 0.0;
+            for (int64_t t = 0; t < n_tokens; ++t)
+                acc += 2.0 * act(x, x_is_fp16, t * ldx + i) * act(x, x_is_fp16, t * ldx + j);
+            out[i * d + j] = acc / (double)n_tokens;
+        }
+    }
+    double diag = 0.0;
+    for (int64_t i = 0; i < d; ++i) diag += out[i * d + i];
+    const double damp = d > 0 ? 0.01 * (diag / (double)d) : 0.0;
+    for (int64_t i = 0; i < d; ++i) out[i * d + i] += damp;
     return 0;
 }
 

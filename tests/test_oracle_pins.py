@@ -404,3 +404,38 @@ def test_rht_layer_identity():
     xt = oracle.rht(x[None, :], sv)[0]                   # V x
     y = oracle.rht((Wt @ xt)[None, :], su, inverse=True)[0]
     assert np.allclose(y, W @ x, atol=1e-12)
+
+
+# -- Hessian collection -----------------------------------------------------------
+
+def test_hessian_closed_forms():
+    """All-ones tokens: H = 2 n J, h = 2 J, damp = 0.01 * 2 -> 2 J + 0.02 I.
+    One-hot tokens e_(t mod d): h = 2 diag(counts) / n + 0.01 * mean."""
+    d, n = 8, 40
+    ones = oracle.f32_to_bf16(np.ones((n, d), np.float32))
+    h = oracle.hessian(ones)
+    assert np.allclose(h, 2.0 * np.ones((d, d)) + 0.02 * np.eye(d), atol=1e-15)
+    onehot = np.zeros((n, d), np.float32)
+    onehot[np.arange(n), np.arange(n) % d] = 1.0
+    h = oracle.hessian(oracle.f32_to_bf16(onehot))
+    counts = np.bincount(np.arange(n) % d, minlength=d)
+    base = 2.0 * np.diag(counts) / n
+    assert np.allclose(h, base + 0.01 * np.trace(base) / d * np.eye(d), atol=1e-15)
+
+
+def test_hessian_matches_numpy():
+    """Against numpy: 2 X^T X / n (fp64 matmul) plus 0.01 * mean(diag) I; symmetric."""
+    rng = np.random.default_rng(9)
+    n, d = 300, 48
+    xb = oracle.f32_to_bf16(rng.standard_normal((n, d), dtype=np.float32))
+    x = oracle.bf16_to_f32(xb).astype(np.float64)
+    h0 = 2.0 * x.T @ x / n
+    ref = h0 + 0.01 * np.mean(np.diag(h0)) * np.eye(d)
+    h = oracle.hessian(xb)
+    assert np.allclose(h, ref, rtol=1e-13, atol=1e-13)
+    assert np.array_equal(h, h.T)
+    xf = oracle.f32_to_f16(rng.standard_normal((n, d), dtype=np.float32))
+    x = oracle.f16_to_f32(xf).astype(np.float64)
+    h0 = 2.0 * x.T @ x / n
+    assert np.allclose(oracle.hessian(xf, x_is_fp16=True), h0 + 0.01 * np.mean(np.diag(h0)) * np.eye(d),
+                       rtol=1e-13, atol=1e-13)
