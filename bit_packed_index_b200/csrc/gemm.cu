@@ -575,6 +575,71 @@ cudaError_t dispatch(const Layer& L, int mode, const CUtensorMap& ma, const CUte
   return launch_kernel<kFused, 0, 0, MSUB>(ma, mb, g, smem, grid, stream);
 }
 
+// ---------------------------------------------------------------------------
+// Hessian collection: H = X^T X on the same tcgen05 pipeline (staged form,
+// A = B = X^T with the tokens as the contraction), then the normalisation
+// and damping of "VPTQ Guide", section "Step 1: Hessian Matrix Collection":
+// h = 2 H / n, h[i][i] += 0.01 * mean_i h[i][i].
+// ---------------------------------------------------------------------------
+
+// xt[i][t] = x[t][i] (t < n, i < d), through 32 x 32 shared-memory tiles.
+__global__ void hess_transpose(const uint16_t* __restrict__ x, int64_t ldx, int n, int d,
+                               uint16_t* __restrict__ xt, int64_t ldt) {
+  __shared__ uint16_t tile[32][33];
+  const int t0 = blockIdx.x * 32, i0 = blockIdx.y * 32;
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    const int t = t0 + r, i = i0 + threadIdx.x;
+    tile[r][threadIdx.x] = (t < n && i < d) ? x[static_cast<int64_t>(t) * ldx + i] : static_cast<uint16_t>(0);
+  }
+  __syncthreads();
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    const int i = i0 + r, t = t0 + threadIdx.x;
+    if (i < d && t < n) xt[static_cast<int64_t>(i) * ldt + t] = tile[threadIdx.x][r];
+  }
+}
+
+// damp = 0.01 * mean_i (2 / n) h[i][i], in fp64 (one block).
+__global__ void hess_damp(const float* __restrict__ h, int64_t ldh, int d, double two_over_n,
+                          double* __restrict__ damp) {
+  __shared__ double red[256];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) s += static_cast<double>(h[static_cast<int64_t>(i) * ldh + i]);
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *damp = 0.01 * (red[0] * two_over_n / d);
+}
+
+// h[i][j] = fp32((2 / n) h[i][j] + (i == j ? damp : 0)), one rounding.
+__global__ void hess_scale(float* __restrict__ h, int64_t ldh, int d, double two_over_n,
+                           const double* __restrict__ damp) {
+  const int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (k >= static_cast<int64_t>(d) * d) return;
+  const int i = static_cast<int>(k / d), j = static_cast<int>(k % d);
+  float* p = h + static_cast<int64_t>(i) * ldh + j;
+  *p = static_cast<float>(static_cast<double>(*p) * two_over_n + (i == j ? *damp : 0.0));
+}
+
+// Instruction descriptor for kind::f16 with bf16 A and B (atype = btype = 1).
+constexpr uint32_t bf16_idesc(int m, int n) { return f16_idesc(m, n) | (1u << 7) | (1u << 10); }
+
+struct HessLayout {
+  int64_t ldt;
+  size_t off_xt, off_damp, total;
+};
+
+HessLayout hess_layout(int n, int d) {
+  HessLayout h;
+  h.ldt = (static_cast<int64_t>(n) + 7) / 8 * 8;
+  h.off_xt = 256;
+  h.off_damp = h.off_xt + round256(static_cast<size_t>(d) * h.ldt * 2);
+  h.total = h.off_damp + 256;
+  return h;
+}
+
 }  // namespace
 
 size_t gemm_workspace_bytes(const Layer& L, int m, bool x_fp16) {
@@ -667,6 +732,63 @@ vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t
   dim3 grid((m + BM * msub - 1) / (BM * msub), (L.n + bn - 1) / bn);
   return cuda_status(msub == 2 ? dispatch<2>(L, lay.mode, ma, mb, g, smem, grid, stream)
                                : dispatch<1>(L, lay.mode, ma, mb, g, smem, grid, stream));
+}
+
+}  // namespace vqk
+
+
+namespace vqk {
+
+size_t hessian_workspace_bytes(int n, int d) { return (n < 1 || d < 1) ? 0 : hess_layout(n, d).total; }
+
+vq_status launch_hessian(const void* x, bool x_fp16, int n, int d, int64_t ldx, float* h, int64_t ldh,
+                         void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const HessLayout lay = hess_layout(n, d);
+  if (ws_bytes < lay.total) return VQ_ERR_WORKSPACE;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(w8);
+  uint16_t* xt = reinterpret_cast<uint16_t*>(w8 + lay.off_xt);
+  double* damp = reinterpret_cast<double*>(w8 + lay.off_damp);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  count_launch();
+  hess_transpose<<<dim3((n + 31) / 32, (d + 31) / 32), dim3(32, 8), 0, stream>>>(
+      static_cast<const uint16_t*>(x), ldx, n, d, xt, lay.ldt);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+
+  int msub = 1, bn = BN;
+  choose_tiles(d, d, device_sm_count(), &msub, &bn);
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, xt, n, d, lay.ldt, BM) || !make_map(&mb, xt, n, d, lay.ldt, bn)) return VQ_ERR_CUDA;
+  GemmArgs g{};
+  g.L.n = d;
+  g.L.kin = n;
+  g.m = d;
+  g.num_kt = (n + BK - 1) / BK;
+  g.rowsum = nullptr;
+  g.y = h;
+  g.yt = VQ_FP32;
+  g.ldy = ldh;
+  g.status = status;
+  const int optin = device_smem_optin();
+  const int kStageBytes = stage_bytes(msub);
+  const size_t fixed = 1024 + 3072;
+  g.stages = std::min(4, static_cast<int>((optin - fixed) / kStageBytes));
+  const size_t smem = fixed + static_cast<size_t>(g.stages) * kStageBytes;
+  g.bn = bn;
+  g.idesc = x_fp16 ? f16_idesc(BM, bn) : bf16_idesc(BM, bn);
+  dim3 grid((d + BM * msub - 1) / (BM * msub), (d + bn - 1) / bn);
+  e = msub == 2 ? launch_kernel<kStaged, 0, 0, 2>(ma, mb, g, smem, grid, stream)
+                : launch_kernel<kStaged, 0, 0, 1>(ma, mb, g, smem, grid, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  const double two_over_n = 2.0 / static_cast<double>(n);
+  count_launch();
+  hess_damp<<<1, 256, 0, stream>>>(h, ldh, d, two_over_n, damp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+  const int64_t cnt = static_cast<int64_t>(d) * d;
+  count_launch();
+  hess_scale<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, stream>>>(h, ldh, d, two_over_n, damp);
+  return cuda_status(cudaGetLastError());
 }
 
 }  // namespace vqk

@@ -180,6 +180,25 @@ using namespace vqk;
 
 extern "C" {
 
+vq_status vq_hessian_workspace_size(int32_t n_tokens, int32_t d_in, size_t* bytes) {
+  if (!bytes || n_tokens < 0 || d_in < 0) return VQ_ERR_INVALID_ARG;
+  *bytes = hessian_workspace_bytes(n_tokens, d_in);
+  return VQ_OK;
+}
+
+vq_status vq_hessian(const void* x, vq_dtype x_dtype, int32_t n_tokens, int32_t d_in, int64_t ldx, float* h,
+                     int64_t ldh, void* workspace, size_t workspace_bytes, void* stream) {
+  if (n_tokens < 1 || d_in < 0 || ldx < d_in || ldh < d_in || !dtype_ok_in(x_dtype)) return VQ_ERR_INVALID_ARG;
+  if (d_in == 0) return VQ_OK;
+  if (!x || !h) return VQ_ERR_INVALID_ARG;
+  if (!aligned(x, 2) || !aligned(h, 4)) return VQ_ERR_ALIGNMENT;
+  const size_t need = hessian_workspace_bytes(n_tokens, d_in);
+  if (!workspace || workspace_bytes < need) return VQ_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return VQ_ERR_ALIGNMENT;
+  return launch_hessian(x, x_dtype == VQ_FP16, n_tokens, d_in, ldx, h, ldh, workspace, workspace_bytes,
+                        static_cast<cudaStream_t>(stream));
+}
+
 vq_status vq_gemv_multi_workspace_size(const vq_layer_desc* const* layers, int32_t n_layers, int32_t batch,
                                        size_t* bytes) {
   if (!bytes) return VQ_ERR_INVALID_ARG;

@@ -82,6 +82,11 @@ vq_status plan_gemv(const Layer& L, int batch, GemvPlan* plan, size_t ws_cap = ~
 // Lookup-table plans (tiled order; a batch runs one table pass per row of x,
 // up to a per-layer limit); false when no table kernel applies.
 bool plan_gemv_lut(const Layer& L, int batch, size_t ws_cap, GemvPlan* plan);
+// Hessian of a layer's inputs on the tensor cores (gemm.cu).
+size_t hessian_workspace_bytes(int n_tokens, int d);
+vq_status launch_hessian(const void* x, bool x_fp16, int n_tokens, int d, int64_t ldx, float* h, int64_t ldh,
+                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 // Layers sharing x in one table launch (tiled 2^16 books, batch 1).
 struct LutMultiPlan {
   int grid;

@@ -5,8 +5,8 @@ turns torch tensors into pointers, sizes and the current CUDA stream.  There
 is no fallback: if ``libvq.so`` is missing or fails to load, every call raises.
 
 Names follow the C ABI: ``dequant``, ``gemv``, ``gemv_multi``, ``gemv_rht``,
-``rht``, ``gemm``, ``repack_tile4``, ``encode``, plus the workspace size
-queries.  A ``Layer`` holds the device tensors of one
+``rht``, ``gemm``, ``repack_tile4``, ``encode``, ``hessian``, plus the
+workspace size queries.  A ``Layer`` holds the device tensors of one
 quantised layer (packed index streams in row order or in the tiled order,
 fp16 codebooks, optional fp16 scale and bias).
 """
@@ -95,12 +95,15 @@ def lib():
             L.vq_rht.argtypes = [P, C.c_int, I32, I32, I64, P, I32, P, C.c_int, I64, P]
             L.vq_gemv_rht_workspace_size.argtypes = [P, I32, C.POINTER(SZ)]
             L.vq_gemv_rht.argtypes = [P, P, P, P, C.c_int, I32, I64, P, C.c_int, I64, P, SZ, P]
+            L.vq_hessian_workspace_size.argtypes = [I32, I32, C.POINTER(SZ)]
+            L.vq_hessian.argtypes = [P, C.c_int, I32, I32, I64, P, I64, P, SZ, P]
             L.vq_encode_workspace_size.argtypes = [P, C.POINTER(SZ)]
             L.vq_encode.argtypes = [P, P, SZ, P]
             for fn in ("vq_dequant", "vq_gemv_workspace_size", "vq_gemv", "vq_gemv_noalloc",
                        "vq_gemm_workspace_size", "vq_gemm", "vq_repack_tile4",
                        "vq_encode_workspace_size", "vq_encode", "vq_gemv_multi_workspace_size",
-                       "vq_gemv_multi", "vq_rht", "vq_gemv_rht_workspace_size", "vq_gemv_rht"):
+                       "vq_gemv_multi", "vq_rht", "vq_gemv_rht_workspace_size", "vq_gemv_rht",
+                       "vq_hessian_workspace_size", "vq_hessian"):
                 getattr(L, fn).restype = C.c_int
             L.vq_status_string.argtypes = [C.c_int]
             L.vq_status_string.restype = C.c_char_p
@@ -389,6 +392,22 @@ def gemv_rht(layer: Layer, signs_in: torch.Tensor, signs_out: torch.Tensor, x: t
     _check("vq_gemv_rht", lib().vq_gemv_rht(C.byref(layer.desc()), _ptr(signs_in), _ptr(signs_out), _ptr(x),
                                             _DTYPE[x.dtype], batch, ldx, _ptr(out), _DTYPE[out.dtype], ldy,
                                             _ptr(ws), ws_bytes, C.c_void_p(_stream(layer.device))))
+    return out
+
+
+def hessian(x: torch.Tensor, out: Optional[torch.Tensor] = None,
+            workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """h = 2 X^T X / n + 0.01 mean(diag) I (float32 [d][d]) of activations x
+    (bf16 or fp16 [n_tokens][d] on the device), through vq_hessian."""
+    n, d = x.shape
+    if out is None:
+        out = torch.empty((d, d), dtype=torch.float32, device=x.device)
+    nb = C.c_size_t(0)
+    _check("vq_hessian_workspace_size", lib().vq_hessian_workspace_size(n, d, C.byref(nb)))
+    ws, ws_bytes = _workspace(nb.value, x.device, workspace)
+    ldx = x.stride(0) if n > 1 else max(d, 1)
+    _check("vq_hessian", lib().vq_hessian(_ptr(x), _DTYPE[x.dtype], n, d, ldx, _ptr(out), out.stride(0),
+                                          _ptr(ws), ws_bytes, C.c_void_p(_stream(x.device))))
     return out
 
 

@@ -384,6 +384,24 @@ VQ_API vq_status vq_gemv_rht(const vq_layer_desc* layer, const uint32_t* signs_i
                              int32_t batch, int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy,
                              void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * vq_hessian -- the normalised, damped Hessian of a layer's inputs ("VPTQ
+ * Guide", section "Step 1: Hessian Matrix Collection"; section "1.
+ * Second-Order Hessian-Weighted Optimization": H = 2 X X^T over the tokens):
+ *   h = 2 X^T X / n_tokens,  h[i][i] += 0.01 * mean_i h[i][i]
+ * X: device, x_dtype (VQ_BF16 or VQ_FP16) [n_tokens][ldx], d_in columns
+ * used; h: device fp32 [d_in][ldh].  X^T X runs on the tcgen05 tensor cores
+ * (bf16 or fp16 operands as given, exact products, fp32 accumulation); the
+ * normalisation and damping in fp64, rounded once to fp32.  The workspace
+ * (vq_hessian_workspace_size, 256-byte aligned) holds X^T and a status word
+ * (first 32 bits: VQ_OK or VQ_ERR_TIMEOUT).
+ * Errors: VQ_ERR_INVALID_ARG (n_tokens < 1, short strides, NULL buffers),
+ * VQ_ERR_ALIGNMENT, VQ_ERR_WORKSPACE, VQ_ERR_CUDA.
+ */
+VQ_API vq_status vq_hessian_workspace_size(int32_t n_tokens, int32_t d_in, size_t* bytes);
+VQ_API vq_status vq_hessian(const void* x, vq_dtype x_dtype, int32_t n_tokens, int32_t d_in, int64_t ldx,
+                            float* h, int64_t ldh, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Static description of a status code (never NULL). */
 VQ_API const char* vq_status_string(vq_status status);
 

@@ -20,7 +20,8 @@ def test_every_declared_symbol_is_exported(lib):
                           "vq_status_string", "vq_last_cuda_error", "vq_abi_version",
                           "vq_kernel_launches", "vq_encode_workspace_size", "vq_encode",
                           "vq_gemv_multi_workspace_size", "vq_gemv_multi", "vq_rht",
-                          "vq_gemv_rht_workspace_size", "vq_gemv_rht"}
+                          "vq_gemv_rht_workspace_size", "vq_gemv_rht", "vq_hessian_workspace_size",
+                          "vq_hessian"}
     for n in names:
         assert hasattr(lib, n), n
 
