@@ -25,6 +25,7 @@ encode = the nearest-centroid encoder (vq_encode) on a 4096 x 4096 matrix
          against one K = 2^16, d = 8 book, in (vector, centroid) pairs/s.
 rht_gate = the 70B gate_proj in the rotated basis (vq_gemv_rht) beside the
          same layer through vq_gemv.
+hessian = vq_hessian on 8192 tokens x 8192 features, in TFLOP/s.
 roofline, cpu_baseline, clocks and gpu_launches are described beside the
 keys they fill.  ``--impl reference`` times the CPU oracle on the same
 metric instead (a bounded sample of the same workload per step).
@@ -72,6 +73,8 @@ ENCODE_SHAPE = (4096, 4096, 8, [16])
 ENCODE_STD = [0.02]
 ENCODE_SEED = 11
 RHT_SEED = 12           # sign bits of the rotated-basis measurement
+HESSIAN_SHAPE = (8192, 8192)   # tokens, features
+HESSIAN_SEED = 13
 
 
 def kernel_sources_sha(files) -> str:
@@ -424,6 +427,7 @@ def run_gpu(args):
     gemm = run_gemm(dev, peaks, peak_src, vq)
     decode_405b = run_decode_405b(dev, peaks, peak_src, vq)
     rht = run_rht(dev, vq)
+    hess = run_hessian(dev, peaks, peak_src, vq)
     encode = run_encode(dev, peaks, peak_src, vq,
                         with_oracle=rank == 0 and world == 1 and not args.no_cpu_baseline)
 
@@ -442,6 +446,7 @@ def run_gpu(args):
         "gemm": gemm,
         "decode_405b_gate": decode_405b,
         "rht_gate": rht,
+        "hessian": hess,
         "encode": encode,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -619,6 +624,34 @@ def run_rht(dev, vq):
                         "(blocks of 8192 on x, 4096 on y)",
             "us": rot, "us_without_rotation": plain, "rotation_overhead_us": rot - plain,
             "achieved_gbs": alg_bytes(spec, 1) / (rot * 1e-6) / 1e9}
+
+
+def run_hessian(dev, peaks, peak_src, vq):
+    """Beside the headline: the Hessian of a layer's inputs (vq_hessian) for
+    8192 bf16 activation tokens of 8192 features (X ~ N(0, 1), 0.1 % outlier
+    columns x20), in TFLOP/s of the X^T X contraction."""
+    import torch
+    n, d = HESSIAN_SHAPE
+    x = synth.make_x(HESSIAN_SEED, n, d, 0.001)
+    xd = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+    out = torch.empty((d, d), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(256, vq.hessian_workspace_size(n, d)), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        vq.hessian(xd, out=out, workspace=ws)
+    times = []
+    for _ in range(10):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        vq.hessian(xd, out=out, workspace=ws)
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    tf = 2.0 * n * d * d / (ms * 1e-3) / 1e12
+    return {"workload": f"hessian: {n} bf16 tokens x {d} features -> fp32 [{d}][{d}]",
+            "ms": ms, "tflops": tf, "device_status": int(ws[:4].view(torch.int32).item()),
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tf / peaks["bf16_tflops"], "peak_source": peak_src + " (bf16 burst)"}}
 
 
 def run_profile(args):

@@ -395,6 +395,12 @@ def gemv_rht(layer: Layer, signs_in: torch.Tensor, signs_out: torch.Tensor, x: t
     return out
 
 
+def hessian_workspace_size(n_tokens: int, d: int) -> int:
+    nb = C.c_size_t(0)
+    _check("vq_hessian_workspace_size", lib().vq_hessian_workspace_size(n_tokens, d, C.byref(nb)))
+    return nb.value
+
+
 def hessian(x: torch.Tensor, out: Optional[torch.Tensor] = None,
             workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
     """h = 2 X^T X / n + 0.01 mean(diag) I (float32 [d][d]) of activations x
@@ -402,9 +408,7 @@ def hessian(x: torch.Tensor, out: Optional[torch.Tensor] = None,
     n, d = x.shape
     if out is None:
         out = torch.empty((d, d), dtype=torch.float32, device=x.device)
-    nb = C.c_size_t(0)
-    _check("vq_hessian_workspace_size", lib().vq_hessian_workspace_size(n, d, C.byref(nb)))
-    ws, ws_bytes = _workspace(nb.value, x.device, workspace)
+    ws, ws_bytes = _workspace(hessian_workspace_size(n, d), x.device, workspace)
     ldx = x.stride(0) if n > 1 else max(d, 1)
     _check("vq_hessian", lib().vq_hessian(_ptr(x), _DTYPE[x.dtype], n, d, ldx, _ptr(out), out.stride(0),
                                           _ptr(ws), ws_bytes, C.c_void_p(_stream(x.device))))
