@@ -426,6 +426,7 @@ def run_gpu(args):
 
     gemm = run_gemm(dev, peaks, peak_src, vq)
     decode_405b = run_decode_405b(dev, peaks, peak_src, vq)
+    qkv_405b = run_405b_qkv(dev, peaks, peak_src, vq)
     rht = run_rht(dev, vq)
     hess = run_hessian(dev, peaks, peak_src, vq)
     encode = run_encode(dev, peaks, peak_src, vq,
@@ -445,6 +446,7 @@ def run_gpu(args):
         "clocks": clocks.summary(),
         "gemm": gemm,
         "decode_405b_gate": decode_405b,
+        "decode_405b_qkv": qkv_405b,
         "rht_gate": rht,
         "hessian": hess,
         "encode": encode,
@@ -526,6 +528,39 @@ def run_decode_405b(dev, peaks, peak_src, vq):
                         "B=1, tiled index order (small-book lookup-table kernel)",
             "us": ms * 1e3, "achieved_gbs": gbs, "frac_of_measured_hbm": gbs / peaks["hbm_gbs"],
             "algorithmic_bytes": alg_bytes(spec, 1), "peak_source": peak_src}
+
+
+def run_405b_qkv(dev, peaks, peak_src, vq):
+    """Beside the headline: the Llama-3.1-405B q/k/v projections (16384, 1024
+    and 1024 rows x 16384, d = 6, K = 2^12 + 2^4) reading the same x, tiled, as
+    one vq_gemv_multi call; L2 flushed between timed calls."""
+    import torch
+    w = WORKLOADS["llama31_405b"]
+    specs = [w.layers[li][0] for li in (0, 1, 2)]
+    layers = [vq.Layer.from_synth(synth.make_layer(*w.layers[li]), dev, layout="tile4") for li in (0, 1, 2)]
+    x = torch.from_numpy(synth.make_x(w.x_seed, 1, specs[0].in_features).view(np.int16)).to(dev)
+    x = x.view(torch.bfloat16)
+    outs = [torch.empty((1, s.out_features), dtype=torch.bfloat16, device=dev) for s in specs]
+    ws = torch.empty(max(256, vq.gemv_multi_workspace_size(layers, 1)), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        vq.gemv_multi(layers, x, outs=outs, workspace=ws)
+    times = []
+    for _ in range(20):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        vq.gemv_multi(layers, x, outs=outs, workspace=ws)
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    nbytes = sum(alg_bytes(s, 1) for s in specs)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": "llama31_405b q_proj + k_proj + v_proj (16384/1024/1024 x 16384), d=6, "
+                        "K=2^12 + residual K=2^4, B=1, tiled, one vq_gemv_multi call",
+            "us": ms * 1e3, "achieved_gbs": gbs, "frac_of_measured_hbm": gbs / peaks["hbm_gbs"],
+            "algorithmic_bytes": nbytes, "peak_source": peak_src}
 
 
 def run_encode(dev, peaks, peak_src, vq, with_oracle: bool):
@@ -660,7 +695,14 @@ def run_profile(args):
     import torch
     from bit_packed_index_b200 import vq
     dev = torch.device("cuda", 0)
-    if args.profile == "encode":
+    if args.profile == "hessian":
+        n, d = HESSIAN_SHAPE
+        x = torch.from_numpy(synth.make_x(HESSIAN_SEED, n, d, 0.001).view(np.int16)).to(dev).view(torch.bfloat16)
+        out = torch.empty((d, d), dtype=torch.float32, device=dev)
+        ws = torch.empty(vq.hessian_workspace_size(n, d), dtype=torch.uint8, device=dev)
+        for _ in range(args.profile_launches):
+            vq.hessian(x, out=out, workspace=ws)
+    elif args.profile == "encode":
         n, kin, d, log2k = ENCODE_SHAPE
         w, books = synth.make_encode_input(n, kin, d, log2k, ENCODE_STD, seed=ENCODE_SEED)
         W = torch.from_numpy(w.view(np.int16)).to(dev).view(torch.float16)
@@ -717,12 +759,12 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", choices=["gemv", "lut", "lut_gateup", "lut_down", "lut_small", "gemm",
-                                          "dequant", "encode"],
+                                          "dequant", "encode", "hessian"],
                     help="run a few untimed launches of one call on its workload (for ncu): "
                          "gemv / lut = 70B gate_proj in row / tiled order, lut_gateup = 70B "
                          "gate_proj + up_proj in one vq_gemv_multi launch, lut_down = 70B "
                          "down_proj in tiled order, lut_small = 405B gate_proj in tiled order, "
-                         "encode = the encoder on its bench workload")
+                         "encode / hessian = the encoder / the Hessian on their bench workloads")
     ap.add_argument("--profile-launches", type=int, default=3)
     args = ap.parse_args(argv)
     if args.profile:
