@@ -279,6 +279,21 @@ __device__ __forceinline__ float lut_pair_bfrag(const uint16_t* __restrict__ x, 
   return __uint_as_float(static_cast<uint32_t>(127 + e) << 23);   // 2^e (inf for e = 128)
 }
 
+// e with mx = m * 2^e, 0.5 <= m < 1, from the float bits (-126 for a
+// subnormal mx; 0 when mx is zero or not finite), and x * 2^-e as two exact
+// power-of-two factors (each a normal float for e in [-126, 128]).
+__device__ __forceinline__ int lut_exp(float mx) {
+  return (mx > 0.0f && mx < INFINITY) ? static_cast<int>(__float_as_uint(mx) >> 23) - 126 : 0;
+}
+__device__ __forceinline__ float lut_scale_down(float v, int e) {
+  const float f1 = __uint_as_float(static_cast<uint32_t>(127 - e / 2) << 23);
+  const float f2 = __uint_as_float(static_cast<uint32_t>(127 - (e - e / 2)) << 23);
+  return v * f1 * f2;
+}
+__device__ __forceinline__ float lut_pow2(int e) {               // 2^e (inf for e = 128)
+  return __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+}
+
 // One 32-centroid tile: D = A x B (fp32), A = afr (rows g and g+8 of the
 // tile, each an 8-byte load), then the eight table entries of this lane in
 // fp16.  Lane (n, t) owns T[32*tile + 2n + t/2][2(t%2), +1] and the same for
@@ -645,11 +660,10 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_small_kernel(Layer L,
       float mx = l1;
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      int e = 0;
-      if (mx > 0.0f && mx < INFINITY) frexpf(mx, &e);
-      const __half2 h = __floats2half2_rn(ldexpf(a, -e), ldexpf(b, -e));
+      const int e = lut_exp(mx);
+      const __half2 h = __floats2half2_rn(lut_scale_down(a, e), lut_scale_down(b, e));
       bfrag = *reinterpret_cast<const uint32_t*>(&h);
-      if (tid == 0) s_scale = ldexpf(1.0f, e);
+      if (tid == 0) s_scale = lut_pow2(e);
       if (warp == 0) {
         float v = a + b;
 #pragma unroll
@@ -809,11 +823,10 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_pair_kernel(LutSet S,
       float mx = l1;
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      int e = 0;
-      if (mx > 0.0f && mx < INFINITY) frexpf(mx, &e);
-      const __half2 h = __floats2half2_rn(ldexpf(a, -e), ldexpf(b, -e));
+      const int e = lut_exp(mx);
+      const __half2 h = __floats2half2_rn(lut_scale_down(a, e), lut_scale_down(b, e));
       bfrag = *reinterpret_cast<const uint32_t*>(&h);
-      if (tid == 0) s_scale = ldexpf(1.0f, e);
+      if (tid == 0) s_scale = lut_pow2(e);
       if (warp == 0 && l == 0) {                    // each group of x once
         float v = a + b;
 #pragma unroll
