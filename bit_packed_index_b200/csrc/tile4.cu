@@ -365,6 +365,9 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(LutSet S, cons
     sm100::tmem_alloc(&s_tmem, TCOLS);
     sm100::tmem_relinquish();
   }
+  // The reduction launch may be scheduled now; it waits for this grid's
+  // completion (griddepcontrol.wait) before reading anything.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
@@ -631,6 +634,9 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_small_kernel(Layer L,
     sm100::tmem_alloc(&s_tmem, TCOLS);
     sm100::tmem_relinquish();
   }
+  // The reduction launch may be scheduled now; it waits for this grid's
+  // completion (griddepcontrol.wait) before reading anything.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
@@ -788,6 +794,9 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_pair_kernel(LutSet S,
     sm100::tmem_alloc(&s_tmem, TCOLS);
     sm100::tmem_relinquish();
   }
+  // The reduction launch may be scheduled now; it waits for this grid's
+  // completion (griddepcontrol.wait) before reading anything.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
@@ -933,6 +942,9 @@ LutOut lut_out_single(const Layer& L, void* y) {
 __global__ void __launch_bounds__(256, 8) gemv_lut_finalize(const float* __restrict__ part,
                                                             const float* __restrict__ xpart, int nparts,
                                                             int ntot, LutOut out, vq_dtype yt) {
+  // Launched as a programmatic dependent of the table kernel: wait for that
+  // grid to complete and its writes to be visible (a no-op otherwise).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ float red[8][33];
   __shared__ float s_xsum;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -973,6 +985,24 @@ __global__ void __launch_bounds__(256, 8) gemv_lut_finalize(const float* __restr
   }
 }
 
+// The reduction of a table launch, as a programmatic dependent launch: its
+// blocks are scheduled while the table kernel drains, instead of after it.
+cudaError_t launch_finalize(const float* part, const float* xpart, int nparts, int ntot, const LutOut& out,
+                            vq_dtype yt, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((ntot + 31) / 32);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, gemv_lut_finalize, part, xpart, nparts, ntot, out, yt);
+}
+
 // The layers of S share x; their partial sums take S.row0[S.nl] rows per block.
 template <int RB8, int LB>
 cudaError_t launch_lut_set(const LutSet& S, const LutOut& out, int grid, const void* x, bool x_fp16,
@@ -986,9 +1016,7 @@ cudaError_t launch_lut_set(const LutSet& S, const LutOut& out, int grid, const v
   count_launch();
   k<<<grid, kLutThreads, kLutSmem, stream>>>(S, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, part, xpart);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  count_launch();
-  gemv_lut_finalize<<<(ntot + 31) / 32, 256, 0, stream>>>(part, xpart, grid, ntot, out, yt);
-  return cudaGetLastError();
+  return launch_finalize(part, xpart, grid, ntot, out, yt, stream);
 }
 
 LutSet lut_set_single(const Layer& L) {
@@ -1063,10 +1091,8 @@ cudaError_t launch_lut_small(const Layer& L, const GemvPlan& p, const void* x, b
                   : launch_lut_small_t<RB8, 6, 2>(L, p, x, x_fp16, ws, stream);
   }
   if (e != cudaSuccess) return e;
-  count_launch();
-  gemv_lut_finalize<<<(L.n + 31) / 32, 256, 0, stream>>>(ws, ws + static_cast<int64_t>(p.grid_x) * L.n,
-                                                        p.grid_x, L.n, lut_out_single(L, y), yt);
-  return cudaGetLastError();
+  return launch_finalize(ws, ws + static_cast<int64_t>(p.grid_x) * L.n, p.grid_x, L.n, lut_out_single(L, y), yt,
+                         stream);
 }
 
 // Tables of the small-book kernels: fp16 [K][4] per book, or fp32 [4][K] on
@@ -1192,10 +1218,7 @@ cudaError_t launch_gemv_lut_multi(const Layer* L, int nl, const LutMultiPlan& p,
              : launch_lut_pair_set<4, 8, 8, 1>(S, p.grid, p.smem, x, x_fp16, ws, stream);
     if (e != cudaSuccess) return e;
     const int ntot = S.row0[nl];
-    count_launch();
-    gemv_lut_finalize<<<(ntot + 31) / 32, 256, 0, stream>>>(ws, ws + static_cast<int64_t>(p.grid) * ntot,
-                                                            p.grid, ntot, out, yt);
-    return cudaGetLastError();
+    return launch_finalize(ws, ws + static_cast<int64_t>(p.grid) * ntot, p.grid, ntot, out, yt, stream);
   }
   if (p.rb8 == 2) return launch_lut_set<2, 1>(S, out, p.grid, x, x_fp16, yt, ws, stream);
   if (p.rb8 == 4) return p.lb == 1 ? launch_lut_set<4, 1>(S, out, p.grid, x, x_fp16, yt, ws, stream)
