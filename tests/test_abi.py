@@ -170,3 +170,37 @@ def test_encode_workspace_and_validation_need_no_device(lib):
     e.idx_row_words[0] = 4
     # vq_encode itself: NULL buffers with data are rejected before any launch
     assert lib.vq_encode(C.byref(e), None, 0, None) == vq.VQ_ERR_INVALID_ARG
+
+
+def test_new_entry_points_validate_before_any_device_call(lib):
+    """Host-side checks of vq_rht, vq_hessian(_workspace_size), vq_gemv_rht
+    and vq_gemv_multi: malformed arguments return a status and launch nothing."""
+    P = C.c_void_p
+    # vq_rht: negative sizes, short strides, bad dtype, NULL buffers with data
+    assert lib.vq_rht(None, vq.VQ_FP32, -1, 8, 8, None, 0, None, vq.VQ_FP32, 8, None) == vq.VQ_ERR_INVALID_ARG
+    assert lib.vq_rht(None, vq.VQ_FP32, 2, 8, 4, None, 0, None, vq.VQ_FP32, 8, None) == vq.VQ_ERR_INVALID_ARG
+    assert lib.vq_rht(None, 7, 2, 8, 8, None, 0, None, vq.VQ_FP32, 8, None) == vq.VQ_ERR_INVALID_ARG
+    assert lib.vq_rht(None, vq.VQ_FP32, 2, 8, 8, None, 0, None, vq.VQ_FP32, 8, None) == vq.VQ_ERR_INVALID_ARG
+    assert lib.vq_rht(None, vq.VQ_FP32, 0, 8, 8, None, 0, None, vq.VQ_FP32, 8, None) == vq.VQ_OK
+    assert lib.vq_rht(P(16), vq.VQ_FP32, 70000, 8, 8, P(16), 0, P(16), vq.VQ_FP32, 8, None) == \
+        vq.VQ_ERR_UNSUPPORTED
+    assert lib.vq_rht(P(18), vq.VQ_FP32, 2, 8, 8, P(16), 0, P(16), vq.VQ_FP32, 8, None) == vq.VQ_ERR_ALIGNMENT
+    # vq_hessian: workspace arithmetic (X^T copy rows padded to 8 tokens) and checks
+    n = C.c_size_t(0)
+    assert lib.vq_hessian_workspace_size(100, 64, C.byref(n)) == vq.VQ_OK
+    assert n.value == 256 + (-(-(64 * 104 * 2) // 256) * 256) + 256
+    assert lib.vq_hessian_workspace_size(-1, 64, C.byref(n)) == vq.VQ_ERR_INVALID_ARG
+    assert lib.vq_hessian(None, vq.VQ_BF16, 0, 64, 64, None, 64, None, 0, None) == vq.VQ_ERR_INVALID_ARG
+    assert lib.vq_hessian(None, vq.VQ_BF16, 10, 64, 32, None, 64, None, 0, None) == vq.VQ_ERR_INVALID_ARG
+    assert lib.vq_hessian(None, vq.VQ_FP32, 10, 64, 64, None, 64, None, 0, None) == vq.VQ_ERR_INVALID_ARG
+    assert lib.vq_hessian(P(16), vq.VQ_BF16, 10, 64, 64, P(16), 64, None, 0, None) == vq.VQ_ERR_WORKSPACE
+    # vq_gemv_multi / vq_gemv_rht: empty or malformed descriptions
+    arr = (C.c_void_p * 1)()
+    assert lib.vq_gemv_multi(arr, 0, None, vq.VQ_BF16, 1, 8, None, vq.VQ_BF16, None, None, 0, None) == \
+        vq.VQ_ERR_INVALID_ARG
+    assert lib.vq_gemv_multi(None, 2, None, vq.VQ_BF16, 1, 8, None, vq.VQ_BF16, None, None, 0, None) == \
+        vq.VQ_ERR_INVALID_ARG
+    d = vq._Desc()
+    d.out_features, d.in_features, d.vec_dim, d.n_books = 4, 16, 0, 1   # d = 0
+    assert lib.vq_gemv_rht(C.byref(d), None, None, None, vq.VQ_BF16, 1, 16, None, vq.VQ_BF16, 4, None, 0,
+                           None) == vq.VQ_ERR_INVALID_ARG
