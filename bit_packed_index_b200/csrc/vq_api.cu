@@ -216,7 +216,9 @@ vq_status vq_gemv_multi(const vq_layer_desc* const* layers, int32_t n_layers, co
   Layer L[kMaxMultiLayers];
   vq_status st = multi_check(layers, n_layers, batch, L);
   if (st != VQ_OK) return st;
-  if (!y || !ldy || !dtype_ok_in(x_dtype) || !dtype_ok_out(y_dtype)) return VQ_ERR_INVALID_ARG;
+  if (!dtype_ok_in(x_dtype) || !dtype_ok_out(y_dtype)) return VQ_ERR_INVALID_ARG;
+  if (batch == 0) return VQ_OK;
+  if (!y || !ldy) return VQ_ERR_INVALID_ARG;
   if (ldx < L[0].kin) return VQ_ERR_INVALID_ARG;
   for (int l = 0; l < n_layers; ++l)
     if (ldy[l] < L[l].n) return VQ_ERR_INVALID_ARG;
