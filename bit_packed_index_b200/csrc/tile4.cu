@@ -9,15 +9,19 @@
 // reorders the sum y[o] = sum_j <x_j, C[i(o, j)]> around the codebook instead
 // of around the rows.  For a group of four vectors j (one tile) and a slice
 // of the 2^16 centroids k (24576, 24576, then 16384) it forms
-// T[k][j] = <x_j, C[k]> once -- a 16 x 8 x 8 tensor-core product per 16
-// centroids -- stores T in shared memory as fp16, and then every row adds the
-// entries its four indices select.  A row's indices sit side by side in the
-// tiled order and consecutive rows follow one another, so each thread reads
-// one 8-byte record per row and a warp reads 256 contiguous bytes.  Each
-// (group, slice) is one task; a block owns every
-// row of the layer for the tasks it runs, and keeps its per-row sums in tensor
-// memory (TMEM) across tasks.  A second kernel adds the per-block sums and
-// applies scale and bias.
+// T[k][j] = <x_j, C[k]> once -- one 16 x 8 x 16 tensor-core product per 32
+// centroids, two centroids per A row -- stores T in shared memory as fp16,
+// and then every row adds the entries its four indices select.  A row's
+// indices sit side by side in the tiled order and consecutive rows follow one
+// another, so each thread reads one 8-byte record per row and a warp reads
+// 256 contiguous bytes.  Each (group, slice) is one task; a block owns every
+// row of the layer for the tasks it runs, and keeps its per-row sums in
+// tensor memory (TMEM) across tasks.  Several layers that read the same x
+// run as one task list, each layer's rows in their own TMEM batches.  A
+// second kernel, launched as a programmatic dependent, adds the per-block
+// sums and applies scale and bias.  Books of at most 2^12 entries use whole
+// tables per group (no slices): gemv_lut_small_kernel and, for 12-bit main
+// books, gemv_lut_pair_kernel.
 #include <algorithm>
 #include <cstdlib>
 
