@@ -346,8 +346,7 @@ __global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
       }
       if (*abort_flag) {   // let copies already in flight land before the block exits
         for (int q = max(0, issued - kEncStages); q < issued; ++q)
-          bounded_wait(&ctrl->full[q % kEncStages], (q / kEncStages) & 1, abort_flag, nullptr,
-                       kEncWaitBudget / 8);
+          drain_phase(&ctrl->full[q % kEncStages], (q / kEncStages) & 1, kEncWaitBudget / 8);
       }
     }
   } else if (warp == 1) {

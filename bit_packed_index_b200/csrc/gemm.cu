@@ -67,10 +67,12 @@ struct GemmArgs {
   int bn;                 // tile width along N (multiple of 32, <= BN)
   uint32_t idesc;         // tcgen05 instruction descriptor for M = 128, N = bn
   const float* rowsum;
+  const float* rowscale;  // 2^e_m of each row of x (its fp16 copy is x * 2^-e_m), or null for 1
   void* y;
   vq_dtype yt;
   int64_t ldy;
   int* status;
+  long long budget;       // SM clocks a wait may take (VQ_WAIT_BUDGET overrides about 2 s)
 };
 
 // Control block at the start of (1024-aligned) dynamic shared memory.
@@ -283,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kt = 0; kt < g.num_kt; ++kt) {
         const int s = kt % g.stages;
         const uint32_t ph = (kt / g.stages) & 1;
-        if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, kWaitBudget)) break;
+        if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, g.budget)) break;
         uint8_t* a = stages + s * kStage;
         mbar_arrive_expect_tx(&ctrl->full[s], MODE == kStaged ? MSUB * kATile + bn * BK * 2 : MSUB * kATile);
 #pragma unroll
@@ -293,9 +295,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued = kt + 1;
       }
       if (*abort_flag) {   // let loads already in flight land before the block exits
+        // (with fused tiles a stage also waits for the producers, who may have
+        // given up: then the time bound, far above a load's latency, ends it)
         for (int kt = max(0, issued - g.stages); kt < issued; ++kt)
-          bounded_wait(&ctrl->full[kt % g.stages], (kt / g.stages) & 1, abort_flag, nullptr,
-                       kWaitBudget / 8);
+          drain_phase(&ctrl->full[kt % g.stages], (kt / g.stages) & 1, kWaitBudget / 64);
       }
     }
   } else if (warp == 1) {
@@ -304,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kt = 0; kt < g.num_kt; ++kt) {
         const int s = kt % g.stages;
         const uint32_t ph = (kt / g.stages) & 1;
-        if (!bounded_wait(&ctrl->full[s], ph, abort_flag, g.status, kWaitBudget)) break;
+        if (!bounded_wait(&ctrl->full[s], ph, abort_flag, g.status, g.budget)) break;
         tc_fence_after();
         const uint32_t a = smem_addr(stages + s * kStage);
         const uint32_t b = a + MSUB * kATile;
@@ -317,6 +320,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&ctrl->empty[s]);
       }
       umma_commit(&ctrl->acc_full);
+      // every product issued has finished before tensor memory is freed, even
+      // when the epilogue gave up waiting for it
+      drain_phase(&ctrl->acc_full, 0, kWaitBudget);
     }
   } else if (warp >= 4) {
     if (MODE == kFused && B1 > 0) {                    // B-tile producers, d = 8 fast path
@@ -341,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int s = kt % g.stages;
         const uint32_t ph = (kt / g.stages) & 1;
-        if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, kWaitBudget)) break;
+        if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, g.budget)) break;
         if (r < bn) d8_store(L, live, kt, cur, stages + s * kStage + MSUB * kATile, r);
         fence_proxy_async_smem();
         mbar_arrive(&ctrl->full[s]);
@@ -351,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kt = 0; kt < g.num_kt; ++kt) {
         const int s = kt % g.stages;
         const uint32_t ph = (kt / g.stages) & 1;
-        if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, kWaitBudget)) break;
+        if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, g.budget)) break;
         uint8_t* btile = stages + s * kStage + MSUB * kATile;
         if (r < bn) {                                  // rows past the tile width stay idle
           if (L.nb == 2) produce_row_generic<2>(L, bv, n0 + r, kt, btile, r);
@@ -364,10 +370,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < 4 + 4 * MSUB) {                         // epilogue: warp & 3 = TMEM lane quarter
       const int q = warp & 3;
       const int sub = (warp - 4) >> 2;                 // which 128-row sub-tile
-      if (bounded_wait(&ctrl->acc_full, 0, abort_flag, g.status, kWaitBudget)) {
+      if (bounded_wait(&ctrl->acc_full, 0, abort_flag, g.status, g.budget)) {
         tc_fence_after();
         const int row = m0 + sub * BM + q * 32 + lane;
         const float rs = (MODE == kFused && L.bias && row < g.m) ? g.rowsum[row] : 0.0f;
+        const float rsc = (g.rowscale && row < g.m) ? g.rowscale[row] : 1.0f;
         const size_t es = g.yt == VQ_FP32 ? 4 : 2;
         for (int c = 0; c < bn / 32; ++c) {
           uint32_t acc[32];
@@ -378,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            v[i] = ctrl->sb[c * 32 + i] * __uint_as_float(acc[i]) + ctrl->sb[BN + c * 32 + i] * rs;
+            v[i] = ctrl->sb[c * 32 + i] * (__uint_as_float(acc[i]) * rsc) + ctrl->sb[BN + c * 32 + i] * rs;
           const int ncols = min(32, L.n - nb);
           uint8_t* dst = reinterpret_cast<uint8_t*>(g.y) + (static_cast<int64_t>(row) * g.ldy + nb) * es;
           if (ncols == 32 && aligned(dst, 16)) {
@@ -413,10 +420,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// x -> fp16 copy [m][kp] (zeros past kin): one 8-element chunk per thread,
-// 16-byte loads and stores when x rows are 16-byte aligned.
+// Per row of bf16 activations: 2^e with max_k |x[m][k]| * 2^-e in [2^14, 2^15)
+// (e kept in [-126, 127]; 1 for an all-zero row), and the row sum of x.  The
+// fp16 operand copy holds x * 2^-e, so no bf16 value overflows fp16 and every
+// value above 2^-29 of its row's largest stays exact; the epilogue multiplies
+// the accumulator by 2^e.  (For typical rows the scaling changes no bit of y:
+// a power of two commutes with every fp32 rounding of the products.)
+__global__ void gemm_rowscale(const uint16_t* __restrict__ x, int m, int kin, int64_t ldx,
+                              float* __restrict__ rowscale, float* __restrict__ rowsum) {
+  const int warps = blockDim.x >> 5;
+  const int row = blockIdx.x * warps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= m) return;
+  const uint16_t* r = x + static_cast<int64_t>(row) * ldx;
+  float mx = 0.0f, s = 0.0f;
+  for (int k = lane; k < kin; k += 32) {
+    const float v = bf2f(r[k]);
+    mx = fmaxf(mx, fabsf(v));
+    s += v;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    s += __shfl_xor_sync(0xffffffffu, s, off);
+  }
+  if (lane == 0) {
+    int e = 0;
+    if (mx > 0.0f && mx < INFINITY) e = max(-126, min(127, static_cast<int>(__float_as_uint(mx) >> 23) - 126 - 15));
+    rowscale[row] = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+    rowsum[row] = s;
+  }
+}
+
+// x -> fp16 copy [m][kp] (zeros past kin), each row times 1 / rowscale[row]
+// (an exact power of two, applied as two factors so each stays a normal
+// float) when rowscale is given: one 8-element chunk per thread, 16-byte
+// loads and stores when x rows are 16-byte aligned.
 __global__ void gemm_convert(const uint16_t* __restrict__ x, int x_fp16, int m, int kin,
-                             int64_t ldx, int vec, uint16_t* __restrict__ x16, int kp) {
+                             int64_t ldx, int vec, uint16_t* __restrict__ x16, int kp,
+                             const float* __restrict__ rowscale) {
   const int cpr = kp / 8;                                   // chunks per row
   const int64_t total = static_cast<int64_t>(m) * cpr;
   for (int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; q < total;
@@ -433,6 +475,13 @@ __global__ void gemm_convert(const uint16_t* __restrict__ x, int x_fp16, int m, 
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[i] = (k + i < kin) ? (x_fp16 ? h2f(xr[k + i]) : bf2f(xr[k + i])) : 0.0f;
+    }
+    if (rowscale) {
+      const int e = static_cast<int>(__float_as_uint(rowscale[row]) >> 23) - 127;
+      const float f1 = __uint_as_float(static_cast<uint32_t>(127 - e / 2) << 23);
+      const float f2 = __uint_as_float(static_cast<uint32_t>(127 - (e - e / 2)) << 23);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = v[i] * f1 * f2;
     }
     uint32_t p[4];
 #pragma unroll
@@ -477,6 +526,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 128-byte swizzle; reads past cols / rows return zeros.
 bool make_map(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int64_t ld,
               int box_rows) {
+  return make_map_f16_sw128(map, base, cols, rows, ld, box_rows);
+}
+
+}  // namespace
+
+bool make_map_f16_sw128(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int64_t ld,
+                        int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -489,13 +545,22 @@ bool make_map(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, in
   return r == CUDA_SUCCESS;
 }
 
+namespace {
+
 size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+// SM clocks a bounded wait may take: about 2 s, or VQ_WAIT_BUDGET (tests use
+// a few clocks to make the waits give up).
+long long wait_budget() {
+  if (const char* env = std::getenv("VQ_WAIT_BUDGET")) return std::atoll(env);
+  return kWaitBudget;
+}
 
 struct GemmLayout {
   int mode;
   int kp;
   bool copy_x;       // bf16 activations (or misaligned fp16) need an fp16 copy
-  size_t off_rowsum, off_x16, off_w, total;
+  size_t off_rowsum, off_rowscale, off_x16, off_w, total;
 };
 
 bool fused_fast_path(const Layer& L) {
@@ -526,7 +591,8 @@ GemmLayout layout_for(const Layer& L, int m, bool x_fp16) {
   g.kp = (L.kin + 7) / 8 * 8;
   g.copy_x = !x_fp16;   // fp16 activations are read in place (16-byte aligned, ldx % 8 == 0)
   g.off_rowsum = 256;
-  g.off_x16 = g.off_rowsum + round256(static_cast<size_t>(m) * 4);
+  g.off_rowscale = g.off_rowsum + round256(static_cast<size_t>(m) * 4);
+  g.off_x16 = g.off_rowscale + (g.copy_x ? round256(static_cast<size_t>(m) * 4) : 0);
   g.off_w = g.off_x16 + (g.copy_x ? round256(static_cast<size_t>(m) * g.kp * 2) : 0);
   g.total = g.off_w + (g.mode == kStaged ? round256(static_cast<size_t>(L.n) * g.kp * 2) : 0);
   return g;
@@ -656,6 +722,7 @@ vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   int* status = reinterpret_cast<int*>(w8);
   float* rowsum = reinterpret_cast<float*>(w8 + lay.off_rowsum);
+  float* rowscale = reinterpret_cast<float*>(w8 + lay.off_rowscale);
   uint16_t* x16 = reinterpret_cast<uint16_t*>(w8 + lay.off_x16);
   uint16_t* what = reinterpret_cast<uint16_t*>(w8 + lay.off_w);
 
@@ -663,20 +730,25 @@ vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t
     cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), stream);
     if (e != cudaSuccess) return cuda_status(e);
     if (lay.copy_x) {
+      // bf16 activations: per-row power-of-two scale (and the row sums), then
+      // the scaled fp16 copy
+      const int warps = 8;
+      count_launch();
+      gemm_rowscale<<<(m + warps - 1) / warps, warps * 32, 0, stream>>>(static_cast<const uint16_t*>(x), m,
+                                                                         L.kin, ldx, rowscale, rowsum);
+      if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
       const int vec = aligned(x, 16) && ldx % 8 == 0;
       const int64_t chunks = static_cast<int64_t>(m) * (lay.kp / 8);
       const int blocks = static_cast<int>(std::min<int64_t>((chunks + 255) / 256, 16 * device_sm_count()));
       count_launch();
       gemm_convert<<<blocks, 256, 0, stream>>>(static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, m,
-                                              L.kin, ldx, vec, x16, lay.kp);
+                                              L.kin, ldx, vec, x16, lay.kp, rowscale);
       if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
-    }
-    if (lay.mode == kFused && L.bias != nullptr) {   // row sums feed the fused bias term only
+    } else if (lay.mode == kFused && L.bias != nullptr) {   // row sums feed the fused bias term only
       const int warps = 8;
       count_launch();
-      gemm_rowsum<<<(m + warps - 1) / warps, warps * 32, 0, stream>>>(
-          lay.copy_x ? x16 : static_cast<const uint16_t*>(x), m, L.kin,
-          lay.copy_x ? lay.kp : ldx, rowsum);
+      gemm_rowsum<<<(m + warps - 1) / warps, warps * 32, 0, stream>>>(static_cast<const uint16_t*>(x), m, L.kin,
+                                                                       ldx, rowsum);
       if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
     }
   }
@@ -698,15 +770,17 @@ vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t
     mb = ma;
   }
 
-  GemmArgs g;
+  GemmArgs g{};
   g.L = L;
   g.m = m;
   g.num_kt = (L.kin + BK - 1) / BK;
   g.rowsum = rowsum;
+  g.rowscale = lay.copy_x ? rowscale : nullptr;
   g.y = y;
   g.yt = yt;
   g.ldy = ldy;
   g.status = status;
+  g.budget = wait_budget();
   g.smem_mask = 0;
   g.book_bytes = 0;
   const int optin = device_smem_optin();
@@ -770,6 +844,7 @@ vq_status launch_hessian(const void* x, bool x_fp16, int n, int d, int64_t ldx, 
   g.yt = VQ_FP32;
   g.ldy = ldh;
   g.status = status;
+  g.budget = wait_budget();
   const int optin = device_smem_optin();
   const int kStageBytes = stage_bytes(msub);
   const size_t fixed = 1024 + 3072;

@@ -218,10 +218,13 @@ cudaError_t launch_d(const Layer& L, const GemvPlan& p, const void* x, bool xf, 
 
 vq_status plan_gemv(const Layer& L, int batch, GemvPlan* p, size_t ws_cap) {
   if (L.layout == VQ_IDX_TILE4) {
-    // batch 1: the lookup-table kernels; everything else: the split-K gather
+    // small batches: the lookup-table kernels; larger batches of 2^16-book
+    // layers: the tensor-core kernel; everything else: the split-K gather
     // kernel below, reading the tiled records
     if (plan_gemv_lut(L, batch, ws_cap, p)) return VQ_OK;
+    if (plan_gemv_tc(L, batch, ws_cap, p)) return VQ_OK;
   } else {
+    if (batch >= 2 && plan_gemv_tc(L, batch, ws_cap, p)) return VQ_OK;
     if (batch == 1 && gemv1_supported(L)) {
       plan_gemv1(L, p);
       if (p->smem <= device_smem_optin()) return VQ_OK;
@@ -274,7 +277,9 @@ vq_status launch_gemv(const Layer& L, const GemvPlan& p, const void* x, bool x_f
   }
   const int D = (L.d == 8) ? 8 : (L.d == 6 ? 6 : 0);
   cudaError_t e;
-  if (p.fast >= 3) {
+  if (p.fast == 7) {
+    return launch_gemv_tc(L, p, x, x_fp16, batch, ldx, y, yt, ldy, ws, stream);
+  } else if (p.fast >= 3) {
     return cuda_status(launch_gemv_lut(L, p, x, x_fp16, batch, ldx, y, yt, ldy, ws, stream));
   } else if (p.fast == 1) {
     e = launch_gemv1(L, p, x, x_fp16, y, yt, ws, stream);

@@ -1,0 +1,421 @@
+// gemvtc.cu -- batched decode (batch 3..16) on the tcgen05 tensor cores, for
+// layers with one 2^16-entry, d = 8 codebook (row or tiled index order).
+//
+// y[b][o] = sum_k x[b][k] * W_hat[o][k] ("VPTQ Guide", section "Step 3";
+// "Vector Quantization for LLM Weights in Production", section "1. Prefill vs.
+// Decode Bottlenecks": decode at B = 1 to 8 is memory bound; the dequantised
+// vectors feed "GEMV / Tensor Core Dot Products").  With a 2^16-entry book
+// every index costs one random 16-byte centroid gather from L2, whatever the
+// batch; the multiply-adds grow with the batch.  So the products go to the
+// tensor cores and the kernel is built to keep the gathers flowing:
+//
+//  * A CTA owns 128 rows of W (the MMA's M) and a range of the input
+//    dimension in steps of 64 (eight vectors, one 128-byte swizzled row of a
+//    K-major tile).  Four producer warps, one thread per row, read the row's
+//    eight indices of a step and issue eight 16-byte cp.async gathers of the
+//    centroids straight into the swizzled A tile: no register staging, three
+//    steps of gathers in flight per thread, three CTAs per SM.
+//  * x, scaled per batch row by a power of two into fp16 (so no value
+//    overflows and the products stay exact), is the N = 16 operand (the batch
+//    padded with zero rows), brought in by TMA per step.
+//  * One thread issues four tcgen05.mma (M = 128, N = 16, K = 16) per step
+//    into a 16-column fp32 accumulator in tensor memory; the producer warps
+//    then read it back (tcgen05.ld) and apply y = s[o] * acc * 2^e_b +
+//    t[o] * sum_k x[b][k].
+//  * Narrow layers split the input dimension across CTAs; fp32 partials go to
+//    the workspace and a second kernel adds them in split order.
+//  * Every wait is bounded: a wait that runs out records VQ_ERR_TIMEOUT in
+//    the workspace's status word and the block drains and ends.
+#include <algorithm>
+#include <cstdlib>
+
+#include "sm100.cuh"
+
+namespace vqk {
+namespace {
+
+using namespace sm100;
+
+constexpr int kTcRows = 128;                     // W rows per CTA (MMA M)
+constexpr int kTcN = 16;                         // batch rows (MMA N; zero rows past the batch)
+constexpr int kTcK = 64;                         // halves per step: 8 vectors of d = 8
+constexpr int kTcATile = kTcRows * kTcK * 2;     // 16 KB
+constexpr int kTcXTile = kTcN * kTcK * 2;        // 2 KB
+constexpr int kTcStage = kTcATile + kTcXTile;    // 18 KB (a multiple of 1024)
+#ifndef VQ_TC_STAGES
+#define VQ_TC_STAGES 4
+#define VQ_TC_LAG 2
+#define VQ_TC_PER_SM 3
+#endif
+constexpr int kTcStages = VQ_TC_STAGES;
+constexpr int kTcLag = VQ_TC_LAG;                // gather steps a producer keeps in flight
+constexpr int kTcThreads = 256;                  // warp 0: x loads, warp 1: MMA, warps 4-7: rows
+constexpr int kTcProducer0 = 128;
+constexpr int kTcSmem = 2048 + kTcStages * kTcStage;   // control block + alignment slack + stages
+constexpr int kTcPerSm = VQ_TC_PER_SM;
+
+struct TcCtrl {
+  uint64_t full[kTcStages];    // the producers' gathers of a stage landed
+  uint64_t xfull[kTcStages];   // the stage's x tile landed (TMA)
+  uint64_t empty[kTcStages];
+  uint64_t acc;
+  uint32_t tmem;
+  int abort;
+};
+
+struct TcArgs {
+  Layer L;
+  int num_kt;             // steps of the whole input dimension
+  int kt_per_split;
+  int batch;
+  const float* xe;        // 2^e of each batch row (x' = x * 2^-e)
+  const float* xsum;      // sum_k x[b][k]
+  void* y;
+  vq_dtype yt;
+  int64_t ldy;
+  float* part;            // [nsplit][batch][N] when the input dimension is split
+  int* status;
+  long long budget;
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Byte offset of 16-byte chunk c of row r in a 128-byte-swizzled tile.
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
+  return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// The 128 bits holding the eight 16-bit indices of row o for vectors
+// 8*kt .. 8*kt+7 (word i: vectors 8kt + 2i and 8kt + 2i + 1).
+template <int LAYOUT>
+__device__ __forceinline__ uint4 step_words(const Layer& L, int64_t o, int kt) {
+  if constexpr (LAYOUT == VQ_IDX_TILE4) {
+    // tiles 2kt and 2kt+1, row o's 64-bit record in each (the second tile may
+    // lie past the last vector)
+    const int ntile = (L.nvec + 3) / 4;
+    const uint2 a = __ldg(reinterpret_cast<const uint2*>(L.idx[0] + (2 * kt) * L.rw[0] + 2 * o));
+    const uint2 b = 2 * kt + 1 < ntile
+                        ? __ldg(reinterpret_cast<const uint2*>(L.idx[0] + (2 * kt + 1) * L.rw[0] + 2 * o))
+                        : make_uint2(0u, 0u);
+    return make_uint4(a.x, a.y, b.x, b.y);
+  } else {
+    // 16 bytes of row o (rows are 16-byte aligned and cover every step)
+    return __ldg(reinterpret_cast<const uint4*>(L.idx[0] + o * L.rw[0] + 4 * kt));
+  }
+}
+
+template <int LAYOUT>
+__global__ void __launch_bounds__(kTcThreads) gemv_tc_kernel(const __grid_constant__ CUtensorMap xmap, TcArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = align1024(smem_raw);
+  TcCtrl* ctrl = reinterpret_cast<TcCtrl*>(base);
+  uint8_t* stages = base + 1024;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Layer& L = g.L;
+  const int row0 = blockIdx.x * kTcRows;
+  const int split = blockIdx.y;
+  const int kt0 = split * g.kt_per_split;
+  const int nkt = min(g.num_kt, kt0 + g.kt_per_split) - kt0;   // >= 1 by construction
+  volatile int* abort_flag = &ctrl->abort;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(&ctrl->full[s], kTcRows);        // every producer thread
+      mbar_init(&ctrl->xfull[s], 1);             // the x load
+      mbar_init(&ctrl->empty[s], 1);
+    }
+    mbar_init(&ctrl->acc, 1);
+    ctrl->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctrl->tmem, 32);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch(&xmap);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem;
+
+  if (warp == 0) {
+    if (lane == 0) {                                   // x tiles by TMA
+      int issued = 0;
+      for (int i = 0; i < nkt; ++i) {
+        const int s = i % kTcStages;
+        const uint32_t ph = (i / kTcStages) & 1;
+        if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, g.budget)) break;
+        mbar_arrive_expect_tx(&ctrl->xfull[s], kTcXTile);
+        tma_load_2d(stages + s * kTcStage + kTcATile, &xmap, &ctrl->xfull[s], (kt0 + i) * kTcK, 0);
+        issued = i + 1;
+      }
+      if (*abort_flag) {   // let loads already in flight land before the block exits
+        for (int i = max(0, issued - kTcStages); i < issued; ++i)
+          drain_phase(&ctrl->xfull[i % kTcStages], (i / kTcStages) & 1, 4000000000LL);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {                                   // MMA issuer
+      const uint32_t idesc = f16_idesc(kTcRows, kTcN);
+      int issued = 0;
+      for (int i = 0; i < nkt; ++i) {
+        const int s = i % kTcStages;
+        const uint32_t ph = (i / kTcStages) & 1;
+        if (!bounded_wait(&ctrl->full[s], ph, abort_flag, g.status, g.budget)) break;
+        if (!bounded_wait(&ctrl->xfull[s], ph, abort_flag, g.status, g.budget)) break;
+        fence_proxy_async_smem();                      // gathered rows were written by cp.async
+        tc_fence_after();
+        const uint32_t a = smem_addr(stages + s * kTcStage);
+        const uint32_t b = a + kTcATile;
+#pragma unroll
+        for (int kk = 0; kk < kTcK / 16; ++kk)
+          umma_f16(tmem, sw128_kmajor_desc(a + kk * 32), sw128_kmajor_desc(b + kk * 32), idesc, (i | kk) != 0);
+        umma_commit(&ctrl->empty[s]);
+        issued = i + 1;
+      }
+      if (issued > 0) {
+        umma_commit(&ctrl->acc);
+        // every product issued has finished before tensor memory is freed,
+        // even when the epilogue gave up waiting for it
+        drain_phase(&ctrl->acc, 0, 4000000000LL);
+      }
+    }
+  } else if (warp >= 4) {
+    // Producers: thread r gathers row row0 + r (rows past N repeat row N-1,
+    // whose results are never stored).
+    const int r = threadIdx.x - kTcProducer0;
+    const int64_t o = min(row0 + r, L.n - 1);
+    const uint16_t* book = L.book[0];
+    int published = 0;
+    // the index words of the next three steps are always in flight
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    uint4 w0 = nkt > 0 ? step_words<LAYOUT>(L, o, kt0) : z;
+    uint4 w1 = nkt > 1 ? step_words<LAYOUT>(L, o, kt0 + 1) : z;
+    uint4 w2 = nkt > 2 ? step_words<LAYOUT>(L, o, kt0 + 2) : z;
+    for (int i = 0; i < nkt; ++i) {
+      const int s = i % kTcStages;
+      const uint32_t ph = (i / kTcStages) & 1;
+      if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, g.budget)) break;
+      const uint32_t wd[4] = {w0.x, w0.y, w0.z, w0.w};
+      w0 = w1;
+      w1 = w2;
+      w2 = i + 3 < nkt ? step_words<LAYOUT>(L, o, kt0 + i + 3) : z;
+      uint8_t* at = stages + s * kTcStage;
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        const uint32_t f = (wd[v >> 1] >> (16 * (v & 1))) & 0xFFFFu;
+        cp_async16(at + sw128_off(r, v), book + static_cast<size_t>(f) * 8);
+      }
+      cp_async_commit();
+      if (i >= kTcLag) {                               // step i - kTcLag has landed: publish it
+        cp_async_wait<kTcLag>();
+        fence_proxy_async_smem();
+        mbar_arrive(&ctrl->full[(i - kTcLag) % kTcStages]);
+        published = i - kTcLag + 1;
+      }
+    }
+    cp_async_wait<0>();                                // nothing of ours may land after the exit
+    fence_proxy_async_smem();
+    if (!*abort_flag)
+      for (int i = published; i < nkt; ++i) mbar_arrive(&ctrl->full[i % kTcStages]);
+    // Epilogue: lane quarter warp & 3, one output row per thread.
+    if (bounded_wait(&ctrl->acc, 0, abort_flag, g.status, g.budget)) {
+      tc_fence_after();
+      uint32_t acc[16];
+      tmem_ld16(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16), acc);
+      tmem_wait_ld();
+      const int row = row0 + r;
+      if (row < L.n) {
+        const float sc = L.scale ? h2f(L.scale[row]) : 1.0f;
+        const float tb = (L.bias && split == 0) ? h2f(L.bias[row]) : 0.0f;
+        for (int b = 0; b < g.batch; ++b) {
+          const float v = sc * (__uint_as_float(acc[b]) * g.xe[b]) + tb * g.xsum[b];
+          if (g.part) g.part[(static_cast<int64_t>(split) * g.batch + b) * L.n + row] = v;
+          else store_out(g.y, g.yt, b * g.ldy + row, v);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 32);
+  }
+}
+
+// x' = x * 2^-e_b in fp16 [16][kp] (zero past kin and for rows b >= batch),
+// 2^e_b and sum_k x[b][k].  e_b puts max_k |x[b][k]| in [2^14, 2^15), so no
+// value overflows fp16 and values above max * 2^-29 stay exact.
+__global__ void gemv_tc_prep(const uint16_t* __restrict__ x, int x_fp16, int64_t ldx, int kin, int kp, int batch,
+                             uint16_t* __restrict__ xh, float* __restrict__ xe, float* __restrict__ xsum) {
+  __shared__ float s_max[32], s_sum[32];
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool live = b < batch;
+  float mx = 0.0f, sm = 0.0f;
+  if (live)
+    for (int k = tid; k < kin; k += blockDim.x) {
+      const uint16_t u = x[b * ldx + k];
+      const float v = x_fp16 ? h2f(u) : bf2f(u);
+      mx = fmaxf(mx, fabsf(v));
+      sm += v;
+    }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    sm += __shfl_xor_sync(0xffffffffu, sm, off);
+  }
+  if (lane == 0) { s_max[warp] = mx; s_sum[warp] = sm; }
+  __syncthreads();
+  if (warp == 0) {
+    mx = lane < static_cast<int>(blockDim.x / 32) ? s_max[lane] : 0.0f;
+    sm = lane < static_cast<int>(blockDim.x / 32) ? s_sum[lane] : 0.0f;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      sm += __shfl_xor_sync(0xffffffffu, sm, off);
+    }
+    if (lane == 0) { s_max[0] = mx; s_sum[0] = sm; }
+  }
+  __syncthreads();
+  mx = s_max[0];
+  // max = m * 2^E with 0.5 <= m < 1; e = E - 15, kept in [-126, 127] (values
+  // below 2^-111 scale to fp16 subnormals or zero).
+  int e = 0;
+  if (mx > 0.0f && mx < INFINITY) e = max(-126, min(127, static_cast<int>(__float_as_uint(mx) >> 23) - 126 - 15));
+  const float f1 = __uint_as_float(static_cast<uint32_t>(127 - e / 2) << 23);
+  const float f2 = __uint_as_float(static_cast<uint32_t>(127 - (e - e / 2)) << 23);
+  for (int k = tid; k < kp; k += blockDim.x) {
+    float v = 0.0f;
+    if (live && k < kin) {
+      const uint16_t u = x[b * ldx + k];
+      v = (x_fp16 ? h2f(u) : bf2f(u)) * f1 * f2;
+    }
+    xh[static_cast<int64_t>(b) * kp + k] = f2h(v);
+  }
+  if (tid == 0) {
+    xe[b] = live ? __uint_as_float(static_cast<uint32_t>(127 + e) << 23) : 0.0f;
+    xsum[b] = live ? s_sum[0] : 0.0f;
+  }
+}
+
+// y[b][o] = sum over splits of part[s][b][o], in split order.
+__global__ void gemv_tc_finalize(const float* __restrict__ part, int nsplit, int batch, int n, void* __restrict__ y,
+                                 vq_dtype yt, int64_t ldy) {
+  const int64_t total = static_cast<int64_t>(batch) * n;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = i / n, o = i - b * n;
+    float v = 0.0f;
+    for (int s = 0; s < nsplit; ++s) v += part[(s * static_cast<int64_t>(batch) + b) * n + o];
+    store_out(y, yt, b * ldy + o, v);
+  }
+}
+
+struct TcLayout {
+  int tiles, nsplit, kt_per_split, num_kt, kp;
+  size_t off_status, off_xh, off_xe, off_part, total;
+};
+
+TcLayout tc_layout(const Layer& L, int batch) {
+  TcLayout t{};
+  t.tiles = (L.n + kTcRows - 1) / kTcRows;
+  t.num_kt = (L.nvec + 7) / 8;
+  t.kp = t.num_kt * kTcK;
+  const int target = kTcPerSm * device_sm_count();
+  int nsplit = std::max(1, std::min(t.num_kt, (target + t.tiles / 2) / t.tiles));
+  t.kt_per_split = (t.num_kt + nsplit - 1) / nsplit;
+  t.nsplit = (t.num_kt + t.kt_per_split - 1) / t.kt_per_split;
+  auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
+  t.off_status = 0;
+  t.off_xh = 256;
+  t.off_xe = t.off_xh + r256(static_cast<size_t>(kTcN) * t.kp * 2);
+  t.off_part = t.off_xe + 256;
+  t.total = t.off_part + (t.nsplit > 1 ? r256(static_cast<size_t>(t.nsplit) * batch * L.n * 4) : 0);
+  return t;
+}
+
+// Smallest batch this kernel serves (VQ_TC_MIN_BATCH overrides, for measurements).
+int tc_min_batch() {
+  if (const char* env = std::getenv("VQ_TC_MIN_BATCH")) return std::atoi(env);
+  return 2;
+}
+
+long long tc_wait_budget() {
+  if (const char* env = std::getenv("VQ_WAIT_BUDGET")) return std::atoll(env);
+  return 4000000000LL;
+}
+
+}  // namespace
+
+bool plan_gemv_tc(const Layer& L, int batch, size_t ws_cap, GemvPlan* p) {
+  if (!(L.layout == VQ_IDX_ROWS || L.layout == VQ_IDX_TILE4) || L.nb != 1 || L.d != 8 || L.b[0] != 16) return false;
+  if (batch < std::max(1, tc_min_batch()) || batch > kTcN || L.n < 1 || L.nvec < 1) return false;
+  if (device_smem_optin() < kTcSmem) return false;
+  const TcLayout t = tc_layout(L, batch);
+  if (t.total > ws_cap) return false;
+  *p = GemvPlan{};
+  p->fast = 7;
+  p->bt = batch;
+  p->nsplit = t.nsplit;
+  p->grid_x = t.tiles;
+  p->smem = kTcSmem;
+  p->ws_bytes = t.total;
+  return true;
+}
+
+vq_status launch_gemv_tc(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, int batch, int64_t ldx,
+                         void* y, vq_dtype yt, int64_t ldy, void* ws, cudaStream_t stream) {
+  const TcLayout t = tc_layout(L, batch);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* xh = reinterpret_cast<uint16_t*>(w + t.off_xh);
+  float* xe = reinterpret_cast<float*>(w + t.off_xe);
+  float* xsum = xe + kTcN;
+  int* status = reinterpret_cast<int*>(w + t.off_status);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  count_launch();
+  gemv_tc_prep<<<kTcN, 256, 0, stream>>>(static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, ldx, L.kin, t.kp, batch,
+                                          xh, xe, xsum);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+  CUtensorMap xmap;
+  if (!make_map_f16_sw128(&xmap, xh, t.kp, kTcN, t.kp, kTcN)) return VQ_ERR_CUDA;
+  TcArgs g{};
+  g.L = L;
+  g.num_kt = t.num_kt;
+  g.kt_per_split = t.kt_per_split;
+  g.batch = batch;
+  g.xe = xe;
+  g.xsum = xsum;
+  g.y = y;
+  g.yt = yt;
+  g.ldy = ldy;
+  g.part = t.nsplit > 1 ? reinterpret_cast<float*>(w + t.off_part) : nullptr;
+  g.status = status;
+  g.budget = tc_wait_budget();
+  auto k = L.layout == VQ_IDX_TILE4 ? gemv_tc_kernel<VQ_IDX_TILE4> : gemv_tc_kernel<VQ_IDX_ROWS>;
+  if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem)) != cudaSuccess)
+    return cuda_status(e);
+  count_launch();
+  k<<<dim3(t.tiles, t.nsplit), kTcThreads, kTcSmem, stream>>>(xmap, g);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+  if (t.nsplit > 1) {
+    const int64_t total = static_cast<int64_t>(batch) * L.n;
+    const int grid = static_cast<int>(std::min<int64_t>((total + 255) / 256, 4LL * device_sm_count()));
+    count_launch();
+    gemv_tc_finalize<<<grid, 256, 0, stream>>>(g.part, t.nsplit, batch, L.n, y, yt, ldy);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+  }
+  return VQ_OK;
+}
+
+}  // namespace vqk

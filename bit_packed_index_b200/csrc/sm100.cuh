@@ -49,12 +49,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Gives up after about
 // `budget` SM clocks (or as soon as another thread has raised *abort): then it
-// raises *abort, records VQ_ERR_TIMEOUT in *status and returns false.
+// raises *abort, records VQ_ERR_TIMEOUT in *status and returns false.  A
+// budget of 0 gives up unless the phase is already complete (tests use it to
+// make a pipeline's waits run out).
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                              int* status, long long budget) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test_wait(bar, parity)) return true;
+  if (budget <= 0) {
+    *abort = 1;
+    if (status) atomicExch(status, static_cast<int>(VQ_ERR_TIMEOUT));
+    return false;
+  }
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -66,6 +86,16 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, vol
       }
     }
   }
+}
+
+// Wait for the phase with the given parity whatever the abort flag says: used
+// to let copies already in flight land before a block that gave up ends.
+// Returns false if about `budget` clocks pass first.
+__device__ __forceinline__ bool drain_phase(uint64_t* bar, uint32_t parity, long long budget) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > budget) return false;
+  return true;
 }
 
 // ---- proxies and TMA ---------------------------------------------------------
@@ -146,6 +176,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// 16 consecutive fp32 columns of one TMEM lane per thread (lanes of the warp's quarter).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
 }
 // 8 consecutive fp32 columns of one TMEM lane per thread, and the store back.
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {

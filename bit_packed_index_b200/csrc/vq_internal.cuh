@@ -6,6 +6,7 @@
 // bf16 conversions (CUDA's own intrinsics).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -74,7 +75,8 @@ struct GemvPlan {
   int fast = 0;       // 0: split-K gather kernel (gemv.cu, either index order),
                       // 1: single-row kernel (gemv1.cu), 2: batched kernel (gemvb.cu),
                       // 3: lookup-table kernel (2^16 book), 5: lookup-table kernel for
-                      // books of <= 2^12 entries (tile4.cu, tiled order, batch 1)
+                      // books of <= 2^12 entries (tile4.cu, tiled order, batch 1),
+                      // 7: tensor-core batched decode (gemvtc.cu)
 };
 // ws_cap: largest workspace the caller can provide (plans that need more
 // either shrink, for the tiled kernels, or are reported by their ws_bytes).
@@ -114,6 +116,17 @@ cudaError_t launch_gemv1(const Layer& L, const GemvPlan& plan, const void* x, bo
 vq_status launch_gemv(const Layer& L, const GemvPlan& plan, const void* x, bool x_fp16, int batch,
                       int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy, float* ws,
                       cudaStream_t stream);
+
+// TMA map of a 2-D fp16 tensor [rows][cols] (row stride ld elements), box
+// {64, box_rows}, 128-byte swizzle, zero fill past the edges (gemm.cu).
+bool make_map_f16_sw128(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int64_t ld,
+                        int box_rows);
+
+// Batched decode on the tensor cores (gemvtc.cu): layers with one 2^16-entry
+// d = 8 book, row or tiled order.
+bool plan_gemv_tc(const Layer& L, int batch, size_t ws_cap, GemvPlan* plan);
+vq_status launch_gemv_tc(const Layer& L, const GemvPlan& plan, const void* x, bool x_fp16, int batch,
+                         int64_t ldx, void* y, vq_dtype y_dtype, int64_t ldy, void* ws, cudaStream_t stream);
 
 size_t gemm_workspace_bytes(const Layer& L, int m, bool x_fp16);
 vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t ldx, void* y,

@@ -61,7 +61,11 @@
  *   default stream).  Argument errors are detected on the host and returned
  *   before anything is launched; nothing is written then.
  * - Launch failures return VQ_ERR_CUDA; vq_last_cuda_error() gives the
- *   cudaError_t.  Kernels never trap and never wait on flags.
+ *   cudaError_t.  Kernels never trap.  Kernels that wait on the device (an
+ *   mbarrier of a TMA / tensor-core pipeline) bound every wait: after about
+ *   2 s (VQ_WAIT_BUDGET in the environment sets the budget in SM clocks) the
+ *   kernel records VQ_ERR_TIMEOUT in the status word of its workspace (see
+ *   each call), lets its copies in flight land, and returns.
  * - fp16 / bf16 values are passed as their 16-bit patterns.
  * - All calls are thread-safe; concurrent calls on different streams may not
  *   share an output or a workspace buffer.
@@ -91,7 +95,7 @@ typedef enum vq_status {
     VQ_ERR_ALIGNMENT = 3,     /* a pointer or leading dimension is misaligned   */
     VQ_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required     */
     VQ_ERR_CUDA = 5,          /* a CUDA call or kernel launch failed            */
-    VQ_ERR_TIMEOUT = 6        /* reserved: a bounded device-side wait gave up   */
+    VQ_ERR_TIMEOUT = 6        /* a bounded device-side wait gave up (status word) */
 } vq_status;
 
 typedef enum vq_idx_layout {
@@ -195,10 +199,19 @@ VQ_API vq_status vq_gemv_workspace_size(const vq_layer_desc* layer, int32_t batc
  * per term, inside the same tolerance as long as the codebook's values are
  * normal fp16 numbers (|c| >= 2^-14).  Books of up to 2^12 entries (one or
  * two, d = 6 or 8) get a table kernel without slices.  Batches of 2 (2^16
- * book) or up to 8 (small books) run one table pass per row of x.  Every
- * other tiled case runs the split-K gather kernel, which reads either index
- * order.  The environment variable VQ_LUT_MAX_BATCH overrides those batch
- * limits (0 turns the table kernels off), for measurements.
+ * book) or up to 8 (small books) run one table pass per row of x.
+ * Batches of 2..16 (3..16 in the tiled order) of layers with one 2^16-entry
+ * d = 8 book run the tensor-core kernel: per 128 rows of W and step of eight
+ * vectors, the centroids are gathered into a shared-memory tile and
+ * multiplied on the tcgen05 tensor cores with x, each row of x scaled by a
+ * power of two into fp16 (exact products, fp32 accumulation); values of a
+ * row below 2^-29 of its largest lose precision as fp16 subnormals.  The
+ * first 32-bit word of its workspace is a status word: VQ_OK, or
+ * VQ_ERR_TIMEOUT if a bounded device-side wait gave up (readable after the
+ * stream completes).  Every other case runs the split-K gather kernel, which
+ * reads either index order.  The environment variables VQ_LUT_MAX_BATCH (0
+ * turns the table kernels off) and VQ_TC_MIN_BATCH (above 16 turns the
+ * tensor-core kernel off) move those limits, for measurements.
  * Errors: VQ_ERR_INVALID_ARG, VQ_ERR_UNSUPPORTED (batch > 16), VQ_ERR_ALIGNMENT
  * (x or y not aligned to its element size), VQ_ERR_WORKSPACE, VQ_ERR_CUDA.
  */
@@ -272,12 +285,17 @@ VQ_API vq_status vq_gemm_workspace_size(const vq_layer_desc* layer, int32_t m, v
  * vs. Decode Bottlenecks", and the "GEMV / Tensor Core Dot Products" stage of
  * its dequantisation diagram).
  *   x        device, x_dtype (VQ_BF16 or VQ_FP16) [m][ldx]; 16-byte aligned,
- *            ldx a multiple of 8, ldx >= Kin.  bf16 activations are converted
- *            to fp16 operands (exact for |x| in [2^-14, 65504]; smaller values
- *            become fp16 subnormals, larger ones overflow).
+ *            ldx a multiple of 8, ldx >= Kin.  bf16 activations become fp16
+ *            operands row by row, each row scaled by a power of two that puts
+ *            its largest magnitude in [2^14, 2^15) and undone in the epilogue:
+ *            any finite bf16 value is accepted, and values above 2^-29 of
+ *            their row's largest are exact (smaller ones lose precision as
+ *            fp16 subnormals).  fp16 activations are used as given.
  *   y        device, y_dtype [m][ldy]; ldy >= N
  *   workspace  device scratch of at least vq_gemm_workspace_size() bytes,
- *            256-byte aligned
+ *            256-byte aligned; its first 32-bit word is a status word (VQ_OK,
+ *            or VQ_ERR_TIMEOUT if a bounded device-side wait gave up),
+ *            readable after the stream completes
  * Scale and bias are applied in the epilogue as for vq_gemv.
  * Errors: as vq_gemv; VQ_ERR_UNSUPPORTED for vec_dim > 8 or m > 2^30.
  */

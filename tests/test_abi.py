@@ -87,14 +87,17 @@ def test_layout_field_validation_needs_no_device(lib):
 
 def test_tiled_workspace_sizes(lib):
     """Batch 1 on a lookup-table-eligible tiled layer needs per-block row sums;
-    batch 3 of a 2^16 book and layers no table kernel takes use the split-K
-    gather kernel, which for this narrow layer runs one split (no workspace)."""
+    batch 3 of a 2^16 book takes the tensor-core kernel (status word, the
+    scaled fp16 copy of x as 16 rows of whole 64-element steps, the per-row
+    scales and sums: 256 + 16 * 64 * 2 + 256 bytes for 8 vectors); layers no
+    table kernel takes use the split-K gather kernel, which for this narrow
+    layer runs one split (no workspace)."""
     n = C.c_size_t(0)
     d = _tiled_desc(n=1000, kin=64)
     assert lib.vq_gemv_workspace_size(C.byref(d), 1, C.byref(n)) == vq.VQ_OK
     assert n.value > 0 and n.value % (1001 * 4) == 0
     assert lib.vq_gemv_workspace_size(C.byref(d), 3, C.byref(n)) == vq.VQ_OK
-    assert n.value == 0
+    assert n.value == 256 + 16 * 64 * 2 + 256
     d.log2k[0] = 12                                    # a 2^12 book: the small-book table plan
     d.idx_row_words[0] = vq.tile4_words(1000, 12)
     assert lib.vq_gemv_workspace_size(C.byref(d), 1, C.byref(n)) == vq.VQ_OK

@@ -154,3 +154,46 @@ def test_gemm_degenerate_and_errors():
     with pytest.raises(vq.VQError) as e:             # d > 8 has no tensor-core path
         vq.gemm(big, x[:, :64])
     assert e.value.status == vq.VQ_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("mode", ["fused", "staged"])
+def test_gemm_bf16_rows_beyond_fp16_range(monkeypatch, mode):
+    """bf16 activations beyond fp16's range (|x| up to 1e30) and rows of tiny
+    values (1e-30): each row is scaled into fp16 by its own power of two, so
+    every row stays within the bar (checked row by row), with scale and bias."""
+    monkeypatch.setenv("VQ_GEMM_MODE", mode)
+    spec = LayerSpec(300, 512, 8, (16, 8), (0.02, 0.005))
+    data = synth.make_layer(spec, seed=91)
+    x = oracle.bf16_to_f32(synth.make_x(92, 130, 512, outlier_frac=0.01))
+    x[0] *= np.float32(1e30)
+    x[1] *= np.float32(1e5)          # past 65504
+    x[2] *= np.float32(1e-30)
+    x[3] = 0.0                       # an all-zero row
+    xb = oracle.f32_to_bf16(x)
+    ref = oracle.linear(data, xb)
+    y = _run(_vq().Layer.from_synth(data), _x_dev(xb), torch.float32, 512).double().cpu().numpy()
+    assert np.isfinite(y).all()
+    for r in range(xb.shape[0]):
+        assert_close(y[r:r + 1], ref[r:r + 1], "float32")
+
+
+@pytest.mark.parametrize("mode", ["fused", "staged"])
+def test_gemm_bounded_wait_gives_up_with_timeout_status(monkeypatch, mode):
+    """With a wait budget of 0 clocks the pipeline's first wait that finds its
+    stage not yet complete gives up: the call completes, the status word reads
+    VQ_ERR_TIMEOUT, and the next call with the normal budget is correct."""
+    vq = _vq()
+    monkeypatch.setenv("VQ_GEMM_MODE", mode)
+    spec = LayerSpec(1024, 2048, 8, (16,), (0.02,))
+    data = synth.make_layer(spec, seed=95)
+    layer = vq.Layer.from_synth(data)
+    x = synth.make_x(96, 512, 2048, outlier_frac=0.01)
+    xd = _x_dev(x)
+    ws = torch.zeros(vq.gemm_workspace_size(layer, 512, xd.dtype), dtype=torch.uint8, device="cuda")
+    monkeypatch.setenv("VQ_WAIT_BUDGET", "0")
+    vq.gemm(layer, xd, out_dtype=torch.float32, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == vq.VQ_ERR_TIMEOUT
+    monkeypatch.delenv("VQ_WAIT_BUDGET")
+    y = _run(layer, xd, torch.float32, 2048)
+    assert_close(y.double().cpu().numpy(), oracle.linear(data, x), "float32")

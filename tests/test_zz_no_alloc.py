@@ -42,9 +42,11 @@ def test_noalloc_matches_workspace_version_twice(spec, batch):
 
 def test_noalloc_rejects_layers_beyond_the_scratch():
     from bit_packed_index_b200 import vq
-    spec = LayerSpec(28672, 8192, 8, (16,), (0.02,))       # split K at batch 16: ~11 MB
+    # a tiled layer with a 2^16 book and a residual book runs only the split-K
+    # kernel at batch 16, whose partial sums take ~10.5 MB
+    spec = LayerSpec(28672, 8192, 8, (16, 8), (0.02, 0.005))
     data = synth.make_layer(spec, seed=4244)
-    layer = vq.Layer.from_synth(data)
+    layer = vq.repack_tile4(vq.Layer.from_synth(data))
     assert vq.gemv_workspace_size(layer, 16) > vq.NOALLOC_SCRATCH_BYTES
     x = _x_dev(synth.make_x(4245, 16, spec.in_features))
     with pytest.raises(vq.VQError) as e:
