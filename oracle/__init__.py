@@ -49,6 +49,7 @@ class _Layer(C.Structure):
         ("d", C.c_int32), ("n_books", C.c_int32), ("log2k", C.c_int32 * 2),
         ("idx", C.c_void_p * 2), ("row_words", C.c_int64 * 2),
         ("codebook", C.c_void_p * 2), ("scale", C.c_void_p), ("bias", C.c_void_p),
+        ("out_bias", C.c_void_p),
     ]
 
 
@@ -186,8 +187,8 @@ def _layer_struct(layer):
         L.idx[m] = w.ctypes.data
         L.row_words[m] = layer.row_words[m]
         L.codebook[m] = c.ctypes.data
-    for name in ("scale", "bias"):
-        a = getattr(layer, name)
+    for name in ("scale", "bias", "out_bias"):
+        a = getattr(layer, name, None)
         if a is not None:
             a = np.ascontiguousarray(a, np.uint16)
             keep.append(a)
@@ -223,9 +224,17 @@ def matmul(x: np.ndarray, w: np.ndarray, kin: Optional[int] = None, x_is_fp16: b
 
 
 def linear(layer, x: np.ndarray, rows: Optional[Sequence[int]] = None,
-           x_is_fp16: bool = False) -> np.ndarray:
-    """Forward pass in fp64: y[M][n] for all output rows, or for ``rows``."""
+           x_is_fp16: bool = False, out_bias: Optional[np.ndarray] = None) -> np.ndarray:
+    """Forward pass in fp64: y[M][n] for all output rows, or for ``rows``.
+    The output bias (fp16 bits [N]) is ``out_bias`` when given, else the
+    layer's ``out_bias`` attribute (if any)."""
     L, keep = _layer_struct(layer)
+    if out_bias is not None:
+        ob = np.ascontiguousarray(out_bias, np.uint16)
+        if ob.shape != (layer.spec.out_features,):
+            raise ValueError("out_bias must hold out_features fp16 values")
+        keep.append(ob)
+        L.out_bias = ob.ctypes.data
     x = np.ascontiguousarray(x, np.uint16)
     M = x.shape[0]
     if rows is None:

@@ -26,7 +26,9 @@
  *    channel scaling).
  *  - products y = x . W_hat^T accumulated in fp64 in ascending k order
  *    ("VPTQ Guide", section "Step 3: Fused Low-Bit VPTQ Linear Layer":
- *    forward computes y = x @ W^T with the dequantised weights).
+ *    forward computes y = x @ W^T with the dequantised weights), plus an
+ *    optional fp16 output bias b_out[o] added once in fp64 (the same
+ *    section's F.linear(x, W_hat, bias)).
  *  - the normalised, damped activation Hessian H = 2 X^T X / n + damping
  *    (section "Hessian collection" below);
  *  - the randomized Hadamard transform of QuIP#-style incoherence processing
@@ -260,6 +262,7 @@ typedef struct {
     const uint16_t* codebook[2];   /* fp16 [K][d] */
     const uint16_t* scale;         /* fp16 [N] or NULL */
     const uint16_t* bias;          /* fp16 [N] or NULL */
+    const uint16_t* out_bias;      /* fp16 [N] or NULL: output-side bias of the product */
 } vqo_layer;
 
 static int64_t nvec_of(const vqo_layer* L) { return (L->in_features + L->d - 1) / L->d; }
@@ -345,8 +348,13 @@ int vqo_matmul(int64_t M, int64_t N, int64_t Kin, const uint16_t* x, int x_is_fp
 
 /* The layer's forward pass for the listed output rows (all rows when rows is
  * NULL): dequantise row o, then y[m][c] = sum_k x[m][k] * w_hat[o][k] in fp64,
- * where c is the position of o in the list.  Uses one row buffer per thread,
- * so it runs on full-size layers without materialising W_hat. */
+ * where c is the position of o in the list, plus out_bias[o] (when given)
+ * added once, in fp64, after the sum: the layer's forward ends in
+ * F.linear(x, W_hat, bias), an output-side bias over the product ("VPTQ
+ * Guide", section "Step 3: Fused Low-Bit VPTQ Linear Layer").  That bias is
+ * separate from the per-row bias t folded into W_hat above.  Uses one row
+ * buffer per thread, so it runs on full-size layers without materialising
+ * W_hat. */
 int vqo_linear(const vqo_layer* L, const uint16_t* x, int x_is_fp16, int64_t M, int64_t ldx,
                const int64_t* rows, int64_t nrows, double* y, int64_t ldy) {
     if (check_layer(L) || M < 0 || ldx < L->in_features) return 1;
@@ -372,6 +380,7 @@ int vqo_linear(const vqo_layer* L, const uint16_t* x, int x_is_fp16, int64_t M, 
                     double s = 0.0;
                     for (int64_t k = 0; k < kin; ++k)
                         s += act(x, x_is_fp16, m * ldx + k) * (double)vqo_f16_to_f32(w[k]);
+                    if (L->out_bias) s += (double)vqo_f16_to_f32(L->out_bias[o]);
                     y[m * ldy + c] = s;
                 }
             }

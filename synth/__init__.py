@@ -73,6 +73,7 @@ class LayerSpec:
     scale_range: Optional[Tuple[float, float]] = (0.5, 1.5)   # None: no scale
     bias_std: Optional[float] = 1e-3                          # None: no bias
     name: str = ""
+    out_bias_std: Optional[float] = None                      # None: no output bias
 
     @property
     def n_books(self) -> int:
@@ -91,11 +92,12 @@ class LayerData:
     codebooks: List[np.ndarray]       # uint16 (fp16 bits) [K_m][d] per book
     scale: Optional[np.ndarray]       # uint16 (fp16 bits) [N] or None
     bias: Optional[np.ndarray]        # uint16 (fp16 bits) [N] or None
+    out_bias: Optional[np.ndarray] = None   # uint16 (fp16 bits) [N] or None
 
     def nbytes(self) -> int:
         n = sum(w.nbytes for w in self.idx_words) + sum(c.nbytes for c in self.codebooks)
-        n += 0 if self.scale is None else self.scale.nbytes
-        n += 0 if self.bias is None else self.bias.nbytes
+        for a in (self.scale, self.bias, self.out_bias):
+            n += 0 if a is None else a.nbytes
         return n
 
 
@@ -148,7 +150,11 @@ def make_layer(spec: LayerSpec, seed: int, row_words: Optional[Sequence[int]] = 
     bias = None
     if spec.bias_std is not None:
         bias = to_f16_bits(rng.standard_normal(n, dtype=np.float32) * np.float32(spec.bias_std))
-    return LayerData(spec, streams, rws, books, scale, bias)
+    out_bias = None
+    if spec.out_bias_std is not None:     # drawn last: the other arrays do not depend on it
+        out_bias = to_f16_bits(rng.standard_normal(n, dtype=np.float32)
+                               * np.float32(spec.out_bias_std))
+    return LayerData(spec, streams, rws, books, scale, bias, out_bias)
 
 
 def make_x(seed: int, rows: int, in_features: int, outlier_frac: float = 0.0,

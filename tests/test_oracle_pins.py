@@ -213,6 +213,51 @@ def test_affine_special_case():
     assert np.allclose(oracle.linear(layer, x), xf.sum(1)[:, None] * tf[None, :], rtol=1e-12)
 
 
+def test_output_bias_closed_form():
+    """All-zero book with an output bias: y[m][o] = t[o] * sum_k x[m][k] + b_out[o]
+    (the layer bias t folded into W_hat, then F.linear's output bias once)."""
+    d, n, kin = 8, 21, 8 * 7 + 3
+    book = np.zeros((16, d), np.uint16)
+    rng = np.random.default_rng(31)
+    idx = rng.integers(0, 16, size=(n, -(-kin // d)), dtype=np.uint32)
+    bias = synth.to_f16_bits(rng.standard_normal(n).astype(np.float32))
+    b_out = synth.to_f16_bits(rng.uniform(-4.0, 4.0, n).astype(np.float32))
+    layer = _layer(n, kin, d, [book], [idx], None, bias)
+    x = synth.make_x(32, 3, kin)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    tf = bias.view(np.float16).astype(np.float64)
+    bf = b_out.view(np.float16).astype(np.float64)
+    want = xf.sum(1)[:, None] * tf[None, :] + bf[None, :]
+    assert np.allclose(oracle.linear(layer, x, out_bias=b_out), want, rtol=1e-12, atol=1e-12)
+    # x = 0 leaves exactly the output bias, row by row (also through ``rows``)
+    z = np.zeros_like(x)
+    assert np.array_equal(oracle.linear(layer, z, out_bias=b_out), np.tile(bf, (3, 1)))
+    rows = [20, 0, 7]
+    assert np.array_equal(oracle.linear(layer, z, rows=rows, out_bias=b_out), np.tile(bf[rows], (3, 1)))
+
+
+def test_output_bias_is_added_once_per_output_row():
+    """Random two-book layer: linear with b_out equals numpy's x . W_hat^T (from
+    the independent dequant restatement) + b_out, and the difference to the
+    call without it is b_out in every row of x (not scaled, not per input)."""
+    spec = LayerSpec(48, 8 * 40, 8, (12, 8), (0.02, 0.005), out_bias_std=0.5)
+    layer = synth.make_layer(spec, seed=33)
+    assert layer.out_bias is not None
+    x = synth.make_x(34, 5, spec.in_features)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    w = _numpy_dequant(layer).view(np.float16).astype(np.float64)
+    bf = layer.out_bias.view(np.float16).astype(np.float64)
+    y = oracle.linear(layer, x)                      # the layer's own out_bias
+    assert np.allclose(y, xf @ w.T + bf[None, :], rtol=1e-12, atol=1e-12)
+    no_bias = oracle.linear(layer, x, out_bias=np.zeros(48, np.uint16))
+    assert np.allclose(y - no_bias, np.tile(bf, (5, 1)), rtol=0, atol=1e-12)
+    # the same seed without an output bias draws the same weights
+    plain = synth.make_layer(LayerSpec(48, 8 * 40, 8, (12, 8), (0.02, 0.005)), seed=33)
+    assert plain.out_bias is None
+    assert all(np.array_equal(a, b) for a, b in zip(plain.idx_words, layer.idx_words))
+    assert np.array_equal(oracle.linear(plain, x), no_bias)
+
+
 def _numpy_dequant(layer) -> np.ndarray:
     """Independent float32 restatement, vectorised: same operation order."""
     s = layer.spec
