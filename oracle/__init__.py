@@ -73,6 +73,8 @@ def _load():
                 "vqo_encode": [P, I64, I32, P, I64, P],
                 "vqo_encode_residual": [P, I64, I32, P, I64, P, I64, P, P],
                 "vqo_encode_joint": [P, I64, I32, P, I64, P, I64, P, P],
+                "vqo_encode_h": [P, I64, I32, P, P, I64, P],
+                "vqo_encode_h_residual": [P, I64, I32, P, P, I64, P, I64, P, P],
                 "vqo_rht": [P, I64, I64, P, I32, P],
                 "vqo_hessian": [P, I32, I64, I64, I64, P],
                 "vqo_rht_block": [I64],
@@ -271,6 +273,53 @@ def encode_residual(v: np.ndarray, book1: np.ndarray, book2: np.ndarray):
     _check(_load().vqo_encode_residual(_p(v), nv, d, _p(b1), b1.shape[0], _p(b2), b2.shape[0],
                                        _p(i1), _p(i2)), "encode_residual")
     return i1, i2
+
+
+def encode_h(v: np.ndarray, hb: np.ndarray, book: np.ndarray) -> np.ndarray:
+    """Hessian-weighted nearest centroid: v [nv][d], hb [nv][d][d] (each
+    vector's sub-matrix of H), book fp16 bits [K][d]."""
+    v = np.ascontiguousarray(v, np.float64)
+    hb = np.ascontiguousarray(hb, np.float64)
+    book = np.ascontiguousarray(book, np.uint16)
+    nv, d = v.shape
+    if hb.shape != (nv, d, d):
+        raise ValueError("hb must be [nv][d][d]")
+    idx = np.empty(nv, np.uint32)
+    _check(_load().vqo_encode_h(_p(v), nv, d, _p(hb), _p(book), book.shape[0], _p(idx)), "encode_h")
+    return idx
+
+
+def encode_h_residual(v: np.ndarray, hb: np.ndarray, book1: np.ndarray, book2: np.ndarray):
+    v = np.ascontiguousarray(v, np.float64)
+    hb = np.ascontiguousarray(hb, np.float64)
+    b1 = np.ascontiguousarray(book1, np.uint16)
+    b2 = np.ascontiguousarray(book2, np.uint16)
+    nv, d = v.shape
+    if hb.shape != (nv, d, d):
+        raise ValueError("hb must be [nv][d][d]")
+    i1 = np.empty(nv, np.uint32)
+    i2 = np.empty(nv, np.uint32)
+    _check(_load().vqo_encode_h_residual(_p(v), nv, d, _p(hb), _p(b1), b1.shape[0], _p(b2), b2.shape[0],
+                                         _p(i1), _p(i2)), "encode_h_residual")
+    return i1, i2
+
+
+def hessian_blocks(h: np.ndarray, kin: int, d: int, rows: int) -> tuple:
+    """The sub-matrices H_v of a layer's vectors, in the encoder's vector
+    order (row o, vector j): for whole vectors the d x d block of h on
+    channels j*d .. j*d+d-1, and for a partial last vector (kin % d != 0)
+    the rem x rem block on its valid channels.  Returns (full, last): full
+    [rows * (kin // d)][d][d] and last [rows][rem][rem] (None if rem == 0)."""
+    h = np.asarray(h, np.float64)
+    nfull, rem = kin // d, kin % d
+    blocks = np.stack([h[j * d:(j + 1) * d, j * d:(j + 1) * d] for j in range(nfull)]) if nfull else \
+        np.zeros((0, d, d))
+    full = np.ascontiguousarray(np.broadcast_to(blocks[None], (rows, nfull, d, d)).reshape(rows * nfull, d, d))
+    last = None
+    if rem:
+        b = h[nfull * d:kin, nfull * d:kin]
+        last = np.ascontiguousarray(np.broadcast_to(b[None], (rows, rem, rem)))
+    return full, last
 
 
 def encode_joint(v: np.ndarray, book1: np.ndarray, book2: np.ndarray):

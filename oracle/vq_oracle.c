@@ -37,6 +37,9 @@
  *    ("VPTQ Guide", section "The Information-Theoretic Superiority of Vector
  *    Quantization": q = argmin_k ||w - c_k||^2; section "2. Multi-Stage
  *    Residual Vector Quantization (RVQ)" for the residual stage).
+ *  - the Hessian-weighted variant, D_H(v, c) = (v - c)^T H_v (v - c) with H_v
+ *    the vector's sub-matrix of the layer Hessian ("VPTQ Guide", section
+ *    "1. Second-Order Hessian-Weighted Optimization"), by brute force.
  *
  * Readings of points the pages leave open (stated once here):
  *  - index fields are unsigned; field j of a row occupies bits [j*b, j*b+b),
@@ -427,6 +430,63 @@ int vqo_encode_residual(const double* v, int64_t nv, int d, const uint16_t* book
         for (int e = 0; e < d; ++e)
             r[i * d + e] = v[i * d + e] - (double)vqo_f16_to_f32(book1[(int64_t)idx1[i] * d + e]);
     int rc = vqo_encode(r, nv, d, book2, K2, idx2);
+    free(r);
+    return rc;
+}
+
+/* Hessian-weighted encoding ("VPTQ Guide: Extreme 2-Bit Vector
+ * Quantization", section "1. Second-Order Hessian-Weighted Optimization"):
+ * the distance of vector v to centroid c is D_H(v, c) = (v - c)^T H_v (v - c),
+ * with H_v the d x d sub-matrix of the layer's Hessian on the channels of v.
+ * For each of nv vectors v[i][0..d) (fp64) with its own sub-matrix
+ * hb[i][e][f] (fp64, row-major d x d), idx[i] = argmin_k D_H(v_i, C[k]) over
+ * the fp16 book C[K][d], ties to the lowest k.  Evaluation order (every
+ * operation rounded once in fp64, no fused multiply-add): t_e = v_e - C[k][e];
+ * g_e = sum_f hb[e][f] t_f, f ascending; D = sum_e t_e g_e, e ascending.  A
+ * NaN distance never wins; with no finite distance the index is 0. */
+static double dist_h(const double* v, const double* h, const uint16_t* c, int d, double* t) {
+    for (int e = 0; e < d; ++e) t[e] = v[e] - (double)vqo_f16_to_f32(c[e]);
+    double dist = 0.0;
+    for (int e = 0; e < d; ++e) {
+        double g = 0.0;
+        for (int f = 0; f < d; ++f) g += h[e * d + f] * t[f];
+        dist += t[e] * g;
+    }
+    return dist;
+}
+
+int vqo_encode_h(const double* v, int64_t nv, int d, const double* hb, const uint16_t* book,
+                 int64_t K, uint32_t* idx) {
+    if (d < 1 || d > 64 || K < 1) return 1;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < nv; ++i) {
+        double t[64];
+        double best = INFINITY;
+        int64_t arg = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            double dist = dist_h(v + i * d, hb + i * d * d, book + k * d, d, t);
+            if (dist < best) { best = dist; arg = k; }
+        }
+        idx[i] = (uint32_t)arg;
+    }
+    return 0;
+}
+
+/* The two-stage cascade under the weighted distance: i1 = argmin_k
+ * D_H(v, C1[k]); r = v - C1[i1] (fp64); i2 = argmin_k D_H(r, C2[k]) with the
+ * same sub-matrix.  The page writes the residual stage with the plain
+ * distance; with H_v = I the two coincide, and weighting it keeps the second
+ * stage minimising the same objective for the final reconstruction. */
+int vqo_encode_h_residual(const double* v, int64_t nv, int d, const double* hb,
+                          const uint16_t* book1, int64_t K1, const uint16_t* book2, int64_t K2,
+                          uint32_t* idx1, uint32_t* idx2) {
+    if (vqo_encode_h(v, nv, d, hb, book1, K1, idx1)) return 1;
+    double* r = (double*)malloc((size_t)(nv > 0 ? nv : 1) * (size_t)d * sizeof(double));
+    if (!r) return 2;
+    for (int64_t i = 0; i < nv; ++i)
+        for (int e = 0; e < d; ++e)
+            r[i * d + e] = v[i * d + e] - (double)vqo_f16_to_f32(book1[(int64_t)idx1[i] * d + e]);
+    int rc = vqo_encode_h(r, nv, d, hb, book2, K2, idx2);
     free(r);
     return rc;
 }

@@ -392,6 +392,144 @@ def test_two_book_encoders():
     assert np.array_equal(g2, dist.argmin(1).astype(np.uint32))
 
 
+# -- Hessian-weighted encoding --------------------------------------------------
+# D_H(v, c) = (v - c)^T H_v (v - c), H_v the sub-matrix of H on the vector's
+# channels ("VPTQ Guide", section "1. Second-Order Hessian-Weighted Optimization").
+
+def _f16(vals) -> np.ndarray:
+    return np.asarray(vals, np.float16).view(np.uint16)
+
+
+def _spd(rng, n: int) -> np.ndarray:
+    a = rng.standard_normal((n, n))
+    return a @ a.T / n + 0.05 * np.eye(n)
+
+
+def test_encode_h_with_identity_is_the_plain_encoder():
+    """H_v = I gives the plain squared distance operation for operation (the
+    products by 0 and 1 are exact), so the indices agree bit for bit, also
+    for 4 I (a power of two scales every distance exactly), and the weighted
+    cascade with I is the plain cascade."""
+    spec = LayerSpec(8, 64, 8, (10, 6), (0.05, 0.01))
+    L = synth.make_layer(spec, seed=41)
+    b1, b2 = L.codebooks
+    rng = np.random.default_rng(42)
+    v = rng.standard_normal((700, 8)) * 0.05
+    eye = np.broadcast_to(np.eye(8), (700, 8, 8))
+    assert np.array_equal(oracle.encode_h(v, eye, b1), oracle.encode(v, b1))
+    assert np.array_equal(oracle.encode_h(v, 4 * eye, b1), oracle.encode(v, b1))
+    g1, g2 = oracle.encode_h_residual(v, eye, b1, b2)
+    p1, p2 = oracle.encode_residual(v, b1, b2)
+    assert np.array_equal(g1, p1) and np.array_equal(g2, p2)
+
+
+def test_encode_h_diagonal_hand_worked():
+    """Book (1, 0), (0, 1.5), (3, 3); D_H = sum_e H_ee (v_e - c_e)^2 for a
+    diagonal H, worked by hand:
+      v = (0, 0),     H = I:             1,     2.25,  18      -> 0
+      v = (0, 0),     H = diag(4, 1):    4,     2.25,  45      -> 1
+      v = (0, 0),     H = diag(1, 4):    1,     9,     45      -> 0
+      v = (0.9, 1.2), H = I:             1.45,  0.9,   7.65    -> 1
+      v = (0.9, 1.2), H = diag(10, 0.1): 0.244, 8.109, 44.424  -> 0"""
+    book = _f16([[1, 0], [0, 1.5], [3, 3]])
+    cases = [((0.0, 0.0), (1.0, 1.0), 0), ((0.0, 0.0), (4.0, 1.0), 1), ((0.0, 0.0), (1.0, 4.0), 0),
+             ((0.9, 1.2), (1.0, 1.0), 1), ((0.9, 1.2), (10.0, 0.1), 0)]
+    for v, hd, want in cases:
+        assert list(oracle.encode_h(np.array([v]), np.diag(hd)[None], book)) == [want], (v, hd)
+    # the same vectors in one call, each with its own sub-matrix
+    vs = np.array([c[0] for c in cases])
+    hs = np.stack([np.diag(c[1]) for c in cases])
+    assert list(oracle.encode_h(vs, hs, book)) == [c[2] for c in cases]
+
+
+def test_encode_h_off_diagonal_hand_worked():
+    """H = [[1, 0.75], [0.75, 1]], v = 0: (1, 1) -> 1 + 1 + 2 * 0.75 = 3.5;
+    (1, -1.25) -> 1 + 1.5625 - 2 * 0.75 * 1.25 = 0.6875: picks 1, where the
+    plain distances 2 and 2.5625 pick 0.  The cross term's sign matters: with
+    -0.75 off the diagonal the distances become 0.5 and 4.4375 (picks 0)."""
+    book = _f16([[1, 1], [1, -1.25]])
+    v = np.zeros((1, 2))
+    assert list(oracle.encode(v, book)) == [0]
+    assert list(oracle.encode_h(v, np.array([[[1.0, 0.75], [0.75, 1.0]]]), book)) == [1]
+    assert list(oracle.encode_h(v, np.array([[[1.0, -0.75], [-0.75, 1.0]]]), book)) == [0]
+    # a non-symmetric H weighs like its symmetric part: (v-c)^T H (v-c)
+    assert list(oracle.encode_h(v, np.array([[[1.0, 1.5], [0.0, 1.0]]]), book)) == [1]
+
+
+def test_encode_h_ties_go_to_lowest_index():
+    book = _f16([[1, 0], [0, 1], [1, 0]])
+    h = np.array([[[2.0, 0.0], [0.0, 2.0]]])
+    assert list(oracle.encode_h(np.array([[1.0, 0.0]]), h, book)) == [0]
+    assert list(oracle.encode_h(np.array([[0.5, 0.5]]), h, book)) == [0]
+
+
+@pytest.mark.parametrize("d,kin", [(8, 8 * 12), (6, 6 * 10 + 4)])
+def test_encode_h_matches_numpy_brute_force_on_layer_blocks(d, kin):
+    """A random SPD Hessian of a small layer: the oracle with each vector's
+    sub-matrix (hessian_blocks) agrees with numpy's einsum distances and
+    argmin, for whole vectors and the partial last one; the chosen distance is
+    numpy's minimum.  Taking the neighbouring block instead changes answers."""
+    rng = np.random.default_rng(43 + d)
+    rows = 9
+    h = _spd(rng, kin)
+    book = synth.to_f16_bits(rng.standard_normal((64, d)).astype(np.float32) * 0.3).reshape(64, d)
+    w = rng.standard_normal((rows, kin)) * 0.3
+    full, last = oracle.hessian_blocks(h, kin, d, rows)
+    nfull, rem = kin // d, kin % d
+    assert (rem == 0) == (last is None)
+    v = w[:, :nfull * d].reshape(rows * nfull, d)
+    got = oracle.encode_h(v, full, book)
+    c = book.view(np.float16).astype(np.float64)
+    jj = np.tile(np.arange(nfull), rows)
+    t = v[:, None, :] - c[None]                                   # [nv][K][d]
+    blocks = np.stack([h[j * d:(j + 1) * d, j * d:(j + 1) * d] for j in jj])
+    dist = np.einsum("nke,nef,nkf->nk", t, blocks, t)
+    assert np.array_equal(got, dist.argmin(1).astype(np.uint32))
+    chosen = dist[np.arange(len(got)), got]
+    assert np.allclose(chosen, dist.min(1), rtol=1e-12, atol=0)
+    # the sub-matrix is the vector's own: the neighbouring block moves answers
+    shifted = np.stack([h[((j + 1) % nfull) * d:((j + 1) % nfull + 1) * d,
+                          ((j + 1) % nfull) * d:((j + 1) % nfull + 1) * d] for j in jj])
+    assert (oracle.encode_h(v, shifted, book) != got).mean() > 0.05
+    # and the weighting moves answers against the plain distance
+    assert (oracle.encode(v, book) != got).mean() > 0.05
+    if rem:
+        vl = np.ascontiguousarray(w[:, nfull * d:])
+        bl = np.ascontiguousarray(book[:, :rem])
+        gl = oracle.encode_h(vl, last, bl)
+        hl = h[nfull * d:, nfull * d:]
+        tl = vl[:, None, :] - bl.view(np.float16).astype(np.float64)[None]
+        dl = np.einsum("nke,ef,nkf->nk", tl, hl, tl)
+        assert np.array_equal(gl, dl.argmin(1).astype(np.uint32))
+
+
+def test_encode_h_residual_matches_numpy():
+    rng = np.random.default_rng(47)
+    d = 8
+    spec = LayerSpec(8, 64, d, (6, 4), (0.3, 0.05))
+    b1, b2 = synth.make_layer(spec, seed=48).codebooks
+    v = rng.standard_normal((200, d)) * 0.3
+    hb = np.stack([_spd(rng, d) for _ in range(200)])
+    g1, g2 = oracle.encode_h_residual(v, hb, b1, b2)
+    c1 = b1.view(np.float16).astype(np.float64)
+    c2 = b2.view(np.float16).astype(np.float64)
+    t1 = v[:, None] - c1[None]
+    assert np.array_equal(g1, np.einsum("nke,nef,nkf->nk", t1, hb, t1).argmin(1))
+    r = v - c1[g1]
+    t2 = r[:, None] - c2[None]
+    assert np.array_equal(g2, np.einsum("nke,nef,nkf->nk", t2, hb, t2).argmin(1))
+
+
+def test_hessian_blocks_pick_the_vector_channels():
+    kin, d, rows = 14, 4, 2
+    h = np.arange(kin)[:, None] * 100.0 + np.arange(kin)[None, :]
+    full, last = oracle.hessian_blocks(h, kin, d, rows)
+    assert full.shape == (rows * 3, d, d) and last.shape == (rows, 2, 2)
+    assert full[1][0, 0] == 4 * 100 + 4 and full[1][3, 2] == 7 * 100 + 6
+    assert full[3 + 2][1, 3] == 9 * 100 + 11                     # row 1, vector 2
+    assert last[1].tolist() == [[1212.0, 1213.0], [1312.0, 1313.0]]
+
+
 # -- randomized Hadamard transform ----------------------------------------------
 
 def _signs(n, seed):
