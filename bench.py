@@ -26,6 +26,10 @@ encode = the nearest-centroid encoder (vq_encode) on a 4096 x 4096 matrix
 rht_gate = the 70B gate_proj in the rotated basis (vq_gemv_rht) beside the
          same layer through vq_gemv.
 hessian = vq_hessian on 8192 tokens x 8192 features, in TFLOP/s.
+sweep  = every other configuration of the measurement plan, one call each
+         (tiny 512^2; 8B up_proj at B 1/4/16; 70B gate_proj and down_proj at
+         B 2/8/16; 405B gate_proj at B 2/4/8/16 and prefill M=1024, 405B q_proj
+         at M=1024; the 8192^2 prefill at M 512/4096).
 roofline, cpu_baseline, clocks and gpu_launches are described beside the
 keys they fill.  ``--impl reference`` times the CPU oracle on the same
 metric instead (a bounded sample of the same workload per step).
@@ -385,7 +389,7 @@ def run_gpu(args):
                 "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                 "row_order_gather_ceiling_us": 120.0,
                 "note": "not HBM-bound: the table kernel is bound by instruction issue and "
-                        "shared-memory lookups (4 slice tests per index), the row-order kernel "
+                        "shared-memory lookups (3 slice tests per index), the row-order kernel "
                         "by random 16-byte centroid gathers through L1/L2 (0.84/clk/SM)"}
 
     # e2e through the public API with pinned host activations and outputs:
@@ -425,6 +429,7 @@ def run_gpu(args):
            "ms_per_step": e2e_ms / args.steps}
 
     gemm = run_gemm(dev, peaks, peak_src, vq)
+    sweep = run_sweep(dev, peaks, peak_src, vq, copies[0])
     decode_405b = run_decode_405b(dev, peaks, peak_src, vq)
     qkv_405b = run_405b_qkv(dev, peaks, peak_src, vq)
     rht = run_rht(dev, vq)
@@ -445,6 +450,7 @@ def run_gpu(args):
         "gpu_launches": int(launches),
         "clocks": clocks.summary(),
         "gemm": gemm,
+        "sweep": sweep,
         "decode_405b_gate": decode_405b,
         "decode_405b_qkv": qkv_405b,
         "rht_gate": rht,
@@ -496,6 +502,108 @@ def run_gemm(dev, peaks, peak_src, vq):
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"],
                          "peak_source": peak_src + " (bf16 burst; fp16 nominal rate is the same)"}}
+
+
+def _median_us(fn, flush, reps=10, warm=3):
+    """Median time of fn() in microseconds from CUDA events on the current
+    stream, a 256 MB write between calls (L2 flushed), after warm-up calls."""
+    import torch
+    for _ in range(warm):
+        fn()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts) * 1e3
+
+
+def run_sweep(dev, peaks, peak_src, vq, layers70):
+    """Every configuration of the measurement plan beside the headline, one
+    call each, L2 flushed between calls: the decode GEMV per layer and batch
+    (both index orders where the planner's kernels differ; the faster is
+    reported first) and the prefill GEMM at the other row counts.  Decode:
+    us, algorithmic GB/s and the fraction of the measured HBM peak; prefill:
+    us, TFLOP/s and the fraction of the measured bf16 burst peak."""
+    import torch
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    hbm = peaks["hbm_gbs"]
+    out = {"protocol": "median of 10 calls, CUDA events, a 256 MB write between calls (L2 flushed)",
+           "peak_source": peak_src, "decode": [], "prefill": []}
+
+    def decode_entry(name, spec, layers_by_order, batches, x_seed, outlier):
+        for bsz in batches:
+            x = torch.from_numpy(synth.make_x(x_seed, bsz, spec.in_features, outlier).view(np.int16)).to(dev)
+            x = x.view(torch.bfloat16)
+            y = torch.empty((bsz, spec.out_features), dtype=torch.bfloat16, device=dev)
+            res = {}
+            for order, layer in layers_by_order.items():
+                ws = torch.empty(max(256, vq.gemv_workspace_size(layer, bsz)), dtype=torch.uint8, device=dev)
+                res[order] = _median_us(lambda: vq.gemv(layer, x, out=y, workspace=ws), flush)
+                del ws
+            best = min(res, key=res.get)
+            gbs = alg_bytes(spec, bsz) / (res[best] * 1e-6) / 1e9
+            out["decode"].append({"workload": name, "batch": bsz, "us": res[best], "index_order": best,
+                                  "us_by_order": res, "gbs": gbs, "frac_of_measured_hbm": gbs / hbm})
+
+    # tiny 512 x 512, one 2^16 book, B = 1
+    w = WORKLOADS["tiny_512"]
+    spec, seed = w.layers[0]
+    rows = vq.Layer.from_synth(synth.make_layer(spec, seed), dev)
+    decode_entry("tiny_512 512x512, d=8, K=2^16 (2.0 bpw)", spec,
+                 {"rows": rows, "tile4": vq.repack_tile4(rows)}, (1,), w.x_seed, 0.0)
+    # Llama-3-8B up_proj, 2^12 + 2^8 books, B in {1, 4, 16}
+    w = WORKLOADS["llama3_8b_up"]
+    spec, seed = w.layers[0]
+    rows = vq.Layer.from_synth(synth.make_layer(spec, seed), dev)
+    decode_entry("llama3_8b_up 14336x4096, d=8, K=2^12 + 2^8 (2.5 bpw)", spec,
+                 {"rows": rows, "tile4": vq.repack_tile4(rows)}, (1, 4, 16), w.x_seed, 0.0)
+    del rows
+    # Llama-3-70B MLP layers (the step's tiled layers), B in {2, 8, 16}
+    w = WORKLOADS[DECODE]
+    for (spec, _), layer in zip(w.layers, layers70):
+        if spec.name == "up_proj":
+            continue                                    # the same shape as gate_proj
+        decode_entry(f"llama3_70b {spec.name} {spec.out_features}x{spec.in_features}, d=8, K=2^16 (2.0 bpw)",
+                     spec, {layer.layout: layer}, (2, 8, 16), w.x_seed, w.outlier_frac)
+    # Llama-3.1-405B gate_proj, 2^12 + 2^4 books at d = 6, B in {2, 4, 8, 16}
+    w = WORKLOADS["llama31_405b"]
+    spec, seed = w.layers[4]
+    rows = vq.Layer.from_synth(synth.make_layer(spec, seed), dev)
+    decode_entry("llama31_405b gate_proj 53248x16384, d=6, K=2^12 + 2^4 (2.67 bpw)", spec,
+                 {"rows": rows, "tile4": vq.repack_tile4(rows)}, (2, 4, 8, 16), w.x_seed + 4, 0.0)
+
+    def prefill_entry(name, spec, layer, m, x_seed):
+        x = torch.from_numpy(synth.make_x(x_seed, m, spec.in_features).view(np.int16)).to(dev).view(torch.bfloat16)
+        y = torch.empty((m, spec.out_features), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(vq.gemm_workspace_size(layer, m), dtype=torch.uint8, device=dev)
+        us = _median_us(lambda: vq.gemm(layer, x, out=y, workspace=ws), flush)
+        torch.cuda.synchronize()
+        tf = 2.0 * m * spec.out_features * spec.in_features / (us * 1e-6) / 1e12
+        out["prefill"].append({"workload": name, "m": m, "us": us, "tflops": tf,
+                               "frac_of_measured_bf16": tf / peaks["bf16_tflops"],
+                               "device_status": int(ws[:4].view(torch.int32).item())})
+
+    # the 405B gate_proj at prefill M = 1024 (the layer above), then q_proj
+    prefill_entry("llama31_405b gate_proj 53248x16384, M=1024", spec, rows, 1024, w.x_seed + 4)
+    del rows
+    qspec, qseed = w.layers[0]
+    q = vq.Layer.from_synth(synth.make_layer(qspec, qseed), dev)
+    prefill_entry("llama31_405b q_proj 16384x16384, M=1024", qspec, q, 1024, w.x_seed)
+    del q
+    # prefill 8192 x 8192 (2^16 + 2^8) at M = 512 and 4096 (2048 is the gemm object)
+    w = WORKLOADS[PREFILL]
+    spec, seed = w.layers[0]
+    layer = vq.Layer.from_synth(synth.make_layer(spec, seed), dev)
+    for m in (512, 4096):
+        prefill_entry(f"prefill_8192 8192x8192, K=2^16 + 2^8 (3.0 bpw), M={m}", spec, layer, m, w.x_seed)
+    del layer, flush
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_decode_405b(dev, peaks, peak_src, vq):
