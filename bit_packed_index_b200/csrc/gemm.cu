@@ -51,7 +51,7 @@ __host__ __device__ constexpr int stage_bytes(int msub) { return msub * kATile +
 constexpr int kThreads = 384;                   // 12 warps
 constexpr int kProducerThread0 = 128;           // warps 4..11 produce B tiles
 constexpr int kProducers = 256;
-constexpr int kCtrlBytes = 3072;                // barriers, flags, scale/bias staging
+constexpr int kCtrlBytes = 4096;                // barriers, flags, scale/bias staging
 constexpr long long kWaitBudget = 4000000000LL; // SM clocks (about 2 s)
 constexpr int kMaxStages = 8;
 
@@ -82,7 +82,7 @@ struct Ctrl {
   uint64_t acc_full;
   uint32_t tmem_base;
   int abort_flag;
-  float sb[2 * BN];   // per-column scale, then bias, of this tile
+  float sb[3 * BN];   // per-column scale, bias and output bias of this tile
 };
 static_assert(sizeof(Ctrl) <= kCtrlBytes, "control block");
 
@@ -248,7 +248,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch(&tmap_a);
     if (MODE == kStaged) tma_prefetch(&tmap_b);
   }
-  // Per-column scale and bias of this tile (fused form applies them).
+  // Per-column scale and bias of this tile (fused form applies them; the
+  // staged form's W_hat already holds them) and the output bias (both forms).
   for (int i = threadIdx.x; i < BN; i += kThreads) {
     const int n = n0 + i;
     float s = 1.0f, t = 0.0f;
@@ -258,6 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ctrl->sb[i] = s;
     ctrl->sb[BN + i] = t;
+    ctrl->sb[2 * BN + i] = n < L.n ? out_bias_of(L.ob, n) : 0.0f;
   }
   BookView bv[2];
   if (MODE == kFused) {
@@ -385,7 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            v[i] = ctrl->sb[c * 32 + i] * (__uint_as_float(acc[i]) * rsc) + ctrl->sb[BN + c * 32 + i] * rs;
+            v[i] = ctrl->sb[c * 32 + i] * (__uint_as_float(acc[i]) * rsc) + ctrl->sb[BN + c * 32 + i] * rs +
+                   ctrl->sb[2 * BN + c * 32 + i];
           const int ncols = min(32, L.n - nb);
           uint8_t* dst = reinterpret_cast<uint8_t*>(g.y) + (static_cast<int64_t>(row) * g.ldy + nb) * es;
           if (ncols == 32 && aligned(dst, 16)) {
@@ -714,9 +717,7 @@ size_t gemm_workspace_bytes(const Layer& L, int m, bool x_fp16) {
 
 vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t ldx, void* y,
                       vq_dtype yt, int64_t ldy, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  const size_t es = yt == VQ_FP32 ? 4 : 2;
-  if (L.kin == 0)
-    return cuda_status(cudaMemset2DAsync(y, ldy * es, 0, static_cast<size_t>(L.n) * es, m, stream));
+  if (L.kin == 0) return launch_empty_rows(L, y, yt, ldy, m, stream);
   const GemmLayout lay = layout_for(L, m, x_fp16);
   if (ws_bytes < lay.total) return VQ_ERR_WORKSPACE;
   uint8_t* w8 = static_cast<uint8_t*>(ws);
@@ -785,7 +786,7 @@ vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t
   g.book_bytes = 0;
   const int optin = device_smem_optin();
   const int kStageBytes = stage_bytes(msub);
-  const size_t fixed = 1024 + 3072;   // alignment slack + control block
+  const size_t fixed = 1024 + kCtrlBytes;   // alignment slack + control block
   if (lay.mode == kFused) {
     // Stage the books that fit next to at least three pipeline stages.
     const size_t budget = static_cast<size_t>(optin) - fixed - 2 * kStageBytes;
@@ -847,7 +848,7 @@ vq_status launch_hessian(const void* x, bool x_fp16, int n, int d, int64_t ldx, 
   g.budget = wait_budget();
   const int optin = device_smem_optin();
   const int kStageBytes = stage_bytes(msub);
-  const size_t fixed = 1024 + 3072;
+  const size_t fixed = 1024 + kCtrlBytes;
   g.stages = std::min(4, static_cast<int>((optin - fixed) / kStageBytes));
   const size_t smem = fixed + static_cast<size_t>(g.stages) * kStageBytes;
   g.bn = bn;

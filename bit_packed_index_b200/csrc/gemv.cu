@@ -164,7 +164,8 @@ __global__ void __launch_bounds__(kGvThreads) gemv_kernel(
           if (lane == 0 && orow < o_end && b < batch) {
             const float sc = L.scale ? h2f(L.scale[orow]) : 1.0f;
             const float t = L.bias ? h2f(L.bias[orow]) : 0.0f;
-            const float val = sc * dot + t * xsum[b];
+            float val = sc * dot + t * xsum[b];
+            if (split == 0) val += out_bias_of(L.ob, orow);   // once, with split 0's part
             if (ws) ws[(static_cast<int64_t>(split) * batch + b) * L.n + orow] = val;
             else store_out(y, yt, b * ldy + orow, val);
           }
@@ -184,6 +185,17 @@ __global__ void gemv_finalize(const float* __restrict__ ws, int nsplit, int batc
     float v = 0.0f;
     for (int s = 0; s < nsplit; ++s) v += ws[(s * static_cast<int64_t>(batch) + b) * n + o];
     store_out(y, yt, b * ldy + o, v);
+  }
+}
+
+// y[b][o] = out_bias[o] for every row b of y (a layer with no inputs).
+__global__ void fill_out_bias(const uint16_t* __restrict__ ob, int rows, int n, void* __restrict__ y,
+                              vq_dtype yt, int64_t ldy) {
+  const int64_t total = static_cast<int64_t>(rows) * n;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = i / n, o = i - b * n;
+    store_out(y, yt, b * ldy + o, h2f(ob[o]));
   }
 }
 
@@ -267,14 +279,24 @@ vq_status plan_gemv(const Layer& L, int batch, GemvPlan* p, size_t ws_cap) {
   return VQ_OK;
 }
 
+vq_status launch_empty_rows(const Layer& L, void* y, vq_dtype yt, int64_t ldy, int rows,
+                            cudaStream_t stream) {
+  if (!L.ob) {   // y = 0: all-zero bits in every output type
+    const size_t es = yt == VQ_FP32 ? 4 : 2;
+    return cuda_status(cudaMemset2DAsync(y, ldy * es, 0, L.n * es, rows, stream));
+  }
+  const int64_t total = static_cast<int64_t>(rows) * L.n;
+  const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 4 * device_sm_count()));
+  count_launch();
+  fill_out_bias<<<blocks, 256, 0, stream>>>(L.ob, rows, L.n, y, yt, ldy);
+  return cuda_status(cudaGetLastError());
+}
+
 vq_status launch_gemv(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, int batch,
                       int64_t ldx, void* y, vq_dtype yt, int64_t ldy, float* ws,
                       cudaStream_t stream) {
   if (L.n == 0 || batch == 0) return VQ_OK;
-  if (L.kin == 0) {   // empty rows: y = 0 (all-zero bits in every output type)
-    const size_t es = yt == VQ_FP32 ? 4 : 2;
-    return cuda_status(cudaMemset2DAsync(y, ldy * es, 0, L.n * es, batch, stream));
-  }
+  if (L.kin == 0) return launch_empty_rows(L, y, yt, ldy, batch, stream);
   const int D = (L.d == 8) ? 8 : (L.d == 6 ? 6 : 0);
   cudaError_t e;
   if (p.fast == 7) {

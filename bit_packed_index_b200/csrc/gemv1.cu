@@ -267,7 +267,8 @@ __global__ void __launch_bounds__(kThreads1, 1) gemv1_kernel(
       for (int c = 0; c < nck; ++c) dot += part[rl * chunks_per_split + c];
       const float sc = L.scale ? h2f(L.scale[o]) : 1.0f;
       const float t = L.bias ? h2f(L.bias[o]) : 0.0f;
-      const float val = sc * dot + t * (*xsum_s);
+      float val = sc * dot + t * (*xsum_s);
+      if (split == 0) val += out_bias_of(L.ob, o);   // once, with split 0's part
       if (ws) ws[static_cast<int64_t>(split) * L.n + o] = val;
       else store_out(y, yt, o, val);
     }

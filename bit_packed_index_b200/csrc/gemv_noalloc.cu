@@ -58,6 +58,14 @@ using namespace vqk;
 extern "C" vq_status vq_gemv_noalloc(const vq_layer_desc* layer, const void* x, vq_dtype x_dtype,
                                      int32_t batch, int64_t ldx, void* y, vq_dtype y_dtype,
                                      int64_t ldy, void* stream) {
+  // The scratch array and the plan belong to the current device: a stream of
+  // another device is rejected.
+  if (stream) {
+    int cur = 0, sdev = 0;
+    if (cudaGetDevice(&cur) == cudaSuccess &&
+        cudaStreamGetDevice(static_cast<cudaStream_t>(stream), &sdev) == cudaSuccess && sdev != cur)
+      return VQ_ERR_INVALID_ARG;
+  }
   size_t need = 0;
   vq_status st = gemv_workspace_bytes(layer, batch, kScratchBytes, &need);
   if (st != VQ_OK) return st;

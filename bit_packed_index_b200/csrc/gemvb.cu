@@ -234,7 +234,8 @@ __global__ void __launch_bounds__(kThreadsB, 1) gemvb_kernel(
       if (o >= L.n) continue;
       const float sc = L.scale ? h2f(L.scale[o]) : 1.0f;
       const float t = L.bias ? h2f(L.bias[o]) : 0.0f;
-      const float val = sc * part[rl * BT + b] + t * xsum[b];
+      float val = sc * part[rl * BT + b] + t * xsum[b];
+      if (split == 0) val += out_bias_of(L.ob, o);   // once, with split 0's part
       if (ws) ws[(static_cast<int64_t>(split) * batch + b) * L.n + o] = val;
       else store_out(y, yt, b * ldy + o, val);
     }

@@ -237,8 +237,9 @@ __global__ void __launch_bounds__(kTcThreads) gemv_tc_kernel(const __grid_consta
       if (row < L.n) {
         const float sc = L.scale ? h2f(L.scale[row]) : 1.0f;
         const float tb = (L.bias && split == 0) ? h2f(L.bias[row]) : 0.0f;
+        const float ob = split == 0 ? out_bias_of(L.ob, row) : 0.0f;
         for (int b = 0; b < g.batch; ++b) {
-          const float v = sc * (__uint_as_float(acc[b]) * g.xe[b]) + tb * g.xsum[b];
+          const float v = sc * (__uint_as_float(acc[b]) * g.xe[b]) + tb * g.xsum[b] + ob;
           if (g.part) g.part[(static_cast<int64_t>(split) * g.batch + b) * L.n + row] = v;
           else store_out(g.y, g.yt, b * g.ldy + row, v);
         }

@@ -40,10 +40,11 @@ __device__ __forceinline__ float rht_sign(const uint32_t* __restrict__ signs, in
   return (__ldg(signs + (t >> 5)) >> (t & 31)) & 1u ? -1.0f : 1.0f;
 }
 
-// grid (n / b, rows); dynamic shared memory b floats.
+// grid (n / b, rows); dynamic shared memory b floats.  `add` (fp16 [n], may
+// be null) is added to every output row after the transform.
 __global__ void rht_kernel(const void* __restrict__ in, int in_t, int64_t ld_in, int b,
                            const uint32_t* __restrict__ signs, int inverse, float scale,
-                           void* __restrict__ out, int out_t, int64_t ld_out) {
+                           void* __restrict__ out, int out_t, int64_t ld_out, const uint16_t* __restrict__ add) {
   extern __shared__ float hv[];
   const int64_t row = blockIdx.y;
   const int64_t k0 = static_cast<int64_t>(blockIdx.x) * b;
@@ -66,6 +67,7 @@ __global__ void rht_kernel(const void* __restrict__ in, int in_t, int64_t ld_in,
   for (int i = threadIdx.x; i < b; i += blockDim.x) {
     float v = hv[i] * scale;
     if (inverse) v *= rht_sign(signs, k0 + i);
+    v += out_bias_of(add, static_cast<int>(k0 + i));
     store_out(out, static_cast<vq_dtype>(out_t), row * ld_out + k0 + i, v);
   }
 }
@@ -77,7 +79,7 @@ template <int E>
 __global__ void __launch_bounds__(1024) rht_big_kernel(const void* __restrict__ in, int in_t, int64_t ld_in,
                                                        int b, const uint32_t* __restrict__ signs, int inverse,
                                                        float scale, void* __restrict__ out, int out_t,
-                                                       int64_t ld_out) {
+                                                       int64_t ld_out, const uint16_t* __restrict__ add) {
   extern __shared__ float hv[];
   const int t = threadIdx.x, T = blockDim.x;
   const int64_t row = blockIdx.y;
@@ -131,12 +133,14 @@ __global__ void __launch_bounds__(1024) rht_big_kernel(const void* __restrict__ 
   for (int r = 0; r < E; ++r) {
     float y = v[r] * scale;
     if (inverse) y *= rht_sign(signs, base + r);
+    y += out_bias_of(add, static_cast<int>(base + r));
     store_out(out, static_cast<vq_dtype>(out_t), row * ld_out + base + r, y);
   }
 }
 
 cudaError_t launch_rht(const void* in, vq_dtype in_t, int rows, int n, int64_t ld_in, const uint32_t* signs,
-                       bool inverse, void* out, vq_dtype out_t, int64_t ld_out, cudaStream_t stream) {
+                       bool inverse, void* out, vq_dtype out_t, int64_t ld_out, cudaStream_t stream,
+                       const uint16_t* add = nullptr) {
   const int b = rht_block(n);
   if (b >= 256) {
     const int T = std::min(1024, b / 8), E = b / T;
@@ -147,7 +151,7 @@ cudaError_t launch_rht(const void* in, vq_dtype in_t, int rows, int n, int64_t l
     if (e != cudaSuccess) return e;
     count_launch();
     k<<<dim3(n / b, rows), T, smem, stream>>>(in, in_t, ld_in, b, signs, inverse ? 1 : 0, scale, out, out_t,
-                                              ld_out);
+                                              ld_out, add);
     return cudaGetLastError();
   }
   const int smem = b * static_cast<int>(sizeof(float));
@@ -157,7 +161,7 @@ cudaError_t launch_rht(const void* in, vq_dtype in_t, int rows, int n, int64_t l
   const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b)));
   count_launch();
   rht_kernel<<<dim3(n / b, rows), threads, smem, stream>>>(in, in_t, ld_in, b, signs, inverse ? 1 : 0, scale,
-                                                          out, out_t, ld_out);
+                                                          out, out_t, ld_out, add);
   return cudaGetLastError();
 }
 
@@ -247,10 +251,13 @@ vq_status vq_gemv_rht(const vq_layer_desc* layer, const uint32_t* signs_in, cons
     cudaError_t e = launch_rht(x, x_dtype, batch, L.kin, ldx, signs_in, false, xt, VQ_FP16, r.ldt, stream);
     if (e != cudaSuccess) return cuda_status(e);
   }
-  st = gemv_run(layer, xt, VQ_FP16, batch, r.ldt, yt, VQ_FP32, L.n, r.gemv_bytes ? ws + r.off_g : nullptr,
+  // The output bias belongs to y, not to y~: the inverse transform adds it.
+  vq_layer_desc inner = *layer;
+  inner.out_bias = nullptr;
+  st = gemv_run(&inner, xt, VQ_FP16, batch, r.ldt, yt, VQ_FP32, L.n, r.gemv_bytes ? ws + r.off_g : nullptr,
                 r.gemv_bytes, ~static_cast<size_t>(0), stream);
   if (st != VQ_OK) return st;
-  return cuda_status(launch_rht(yt, VQ_FP32, batch, L.n, L.n, signs_out, true, y, y_dtype, ldy, stream));
+  return cuda_status(launch_rht(yt, VQ_FP32, batch, L.n, L.n, signs_out, true, y, y_dtype, ldy, stream, L.ob));
 }
 
 }  // extern "C"

@@ -927,6 +927,7 @@ struct LutOut {
   int row0[kLutMaxLayers + 1];
   const uint16_t* scale[kLutMaxLayers];
   const uint16_t* bias[kLutMaxLayers];
+  const uint16_t* ob[kLutMaxLayers];     // output bias, may be null
   void* y[kLutMaxLayers];
 };
 
@@ -937,12 +938,13 @@ LutOut lut_out_single(const Layer& L, void* y) {
   o.row0[1] = L.n;
   o.scale[0] = L.scale;
   o.bias[0] = L.bias;
+  o.ob[0] = L.ob;
   o.y[0] = y;
   return o;
 }
 
-// y_l[o] = s_l[o] * sum_b part[b][row0_l + o] + t_l[o] * sum_b xpart[b], the
-// partial sums added in a fixed order.
+// y_l[o] = s_l[o] * sum_b part[b][row0_l + o] + t_l[o] * sum_b xpart[b]
+// + ob_l[o], the partial sums added in a fixed order.
 __global__ void __launch_bounds__(256, 8) gemv_lut_finalize(const float* __restrict__ part,
                                                             const float* __restrict__ xpart, int nparts,
                                                             int ntot, LutOut out, vq_dtype yt) {
@@ -985,7 +987,7 @@ __global__ void __launch_bounds__(256, 8) gemv_lut_finalize(const float* __restr
     const int o = v - out.row0[l];
     const float sc = out.scale[l] ? h2f(out.scale[l][o]) : 1.0f;
     const float tb = out.bias[l] ? h2f(out.bias[l][o]) : 0.0f;
-    store_out(out.y[l], yt, o, sc * t + tb * s_xsum);
+    store_out(out.y[l], yt, o, sc * t + tb * s_xsum + out_bias_of(out.ob[l], o));
   }
 }
 
@@ -1206,6 +1208,7 @@ cudaError_t launch_gemv_lut_multi(const Layer* L, int nl, const LutMultiPlan& p,
     S.row0[l + 1] = out.row0[l + 1] = S.row0[l] + L[l].n;
     out.scale[l] = L[l].scale;
     out.bias[l] = L[l].bias;
+    out.ob[l] = L[l].ob;
     out.y[l] = y[l];
   }
   if (p.kind == 1) {                                 // paired-row small-book kernel

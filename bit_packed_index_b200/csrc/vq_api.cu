@@ -8,7 +8,7 @@
 
 #include "vq_internal.cuh"
 
-static_assert(sizeof(vq_layer_desc) == 96, "vq_layer_desc layout is part of the ABI");
+static_assert(sizeof(vq_layer_desc) == 104, "vq_layer_desc layout is part of the ABI");
 
 namespace vqk {
 namespace {
@@ -93,9 +93,12 @@ vq_status check_layer(const vq_layer_desc* desc, Layer* out) {
     L.idx[1] = L.idx[0];
     L.book[1] = L.book[0];
   }
-  if ((D.scale && !aligned(D.scale, 2)) || (D.bias && !aligned(D.bias, 2))) return VQ_ERR_ALIGNMENT;
+  if ((D.scale && !aligned(D.scale, 2)) || (D.bias && !aligned(D.bias, 2)) ||
+      (D.out_bias && !aligned(D.out_bias, 2)))
+    return VQ_ERR_ALIGNMENT;
   L.scale = D.scale;
   L.bias = D.bias;
+  L.ob = D.out_bias;
   *out = L;
   return VQ_OK;
 }

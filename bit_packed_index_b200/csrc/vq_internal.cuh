@@ -32,6 +32,7 @@ struct Layer {
   const uint16_t* book[2];
   const uint16_t* scale;  // may be null
   const uint16_t* bias;   // may be null
+  const uint16_t* ob;     // output bias added to y after the product, may be null
   int layout;             // VQ_IDX_ROWS or VQ_IDX_TILE4
 };
 
@@ -56,6 +57,9 @@ __host__ __device__ inline bool aligned(const void* p, size_t a) { return (reint
 // Kernel launchers (one per .cu file).
 // ---------------------------------------------------------------------------
 vq_status launch_dequant(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream);
+// y of a layer without inputs (Kin = 0): its output bias, else zeros (gemv.cu).
+vq_status launch_empty_rows(const Layer& L, void* y, vq_dtype yt, int64_t ldy, int rows,
+                            cudaStream_t stream);
 
 // Tiled index order (tile4.cu).
 vq_status launch_repack_tile4(const Layer& src, uint32_t* const dst[2], const int64_t tile_words[2],
@@ -149,6 +153,8 @@ __device__ __forceinline__ uint32_t load_field(const uint32_t* __restrict__ row,
 }
 
 __device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+// Output bias of row o (0 without one).
+__device__ __forceinline__ float out_bias_of(const uint16_t* ob, int o) { return ob ? h2f(ob[o]) : 0.0f; }
 __device__ __forceinline__ float bf2f(uint16_t h) {
   return __bfloat162float(__ushort_as_bfloat16(h));
 }

@@ -8,7 +8,7 @@ Names follow the C ABI: ``dequant``, ``gemv``, ``gemv_multi``, ``gemv_rht``,
 ``rht``, ``gemm``, ``repack_tile4``, ``encode``, ``hessian``, plus the
 workspace size queries.  A ``Layer`` holds the device tensors of one
 quantised layer (packed index streams in row order or in the tiled order,
-fp16 codebooks, optional fp16 scale and bias).
+fp16 codebooks, optional fp16 scale and bias, optional fp16 output bias).
 """
 from __future__ import annotations
 
@@ -48,7 +48,7 @@ class _Desc(C.Structure):
         ("vec_dim", C.c_int32), ("n_books", C.c_int32), ("log2k", C.c_int32 * 2),
         ("idx", C.c_void_p * 2), ("idx_row_words", C.c_int64 * 2),
         ("codebook", C.c_void_p * 2), ("scale", C.c_void_p), ("bias", C.c_void_p),
-        ("idx_layout", C.c_int32), ("reserved", C.c_int32),
+        ("idx_layout", C.c_int32), ("reserved", C.c_int32), ("out_bias", C.c_void_p),
     ]
 
 
@@ -142,6 +142,7 @@ class Layer:
     scale: Optional[torch.Tensor] = None   # float16 [N]
     bias: Optional[torch.Tensor] = None    # float16 [N]
     layout: str = "rows"               # "rows" or "tile4"
+    out_bias: Optional[torch.Tensor] = None   # float16 [N], added to y after the product
     _desc: Optional[_Desc] = field(default=None, repr=False)
 
     @property
@@ -165,14 +166,16 @@ class Layer:
             d.scale = None if self.scale is None else self.scale.data_ptr()
             d.bias = None if self.bias is None else self.bias.data_ptr()
             d.idx_layout = _LAYOUT[self.layout]
+            d.out_bias = None if self.out_bias is None else self.out_bias.data_ptr()
             self._desc = d
         return self._desc
 
     @classmethod
     def from_host(cls, out_features: int, in_features: int, vec_dim: int, log2k: Sequence[int],
                   idx_words: Sequence, codebooks: Sequence, scale=None, bias=None,
-                  device="cuda") -> "Layer":
-        """From numpy arrays: uint32 streams, fp16-bit (uint16) codebooks/scale/bias."""
+                  device="cuda", out_bias=None) -> "Layer":
+        """From numpy arrays: uint32 streams, fp16-bit (uint16) codebooks, scale,
+        bias and output bias."""
         import numpy as np
 
         def words(a):
@@ -187,7 +190,7 @@ class Layer:
 
         return cls(out_features, in_features, vec_dim, list(log2k),
                    [words(w) for w in idx_words], [halves(c) for c in codebooks],
-                   halves(scale), halves(bias))
+                   halves(scale), halves(bias), out_bias=halves(out_bias))
 
     @classmethod
     def from_synth(cls, data, device="cuda", layout: str = "rows") -> "Layer":
@@ -195,7 +198,8 @@ class Layer:
         them on the device with vq_repack_tile4."""
         s = data.spec
         layer = cls.from_host(s.out_features, s.in_features, s.d, s.log2k, data.idx_words,
-                              data.codebooks, data.scale, data.bias, device)
+                              data.codebooks, data.scale, data.bias, device,
+                              getattr(data, "out_bias", None))
         if layout == "tile4":
             layer = repack_tile4(layer)
         elif layout != "rows":
@@ -204,7 +208,7 @@ class Layer:
 
     def nbytes(self) -> int:
         n = sum(t.numel() * t.element_size() for t in self.idx + self.codebooks)
-        for t in (self.scale, self.bias):
+        for t in (self.scale, self.bias, self.out_bias):
             n += 0 if t is None else t.numel() * 2
         return n
 
@@ -229,7 +233,7 @@ def repack_tile4(layer: Layer, tile_words: Optional[Sequence[int]] = None) -> La
     _check("vq_repack_tile4", lib().vq_repack_tile4(C.byref(layer.desc()), ptrs, words,
                                                     C.c_void_p(_stream(layer.device))))
     return Layer(layer.out_features, layer.in_features, layer.vec_dim, list(layer.log2k), dst,
-                 layer.codebooks, layer.scale, layer.bias, layout="tile4")
+                 layer.codebooks, layer.scale, layer.bias, layout="tile4", out_bias=layer.out_bias)
 
 
 def dequant(layer: Layer, out: Optional[torch.Tensor] = None) -> torch.Tensor:

@@ -80,7 +80,7 @@
 extern "C" {
 #endif
 
-#define VQ_ABI_VERSION 3
+#define VQ_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define VQ_API __attribute__((visibility("default")))
@@ -126,6 +126,14 @@ typedef enum vq_dtype {
  *   bias           fp16 [N], or NULL for no bias
  *   idx_layout     VQ_IDX_ROWS or VQ_IDX_TILE4 (a zero-filled struct means rows)
  *   reserved       must be 0
+ *   out_bias       fp16 [N], or NULL: the output-side bias of the product,
+ *                  y[b][o] = sum_k x[b][k] W_hat[o][k] + out_bias[o], added in
+ *                  fp32 to the accumulated product before y is rounded to its
+ *                  type.  The layer's forward ends in F.linear(x, W_hat, bias)
+ *                  ("VPTQ Guide", section "Step 3: Fused Low-Bit VPTQ Linear
+ *                  Layer"); this is that bias, distinct from the per-row bias
+ *                  t above, which is part of W_hat.  vq_dequant ignores it.
+ *                  (Added in ABI version 4, which made the struct 104 bytes.)
  * Entries for m >= n_books are ignored.
  */
 typedef struct vq_layer_desc {
@@ -141,6 +149,7 @@ typedef struct vq_layer_desc {
     const uint16_t* bias;
     int32_t idx_layout;
     int32_t reserved;
+    const uint16_t* out_bias;
 } vq_layer_desc;
 
 /*
@@ -229,8 +238,14 @@ VQ_API vq_status vq_gemv(const vq_layer_desc* layer, const void* x, vq_dtype x_d
  * fixed device array of VQ_NOALLOC_SCRATCH_BYTES inside the library, which
  * every GPU that loads the library holds until the process exits.  The call
  * allocates nothing (no cudaMalloc, no allocating library routine).
- *   - Returns VQ_ERR_WORKSPACE when this layer and batch need more scratch than
- *     VQ_NOALLOC_SCRATCH_BYTES (vq_gemv_workspace_size() tells in advance).
+ *   - Plans whose scratch can shrink run within the array (the table kernels'
+ *     per-block row sums: fewer blocks); a plan that needs more scratch than
+ *     VQ_NOALLOC_SCRATCH_BYTES and cannot shrink (split-K partial sums) makes
+ *     the call return VQ_ERR_WORKSPACE.  vq_gemv_workspace_size() reports the
+ *     unconstrained plan, so a size above the array does not by itself mean
+ *     that this call fails.
+ *   - The array and the plan belong to the current device: `stream` must be a
+ *     stream of the current device (or NULL), else VQ_ERR_INVALID_ARG.
  *   - The first call on each device looks up the array's device address (with
  *     that device current) and caches it; make that first call before any
  *     stream capture.

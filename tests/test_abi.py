@@ -27,8 +27,8 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_host_only_calls(lib):
-    assert lib.vq_abi_version() == 3
-    assert C.sizeof(vq._Desc) == 96       # static_assert'ed in the library
+    assert lib.vq_abi_version() == 4
+    assert C.sizeof(vq._Desc) == 104      # static_assert'ed in the library
     assert C.sizeof(vq._EncDesc) == 88
     assert vq.kernel_launches() == 0          # nothing launched in this process
     for s in range(7):
@@ -83,6 +83,19 @@ def test_layout_field_validation_needs_no_device(lib):
     # but 1000 records of 64 bits need 2000 words per tile
     d.idx_row_words[0] = 4
     assert lib.vq_gemv_workspace_size(C.byref(d), 1, C.byref(n)) == vq.VQ_ERR_INVALID_ARG
+
+
+def test_output_bias_field_is_checked_on_the_host(lib):
+    """The output bias pointer (ABI version 4) is optional, and an fp16 array
+    that is not 2-byte aligned is refused before anything runs."""
+    n = C.c_size_t(0)
+    d = _tiled_desc()
+    assert C.sizeof(vq._Desc) - vq._Desc.out_bias.offset == 8      # the last field
+    d.out_bias = 0x30000
+    assert lib.vq_gemv_workspace_size(C.byref(d), 1, C.byref(n)) == vq.VQ_OK
+    d.out_bias = 0x30001
+    assert lib.vq_gemv_workspace_size(C.byref(d), 1, C.byref(n)) == vq.VQ_ERR_ALIGNMENT
+    assert lib.vq_gemm_workspace_size(C.byref(d), 64, vq.VQ_BF16, C.byref(n)) == vq.VQ_ERR_ALIGNMENT
 
 
 def test_tiled_workspace_sizes(lib):
@@ -207,3 +220,13 @@ def test_new_entry_points_validate_before_any_device_call(lib):
     d.out_features, d.in_features, d.vec_dim, d.n_books = 4, 16, 0, 1   # d = 0
     assert lib.vq_gemv_rht(C.byref(d), None, None, None, vq.VQ_BF16, 1, 16, None, vq.VQ_BF16, 4, None, 0,
                            None) == vq.VQ_ERR_INVALID_ARG
+
+
+def test_noalloc_scratch_size_matches_the_header():
+    """The binding's NOALLOC_SCRATCH_BYTES is the header's
+    VQ_NOALLOC_SCRATCH_BYTES (the tests size their layers against it)."""
+    import re
+    with open(vq.HEADER) as fh:
+        m = re.search(r"#define\s+VQ_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", fh.read())
+    assert m, "macro not found"
+    assert vq.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))

@@ -1,16 +1,17 @@
 """vq_gemv_noalloc: the decode GEMV for callers that cannot allocate device
 memory where they run the layer (it takes its split-K scratch from a fixed
 array inside the library).  Its output must match vq_gemv's, which gets a
-caller-allocated workspace, on two calls in a row (the second call finds the
-first call's leftovers in the shared array).  This file is collected last so
+caller-allocated workspace, and the fp64 oracle, on two calls in a row (the
+second call finds the first call's leftovers in the shared array).  This file is collected last so
 that a run stopping at the first failure has already run every other test."""
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 from synth import LayerSpec
-from tests._util import TOL, normwise_err
+from tests._util import TOL, assert_close, normwise_err
 
 pytestmark = pytest.mark.gpu
 
@@ -30,7 +31,9 @@ def test_noalloc_matches_workspace_version_twice(spec, batch):
     layer = vq.Layer.from_synth(data)
     need = vq.gemv_workspace_size(layer, batch)
     assert 0 < need <= vq.NOALLOC_SCRATCH_BYTES        # the scratch is really used
-    x = _x_dev(synth.make_x(4243, batch, spec.in_features))
+    xb = synth.make_x(4243, batch, spec.in_features)
+    x = _x_dev(xb)
+    exact = oracle.linear(data, xb)                      # the fp64 definition
     ref = vq.gemv(layer, x, out_dtype=torch.float32).double().cpu().numpy()
     for _ in range(2):
         out = torch.full((batch, spec.out_features), float("nan"), device="cuda")
@@ -38,6 +41,7 @@ def test_noalloc_matches_workspace_version_twice(spec, batch):
         got = out.double().cpu().numpy()
         assert np.isfinite(got).all()
         assert normwise_err(got, ref) <= TOL
+        assert_close(got, exact, "float32")
 
 
 def test_noalloc_rejects_layers_beyond_the_scratch():
