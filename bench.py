@@ -76,6 +76,10 @@ LAYOUTS = ("tile4", "tile4", "tile4")
 ENCODE_SHAPE = (4096, 4096, 8, [16])
 ENCODE_STD = [0.02]
 ENCODE_SEED = 11
+# The Hessian-weighted encoder's H: 2 X^T X / n + 0.01 mean(diag) I of 1024
+# synthetic bf16 tokens ~ N(0, 1) with 0.1 % outlier channels x20 (vq_hessian).
+ENCODE_H_TOKENS = 1024
+ENCODE_H_SEED = 14
 RHT_SEED = 12           # sign bits of the rotated-basis measurement
 HESSIAN_SHAPE = (8192, 8192)   # tokens, features
 HESSIAN_SEED = 13
@@ -436,6 +440,8 @@ def run_gpu(args):
     hess = run_hessian(dev, peaks, peak_src, vq)
     encode = run_encode(dev, peaks, peak_src, vq,
                         with_oracle=rank == 0 and world == 1 and not args.no_cpu_baseline)
+    encode_h = run_encode(dev, peaks, peak_src, vq,
+                          with_oracle=rank == 0 and world == 1 and not args.no_cpu_baseline, hessian=True)
 
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -456,6 +462,7 @@ def run_gpu(args):
         "rht_gate": rht,
         "hessian": hess,
         "encode": encode,
+        "encode_h": encode_h,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gbs, rows, dt, cores = oracle_rate(10.0, w.layers, xs_host)
@@ -671,26 +678,31 @@ def run_405b_qkv(dev, peaks, peak_src, vq):
             "algorithmic_bytes": nbytes, "peak_source": peak_src}
 
 
-def run_encode(dev, peaks, peak_src, vq, with_oracle: bool):
+def run_encode(dev, peaks, peak_src, vq, with_oracle: bool, hessian: bool = False):
     """Beside the headline: the nearest-centroid encoder (vq_encode) on a
     4096 x 4096 fp16 matrix against one K = 2^16, d = 8 book (2M vectors x
     65536 centroids), L2 flushed between timed calls; the oracle's brute force
-    on a sample of the same vectors for scale."""
+    on a sample of the same vectors for scale.  With ``hessian`` the
+    Hessian-weighted distance, H from vq_hessian of synthetic activations."""
     import torch
     n, kin, d, log2k = ENCODE_SHAPE
     w, books = synth.make_encode_input(n, kin, d, log2k, ENCODE_STD, seed=ENCODE_SEED)
     W = torch.from_numpy(w.view(np.int16)).to(dev).view(torch.float16)
     B = [torch.from_numpy(b.view(np.int16)).to(dev).view(torch.float16) for b in books]
-    ws = torch.empty(vq.encode_workspace_size(n, kin, log2k, d), dtype=torch.uint8, device=dev)
+    H = None
+    if hessian:
+        xt = synth.make_x(ENCODE_H_SEED, ENCODE_H_TOKENS, kin, 0.001)
+        H = vq.hessian(torch.from_numpy(xt.view(np.int16)).to(dev).view(torch.bfloat16))
+    ws = torch.empty(vq.encode_workspace_size(n, kin, log2k, d, hessian=hessian), dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     for _ in range(3):
-        vq.encode(W, B, log2k, d, workspace=ws)
+        vq.encode(W, B, log2k, d, workspace=ws, hessian=H)
     times = []
     for _ in range(5):
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        vq.encode(W, B, log2k, d, workspace=ws)
+        vq.encode(W, B, log2k, d, workspace=ws, hessian=H)
         b.record()
         b.synchronize()
         times.append(a.elapsed_time(b))
@@ -702,7 +714,9 @@ def run_encode(dev, peaks, peak_src, vq, with_oracle: bool):
     # ALU roofline: one minimum operation per (vector, centroid) pair at full
     # issue on every SM sub-partition (148 SMs x 4 x 32 lanes x max SM clock).
     alu_peak = 148 * 4 * 32 * 1.965e9
-    out = {"workload": f"encode {n}x{kin} fp16 W ~ N(0, {ENCODE_STD[0]}), d={d}, one K=2^{log2k[0]} book: "
+    what = ("Hessian-weighted (v-c)^T H_v (v-c), H of 1024 synthetic tokens with 0.1% outlier channels, "
+            if hessian else "")
+    out = {"workload": f"encode {what}{n}x{kin} fp16 W ~ N(0, {ENCODE_STD[0]}), d={d}, one K=2^{log2k[0]} book: "
                        f"{nv} vectors x {1 << log2k[0]} centroids",
            "ms": ms, "pairs_per_s": rate, "device_status": int(ctrl[0]),
            "exact_pass_vectors": int(ctrl[1]), "exact_pass_share": int(ctrl[1]) / nv,
@@ -710,16 +724,24 @@ def run_encode(dev, peaks, peak_src, vq, with_oracle: bool):
                         "frac": rate / alu_peak,
                         "peak_source": "derived: one ALU operation per pair at full issue, "
                                        "148 SMs x 128 lanes x 1965 MHz"},
-           "tensor_tflops": 2.0 * d * pairs / (ms * 1e-3) / 1e12}
+           "tensor_tflops": 2.0 * (2 * d if hessian else d) * pairs / (ms * 1e-3) / 1e12}
+    if hessian:
+        out["roofline"]["note"] = ("the weighted epilogue spends two operations per pair (an fma adding "
+                                   "c^T H_j c, then the minimum), so 0.5 of this peak is its ceiling")
     if not with_oracle:
         return out
     # CPU baseline: the oracle on a bounded sample of the same vectors (host cores)
     import oracle
     import time as _time
-    sample = 256
+    sample = 256 if not hessian else 64
     v = oracle.f16_to_f32(w[:sample * d // kin + 1]).astype(np.float64).reshape(-1, d)[:sample]
     t0 = _time.perf_counter()
-    oracle.encode(v, books[0])
+    if hessian:
+        hb = oracle.hessian_blocks(H.double().cpu().numpy(), kin, d, sample * d // kin + 1)[0][:sample]
+        t0 = _time.perf_counter()
+        oracle.encode_h(v, hb, books[0])
+    else:
+        oracle.encode(v, books[0])
     dt = _time.perf_counter() - t0
     out["cpu_baseline"] = {"value": sample * (1 << log2k[0]) / dt, "unit": "pairs/s",
                            "cores": oracle.num_threads(), "kind": "oracle",

@@ -31,6 +31,16 @@
 //    other vector -- near-ties, partial last vectors, values fp16 cannot hold
 //    -- is decided by an fp64 pass over the whole book that repeats the
 //    definition operation by operation, so the output equals the definition.
+//  * Hessian-weighted form ("VPTQ Guide", section "1. Second-Order
+//    Hessian-Weighted Optimization": D_H(v, c) = (v - c)^T H_v (v - c), H_v
+//    the sub-matrix of H on the vector's channels).  D_H = v^T H v + (c^T H_v
+//    c - 2 c^T H_s v) with H_s = (H_v + H_v^T) / 2, and again only the bracket
+//    depends on c.  A block holds 128 rows of one block of channels j, so all
+//    its vectors share H_j: the A row is z = H_s v (scaled, split into fp16 hi
+//    and lo halves), the B row [-2 c~, -2 c~] (the same for every j), and the
+//    epilogue adds nc[j][k] = c~^T H_j c~ (a table of fp32 values per block
+//    of channels, made once per call) with one fma per value.  The exact
+//    paths evaluate (v - c)^T H_v (v - c) as the definition does.
 //  * Every mbarrier wait is bounded; a wait that runs out of budget raises
 //    the block's abort flag, records VQ_ERR_TIMEOUT in the workspace's status
 //    word and lets every warp fall through to the teardown.
@@ -56,6 +66,7 @@ constexpr int kEncATile = kEncM * 128;              // 16 KB: rows of 128 B, fir
 constexpr long long kEncWaitBudget = 4000000000LL;  // SM clocks (about 2 s)
 constexpr float kEncPadNorm = 30000.0f;             // hi = lo of padding centroids
 constexpr int kEncMaxD = 14;                        // d + 2 <= 16
+constexpr int kEncHMaxD = 8;                        // Hessian-weighted form: 2 d <= 16
 constexpr int kEncExactThreads = 256;
 
 struct EncCtrl {
@@ -71,7 +82,12 @@ struct EncCtrl {
   float second[4][kEncM];        //   smallest chunk minimum of the other chunks,
   int chunk[4][kEncM];           //   first centroid of the chunk holding the smallest
   double v[kEncM][kEncMaxD];     // the vectors, exactly (fp64)
-  double vnorm[kEncM];           // ||v||^2 (fp64)
+  double vnorm[kEncM];           // ||v||^2 (fp64); v^T H v in the weighted form
+  // Hessian-weighted form only:
+  float zsc[kEncM];              // 2^u: the vector's scale of z = H_s v~
+  double slack[kEncM];           // size of the fp64 rounding in its exact distances
+  double hj[kEncHMaxD][kEncHMaxD];   // H on this block's channels (fp64)
+  float ncw[kEncEpiWarps][64];   // each epilogue warp's nc values of the current tile
 };
 
 // Workspace control words (first 256 bytes).
@@ -132,16 +148,26 @@ __global__ void enc_book_norm_kernel(const uint16_t* __restrict__ book, int K, i
 // Prepared book: centroid k = 1024 q + 256 sl + r sits in block q (32 KB),
 // row r, 16-half column slot sl, 128-byte swizzled; halves [-2 c~ (d), hi,
 // lo, 0...], c~ = fp16(c * 2^s), hi + lo = ||c~||^2.  Centroids k >= K (the
-// padding up to a whole block) get hi = lo = kEncPadNorm and zero c~.
+// padding up to a whole block) get hi = lo = kEncPadNorm and zero c~.  The
+// Hessian-weighted form (hw) stores [-2 c~ (d), -2 c~ (d), 0...] instead (the
+// two copies multiply the two fp16 halves of z) and zero for the padding,
+// whose c^T H c term is infinite.
 __global__ void enc_book_prep_kernel(const uint16_t* __restrict__ book, int K, int d, int kp,
-                                     const unsigned* __restrict__ cmax_bits, uint8_t* __restrict__ bprep) {
+                                     const unsigned* __restrict__ cmax_bits, uint8_t* __restrict__ bprep,
+                                     int hw) {
   const int k = blockIdx.x * blockDim.x + threadIdx.x;
   if (k >= kp) return;
   const float f = enc_pow2(enc_scale_exp(__uint_as_float(*cmax_bits)));
   uint16_t h[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) h[i] = 0;
-  if (k < K) {
+  if (hw) {
+    if (k < K)
+      for (int e = 0; e < d; ++e) {
+        const float c = h2f(f2h(h2f(book[static_cast<int64_t>(k) * d + e]) * f));
+        h[e] = h[d + e] = f2h(-2.0f * c);
+      }
+  } else if (k < K) {
     float nrm = 0.0f;
     for (int e = 0; e < d; ++e) {
       const float c = h2f(f2h(h2f(book[static_cast<int64_t>(k) * d + e]) * f));
@@ -170,6 +196,61 @@ __global__ void enc_book_prep_kernel(const uint16_t* __restrict__ book, int K, i
   *reinterpret_cast<uint4*>(base + enc_sw128(r, 2 * sl + 1)) = c1;
 }
 
+// Hessian-weighted form: nc[j][k] = c~_k^T H_j c~_k in fp32 for every block j
+// of d channels (j < nfull) and centroid k < kp, with c~ = fp16(c 2^s) as in
+// the prepared book and H_j the d x d block of h on channels j d .. j d + d - 1;
+// +infinity for the padding k >= K.  Also ncabs[j] = max_k |c~_k|^T |H_j|
+// |c~_k| (as fp32 bits; zero on entry), the scale of nc's rounding error.
+// Grid (kp / 256, nfull).
+__global__ void enc_nc_kernel(const uint16_t* __restrict__ book, int K, int d, int kp,
+                              const unsigned* __restrict__ cmax_bits, const float* __restrict__ h,
+                              int64_t ldh, float* __restrict__ nc, unsigned* __restrict__ ncabs) {
+  __shared__ float hs[kEncHMaxD * kEncHMaxD];
+  __shared__ float red[8];
+  const int j = blockIdx.y;
+  if (threadIdx.x < d * d) {
+    const int e = threadIdx.x / d, g = threadIdx.x % d;
+    hs[threadIdx.x] = h[static_cast<int64_t>(j * d + e) * ldh + j * d + g];
+  }
+  __syncthreads();
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;   // kp is a multiple of 256: always < kp
+  float v = INFINITY, va = 0.0f;
+  if (k < K) {
+    const float f = enc_pow2(enc_scale_exp(__uint_as_float(*cmax_bits)));
+    float c[kEncHMaxD];
+#pragma unroll
+    for (int e = 0; e < kEncHMaxD; ++e)
+      c[e] = e < d ? h2f(f2h(h2f(book[static_cast<int64_t>(k) * d + e]) * f)) : 0.0f;
+    v = 0.0f;
+#pragma unroll
+    for (int e = 0; e < kEncHMaxD; ++e) {
+      if (e < d) {
+        float g = 0.0f, ga = 0.0f;
+#pragma unroll
+        for (int q = 0; q < kEncHMaxD; ++q)
+          if (q < d) {
+            g = fmaf(hs[e * d + q], c[q], g);
+            ga = fmaf(fabsf(hs[e * d + q]), fabsf(c[q]), ga);
+          }
+        v = fmaf(c[e], g, v);
+        va = fmaf(fabsf(c[e]), ga, va);
+      }
+    }
+  }
+  nc[static_cast<int64_t>(j) * kp + k] = v;
+  // the block's largest |c|^T |H| |c| (non-negative, so the bits order as the values)
+  va *= 1.0f + 0x1p-20f;                               // covers the rounding of va itself
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) va = fmaxf(va, __shfl_xor_sync(0xffffffffu, va, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = va;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.0f;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+    atomicMax(ncabs + j, __float_as_uint(m));
+  }
+}
+
 // The book in fp64 (exact), for the exact distances.
 __global__ void enc_book64_kernel(const uint16_t* __restrict__ book, int64_t count, double* __restrict__ out) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -194,6 +275,13 @@ struct EncArgs {
   int* list;                     // vector ids o * nvec + j left to the exact pass
   int* list_count;
   int* status;
+  // Hessian-weighted form: a block's 128 vectors are rows o0 .. o0+127 of one
+  // block of channels j (mt blocks per j), nc = c~^T H_j c~ [nfull][kp].
+  const float* h;
+  int64_t ldh;
+  const float* nc;
+  const unsigned* ncabs;         // max_k |c~_k|^T |H_j| |c~_k| per block j (fp32 bits)
+  int mt;
 };
 
 // sum_e (v_e - c_e)^2 with each difference, square and sum rounded once in
@@ -203,6 +291,28 @@ __device__ __forceinline__ double enc_dist64(const double* v, const double* c, i
   for (int e = 0; e < d; ++e) {
     const double t = __dsub_rn(v[e], c[e]);
     dist = __dadd_rn(dist, __dmul_rn(t, t));
+  }
+  return dist;
+}
+
+// (v - c)^T H (v - c) with t_e = v_e - c_e, g_e = sum_f H[e][f] t_f (f
+// ascending), the sum over e ascending, every operation rounded once in
+// fp64: the weighted distance of the definition.
+__device__ __forceinline__ double enc_dist64h(const double* v, const double* c,
+                                              const double (*hj)[kEncHMaxD], int d) {
+  double t[kEncHMaxD];
+#pragma unroll
+  for (int e = 0; e < kEncHMaxD; ++e) t[e] = e < d ? __dsub_rn(v[e], c[e]) : 0.0;
+  double dist = 0.0;
+#pragma unroll
+  for (int e = 0; e < kEncHMaxD; ++e) {
+    if (e < d) {
+      double g = 0.0;
+#pragma unroll
+      for (int f = 0; f < kEncHMaxD; ++f)
+        if (f < d) g = __dadd_rn(g, __dmul_rn(hj[e][f], t[f]));
+      dist = __dadd_rn(dist, __dmul_rn(t[e], g));
+    }
   }
   return dist;
 }
@@ -233,6 +343,9 @@ __device__ __forceinline__ void enc_chunk(const uint32_t (&r)[32], int k0, float
   chunk = p ? k0 : chunk;
 }
 
+// HW: the Hessian-weighted form (see EncArgs).  The plain form's blocks take
+// 128 consecutive vectors in (row, vector) order.
+template <bool HW>
 __global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
   extern __shared__ __align__(1024) uint8_t enc_smem[];
   EncCtrl* ctrl = reinterpret_cast<EncCtrl*>(enc_smem);
@@ -240,7 +353,9 @@ __global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
   uint8_t* stages = atile + kEncATile;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &ctrl->abort_flag;
-  const int64_t v0 = static_cast<int64_t>(blockIdx.x) * kEncM;
+  const int64_t v0 = HW ? 0 : static_cast<int64_t>(blockIdx.x) * kEncM;
+  const int hblk = HW ? static_cast<int>(blockIdx.x / a.mt) : 0;          // block of channels
+  const int obase = HW ? static_cast<int>(blockIdx.x % a.mt) * kEncM : 0;  // its first row
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kEncStages; ++s) {
@@ -258,6 +373,15 @@ __global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
     tmem_alloc(&ctrl->tmem_base, 512);
     tmem_relinquish();
   }
+  if (HW) {                                            // H on this block's channels, in fp64
+    if (threadIdx.x < kEncHMaxD * kEncHMaxD) {
+      const int e = threadIdx.x / kEncHMaxD, g = threadIdx.x % kEncHMaxD;
+      ctrl->hj[e][g] = (e < a.d && g < a.d)
+                           ? static_cast<double>(a.h[static_cast<int64_t>(hblk * a.d + e) * a.ldh + hblk * a.d + g])
+                           : 0.0;
+    }
+    __syncthreads();
+  }
 
   // A operand: row t = [v~ (d halves), 1, 1, 0...] of vector v0 + t, and the
   // vector's error bound.  With s the book's exponent and v~ = fp16(v 2^s),
@@ -267,9 +391,18 @@ __global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
   //      + 2^-22 ||v~||_1 (1 + sqrt C)     fp16 rounding of tiny c~ components
   //      + 2 delta (sqrt C + 1)            v~ against v 2^s (delta: its L1 error)
   // with C = max_k ||c~_k||^2 < 2^10; the terms are loose by design.
+  //
+  // Weighted form: row t = [z~ hi (d halves), z~ lo (d halves), 0...] with
+  // z = H_s v 2^s (fp32), z~ = z 2^u (u puts max |z~| in [2^13, 2^14)) split
+  // into two fp16 halves; the MMA returns -2<z~, c~> and the epilogue adds
+  // nc_k 2^u, so D(k) approximates (c~^T H c~ - 2 c~^T H_s v~) 2^u =
+  // (D_H(v, c) - v^T H v) 4^s 2^u.  The bound (eps) sums, each with a factor
+  // of four to spare: fp32 rounding of nc (d + 2 roundings of terms up to
+  // Hmax d C), of z (d + 2 roundings of |H_s| |v~|), of the MMA's sums and
+  // the epilogue's fma, the fp16 hi/lo split of z~ (2^-22 relative, 2^-25
+  // absolute) and the fp16 rounding of tiny c~ components (2^-25 absolute).
   if (threadIdx.x < kEncM) {
     const int t = threadIdx.x;
-    const int64_t gv = v0 + t;
     const float cmax = __uint_as_float(*a.cmax_bits);
     const int se = enc_scale_exp(cmax);
     const float f = enc_pow2(se);
@@ -278,37 +411,141 @@ __global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
     for (int i = 0; i < 16; ++i) h[i] = 0;
     float eps = 0.0f;
     int flag = 2;
-    if (gv < a.nv_full) {
-      flag = 0;
-      const int o = static_cast<int>(gv / a.nfull), j = static_cast<int>(gv % a.nfull);
-      const uint16_t* wr = a.w + static_cast<int64_t>(o) * a.ldw + static_cast<int64_t>(j) * a.d;
-      const uint16_t* c1 = a.book1 ? a.book1 + static_cast<int64_t>(a.idx1[static_cast<int64_t>(o) * a.nvec + j]) * a.d
-                                   : nullptr;
-      float n2 = 0.0f, l1 = 0.0f, dl = 0.0f;
-      double vn = 0.0;
-      for (int e = 0; e < a.d; ++e) {
-        double ve = static_cast<double>(h2f(wr[e]));
-        if (c1) ve = __dsub_rn(ve, static_cast<double>(h2f(c1[e])));
-        ctrl->v[t][e] = ve;
-        vn = __dadd_rn(vn, __dmul_rn(ve, ve));
-        float v = h2f(wr[e]);
-        if (c1) v = __fsub_rn(v, h2f(c1[e]));
-        const float vs = v * f;                      // exact: a power-of-two scale in range
-        const uint16_t hv = f2h(vs);
-        const float vt = h2f(hv);
-        if (!(fabsf(vt) <= 65504.0f)) flag = 1;      // overflow or NaN: exact pass
-        h[e] = hv;
-        n2 = fmaf(vt, vt, n2);
-        l1 += fabsf(vt);
-        dl += fabsf(vt - vs) + fabsf(vs) * 0x1p-22f + 0x1p-24f;
+    if (HW) {
+      const int o = obase + t, j = hblk;
+      if (o < a.n) {
+        flag = 0;
+        const uint16_t* wr = a.w + static_cast<int64_t>(o) * a.ldw + static_cast<int64_t>(j) * a.d;
+        const uint16_t* c1 = a.book1 ? a.book1 + static_cast<int64_t>(a.idx1[static_cast<int64_t>(o) * a.nvec + j]) * a.d
+                                     : nullptr;
+        double vd[kEncHMaxD];
+        float vs[kEncHMaxD];
+#pragma unroll
+        for (int e = 0; e < kEncHMaxD; ++e) {
+          vd[e] = 0.0;
+          vs[e] = 0.0f;
+          if (e < a.d) {
+            double ve = static_cast<double>(h2f(wr[e]));
+            if (c1) ve = __dsub_rn(ve, static_cast<double>(h2f(c1[e])));
+            vd[e] = ve;
+            ctrl->v[t][e] = ve;
+            float v = h2f(wr[e]);
+            if (c1) v = __fsub_rn(v, h2f(c1[e]));
+            vs[e] = v * f;                             // a power-of-two scale
+          }
+        }
+        // v^T H v in fp64 (the definition's order), |v|^T |H| |v|, ||v||^2, max |H|
+        double vhv = 0.0, vha = 0.0, vn = 0.0;
+        float hmax = 0.0f;
+#pragma unroll
+        for (int e = 0; e < kEncHMaxD; ++e) {
+          if (e < a.d) {
+            double g = 0.0, ga = 0.0;
+#pragma unroll
+            for (int q = 0; q < kEncHMaxD; ++q) {
+              if (q < a.d) {
+                const double hv = ctrl->hj[e][q];
+                g = __dadd_rn(g, __dmul_rn(hv, vd[q]));
+                ga += fabs(hv) * fabs(vd[q]);
+                hmax = fmaxf(hmax, fabsf(static_cast<float>(hv)));
+              }
+            }
+            vhv = __dadd_rn(vhv, __dmul_rn(vd[e], g));
+            vha += fabs(vd[e]) * ga;
+            vn += vd[e] * vd[e];
+          }
+        }
+        // z = H_s v~ in fp32, and the 2-norm of the terms' magnitudes (|H_s| |v~|)
+        float z[kEncHMaxD], hv2 = 0.0f, zmax = 0.0f;
+#pragma unroll
+        for (int e = 0; e < kEncHMaxD; ++e) {
+          z[e] = 0.0f;
+          if (e < a.d) {
+            float ha = 0.0f;
+#pragma unroll
+            for (int q = 0; q < kEncHMaxD; ++q) {
+              if (q < a.d) {
+                const float hs = 0.5f * (static_cast<float>(ctrl->hj[e][q]) + static_cast<float>(ctrl->hj[q][e]));
+                z[e] = fmaf(hs, vs[q], z[e]);
+                ha += fabsf(hs) * fabsf(vs[q]);
+              }
+            }
+            hv2 += ha * ha;
+            zmax = fmaxf(zmax, fabsf(z[e]));
+          }
+        }
+        hv2 = sqrtf(hv2) * 1.001f;
+        float zs = 1.0f;
+        if (zmax > 0.0f && zmax < INFINITY) {
+          const int ez = static_cast<int>((__float_as_uint(zmax) >> 23) & 0xffu) - 127;
+          zs = enc_pow2(max(-126, min(127, 13 - ez)));
+        }
+        float z2 = 0.0f, zmx = 0.0f;
+#pragma unroll
+        for (int e = 0; e < kEncHMaxD; ++e) {
+          if (e < a.d) {
+            const float zt = z[e] * zs;
+            const uint16_t hi = f2h(zt);
+            const uint16_t lo = f2h(zt - h2f(hi));
+            h[e] = hi;
+            h[a.d + e] = lo;
+            z2 += zt * zt;
+            zmx = fmaxf(zmx, fabsf(zt));
+          }
+        }
+        z2 = sqrtf(z2) * 1.001f;
+        const float dd = static_cast<float>(a.d);
+        const float cs = cmax * f * f;
+        const float rc = sqrtf(cs) * 1.001f;           // >= |c~_k| for every k
+        const float na = __uint_as_float(a.ncabs[j]) * zs;   // >= |c~|^T |H_j| |c~| 2^u
+        const float hm = hmax * zs, hv = hv2 * zs;
+        // nc's fp32 sums (2 d roundings), the epilogue's fma, the MMA's fp32
+        // sums of 2 d products (|sum| <= 2 rc ||z~||), z's own rounding and
+        // fp16 split, and the fp16 rounding of tiny c~ components
+        eps = 2.0f * ((2.0f * dd + 2.0f) * 0x1p-24f * na + 0x1p-24f * (na + 2.0f * rc * z2) +
+                      (2.0f * dd + 1.0f) * 0x1p-24f * 2.0f * rc * z2 +
+                      2.0f * rc * ((dd + 2.0f) * 0x1p-24f * hv + 0x1p-22f * z2 + 3.0f * 0x1p-25f) +
+                      0x1p-23f * dd * (hm * dd * rc + zmx));
+        if (!(eps < INFINITY) || !(fabs(vhv) < INFINITY) || !(zmx < 16384.0f)) flag = 1;
+        ctrl->vnorm[t] = vhv;
+        ctrl->zsc[t] = zs;
+        // fp64 rounding of the exact distances and of v^T H v, before scaling
+        ctrl->slack[t] = 0x1p-36 * (vha + 2.0 * static_cast<double>(hmax) * a.d * (vn + static_cast<double>(cmax)));
       }
-      ctrl->vnorm[t] = vn;
-      h[a.d] = 0x3C00u;                              // 1.0 (times hi)
-      h[a.d + 1] = 0x3C00u;                          // 1.0 (times lo)
-      const float cs = cmax * f * f;
-      const float rc = sqrtf(cs);
-      eps = 0x1p-18f * (n2 + 2.0f * cs + 1.0f) + 0x1p-22f * l1 * (1.0f + rc) + 2.0f * dl * (rc + 1.0f);
-      if (!(eps < INFINITY)) flag = 1;
+    } else {
+      const int64_t gv = v0 + t;
+      if (gv < a.nv_full) {
+        flag = 0;
+        const int o = static_cast<int>(gv / a.nfull), j = static_cast<int>(gv % a.nfull);
+        const uint16_t* wr = a.w + static_cast<int64_t>(o) * a.ldw + static_cast<int64_t>(j) * a.d;
+        const uint16_t* c1 = a.book1 ? a.book1 + static_cast<int64_t>(a.idx1[static_cast<int64_t>(o) * a.nvec + j]) * a.d
+                                     : nullptr;
+        float n2 = 0.0f, l1 = 0.0f, dl = 0.0f;
+        double vn = 0.0;
+        for (int e = 0; e < a.d; ++e) {
+          double ve = static_cast<double>(h2f(wr[e]));
+          if (c1) ve = __dsub_rn(ve, static_cast<double>(h2f(c1[e])));
+          ctrl->v[t][e] = ve;
+          vn = __dadd_rn(vn, __dmul_rn(ve, ve));
+          float v = h2f(wr[e]);
+          if (c1) v = __fsub_rn(v, h2f(c1[e]));
+          const float vs = v * f;                      // exact: a power-of-two scale in range
+          const uint16_t hv = f2h(vs);
+          const float vt = h2f(hv);
+          if (!(fabsf(vt) <= 65504.0f)) flag = 1;      // overflow or NaN: exact pass
+          h[e] = hv;
+          n2 = fmaf(vt, vt, n2);
+          l1 += fabsf(vt);
+          dl += fabsf(vt - vs) + fabsf(vs) * 0x1p-22f + 0x1p-24f;
+        }
+        ctrl->vnorm[t] = vn;
+        h[a.d] = 0x3C00u;                              // 1.0 (times hi)
+        h[a.d + 1] = 0x3C00u;                          // 1.0 (times lo)
+        const float cs = cmax * f * f;
+        const float rc = sqrtf(cs);
+        eps = 0x1p-18f * (n2 + 2.0f * cs + 1.0f) + 0x1p-22f * l1 * (1.0f + rc) + 2.0f * dl * (rc + 1.0f);
+        if (!(eps < INFINITY)) flag = 1;
+      }
     }
     ctrl->eps[t] = eps;
     ctrl->flag[t] = flag;
@@ -371,6 +608,15 @@ __global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
     const int row = lq * 32 + lane;
     float best = INFINITY, second = INFINITY;
     int chunk = 0;
+    // Weighted form: this warp's 64 values of nc for the next tile, fetched a
+    // tile ahead (two per lane) and passed through its own shared-memory row.
+    const float* ncr = HW ? a.nc + static_cast<int64_t>(hblk) * a.kp : nullptr;
+    float p0 = 0.0f, p1 = 0.0f, zs = 1.0f;
+    if (HW) {
+      p0 = ncr[cq * 64 + lane];
+      p1 = ncr[cq * 64 + 32 + lane];
+      zs = ctrl->zsc[row];
+    }
     for (int t = 0; t < ntiles; ++t) {
       const int ab = t & 1;
       if (!bounded_wait(&ctrl->acc_full[ab], (t >> 1) & 1, abort_flag, a.status, kEncWaitBudget)) break;
@@ -384,6 +630,23 @@ __global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctrl->acc_empty[ab]);
       const int k0 = (t >> 2) * kEncBlockK + (t & 3) * kEncN + cq * 64;
+      if (HW) {
+        float* ns = ctrl->ncw[warp - 4];
+        ns[lane] = p0;
+        ns[32 + lane] = p1;
+        __syncwarp();
+        if (t + 1 < ntiles) {
+          const int k1 = ((t + 1) >> 2) * kEncBlockK + ((t + 1) & 3) * kEncN + cq * 64;
+          p0 = ncr[k1 + lane];
+          p1 = ncr[k1 + 32 + lane];
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          r0[i] = __float_as_uint(fmaf(ns[i], zs, __uint_as_float(r0[i])));
+          r1[i] = __float_as_uint(fmaf(ns[32 + i], zs, __uint_as_float(r1[i])));
+        }
+        __syncwarp();
+      }
       enc_chunk(r0, k0, best, second, chunk);
       enc_chunk(r1, k0 + 32, best, second, chunk);
     }
@@ -425,7 +688,9 @@ __global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
       double e = INFINITY;
       if (ctrl->flag[t] == 0) {
         const int k = ctrl->chunk[0][t] + c;
-        if (k < a.K) e = enc_dist64(ctrl->v[t], a.book64 + static_cast<int64_t>(k) * a.d, a.d);
+        if (k < a.K)
+          e = HW ? enc_dist64h(ctrl->v[t], a.book64 + static_cast<int64_t>(k) * a.d, ctrl->hj, a.d)
+                 : enc_dist64(ctrl->v[t], a.book64 + static_cast<int64_t>(k) * a.d, a.d);
       }
       ex[p] = e;
     }
@@ -435,12 +700,20 @@ __global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
   // chunk's exact minimum, that minimum (lowest k on ties) is the answer.
   //   outside:  D(k) >= second  =>  exact bracket >= second - eps
   //   inside:   exact bracket of the best = (dist - ||v||^2) 4^s
+  //             (weighted: (dist - v^T H v) 4^s 2^u)
   if (threadIdx.x < kEncM && live) {
     const int t = threadIdx.x;
     const int flag = ctrl->flag[t];
     if (flag != 2) {
-      const int64_t gv = v0 + t;
-      const int o = static_cast<int>(gv / a.nfull), j = static_cast<int>(gv % a.nfull);
+      int o, j;
+      if (HW) {
+        o = obase + t;
+        j = hblk;
+      } else {
+        const int64_t gv = v0 + t;
+        o = static_cast<int>(gv / a.nfull);
+        j = static_cast<int>(gv % a.nfull);
+      }
       const int64_t vid = static_cast<int64_t>(o) * a.nvec + j;
       bool done = false;
       if (flag == 0) {
@@ -455,9 +728,11 @@ __global__ void __launch_bounds__(kEncThreads, 1) enc_tc_kernel(EncArgs a) {
         }
         if (kmin >= 0) {
           const int se2 = 2 * enc_scale_exp(__uint_as_float(*a.cmax_bits));   // 4^s as a double
-          const double s4 = __longlong_as_double(static_cast<long long>(1023 + se2) << 52);
-          const double dex = (emin - ctrl->vnorm[t]) * s4;
-          const double slack = 0x1p-40 * (fabs(emin) + ctrl->vnorm[t]) * s4;
+          double sc = __longlong_as_double(static_cast<long long>(1023 + se2) << 52);
+          if (HW) sc *= static_cast<double>(ctrl->zsc[t]);
+          const double dex = (emin - ctrl->vnorm[t]) * sc;
+          double slack = 0x1p-40 * (fabs(emin) + fabs(ctrl->vnorm[t])) * sc;
+          if (HW) slack += ctrl->slack[t] * sc;
           if (static_cast<double>(ctrl->second[0][t]) - dex > static_cast<double>(ctrl->eps[t]) + slack) {
             a.idx_out[vid] = static_cast<uint32_t>(kmin);
             done = true;
@@ -491,6 +766,8 @@ struct EncExactArgs {
   const int* list;
   const int* list_count;
   int partial_rows;              // n when the last vector of every row is partial, else 0
+  const float* h;                // weighted form: the Hessian (else null)
+  int64_t ldh;
 };
 
 // Work items: the listed vectors, then the partial last vector of every row.
@@ -503,6 +780,9 @@ struct EncExactArgs {
 // vector with no finite distance gets index 0.
 constexpr int kEncExactTile = 512;
 
+// The weighted form (HW) takes (v - c)^T H_v (v - c) instead, H_v read once
+// per vector into registers (fp64), in the order of enc_dist64h.
+template <bool HW>
 __global__ void __launch_bounds__(kEncExactThreads) enc_exact_kernel(EncExactArgs a) {
   constexpr int NW = kEncExactThreads / 32;
   extern __shared__ double tile[];                 // [d][kEncExactTile]
@@ -536,6 +816,16 @@ __global__ void __launch_bounds__(kEncExactThreads) enc_exact_kernel(EncExactArg
           v[e] = __dsub_rn(v[e], static_cast<double>(h2f(a.book1[static_cast<int64_t>(a.idx1[vid]) * a.d + e])));
       }
     }
+    double hr[HW ? kEncHMaxD : 1][HW ? kEncHMaxD : 1];
+    if (HW) {
+#pragma unroll
+      for (int e = 0; e < (HW ? kEncHMaxD : 1); ++e)
+#pragma unroll
+        for (int g = 0; g < (HW ? kEncHMaxD : 1); ++g)
+          hr[e][g] = (e < dv && g < dv)
+                         ? static_cast<double>(a.h[static_cast<int64_t>(j * a.d + e) * a.ldh + j * a.d + g])
+                         : 0.0;
+    }
     double best = INFINITY;
     int arg = INT_MAX;
     for (int k0 = 0; k0 < a.K; k0 += kEncExactTile) {
@@ -547,11 +837,27 @@ __global__ void __launch_bounds__(kEncExactThreads) enc_exact_kernel(EncExactArg
       if (has) {
         for (int kk = lane; kk < nk; kk += 32) {
           double dist = 0.0;
+          if (HW) {
+            double t[kEncHMaxD];
 #pragma unroll
-          for (int e = 0; e < kEncMaxD; ++e) {
-            if (e < dv) {
-              const double t = __dsub_rn(v[e], tile[e * kEncExactTile + kk]);
-              dist = __dadd_rn(dist, __dmul_rn(t, t));
+            for (int e = 0; e < kEncHMaxD; ++e) t[e] = e < dv ? __dsub_rn(v[e], tile[e * kEncExactTile + kk]) : 0.0;
+#pragma unroll
+            for (int e = 0; e < (HW ? kEncHMaxD : 1); ++e) {
+              if (e < dv) {
+                double g = 0.0;
+#pragma unroll
+                for (int f = 0; f < (HW ? kEncHMaxD : 1); ++f)
+                  if (f < dv) g = __dadd_rn(g, __dmul_rn(hr[e][f], t[f]));
+                dist = __dadd_rn(dist, __dmul_rn(t[e], g));
+              }
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < kEncMaxD; ++e) {
+              if (e < dv) {
+                const double t = __dsub_rn(v[e], tile[e * kEncExactTile + kk]);
+                dist = __dadd_rn(dist, __dmul_rn(t, t));
+              }
             }
           }
           if (dist < best) {       // k ascends per lane: the first minimum
@@ -595,13 +901,15 @@ __global__ void enc_pack_kernel(const uint32_t* __restrict__ idx, int n, int nve
 // ---------------------------------------------------------------------------
 // Host side.
 // ---------------------------------------------------------------------------
-static_assert(sizeof(vq_encode_desc) == 88, "vq_encode_desc layout");
+static_assert(sizeof(vq_encode_desc) == 104, "vq_encode_desc layout");
 
 struct EncPlan {
   int n, kin, d, nb, nvec, nfull;
   int b[2], K[2], kp[2];
   int64_t nv_full;
-  size_t off_bprep[2], off_book64[2], off_idx[2], off_list, total;
+  bool hw;                       // Hessian-weighted form
+  int mt;                        // weighted form: blocks of 128 rows
+  size_t off_bprep[2], off_book64[2], off_idx[2], off_nc[2], off_ncabs[2], off_list, total;
 };
 
 size_t enc_round256(size_t x) { return (x + 255) / 256 * 256; }
@@ -625,6 +933,15 @@ vq_status enc_check(const vq_encode_desc* e, EncPlan* p, bool ptrs) {
   if (e->ldw < p->kin) return VQ_ERR_INVALID_ARG;
   if (data && !e->w) return VQ_ERR_INVALID_ARG;
   if (data && !aligned(e->w, 2)) return VQ_ERR_ALIGNMENT;
+  p->hw = e->h != nullptr;
+  p->mt = (p->n + kEncM - 1) / kEncM;
+  if (p->hw) {
+    if (p->d > kEncHMaxD) return VQ_ERR_UNSUPPORTED;
+    if (e->ldh < p->kin) return VQ_ERR_INVALID_ARG;
+    if (!aligned(e->h, 4)) return VQ_ERR_ALIGNMENT;
+    if (static_cast<int64_t>(p->nfull) * p->mt >= (int64_t{1} << 31) || p->nfull > 65535)
+      return VQ_ERR_UNSUPPORTED;
+  }
   size_t off = 256;
   for (int m = 0; m < p->nb; ++m) {
     if (e->log2k[m] < 1 || e->log2k[m] > 16) return VQ_ERR_INVALID_ARG;
@@ -647,6 +964,12 @@ vq_status enc_check(const vq_encode_desc* e, EncPlan* p, bool ptrs) {
   for (int m = 0; m < p->nb; ++m) {
     p->off_idx[m] = off;
     off = enc_round256(off + nv * 4);
+  }
+  for (int m = 0; m < p->nb; ++m) {   // weighted form: c~^T H_j c~ per block and centroid,
+    p->off_nc[m] = off;                 // then its error scale per block
+    if (p->hw) off = enc_round256(off + static_cast<size_t>(p->nfull) * p->kp[m] * 4);
+    p->off_ncabs[m] = off;
+    if (p->hw) off = enc_round256(off + static_cast<size_t>(p->nfull) * 4);
   }
   p->off_list = off;
   off = enc_round256(off + nv * 4);
@@ -700,8 +1023,17 @@ vq_status vq_encode(const vq_encode_desc* desc, void* workspace, size_t workspac
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
     count_launch();
     enc_book_prep_kernel<<<(p.kp[m] + 255) / 256, 256, 0, stream>>>(
-        desc->codebook[m], p.K[m], p.d, p.kp[m], &wc->cmax_bits[m], ws + p.off_bprep[m]);
+        desc->codebook[m], p.K[m], p.d, p.kp[m], &wc->cmax_bits[m], ws + p.off_bprep[m], p.hw ? 1 : 0);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+    if (p.hw && p.nfull > 0) {
+      e = cudaMemsetAsync(ws + p.off_ncabs[m], 0, static_cast<size_t>(p.nfull) * 4, stream);
+      if (e != cudaSuccess) return cuda_status(e);
+      count_launch();
+      enc_nc_kernel<<<dim3(p.kp[m] / 256, p.nfull), 256, 0, stream>>>(
+          desc->codebook[m], p.K[m], p.d, p.kp[m], &wc->cmax_bits[m], desc->h, desc->ldh,
+          reinterpret_cast<float*>(ws + p.off_nc[m]), reinterpret_cast<unsigned*>(ws + p.off_ncabs[m]));
+      if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+    }
     const int64_t cnt = static_cast<int64_t>(p.K[m]) * p.d;
     count_launch();
     enc_book64_kernel<<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, stream>>>(
@@ -710,7 +1042,8 @@ vq_status vq_encode(const vq_encode_desc* desc, void* workspace, size_t workspac
   }
 
   const int smem = static_cast<int>(sizeof(EncCtrl)) + 1024 + kEncATile + kEncStages * kEncBlockBytes;
-  e = cudaFuncSetAttribute(enc_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  auto tck = p.hw ? enc_tc_kernel<true> : enc_tc_kernel<false>;
+  e = cudaFuncSetAttribute(tck, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_status(e);
   int* list = reinterpret_cast<int*>(ws + p.off_list);
   for (int m = 0; m < p.nb; ++m) {
@@ -738,9 +1071,14 @@ vq_status vq_encode(const vq_encode_desc* desc, void* workspace, size_t workspac
       a.list = list;
       a.list_count = &wc->list_count[m];
       a.status = &wc->status;
-      const int64_t grid = (p.nv_full + kEncM - 1) / kEncM;
+      a.h = desc->h;
+      a.ldh = desc->ldh;
+      a.nc = p.hw ? reinterpret_cast<const float*>(ws + p.off_nc[m]) : nullptr;
+      a.ncabs = p.hw ? reinterpret_cast<const unsigned*>(ws + p.off_ncabs[m]) : nullptr;
+      a.mt = p.mt;
+      const int64_t grid = p.hw ? static_cast<int64_t>(p.nfull) * p.mt : (p.nv_full + kEncM - 1) / kEncM;
       count_launch();
-      enc_tc_kernel<<<static_cast<unsigned>(grid), kEncThreads, smem, stream>>>(a);
+      tck<<<static_cast<unsigned>(grid), kEncThreads, smem, stream>>>(a);
       if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
     }
     EncExactArgs x;
@@ -758,14 +1096,17 @@ vq_status vq_encode(const vq_encode_desc* desc, void* workspace, size_t workspac
     x.list = list;
     x.list_count = &wc->list_count[m];
     x.partial_rows = p.nfull < p.nvec ? p.n : 0;
+    x.h = desc->h;
+    x.ldh = desc->ldh;
     count_launch();
     const int xsmem = kEncExactTile * p.d * static_cast<int>(sizeof(double));
+    auto xk = p.hw ? enc_exact_kernel<true> : enc_exact_kernel<false>;
     if (m == 0) {
-      e = cudaFuncSetAttribute(enc_exact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = cudaFuncSetAttribute(xk, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kEncExactTile * kEncMaxD * static_cast<int>(sizeof(double)));
       if (e != cudaSuccess) return cuda_status(e);
     }
-    enc_exact_kernel<<<2 * device_sm_count(), kEncExactThreads, xsmem, stream>>>(x);
+    xk<<<2 * device_sm_count(), kEncExactThreads, xsmem, stream>>>(x);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   }
   for (int m = 0; m < p.nb; ++m) {

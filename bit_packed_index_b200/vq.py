@@ -59,6 +59,7 @@ class _EncDesc(C.Structure):
         ("w", C.c_void_p), ("ldw", C.c_int64),
         ("codebook", C.c_void_p * 2),
         ("idx", C.c_void_p * 2), ("idx_row_words", C.c_int64 * 2),
+        ("h", C.c_void_p), ("ldh", C.c_int64),
     ]
 
 
@@ -425,7 +426,8 @@ def row_words(in_features: int, vec_dim: int, log2k: int) -> int:
     return -(-(nvec * log2k) // 128) * 4
 
 
-def _encode_desc(w: torch.Tensor, codebooks, log2k, vec_dim: int, idx) -> _EncDesc:
+def _encode_desc(w: torch.Tensor, codebooks, log2k, vec_dim: int, idx,
+                 hessian: Optional[torch.Tensor] = None) -> _EncDesc:
     d = _EncDesc()
     d.out_features, d.in_features = w.shape[0], w.shape[1]
     d.vec_dim, d.n_books = vec_dim, len(log2k)
@@ -436,14 +438,22 @@ def _encode_desc(w: torch.Tensor, codebooks, log2k, vec_dim: int, idx) -> _EncDe
         d.codebook[m] = codebooks[m].data_ptr()
         d.idx[m] = idx[m].data_ptr() if idx[m].numel() else None
         d.idx_row_words[m] = idx[m].shape[1]
+    if hessian is not None:
+        if hessian.dtype != torch.float32 or hessian.dim() != 2 or hessian.stride(1) != 1:
+            raise ValueError("the Hessian must be a row-major float32 matrix")
+        d.h = hessian.data_ptr()
+        d.ldh = hessian.stride(0)
     return d
 
 
 def encode_workspace_size(out_features: int, in_features: int, log2k: Sequence[int],
-                          vec_dim: int) -> int:
+                          vec_dim: int, hessian: bool = False) -> int:
     d = _EncDesc()
     d.out_features, d.in_features, d.vec_dim, d.n_books = out_features, in_features, vec_dim, len(log2k)
     d.ldw = max(in_features, 1)
+    if hessian:                        # any aligned non-null pointer: only sizes are read
+        d.h = 256
+        d.ldh = max(in_features, 1)
     for m, b in enumerate(log2k):
         d.log2k[m] = int(b)
         d.idx_row_words[m] = row_words(in_features, vec_dim, int(b))
@@ -453,18 +463,19 @@ def encode_workspace_size(out_features: int, in_features: int, log2k: Sequence[i
 
 
 def encode(w: torch.Tensor, codebooks: Sequence[torch.Tensor], log2k: Sequence[int], vec_dim: int,
-           workspace: Optional[torch.Tensor] = None) -> Layer:
+           workspace: Optional[torch.Tensor] = None, hessian: Optional[torch.Tensor] = None) -> Layer:
     """Nearest-centroid encoding of W (float16 [N][Kin] on the device) against
     one book, or two as a greedy residual cascade (vq_encode): a row-order
     Layer holding the packed streams and the given codebooks (no scale or
-    bias)."""
+    bias).  With ``hessian`` (float32 [Kin][Kin] on the device, e.g. from
+    ``hessian()``) the distance is the Hessian-weighted (v-c)^T H_v (v-c)."""
     if w.dtype != torch.float16 or w.dim() != 2 or (w.shape[0] > 1 and w.stride(1) != 1):
         raise ValueError("w must be a row-major float16 matrix")
     log2k = [int(b) for b in log2k]
     books = [c.contiguous() for c in codebooks[:len(log2k)]]
     idx = [torch.empty((w.shape[0], row_words(w.shape[1], vec_dim, b)), dtype=torch.int32,
                        device=w.device) for b in log2k]
-    d = _encode_desc(w, books, log2k, vec_dim, idx)
+    d = _encode_desc(w, books, log2k, vec_dim, idx, hessian)
     n = C.c_size_t(0)
     _check("vq_encode_workspace_size", lib().vq_encode_workspace_size(C.byref(d), C.byref(n)))
     ws, ws_bytes = _workspace(n.value, w.device, workspace)

@@ -343,6 +343,21 @@ VQ_API vq_status vq_gemm(const vq_layer_desc* layer, const void* x, vq_dtype x_d
  * other vector (and every partial last vector) is decided by an fp64 pass
  * over the whole book.  The result therefore equals the exact definition.
  *
+ * Hessian-weighted form (h != NULL): the distance becomes
+ *     D_H(v, c) = (v - c)^T H_v (v - c),
+ * H_v the sub-matrix of the layer's Hessian h on the vector's channels
+ * (rows and columns j*d .. j*d+d-1, fewer for a partial last vector), for
+ * both stages of the cascade ("VPTQ Guide", section "1. Second-Order
+ * Hessian-Weighted Optimization": D_H(w, c_k) = (w - c_k)^T H_Iv (w - c_k);
+ * the page writes the residual stage unweighted, which is the case H = I).
+ * Exactly as in fp64: t_e = v_e - c_e, g_e = sum_f H[e][f] t_f (f ascending),
+ * D = sum_e t_e g_e (e ascending), every operation rounded once, ties to the
+ * lowest k.  Method: per vector z = H_s v (H_s = (H + H^T) / 2) is split
+ * into two fp16 halves for the tensor cores, which give -2<z, c>; the
+ * epilogue adds c^T H_v c, precomputed per (block of channels, centroid) in
+ * the workspace; near ties and partial last vectors take the fp64 pass as
+ * above.  vec_dim must be <= 8.  h is typically vq_hessian's output.
+ *
  *   out_features, in_features   N, Kin >= 0
  *   vec_dim        d, 1..14
  *   n_books        1 or 2;  log2k[m] in 1..16
@@ -352,6 +367,9 @@ VQ_API vq_status vq_gemm(const vq_layer_desc* layer, const void* x, vq_dtype x_d
  *                  format above): 16-byte aligned, idx_row_words[m] a multiple
  *                  of 4 and >= ceil(nvec*b_m/128)*4; every word of the N rows
  *                  is written (fields, then zero padding)
+ *   h, ldh         NULL for the plain distance, or device fp32 [Kin][ldh],
+ *                  ldh >= Kin, 4-byte aligned, finite values (read only on
+ *                  the diagonal blocks); ABI version 4
  */
 typedef struct vq_encode_desc {
     int32_t out_features;
@@ -364,6 +382,8 @@ typedef struct vq_encode_desc {
     const uint16_t* codebook[2];
     uint32_t* idx[2];
     int64_t idx_row_words[2];
+    const float* h;
+    int64_t ldh;
 } vq_encode_desc;
 
 /* Bytes of device workspace vq_encode needs (host-only, launches nothing;
@@ -376,7 +396,8 @@ VQ_API vq_status vq_encode_workspace_size(const vq_encode_desc* desc, size_t* by
  * 32-bit word is a status word (VQ_OK, or VQ_ERR_TIMEOUT if a bounded
  * device-side wait gave up), readable after the stream completes.
  * Errors: VQ_ERR_INVALID_ARG (sizes, NULL pointers with data, short strides),
- * VQ_ERR_ALIGNMENT, VQ_ERR_WORKSPACE, VQ_ERR_CUDA.
+ * VQ_ERR_UNSUPPORTED (vec_dim > 8 with h), VQ_ERR_ALIGNMENT,
+ * VQ_ERR_WORKSPACE, VQ_ERR_CUDA.
  */
 VQ_API vq_status vq_encode(const vq_encode_desc* desc, void* workspace, size_t workspace_bytes,
                            void* stream);

@@ -29,7 +29,7 @@ def test_every_declared_symbol_is_exported(lib):
 def test_host_only_calls(lib):
     assert lib.vq_abi_version() == 4
     assert C.sizeof(vq._Desc) == 104      # static_assert'ed in the library
-    assert C.sizeof(vq._EncDesc) == 88
+    assert C.sizeof(vq._EncDesc) == 104
     assert vq.kernel_launches() == 0          # nothing launched in this process
     for s in range(7):
         assert lib.vq_status_string(s)
@@ -186,6 +186,34 @@ def test_encode_workspace_and_validation_need_no_device(lib):
     e.idx_row_words[0] = 4
     # vq_encode itself: NULL buffers with data are rejected before any launch
     assert lib.vq_encode(C.byref(e), None, 0, None) == vq.VQ_ERR_INVALID_ARG
+
+
+def test_weighted_encode_workspace_and_validation(lib):
+    """With a Hessian the workspace adds, per book, one fp32 c^T H_j c value
+    per (whole block of channels j, padded centroid); vec_dim > 8, a short
+    ldh or a misaligned H is refused on the host."""
+    r256 = lambda x: -(-x // 256) * 256
+    n, kin, d = 300, 8 * 100 + 5, 8
+    plain = vq.encode_workspace_size(n, kin, [16, 4], d)
+    got = vq.encode_workspace_size(n, kin, [16, 4], d, hessian=True)
+    assert got == plain + r256(100 * 65536 * 4) + r256(100 * 4) + r256(100 * 1024 * 4) + r256(100 * 4)
+    e = vq._EncDesc()
+    e.out_features, e.in_features, e.vec_dim, e.n_books = 4, 16, 8, 1
+    e.log2k[0] = 8
+    e.ldw = 16
+    e.idx_row_words[0] = 4
+    e.h, e.ldh = 0x40000, 16
+    n_ = C.c_size_t(0)
+    assert lib.vq_encode_workspace_size(C.byref(e), C.byref(n_)) == vq.VQ_OK
+    e.ldh = 15
+    assert lib.vq_encode_workspace_size(C.byref(e), C.byref(n_)) == vq.VQ_ERR_INVALID_ARG
+    e.ldh = 16
+    e.h = 0x40002
+    assert lib.vq_encode_workspace_size(C.byref(e), C.byref(n_)) == vq.VQ_ERR_ALIGNMENT
+    e.h = 0x40000
+    e.vec_dim, e.in_features, e.ldw, e.ldh = 9, 18, 18, 18
+    e.idx_row_words[0] = 4
+    assert lib.vq_encode_workspace_size(C.byref(e), C.byref(n_)) == vq.VQ_ERR_UNSUPPORTED
 
 
 def test_new_entry_points_validate_before_any_device_call(lib):
