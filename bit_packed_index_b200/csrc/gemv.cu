@@ -299,7 +299,7 @@ vq_status launch_gemv(const Layer& L, const GemvPlan& p, const void* x, bool x_f
   if (L.kin == 0) return launch_empty_rows(L, y, yt, ldy, batch, stream);
   const int D = (L.d == 8) ? 8 : (L.d == 6 ? 6 : 0);
   cudaError_t e;
-  if (p.fast == 7) {
+  if (p.fast == 7 || p.fast == 8) {
     return launch_gemv_tc(L, p, x, x_fp16, batch, ldx, y, yt, ldy, ws, stream);
   } else if (p.fast >= 3) {
     return cuda_status(launch_gemv_lut(L, p, x, x_fp16, batch, ldx, y, yt, ldy, ws, stream));

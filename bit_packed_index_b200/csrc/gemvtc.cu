@@ -1,5 +1,7 @@
-// gemvtc.cu -- batched decode (batch 3..16) on the tcgen05 tensor cores, for
-// layers with one 2^16-entry, d = 8 codebook (row or tiled index order).
+// gemvtc.cu -- batched decode (batch 2..16) on the tcgen05 tensor cores, for
+// layers with one 2^16-entry, d = 8 codebook, and for layers whose books fit
+// shared memory (at most 2^12 + 2^12 entries, d = 6 or 8), in row or tiled
+// index order.
 //
 // y[b][o] = sum_k x[b][k] * W_hat[o][k] ("VPTQ Guide", section "Step 3";
 // "Vector Quantization for LLM Weights in Production", section "1. Prefill vs.
@@ -254,11 +256,245 @@ __global__ void __launch_bounds__(kTcThreads) gemv_tc_kernel(const __grid_consta
   }
 }
 
+// ---------------------------------------------------------------------------
+// Small books (the 8B and 405B layers: a 2^12-entry main book plus a 2^4 or
+// 2^8 residual, d = 6 or 8).  Both books fit shared memory, so no gather
+// leaves the SM: the books are staged once per CTA as 16-byte rows (d = 6
+// rows zero-padded to 8 halves), and eight producer warps -- two threads per
+// row, four vectors of each step per thread -- read a vector's two centroids
+// from shared memory, add them (one fp16 rounding of c1 + c2, the rounding
+// W_hat itself carries) and store the sum into the swizzled A tile.  x' puts
+// vector j at columns 8 j .. 8 j + 7 (gemv_tc_prep), so the MMA, the x loads
+// and the epilogue are those of the kernel above.
+// ---------------------------------------------------------------------------
+constexpr int kTsThreads = 384;                  // warps 4-11: producers, two per row
+constexpr int kTsProducers = 256;
+constexpr int kTsMaxEntries = 8192;              // K1 + K2 staged (128 KB)
+constexpr int kTsFixed = 2048 + kTcStages * kTcStage;   // control block, slack, stages; books follow
+
+// Words holding the four fields of book m for vectors 8 kt + 4 p .. + 3 of
+// row o, and the bit position of the first (fields are b bits, LSB first).
+template <int LAYOUT>
+__device__ __forceinline__ void tcs_words(const Layer& L, int m, int64_t o, int kt, int p, uint32_t (&w)[3],
+                                          int& sh) {
+  const int b = L.b[m];
+  const uint32_t* src;
+  int64_t w0, avail;
+  if constexpr (LAYOUT == VQ_IDX_TILE4) {
+    const int t = 2 * kt + p;
+    if (t >= (L.nvec + 3) / 4) {                     // a tile past the last vector
+      w[0] = w[1] = w[2] = 0u;
+      sh = 0;
+      return;
+    }
+    const int64_t bit0 = o * 4 * b;
+    src = L.idx[m] + static_cast<int64_t>(t) * L.rw[m];
+    w0 = bit0 >> 5;
+    sh = static_cast<int>(bit0 & 31);
+  } else {
+    const int64_t bit0 = static_cast<int64_t>(8 * kt + 4 * p) * b;
+    src = L.idx[m] + o * L.rw[m];
+    w0 = bit0 >> 5;
+    sh = static_cast<int>(bit0 & 31);
+  }
+  avail = L.rw[m] - w0;                              // words of the row (tile) left
+#pragma unroll
+  for (int i = 0; i < 3; ++i) w[i] = i < avail ? __ldg(src + w0 + i) : 0u;
+}
+
+__device__ __forceinline__ uint32_t tcs_field(const uint32_t (&w)[3], int bit, uint32_t mask) {
+  const int q = bit >> 5, s = bit & 31;
+  const uint32_t lo = q == 0 ? w[0] : (q == 1 ? w[1] : w[2]);
+  const uint32_t hi = q == 0 ? w[1] : (q == 1 ? w[2] : 0u);
+  return __funnelshift_r(lo, hi, s) & mask;
+}
+
+__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+template <int LAYOUT>
+__global__ void __launch_bounds__(kTsThreads, 1) gemv_tcs_kernel(const __grid_constant__ CUtensorMap xmap, TcArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = align1024(smem_raw);
+  TcCtrl* ctrl = reinterpret_cast<TcCtrl*>(base);
+  uint8_t* stages = base + 1024;
+  uint8_t* books = stages + kTcStages * kTcStage;   // [K1][16 B], then [K2][16 B]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Layer& L = g.L;
+  const int row0 = blockIdx.x * kTcRows;
+  const int split = blockIdx.y;
+  const int kt0 = split * g.kt_per_split;
+  const int nkt = min(g.num_kt, kt0 + g.kt_per_split) - kt0;   // >= 1 by construction
+  volatile int* abort_flag = &ctrl->abort;
+  const int k1 = 1 << L.b[0];
+  const int k2 = L.nb == 2 ? 1 << L.b[1] : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(&ctrl->full[s], kTsProducers);   // every producer thread
+      mbar_init(&ctrl->xfull[s], 1);             // the x load
+      mbar_init(&ctrl->empty[s], 1);
+    }
+    mbar_init(&ctrl->acc, 1);
+    ctrl->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctrl->tmem, 32);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch(&xmap);
+  // Stage the books: entry k of book m as 8 halves (d of them from the book,
+  // zeros after).
+  for (int i = threadIdx.x; i < k1 + k2; i += kTsThreads) {
+    const int m = i < k1 ? 0 : 1;
+    const int k = i - m * k1;
+    const uint16_t* c = L.book[m] + static_cast<int64_t>(k) * L.d;
+    uint4 v;
+    if (L.d == 8) {
+      v = __ldg(reinterpret_cast<const uint4*>(c));
+    } else {                                         // d = 6: 12 bytes, 4-byte aligned
+      const uint32_t* c32 = reinterpret_cast<const uint32_t*>(c);
+      v = make_uint4(__ldg(c32), __ldg(c32 + 1), __ldg(c32 + 2), 0u);
+    }
+    *reinterpret_cast<uint4*>(books + static_cast<size_t>(i) * 16) = v;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem;
+
+  if (warp == 0) {
+    if (lane == 0) {                                   // x tiles by TMA
+      int issued = 0;
+      for (int i = 0; i < nkt; ++i) {
+        const int s = i % kTcStages;
+        const uint32_t ph = (i / kTcStages) & 1;
+        if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, g.budget)) break;
+        mbar_arrive_expect_tx(&ctrl->xfull[s], kTcXTile);
+        tma_load_2d(stages + s * kTcStage + kTcATile, &xmap, &ctrl->xfull[s], (kt0 + i) * kTcK, 0);
+        issued = i + 1;
+      }
+      if (*abort_flag) {   // let loads already in flight land before the block exits
+        for (int i = max(0, issued - kTcStages); i < issued; ++i)
+          drain_phase(&ctrl->xfull[i % kTcStages], (i / kTcStages) & 1, 4000000000LL);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {                                   // MMA issuer
+      const uint32_t idesc = f16_idesc(kTcRows, kTcN);
+      int issued = 0;
+      for (int i = 0; i < nkt; ++i) {
+        const int s = i % kTcStages;
+        const uint32_t ph = (i / kTcStages) & 1;
+        if (!bounded_wait(&ctrl->full[s], ph, abort_flag, g.status, g.budget)) break;
+        if (!bounded_wait(&ctrl->xfull[s], ph, abort_flag, g.status, g.budget)) break;
+        tc_fence_after();
+        const uint32_t a = smem_addr(stages + s * kTcStage);
+        const uint32_t b = a + kTcATile;
+#pragma unroll
+        for (int kk = 0; kk < kTcK / 16; ++kk)
+          umma_f16(tmem, sw128_kmajor_desc(a + kk * 32), sw128_kmajor_desc(b + kk * 32), idesc, (i | kk) != 0);
+        umma_commit(&ctrl->empty[s]);
+        issued = i + 1;
+      }
+      if (issued > 0) {
+        umma_commit(&ctrl->acc);
+        drain_phase(&ctrl->acc, 0, 4000000000LL);     // products done before TMEM is freed
+      }
+    }
+  } else if (warp >= 4) {
+    // Producers: thread (r, p) builds vectors 4p .. 4p+3 of each step of row
+    // row0 + r (rows past N repeat row N-1, whose results are never stored).
+    const int pr = threadIdx.x - kTcProducer0;
+    const int r = pr & (kTcRows - 1), p = pr >> 7;
+    const int64_t o = min(row0 + r, L.n - 1);
+    const uint32_t m1 = (1u << L.b[0]) - 1u, m2 = L.nb == 2 ? (1u << L.b[1]) - 1u : 0u;
+    const int b1 = L.b[0], b2 = L.nb == 2 ? L.b[1] : 0;
+    const uint8_t* book2 = books + static_cast<size_t>(k1) * 16;
+    // index words of the next two steps in flight
+    uint32_t wa[3], wb[3], na[3] = {0u, 0u, 0u}, nbw[3] = {0u, 0u, 0u};
+    int sa = 0, sb = 0, nsa = 0, nsb = 0;
+    tcs_words<LAYOUT>(L, 0, o, kt0, p, wa, sa);
+    if (L.nb == 2) tcs_words<LAYOUT>(L, 1, o, kt0, p, wb, sb);
+    if (nkt > 1) {
+      tcs_words<LAYOUT>(L, 0, o, kt0 + 1, p, na, nsa);
+      if (L.nb == 2) tcs_words<LAYOUT>(L, 1, o, kt0 + 1, p, nbw, nsb);
+    }
+    for (int i = 0; i < nkt; ++i) {
+      const int s = i % kTcStages;
+      const uint32_t ph = (i / kTcStages) & 1;
+      uint32_t f1[4], f2[4];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        f1[v] = tcs_field(wa, sa + v * b1, m1);
+        f2[v] = L.nb == 2 ? tcs_field(wb, sb + v * b2, m2) : 0u;
+      }
+#pragma unroll
+      for (int q = 0; q < 3; ++q) {
+        wa[q] = na[q];
+        wb[q] = nbw[q];
+      }
+      sa = nsa;
+      sb = nsb;
+      if (i + 2 < nkt) {
+        tcs_words<LAYOUT>(L, 0, o, kt0 + i + 2, p, na, nsa);
+        if (L.nb == 2) tcs_words<LAYOUT>(L, 1, o, kt0 + i + 2, p, nbw, nsb);
+      }
+      uint4 c[4];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        c[v] = *reinterpret_cast<const uint4*>(books + static_cast<size_t>(f1[v]) * 16);
+        if (L.nb == 2) {
+          const uint4 c2 = *reinterpret_cast<const uint4*>(book2 + static_cast<size_t>(f2[v]) * 16);
+          c[v] = make_uint4(hadd2_u32(c[v].x, c2.x), hadd2_u32(c[v].y, c2.y), hadd2_u32(c[v].z, c2.z),
+                            hadd2_u32(c[v].w, c2.w));
+        }
+      }
+      if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, g.budget)) break;
+      uint8_t* at = stages + s * kTcStage;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) *reinterpret_cast<uint4*>(at + sw128_off(r, 4 * p + v)) = c[v];
+      fence_proxy_async_smem();                        // visible to the tensor cores
+      mbar_arrive(&ctrl->full[s]);
+    }
+    // Epilogue (warps 4-7): lane quarter warp & 3, one output row per thread.
+    if (p == 0 && bounded_wait(&ctrl->acc, 0, abort_flag, g.status, g.budget)) {
+      tc_fence_after();
+      uint32_t acc[16];
+      tmem_ld16(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16), acc);
+      tmem_wait_ld();
+      const int row = row0 + r;
+      if (row < L.n) {
+        const float sc = L.scale ? h2f(L.scale[row]) : 1.0f;
+        const float tb = (L.bias && split == 0) ? h2f(L.bias[row]) : 0.0f;
+        const float ob = split == 0 ? out_bias_of(L.ob, row) : 0.0f;
+        for (int b = 0; b < g.batch; ++b) {
+          const float v = sc * (__uint_as_float(acc[b]) * g.xe[b]) + tb * g.xsum[b] + ob;
+          if (g.part) g.part[(static_cast<int64_t>(split) * g.batch + b) * L.n + row] = v;
+          else store_out(g.y, g.yt, b * g.ldy + row, v);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 32);
+  }
+}
+
 // x' = x * 2^-e_b in fp16 [16][kp] (zero past kin and for rows b >= batch),
 // 2^e_b and sum_k x[b][k].  e_b puts max_k |x[b][k]| in [2^14, 2^15), so no
-// value overflows fp16 and values above max * 2^-29 stay exact.
+// value overflows fp16 and values above max * 2^-29 stay exact.  x' holds
+// vector j of the layer (d elements) at columns 8 j .. 8 j + d - 1 and zeros
+// in the rest of its 8 columns (d = 8: x' is x itself, scaled).
 __global__ void gemv_tc_prep(const uint16_t* __restrict__ x, int x_fp16, int64_t ldx, int kin, int kp, int batch,
-                             uint16_t* __restrict__ xh, float* __restrict__ xe, float* __restrict__ xsum) {
+                             int d, uint16_t* __restrict__ xh, float* __restrict__ xe, float* __restrict__ xsum) {
   __shared__ float s_max[32], s_sum[32];
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool live = b < batch;
@@ -297,8 +533,10 @@ __global__ void gemv_tc_prep(const uint16_t* __restrict__ x, int x_fp16, int64_t
   const float f2 = __uint_as_float(static_cast<uint32_t>(127 - (e - e / 2)) << 23);
   for (int k = tid; k < kp; k += blockDim.x) {
     float v = 0.0f;
-    if (live && k < kin) {
-      const uint16_t u = x[b * ldx + k];
+    const int e8 = k & 7;
+    const int src = (k >> 3) * d + e8;               // element of x in column k
+    if (live && e8 < d && src < kin) {
+      const uint16_t u = x[b * ldx + src];
       v = (x_fp16 ? h2f(u) : bf2f(u)) * f1 * f2;
     }
     xh[static_cast<int64_t>(b) * kp + k] = f2h(v);
@@ -327,13 +565,32 @@ struct TcLayout {
   size_t off_status, off_xh, off_xe, off_part, total;
 };
 
-TcLayout tc_layout(const Layer& L, int batch) {
+// The 2^16-book kernel runs three CTAs per SM and splits the input dimension
+// so that the grid fills about one wave of them; the small-book kernel runs
+// one CTA per SM and picks the split (up to 8) that wastes the least of the
+// last wave.
+TcLayout tc_layout(const Layer& L, int batch, bool small) {
   TcLayout t{};
   t.tiles = (L.n + kTcRows - 1) / kTcRows;
   t.num_kt = (L.nvec + 7) / 8;
   t.kp = t.num_kt * kTcK;
-  const int target = kTcPerSm * device_sm_count();
-  int nsplit = std::max(1, std::min(t.num_kt, (target + t.tiles / 2) / t.tiles));
+  int nsplit = 1;
+  if (!small) {
+    const int target = kTcPerSm * device_sm_count();
+    nsplit = std::max(1, std::min(t.num_kt, (target + t.tiles / 2) / t.tiles));
+  } else {
+    const int sms = device_sm_count();
+    double best = -1.0;
+    for (int ns = 1; ns <= std::min(8, t.num_kt); ++ns) {
+      const int64_t ctas = static_cast<int64_t>(t.tiles) * ns;
+      const int64_t waves = (ctas + sms - 1) / sms;
+      const double score = static_cast<double>(ctas) / static_cast<double>(waves * sms) - 0.02 * (ns - 1);
+      if (score > best + 1e-9) {
+        best = score;
+        nsplit = ns;
+      }
+    }
+  }
   t.kt_per_split = (t.num_kt + nsplit - 1) / nsplit;
   t.nsplit = (t.num_kt + t.kt_per_split - 1) / t.kt_per_split;
   auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
@@ -345,11 +602,22 @@ TcLayout tc_layout(const Layer& L, int batch) {
   return t;
 }
 
-// Smallest batch this kernel serves (VQ_TC_MIN_BATCH overrides, for measurements).
+// Smallest batch the kernels serve (VQ_TC_MIN_BATCH and VQ_TCS_MIN_BATCH
+// override, for measurements).
 int tc_min_batch() {
   if (const char* env = std::getenv("VQ_TC_MIN_BATCH")) return std::atoi(env);
   return 2;
 }
+int tcs_min_batch() {
+  if (const char* env = std::getenv("VQ_TCS_MIN_BATCH")) return std::atoi(env);
+  return 3;
+}
+
+bool tcs_supported(const Layer& L) {
+  if (!(L.d == 6 || L.d == 8) || L.b[0] > 12 || (L.nb == 2 && L.b[1] > 12)) return false;
+  return (1 << L.b[0]) + (L.nb == 2 ? 1 << L.b[1] : 0) <= kTsMaxEntries;
+}
+int tcs_smem(const Layer& L) { return kTsFixed + ((1 << L.b[0]) + (L.nb == 2 ? 1 << L.b[1] : 0)) * 16; }
 
 long long tc_wait_budget() {
   if (const char* env = std::getenv("VQ_WAIT_BUDGET")) return std::atoll(env);
@@ -359,24 +627,29 @@ long long tc_wait_budget() {
 }  // namespace
 
 bool plan_gemv_tc(const Layer& L, int batch, size_t ws_cap, GemvPlan* p) {
-  if (!(L.layout == VQ_IDX_ROWS || L.layout == VQ_IDX_TILE4) || L.nb != 1 || L.d != 8 || L.b[0] != 16) return false;
-  if (batch < std::max(1, tc_min_batch()) || batch > kTcN || L.n < 1 || L.nvec < 1) return false;
-  if (device_smem_optin() < kTcSmem) return false;
-  const TcLayout t = tc_layout(L, batch);
+  if (!(L.layout == VQ_IDX_ROWS || L.layout == VQ_IDX_TILE4) || L.n < 1 || L.nvec < 1 || batch > kTcN) return false;
+  const bool big = L.nb == 1 && L.d == 8 && L.b[0] == 16;
+  const bool small = !big && tcs_supported(L);
+  if (!big && !small) return false;
+  if (batch < std::max(1, big ? tc_min_batch() : tcs_min_batch())) return false;
+  const int smem = big ? kTcSmem : tcs_smem(L);
+  if (device_smem_optin() < smem) return false;
+  const TcLayout t = tc_layout(L, batch, small);
   if (t.total > ws_cap) return false;
   *p = GemvPlan{};
-  p->fast = 7;
+  p->fast = big ? 7 : 8;
   p->bt = batch;
   p->nsplit = t.nsplit;
   p->grid_x = t.tiles;
-  p->smem = kTcSmem;
+  p->smem = smem;
   p->ws_bytes = t.total;
   return true;
 }
 
 vq_status launch_gemv_tc(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, int batch, int64_t ldx,
                          void* y, vq_dtype yt, int64_t ldy, void* ws, cudaStream_t stream) {
-  const TcLayout t = tc_layout(L, batch);
+  const bool small = p.fast == 8;
+  const TcLayout t = tc_layout(L, batch, small);
   uint8_t* w = static_cast<uint8_t*>(ws);
   uint16_t* xh = reinterpret_cast<uint16_t*>(w + t.off_xh);
   float* xe = reinterpret_cast<float*>(w + t.off_xe);
@@ -386,7 +659,7 @@ vq_status launch_gemv_tc(const Layer& L, const GemvPlan& p, const void* x, bool 
   if (e != cudaSuccess) return cuda_status(e);
   count_launch();
   gemv_tc_prep<<<kTcN, 256, 0, stream>>>(static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, ldx, L.kin, t.kp, batch,
-                                          xh, xe, xsum);
+                                          L.d, xh, xe, xsum);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   CUtensorMap xmap;
   if (!make_map_f16_sw128(&xmap, xh, t.kp, kTcN, t.kp, kTcN)) return VQ_ERR_CUDA;
@@ -403,11 +676,13 @@ vq_status launch_gemv_tc(const Layer& L, const GemvPlan& p, const void* x, bool 
   g.part = t.nsplit > 1 ? reinterpret_cast<float*>(w + t.off_part) : nullptr;
   g.status = status;
   g.budget = tc_wait_budget();
-  auto k = L.layout == VQ_IDX_TILE4 ? gemv_tc_kernel<VQ_IDX_TILE4> : gemv_tc_kernel<VQ_IDX_ROWS>;
-  if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem)) != cudaSuccess)
+  auto k = small ? (L.layout == VQ_IDX_TILE4 ? gemv_tcs_kernel<VQ_IDX_TILE4> : gemv_tcs_kernel<VQ_IDX_ROWS>)
+                 : (L.layout == VQ_IDX_TILE4 ? gemv_tc_kernel<VQ_IDX_TILE4> : gemv_tc_kernel<VQ_IDX_ROWS>);
+  const int threads = small ? kTsThreads : kTcThreads;
+  if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem)) != cudaSuccess)
     return cuda_status(e);
   count_launch();
-  k<<<dim3(t.tiles, t.nsplit), kTcThreads, kTcSmem, stream>>>(xmap, g);
+  k<<<dim3(t.tiles, t.nsplit), threads, p.smem, stream>>>(xmap, g);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   if (t.nsplit > 1) {
     const int64_t total = static_cast<int64_t>(batch) * L.n;

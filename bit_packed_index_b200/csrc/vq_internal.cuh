@@ -80,7 +80,8 @@ struct GemvPlan {
                       // 1: single-row kernel (gemv1.cu), 2: batched kernel (gemvb.cu),
                       // 3: lookup-table kernel (2^16 book), 5: lookup-table kernel for
                       // books of <= 2^12 entries (tile4.cu, tiled order, batch 1),
-                      // 7: tensor-core batched decode (gemvtc.cu)
+                      // 7: tensor-core batched decode, 2^16 book (gemvtc.cu),
+                      // 8: the same for books staged in shared memory
 };
 // ws_cap: largest workspace the caller can provide (plans that need more
 // either shrink, for the tiled kernels, or are reported by their ws_bytes).
