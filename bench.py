@@ -849,6 +849,45 @@ def run_profile(args):
         ws = torch.empty(vq.gemv_multi_workspace_size(layers, BATCH), dtype=torch.uint8, device=dev)
         for _ in range(args.profile_launches):
             vq.gemv_multi(layers, x, outs=outs, workspace=ws)
+    elif args.profile in ("tc_gate16", "tcs_q16", "tcs_8b16"):
+        # batch-16 decode on the tensor cores, tiled order: the 70B gate_proj
+        # (2^16 book), the 405B q_proj and the 8B up_proj (small books)
+        name, li = {"tc_gate16": (DECODE, 0), "tcs_q16": ("llama31_405b", 0),
+                    "tcs_8b16": ("llama3_8b_up", 0)}[args.profile]
+        w = WORKLOADS[name]
+        spec, seed = w.layers[li]
+        layer = vq.Layer.from_synth(synth.make_layer(spec, seed), dev, layout="tile4")
+        x = torch.from_numpy(synth.make_x(w.x_seed, 16, spec.in_features, w.outlier_frac)
+                             .view(np.int16)).to(dev).view(torch.bfloat16)
+        out = torch.empty((16, spec.out_features), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(256, vq.gemv_workspace_size(layer, 16)), dtype=torch.uint8, device=dev)
+        for _ in range(args.profile_launches):
+            vq.gemv(layer, x, out=out, workspace=ws)
+    elif args.profile == "encode_h":
+        n, kin, d, log2k = ENCODE_SHAPE
+        w, books = synth.make_encode_input(n, kin, d, log2k, ENCODE_STD, seed=ENCODE_SEED)
+        W = torch.from_numpy(w.view(np.int16)).to(dev).view(torch.float16)
+        B = [torch.from_numpy(b.view(np.int16)).to(dev).view(torch.float16) for b in books]
+        xt = synth.make_x(ENCODE_H_SEED, ENCODE_H_TOKENS, kin, 0.001)
+        H = vq.hessian(torch.from_numpy(xt.view(np.int16)).to(dev).view(torch.bfloat16))
+        ws = torch.empty(vq.encode_workspace_size(n, kin, log2k, d, hessian=True), dtype=torch.uint8, device=dev)
+        for _ in range(args.profile_launches):
+            vq.encode(W, B, log2k, d, workspace=ws, hessian=H)
+    elif args.profile == "rht_gate":
+        w = WORKLOADS[DECODE]
+        spec, seed = w.layers[0]
+        layer = vq.Layer.from_synth(synth.make_layer(spec, seed), dev, layout="tile4")
+        x = torch.from_numpy(synth.make_x(w.x_seed, 1, spec.in_features, w.outlier_frac)
+                             .view(np.int16)).to(dev).view(torch.bfloat16)
+        rng = np.random.default_rng(RHT_SEED)
+        s_in = torch.from_numpy(rng.integers(0, 2**31, size=(spec.in_features + 31) // 32, dtype=np.int64)
+                                .astype(np.int32)).to(dev)
+        s_out = torch.from_numpy(rng.integers(0, 2**31, size=(spec.out_features + 31) // 32, dtype=np.int64)
+                                 .astype(np.int32)).to(dev)
+        y = torch.empty((1, spec.out_features), dtype=torch.bfloat16, device=dev)
+        wr = torch.empty(vq.gemv_rht_workspace_size(layer, 1), dtype=torch.uint8, device=dev)
+        for _ in range(args.profile_launches):
+            vq.gemv_rht(layer, s_in, s_out, x, out=y, workspace=wr)
     elif args.profile in ("gemv", "lut", "lut_down", "lut_small", "dequant"):
         w = WORKLOADS[DECODE if args.profile != "lut_small" else "llama31_405b"]
         spec, seed = w.layers[{"lut_small": 4, "lut_down": 2}.get(args.profile, 0)]
@@ -889,6 +928,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", choices=["gemv", "lut", "lut_gateup", "lut_down", "lut_small", "gemm",
+                                          "tc_gate16", "tcs_q16", "tcs_8b16", "encode_h", "rht_gate",
                                           "dequant", "encode", "hessian"],
                     help="run a few untimed launches of one call on its workload (for ncu): "
                          "gemv / lut = 70B gate_proj in row / tiled order, lut_gateup = 70B "

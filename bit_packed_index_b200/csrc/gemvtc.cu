@@ -61,9 +61,15 @@ struct TcCtrl {
   uint64_t xfull[kTcStages];   // the stage's x tile landed (TMA)
   uint64_t empty[kTcStages];
   uint64_t acc;
+  uint64_t accf[2];            // small-book kernel: accumulator b complete
+  uint64_t acce[2];            //   accumulator b read by the epilogue
+  uint64_t xf[16];             //   x ring: tile landed (TMA)
+  uint64_t xe[16];             //   x ring: tile consumed by the MMAs
   uint32_t tmem;
   int abort;
 };
+
+static_assert(sizeof(TcCtrl) <= 1024, "control block");
 
 struct TcArgs {
   Layer L;
@@ -78,6 +84,7 @@ struct TcArgs {
   float* part;            // [nsplit][batch][N] when the input dimension is split
   int* status;
   long long budget;
+  int tiles, nitems;      // small-book kernel: work items (row tile, split), split-major
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -131,7 +138,7 @@ __global__ void __launch_bounds__(kTcThreads) gemv_tc_kernel(const __grid_consta
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&ctrl->full[s], kTcRows);        // every producer thread
+      mbar_init(&ctrl->full[s], kTcRows / 32);   // one arrival per producer warp
       mbar_init(&ctrl->xfull[s], 1);             // the x load
       mbar_init(&ctrl->empty[s], 1);
     }
@@ -206,7 +213,8 @@ __global__ void __launch_bounds__(kTcThreads) gemv_tc_kernel(const __grid_consta
     for (int i = 0; i < nkt; ++i) {
       const int s = i % kTcStages;
       const uint32_t ph = (i / kTcStages) & 1;
-      if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, g.budget)) break;
+      // warp-uniform: the warp publishes its steps with one arrival
+      if (!__all_sync(0xffffffffu, bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, g.budget))) break;
       const uint32_t wd[4] = {w0.x, w0.y, w0.z, w0.w};
       w0 = w1;
       w1 = w2;
@@ -221,13 +229,15 @@ __global__ void __launch_bounds__(kTcThreads) gemv_tc_kernel(const __grid_consta
       if (i >= kTcLag) {                               // step i - kTcLag has landed: publish it
         cp_async_wait<kTcLag>();
         fence_proxy_async_smem();
-        mbar_arrive(&ctrl->full[(i - kTcLag) % kTcStages]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->full[(i - kTcLag) % kTcStages]);
         published = i - kTcLag + 1;
       }
     }
     cp_async_wait<0>();                                // nothing of ours may land after the exit
     fence_proxy_async_smem();
-    if (!*abort_flag)
+    __syncwarp();
+    if (__all_sync(0xffffffffu, !*abort_flag) && lane == 0)
       for (int i = published; i < nkt; ++i) mbar_arrive(&ctrl->full[i % kTcStages]);
     // Epilogue: lane quarter warp & 3, one output row per thread.
     if (bounded_wait(&ctrl->acc, 0, abort_flag, g.status, g.budget)) {
@@ -260,20 +270,43 @@ __global__ void __launch_bounds__(kTcThreads) gemv_tc_kernel(const __grid_consta
 // Small books (the 8B and 405B layers: a 2^12-entry main book plus a 2^4 or
 // 2^8 residual, d = 6 or 8).  Both books fit shared memory, so no gather
 // leaves the SM: the books are staged once per CTA as 16-byte rows (d = 6
-// rows zero-padded to 8 halves), and eight producer warps -- two threads per
-// row, four vectors of each step per thread -- read a vector's two centroids
+// rows zero-padded to 8 halves), and the producer warps -- two or four
+// threads per row, each with its share of a step's eight vectors -- read a vector's two centroids
 // from shared memory, add them (one fp16 rounding of c1 + c2, the rounding
 // W_hat itself carries) and store the sum into the swizzled A tile.  x' puts
 // vector j at columns 8 j .. 8 j + 7 (gemv_tc_prep), so the MMA, the x loads
 // and the epilogue are those of the kernel above.
 // ---------------------------------------------------------------------------
-constexpr int kTsThreads = 384;                  // warps 4-11: producers, two per row
-constexpr int kTsProducers = 256;
+// Producer threads per row: four in the tiled order (a warp's loads of a
+// tile's records are contiguous), two in row order (each thread's index
+// words come from its own row, so fewer, longer reads measured faster).
+template <int LAYOUT>
+struct TsShape {
+  static constexpr int per_row = LAYOUT == VQ_IDX_TILE4 ? 4 : 2;
+  static constexpr int vpt = 8 / per_row;                  // vectors of a step per producer thread
+  static constexpr int producers = kTcRows * per_row;
+  static constexpr int threads = kTcProducer0 + producers;   // warps 4..: producers
+};
+#ifndef VQ_TS_NACC
+#define VQ_TS_NACC 4
+#endif
+constexpr int kTsNacc = VQ_TS_NACC;              // accumulators per item: the K slices of a step alternate
+constexpr int kTsTmemCols = 2 * 16 * kTsNacc < 32 ? 32 : 2 * 16 * kTsNacc;
+#ifndef VQ_TS_PF
+#define VQ_TS_PF 4
+#endif
+constexpr int kTsPf = VQ_TS_PF;                  // steps of index words a producer keeps in flight
 constexpr int kTsMaxEntries = 8192;              // K1 + K2 staged (128 KB)
-constexpr int kTsFixed = 2048 + kTcStages * kTcStage;   // control block, slack, stages; books follow
+#ifndef VQ_TS_XS
+#define VQ_TS_XS 8
+#endif
+constexpr int kTsXs = VQ_TS_XS;                  // x tiles in flight (their own ring, deeper than the A ring)
+constexpr int kTsFixed = 2048 + kTcStages * kTcATile + kTsXs * kTcXTile;   // control, slack, A ring, x ring
+static_assert(kTsXs >= 2 && kTsXs <= 16, "x ring of 2..16 tiles");
 
-// Words holding the four fields of book m for vectors 8 kt + 4 p .. + 3 of
-// row o, and the bit position of the first (fields are b bits, LSB first).
+// Words holding the TsShape<LAYOUT>::vpt fields of book m for vectors 8 kt + TsShape<LAYOUT>::vpt p ..
+// of row o, and the bit position of the first (fields are b bits, LSB
+// first).
 template <int LAYOUT>
 __device__ __forceinline__ void tcs_words(const Layer& L, int m, int64_t o, int kt, int p, uint32_t (&w)[3],
                                           int& sh) {
@@ -281,18 +314,18 @@ __device__ __forceinline__ void tcs_words(const Layer& L, int m, int64_t o, int 
   const uint32_t* src;
   int64_t w0, avail;
   if constexpr (LAYOUT == VQ_IDX_TILE4) {
-    const int t = 2 * kt + p;
+    const int t = 2 * kt + (TsShape<LAYOUT>::vpt * p) / 4;
     if (t >= (L.nvec + 3) / 4) {                     // a tile past the last vector
       w[0] = w[1] = w[2] = 0u;
       sh = 0;
       return;
     }
-    const int64_t bit0 = o * 4 * b;
+    const int64_t bit0 = o * 4 * b + ((TsShape<LAYOUT>::vpt * p) % 4) * b;
     src = L.idx[m] + static_cast<int64_t>(t) * L.rw[m];
     w0 = bit0 >> 5;
     sh = static_cast<int>(bit0 & 31);
   } else {
-    const int64_t bit0 = static_cast<int64_t>(8 * kt + 4 * p) * b;
+    const int64_t bit0 = static_cast<int64_t>(8 * kt + TsShape<LAYOUT>::vpt * p) * b;
     src = L.idx[m] + o * L.rw[m];
     w0 = bit0 >> 5;
     sh = static_cast<int>(bit0 & 31);
@@ -315,41 +348,50 @@ __device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
   return r;
 }
 
+// Persistent: one CTA per SM stages the books once and takes work items
+// (row tile, split) in turn; the stage ring and its phases run on across
+// items, and two 16-column accumulators alternate so that the epilogue of
+// one item overlaps the products of the next.
 template <int LAYOUT>
-__global__ void __launch_bounds__(kTsThreads, 1) gemv_tcs_kernel(const __grid_constant__ CUtensorMap xmap, TcArgs g) {
+__global__ void __launch_bounds__(TsShape<LAYOUT>::threads, 1) gemv_tcs_kernel(const __grid_constant__ CUtensorMap xmap, TcArgs g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
   TcCtrl* ctrl = reinterpret_cast<TcCtrl*>(base);
   uint8_t* stages = base + 1024;
-  uint8_t* books = stages + kTcStages * kTcStage;   // [K1][16 B], then [K2][16 B]
+  uint8_t* xring = stages + kTcStages * kTcATile;   // kTsXs x tiles
+  uint8_t* books = xring + kTsXs * kTcXTile;        // [K1][16 B], then [K2][16 B]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Layer& L = g.L;
-  const int row0 = blockIdx.x * kTcRows;
-  const int split = blockIdx.y;
-  const int kt0 = split * g.kt_per_split;
-  const int nkt = min(g.num_kt, kt0 + g.kt_per_split) - kt0;   // >= 1 by construction
   volatile int* abort_flag = &ctrl->abort;
   const int k1 = 1 << L.b[0];
   const int k2 = L.nb == 2 ? 1 << L.b[1] : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&ctrl->full[s], kTsProducers);   // every producer thread
+      mbar_init(&ctrl->full[s], TsShape<LAYOUT>::producers / 32);   // one arrival per producer warp
       mbar_init(&ctrl->xfull[s], 1);             // the x load
       mbar_init(&ctrl->empty[s], 1);
     }
     mbar_init(&ctrl->acc, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctrl->accf[b], 1);
+      mbar_init(&ctrl->acce[b], 4);              // the four epilogue warps
+    }
+    for (int q = 0; q < kTsXs; ++q) {
+      mbar_init(&ctrl->xf[q], 1);
+      mbar_init(&ctrl->xe[q], 1);
+    }
     ctrl->abort = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&ctrl->tmem, 32);
+    tmem_alloc(&ctrl->tmem, kTsTmemCols);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) tma_prefetch(&xmap);
   // Stage the books: entry k of book m as 8 halves (d of them from the book,
   // zeros after).
-  for (int i = threadIdx.x; i < k1 + k2; i += kTsThreads) {
+  for (int i = threadIdx.x; i < k1 + k2; i += TsShape<LAYOUT>::threads) {
     const int m = i < k1 ? 0 : 1;
     const int k = i - m * k1;
     const uint16_t* c = L.book[m] + static_cast<int64_t>(k) * L.d;
@@ -369,113 +411,184 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemv_tcs_kernel(const __grid_co
 
   if (warp == 0) {
     if (lane == 0) {                                   // x tiles by TMA
-      int issued = 0;
-      for (int i = 0; i < nkt; ++i) {
-        const int s = i % kTcStages;
-        const uint32_t ph = (i / kTcStages) & 1;
-        if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, g.budget)) break;
-        mbar_arrive_expect_tx(&ctrl->xfull[s], kTcXTile);
-        tma_load_2d(stages + s * kTcStage + kTcATile, &xmap, &ctrl->xfull[s], (kt0 + i) * kTcK, 0);
-        issued = i + 1;
+      int gs = 0;                                      // steps issued over all items
+      bool stop = false;
+      for (int item = blockIdx.x; item < g.nitems && !stop; item += gridDim.x) {
+        const int kt0 = (item / g.tiles) * g.kt_per_split;
+        const int nkt = min(g.num_kt, kt0 + g.kt_per_split) - kt0;
+        for (int i = 0; i < nkt; ++i, ++gs) {
+          const int q = gs % kTsXs;
+          const uint32_t ph = (gs / kTsXs) & 1;
+          if (!bounded_wait(&ctrl->xe[q], ph ^ 1, abort_flag, g.status, g.budget)) {
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx(&ctrl->xf[q], kTcXTile);
+          tma_load_2d(xring + q * kTcXTile, &xmap, &ctrl->xf[q], (kt0 + i) * kTcK, 0);
+        }
       }
       if (*abort_flag) {   // let loads already in flight land before the block exits
-        for (int i = max(0, issued - kTcStages); i < issued; ++i)
-          drain_phase(&ctrl->xfull[i % kTcStages], (i / kTcStages) & 1, 4000000000LL);
+        for (int i = max(0, gs - kTsXs); i < gs; ++i)
+          drain_phase(&ctrl->xf[i % kTsXs], (i / kTsXs) & 1, 4000000000LL);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {                                   // MMA issuer
       const uint32_t idesc = f16_idesc(kTcRows, kTcN);
-      int issued = 0;
-      for (int i = 0; i < nkt; ++i) {
-        const int s = i % kTcStages;
-        const uint32_t ph = (i / kTcStages) & 1;
-        if (!bounded_wait(&ctrl->full[s], ph, abort_flag, g.status, g.budget)) break;
-        if (!bounded_wait(&ctrl->xfull[s], ph, abort_flag, g.status, g.budget)) break;
+      int gs = 0, it = 0;
+      bool any = false, stop = false;
+      for (int item = blockIdx.x; item < g.nitems && !stop; item += gridDim.x, ++it) {
+        const int kt0 = (item / g.tiles) * g.kt_per_split;
+        const int nkt = min(g.num_kt, kt0 + g.kt_per_split) - kt0;
+        const int buf = it & 1;
+        // the epilogue has read what this accumulator held two items ago
+        if (it >= 2 && !bounded_wait(&ctrl->acce[buf], ((it >> 1) & 1) ^ 1, abort_flag, g.status, g.budget))
+          break;
         tc_fence_after();
-        const uint32_t a = smem_addr(stages + s * kTcStage);
-        const uint32_t b = a + kTcATile;
+        for (int i = 0; i < nkt; ++i, ++gs) {
+          const int s = gs % kTcStages;
+          const uint32_t ph = (gs / kTcStages) & 1;
+          const int xq = gs % kTsXs;
+          if (!bounded_wait(&ctrl->full[s], ph, abort_flag, g.status, g.budget) ||
+              !bounded_wait(&ctrl->xf[xq], (gs / kTsXs) & 1, abort_flag, g.status, g.budget)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = smem_addr(stages + s * kTcATile);
+          const uint32_t b = smem_addr(xring + xq * kTcXTile);
+          // consecutive products go to different accumulators, so none waits
+          // for the previous one to finish accumulating
 #pragma unroll
-        for (int kk = 0; kk < kTcK / 16; ++kk)
-          umma_f16(tmem, sw128_kmajor_desc(a + kk * 32), sw128_kmajor_desc(b + kk * 32), idesc, (i | kk) != 0);
-        umma_commit(&ctrl->empty[s]);
-        issued = i + 1;
+          for (int kk = 0; kk < kTcK / 16; ++kk)
+            umma_f16(tmem + 16 * (kTsNacc * buf + kk % kTsNacc), sw128_kmajor_desc(a + kk * 32),
+                     sw128_kmajor_desc(b + kk * 32), idesc, (i != 0) || (kk >= kTsNacc));
+          umma_commit(&ctrl->empty[s]);
+          umma_commit(&ctrl->xe[xq]);
+          any = true;
+        }
+        if (!stop) umma_commit(&ctrl->accf[buf]);
       }
-      if (issued > 0) {
+      if (any) {
+        // every product issued has finished before tensor memory is freed
         umma_commit(&ctrl->acc);
-        drain_phase(&ctrl->acc, 0, 4000000000LL);     // products done before TMEM is freed
+        drain_phase(&ctrl->acc, 0, 4000000000LL);
       }
     }
   } else if (warp >= 4) {
-    // Producers: thread (r, p) builds vectors 4p .. 4p+3 of each step of row
-    // row0 + r (rows past N repeat row N-1, whose results are never stored).
+    // Producers: thread (r, p) builds vectors TsShape<LAYOUT>::vpt p .. of each step of
+    // row row0 + r (rows past N repeat row N-1, whose results are never
+    // stored); warps 4-7 (p = 0) then run the item's epilogue.
     const int pr = threadIdx.x - kTcProducer0;
     const int r = pr & (kTcRows - 1), p = pr >> 7;
-    const int64_t o = min(row0 + r, L.n - 1);
     const uint32_t m1 = (1u << L.b[0]) - 1u, m2 = L.nb == 2 ? (1u << L.b[1]) - 1u : 0u;
     const int b1 = L.b[0], b2 = L.nb == 2 ? L.b[1] : 0;
     const uint8_t* book2 = books + static_cast<size_t>(k1) * 16;
-    // index words of the next two steps in flight
-    uint32_t wa[3], wb[3], na[3] = {0u, 0u, 0u}, nbw[3] = {0u, 0u, 0u};
-    int sa = 0, sb = 0, nsa = 0, nsb = 0;
-    tcs_words<LAYOUT>(L, 0, o, kt0, p, wa, sa);
-    if (L.nb == 2) tcs_words<LAYOUT>(L, 1, o, kt0, p, wb, sb);
-    if (nkt > 1) {
-      tcs_words<LAYOUT>(L, 0, o, kt0 + 1, p, na, nsa);
-      if (L.nb == 2) tcs_words<LAYOUT>(L, 1, o, kt0 + 1, p, nbw, nsb);
-    }
-    for (int i = 0; i < nkt; ++i) {
-      const int s = i % kTcStages;
-      const uint32_t ph = (i / kTcStages) & 1;
-      uint32_t f1[4], f2[4];
+    int gs = 0, it = 0;
+    bool stop = false;
+    for (int item = blockIdx.x; item < g.nitems && !stop; item += gridDim.x, ++it) {
+      const int split = item / g.tiles;
+      const int row0 = (item - split * g.tiles) * kTcRows;
+      const int kt0 = split * g.kt_per_split;
+      const int nkt = min(g.num_kt, kt0 + g.kt_per_split) - kt0;
+      const int64_t o = min(row0 + r, L.n - 1);
+      // index words of the next kTsPf steps in flight (a register window
+      // that slides by one step per iteration)
+      uint32_t pw[kTsPf][2][3];
+      int psh[kTsPf][2];
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        f1[v] = tcs_field(wa, sa + v * b1, m1);
-        f2[v] = L.nb == 2 ? tcs_field(wb, sb + v * b2, m2) : 0u;
-      }
-#pragma unroll
-      for (int q = 0; q < 3; ++q) {
-        wa[q] = na[q];
-        wb[q] = nbw[q];
-      }
-      sa = nsa;
-      sb = nsb;
-      if (i + 2 < nkt) {
-        tcs_words<LAYOUT>(L, 0, o, kt0 + i + 2, p, na, nsa);
-        if (L.nb == 2) tcs_words<LAYOUT>(L, 1, o, kt0 + i + 2, p, nbw, nsb);
-      }
-      uint4 c[4];
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        c[v] = *reinterpret_cast<const uint4*>(books + static_cast<size_t>(f1[v]) * 16);
-        if (L.nb == 2) {
-          const uint4 c2 = *reinterpret_cast<const uint4*>(book2 + static_cast<size_t>(f2[v]) * 16);
-          c[v] = make_uint4(hadd2_u32(c[v].x, c2.x), hadd2_u32(c[v].y, c2.y), hadd2_u32(c[v].z, c2.z),
-                            hadd2_u32(c[v].w, c2.w));
+      for (int q = 0; q < kTsPf; ++q) {
+        pw[q][1][0] = pw[q][1][1] = pw[q][1][2] = 0u;
+        psh[q][1] = 0;
+        if (q < nkt) {
+          tcs_words<LAYOUT>(L, 0, o, kt0 + q, p, pw[q][0], psh[q][0]);
+          if (L.nb == 2) tcs_words<LAYOUT>(L, 1, o, kt0 + q, p, pw[q][1], psh[q][1]);
+        } else {
+          pw[q][0][0] = pw[q][0][1] = pw[q][0][2] = 0u;
+          psh[q][0] = 0;
         }
       }
-      if (!bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, g.budget)) break;
-      uint8_t* at = stages + s * kTcStage;
+      for (int i = 0; i < nkt; ++i, ++gs) {
+        const int s = gs % kTcStages;
+        const uint32_t ph = (gs / kTcStages) & 1;
+        uint32_t f1[TsShape<LAYOUT>::vpt], f2[TsShape<LAYOUT>::vpt];
 #pragma unroll
-      for (int v = 0; v < 4; ++v) *reinterpret_cast<uint4*>(at + sw128_off(r, 4 * p + v)) = c[v];
-      fence_proxy_async_smem();                        // visible to the tensor cores
-      mbar_arrive(&ctrl->full[s]);
-    }
-    // Epilogue (warps 4-7): lane quarter warp & 3, one output row per thread.
-    if (p == 0 && bounded_wait(&ctrl->acc, 0, abort_flag, g.status, g.budget)) {
+        for (int v = 0; v < TsShape<LAYOUT>::vpt; ++v) {
+          f1[v] = tcs_field(pw[0][0], psh[0][0] + v * b1, m1);
+          f2[v] = L.nb == 2 ? tcs_field(pw[0][1], psh[0][1] + v * b2, m2) : 0u;
+        }
+#pragma unroll
+        for (int q = 0; q + 1 < kTsPf; ++q) {
+#pragma unroll
+          for (int m = 0; m < 2; ++m) {
+            pw[q][m][0] = pw[q + 1][m][0];
+            pw[q][m][1] = pw[q + 1][m][1];
+            pw[q][m][2] = pw[q + 1][m][2];
+            psh[q][m] = psh[q + 1][m];
+          }
+        }
+        if (i + kTsPf < nkt) {
+          tcs_words<LAYOUT>(L, 0, o, kt0 + i + kTsPf, p, pw[kTsPf - 1][0], psh[kTsPf - 1][0]);
+          if (L.nb == 2) tcs_words<LAYOUT>(L, 1, o, kt0 + i + kTsPf, p, pw[kTsPf - 1][1], psh[kTsPf - 1][1]);
+        }
+        uint4 c[TsShape<LAYOUT>::vpt];
+#pragma unroll
+        for (int v = 0; v < TsShape<LAYOUT>::vpt; ++v) {
+          c[v] = *reinterpret_cast<const uint4*>(books + static_cast<size_t>(f1[v]) * 16);
+          if (L.nb == 2) {
+            const uint4 c2 = *reinterpret_cast<const uint4*>(book2 + static_cast<size_t>(f2[v]) * 16);
+            c[v] = make_uint4(hadd2_u32(c[v].x, c2.x), hadd2_u32(c[v].y, c2.y), hadd2_u32(c[v].z, c2.z),
+                              hadd2_u32(c[v].w, c2.w));
+          }
+        }
+        // warp-uniform: the warp publishes its rows of a step with one arrival
+        if (!__all_sync(0xffffffffu, bounded_wait(&ctrl->empty[s], ph ^ 1, abort_flag, g.status, g.budget))) {
+          stop = true;
+          break;
+        }
+        uint8_t* at = stages + s * kTcATile;
+#pragma unroll
+        for (int v = 0; v < TsShape<LAYOUT>::vpt; ++v) *reinterpret_cast<uint4*>(at + sw128_off(r, TsShape<LAYOUT>::vpt * p + v)) = c[v];
+        fence_proxy_async_smem();                      // visible to the tensor cores
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->full[s]);
+      }
+      if (stop || p != 0) continue;
+      // Epilogue (warps 4-7): lane quarter warp & 3, one output row per thread.
+      const int buf = it & 1;
+      if (!__all_sync(0xffffffffu, bounded_wait(&ctrl->accf[buf], (it >> 1) & 1, abort_flag, g.status, g.budget))) {
+        stop = true;
+        continue;
+      }
       tc_fence_after();
       uint32_t acc[16];
-      tmem_ld16(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16), acc);
+      float accs[16];
+      tmem_ld16(tmem + 16 * kTsNacc * buf + (static_cast<uint32_t>(32 * (warp & 3)) << 16), acc);
       tmem_wait_ld();
+#pragma unroll
+      for (int b = 0; b < 16; ++b) accs[b] = __uint_as_float(acc[b]);
+#pragma unroll
+      for (int q = 1; q < kTsNacc; ++q) {
+        tmem_ld16(tmem + 16 * (kTsNacc * buf + q) + (static_cast<uint32_t>(32 * (warp & 3)) << 16), acc);
+        tmem_wait_ld();
+#pragma unroll
+        for (int b = 0; b < 16; ++b) accs[b] += __uint_as_float(acc[b]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctrl->acce[buf]);
       const int row = row0 + r;
       if (row < L.n) {
         const float sc = L.scale ? h2f(L.scale[row]) : 1.0f;
         const float tb = (L.bias && split == 0) ? h2f(L.bias[row]) : 0.0f;
         const float ob = split == 0 ? out_bias_of(L.ob, row) : 0.0f;
-        for (int b = 0; b < g.batch; ++b) {
-          const float v = sc * (__uint_as_float(acc[b]) * g.xe[b]) + tb * g.xsum[b] + ob;
-          if (g.part) g.part[(static_cast<int64_t>(split) * g.batch + b) * L.n + row] = v;
-          else store_out(g.y, g.yt, b * g.ldy + row, v);
+#pragma unroll
+        for (int b = 0; b < kTcN; ++b) {
+          if (b < g.batch) {
+            const float v = sc * (accs[b] * g.xe[b]) + tb * g.xsum[b] + ob;
+            if (g.part) g.part[(static_cast<int64_t>(split) * g.batch + b) * L.n + row] = v;
+            else store_out(g.y, g.yt, b * g.ldy + row, v);
+          }
         }
       }
     }
@@ -484,7 +597,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemv_tcs_kernel(const __grid_co
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 32);
+    tmem_dealloc(tmem, kTsTmemCols);
   }
 }
 
@@ -584,7 +697,7 @@ TcLayout tc_layout(const Layer& L, int batch, bool small) {
     for (int ns = 1; ns <= std::min(8, t.num_kt); ++ns) {
       const int64_t ctas = static_cast<int64_t>(t.tiles) * ns;
       const int64_t waves = (ctas + sms - 1) / sms;
-      const double score = static_cast<double>(ctas) / static_cast<double>(waves * sms) - 0.02 * (ns - 1);
+      const double score = static_cast<double>(ctas) / static_cast<double>(waves * sms) - 0.005 * (ns - 1);
       if (score > best + 1e-9) {
         best = score;
         nsplit = ns;
@@ -678,11 +791,16 @@ vq_status launch_gemv_tc(const Layer& L, const GemvPlan& p, const void* x, bool 
   g.budget = tc_wait_budget();
   auto k = small ? (L.layout == VQ_IDX_TILE4 ? gemv_tcs_kernel<VQ_IDX_TILE4> : gemv_tcs_kernel<VQ_IDX_ROWS>)
                  : (L.layout == VQ_IDX_TILE4 ? gemv_tc_kernel<VQ_IDX_TILE4> : gemv_tc_kernel<VQ_IDX_ROWS>);
-  const int threads = small ? kTsThreads : kTcThreads;
+  const int threads = small ? (L.layout == VQ_IDX_TILE4 ? TsShape<VQ_IDX_TILE4>::threads
+                                                      : TsShape<VQ_IDX_ROWS>::threads)
+                            : kTcThreads;
   if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem)) != cudaSuccess)
     return cuda_status(e);
+  g.tiles = t.tiles;
+  g.nitems = t.tiles * t.nsplit;
+  const dim3 grid = small ? dim3(std::min(g.nitems, device_sm_count())) : dim3(t.tiles, t.nsplit);
   count_launch();
-  k<<<dim3(t.tiles, t.nsplit), threads, p.smem, stream>>>(xmap, g);
+  k<<<grid, threads, p.smem, stream>>>(xmap, g);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   if (t.nsplit > 1) {
     const int64_t total = static_cast<int64_t>(batch) * L.n;

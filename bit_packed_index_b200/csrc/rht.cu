@@ -46,6 +46,10 @@ __global__ void rht_kernel(const void* __restrict__ in, int in_t, int64_t ld_in,
                            const uint32_t* __restrict__ signs, int inverse, float scale,
                            void* __restrict__ out, int out_t, int64_t ld_out, const uint16_t* __restrict__ add) {
   extern __shared__ float hv[];
+  // launched as a programmatic dependent (launch_pdl): the input may be the
+  // previous kernel's output
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t row = blockIdx.y;
   const int64_t k0 = static_cast<int64_t>(blockIdx.x) * b;
   for (int i = threadIdx.x; i < b; i += blockDim.x) {
@@ -81,6 +85,8 @@ __global__ void __launch_bounds__(1024) rht_big_kernel(const void* __restrict__ 
                                                        float scale, void* __restrict__ out, int out_t,
                                                        int64_t ld_out, const uint16_t* __restrict__ add) {
   extern __shared__ float hv[];
+  asm volatile("griddepcontrol.wait;" ::: "memory");      // as rht_kernel
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int t = threadIdx.x, T = blockDim.x;
   const int64_t row = blockIdx.y;
   const int64_t k0 = static_cast<int64_t>(blockIdx.x) * b;
@@ -150,9 +156,8 @@ cudaError_t launch_rht(const void* in, vq_dtype in_t, int rows, int n, int64_t l
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    k<<<dim3(n / b, rows), T, smem, stream>>>(in, in_t, ld_in, b, signs, inverse ? 1 : 0, scale, out, out_t,
-                                              ld_out, add);
-    return cudaGetLastError();
+    return launch_pdl(k, dim3(n / b, rows), T, smem, stream, in, static_cast<int>(in_t), ld_in, b, signs,
+                      inverse ? 1 : 0, scale, out, static_cast<int>(out_t), ld_out, add);
   }
   const int smem = b * static_cast<int>(sizeof(float));
   cudaError_t e = cudaFuncSetAttribute(rht_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -160,9 +165,8 @@ cudaError_t launch_rht(const void* in, vq_dtype in_t, int rows, int n, int64_t l
   const int threads = std::min(1024, std::max(32, b / 2));
   const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b)));
   count_launch();
-  rht_kernel<<<dim3(n / b, rows), threads, smem, stream>>>(in, in_t, ld_in, b, signs, inverse ? 1 : 0, scale,
-                                                          out, out_t, ld_out, add);
-  return cudaGetLastError();
+  return launch_pdl(rht_kernel, dim3(n / b, rows), threads, smem, stream, in, static_cast<int>(in_t), ld_in, b,
+                    signs, inverse ? 1 : 0, scale, out, static_cast<int>(out_t), ld_out, add);
 }
 
 size_t rht_round256(size_t x) { return (x + 255) / 256 * 256; }

@@ -383,6 +383,9 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(LutSet S, cons
     for (int b = 0; b < RB8; ++b) sm100::tmem_st8(tbase + 8 * b, z);
     sm100::tmem_wait_st();
   }
+  // Launched as a programmatic dependent: x may come from the kernel before
+  // (a transform of it); everything above overlapped that kernel's tail.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   float xs_acc = 0.0f;   // warp 0: sum of x, one group per slice-0 task
 
   // Work items: the tasks of the whole rounds, then the last partial round's
@@ -652,6 +655,9 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_small_kernel(Layer L,
     for (int b = 0; b < RB8; ++b) sm100::tmem_st8(tbase + 8 * b, z);
     sm100::tmem_wait_st();
   }
+  // Launched as a programmatic dependent: x may come from the kernel before
+  // (a transform of it); everything above overlapped that kernel's tail.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   float xs_acc = 0.0f;
 
   for (int g = blockIdx.x; g < ntasks; g += gridDim.x) {
@@ -812,6 +818,9 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_pair_kernel(LutSet S,
     for (int b = 0; b < RB8; ++b) sm100::tmem_st8(tbase + 8 * b, z);
     sm100::tmem_wait_st();
   }
+  // Launched as a programmatic dependent: x may come from the kernel before
+  // (a transform of it); everything above overlapped that kernel's tail.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   float xs_acc = 0.0f;
 
   for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
@@ -949,8 +958,10 @@ __global__ void __launch_bounds__(256, 8) gemv_lut_finalize(const float* __restr
                                                             const float* __restrict__ xpart, int nparts,
                                                             int ntot, LutOut out, vq_dtype yt) {
   // Launched as a programmatic dependent of the table kernel: wait for that
-  // grid to complete and its writes to be visible (a no-op otherwise).
+  // grid to complete and its writes to be visible (a no-op otherwise).  The
+  // next launch may then be scheduled (it waits for this grid the same way).
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ float red[8][33];
   __shared__ float s_xsum;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1020,7 +1031,9 @@ cudaError_t launch_lut_set(const LutSet& S, const LutOut& out, int grid, const v
   float* part = ws;
   float* xpart = ws + static_cast<int64_t>(grid) * ntot;
   count_launch();
-  k<<<grid, kLutThreads, kLutSmem, stream>>>(S, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, part, xpart);
+  e = launch_pdl(k, grid, kLutThreads, kLutSmem, stream, S, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, part,
+                 xpart);
+  if (e != cudaSuccess) return e;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return launch_finalize(part, xpart, grid, ntot, out, yt, stream);
 }
@@ -1047,9 +1060,8 @@ cudaError_t launch_lut_small_t(const Layer& L, const GemvPlan& p, const void* x,
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
   if (e != cudaSuccess) return e;
   count_launch();
-  k<<<p.grid_x, kLutThreads, p.smem, stream>>>(L, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, ws,
-                                               ws + static_cast<int64_t>(p.grid_x) * L.n);
-  return cudaGetLastError();
+  return launch_pdl(k, p.grid_x, kLutThreads, p.smem, stream, L, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0,
+                    ws, ws + static_cast<int64_t>(p.grid_x) * L.n);
 }
 
 bool lut_pair_path(const Layer& L) {
@@ -1064,9 +1076,8 @@ cudaError_t launch_lut_pair_set(const LutSet& S, int grid, int smem, const void*
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   count_launch();
-  k<<<grid, kLutThreads, smem, stream>>>(S, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, ws,
-                                         ws + static_cast<int64_t>(grid) * S.row0[S.nl]);
-  return cudaGetLastError();
+  return launch_pdl(k, grid, kLutThreads, smem, stream, S, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, ws,
+                    ws + static_cast<int64_t>(grid) * S.row0[S.nl]);
 }
 
 template <int RB8, int D, int B2>
@@ -1123,19 +1134,26 @@ bool lut_supported(const Layer& L) {
 
 cudaError_t launch_gemv_lut_row(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, void* y,
                                 vq_dtype yt, float* ws, cudaStream_t stream);
-// Measured crossovers against the split-K kernel on tiled layers (B200): a
-// 2^16 book pays up to batch 2 (70B gate: 187 against 352 us at B = 2, 276
-// against 263 at B = 3); books of <= 2^12 entries up to batch 8 and beyond
-// (405B q at B = 8: 484 against 872 us).
+// Measured crossovers against the tensor-core batched kernels (gemvtc.cu) on
+// tiled layers (B200, L2 flushed): the table pass costs about the same per
+// row of x whatever the batch, the tensor-core kernels about the same per
+// call.  A 2^16 book pays up to batch 2 (70B gate: 169 us at B = 2; the
+// tensor-core kernel 190 at any batch).  Books of <= 2^12 entries: up to
+// batch 3 on short rows (8B up, 512 vectors per row: 73 us at B = 3 against
+// 80) and batch 5 on long ones (405B q, 2731 vectors: 62 us per row of x
+// against 309; 405B gate: 136 per row against 856).
 constexpr int kLutMaxBatchBig = 2;
-constexpr int kLutMaxBatchSmall = 8;
+constexpr int kLutMaxBatchSmallShort = 3;
+constexpr int kLutMaxBatchSmallLong = 5;
 
 // Largest batch served by running the batch-1 table kernel once per row of x
-// (each run reads the index streams again); larger batches take the split-K
-// gather kernel.  Environment override for measurements: VQ_LUT_MAX_BATCH.
+// (each run reads the index streams again); larger batches take the
+// tensor-core kernels, else the split-K gather kernel.  Environment override
+// for measurements: VQ_LUT_MAX_BATCH.
 int lut_batch_limit(const Layer& L, bool big) {
   if (const char* env = std::getenv("VQ_LUT_MAX_BATCH")) return std::atoi(env);
-  return big ? kLutMaxBatchBig : kLutMaxBatchSmall;
+  if (big) return kLutMaxBatchBig;
+  return L.nvec > 1024 ? kLutMaxBatchSmallLong : kLutMaxBatchSmallShort;
 }
 
 bool plan_gemv_lut(const Layer& L, int batch, size_t ws_cap, GemvPlan* p) {

@@ -12,6 +12,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "vq.h"
 
 namespace vqk {
@@ -52,6 +54,27 @@ int device_sm_count();
 int device_smem_optin();               // max dynamic shared memory per block, bytes
 
 __host__ __device__ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Launch `kernel` as a programmatic dependent of the previous work on the
+// stream: it may start while that kernel drains, and must execute
+// griddepcontrol.wait before it reads what that kernel wrote or writes what
+// that kernel reads.  (Without a trigger in the previous kernel it starts
+// when that kernel completes, as a plain launch would.)
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ---------------------------------------------------------------------------
 // Kernel launchers (one per .cu file).

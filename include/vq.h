@@ -207,20 +207,24 @@ VQ_API vq_status vq_gemv_workspace_size(const vq_layer_desc* layer, int32_t batc
  * entries the indices select.  That rounding adds about 2^-12 relative error
  * per term, inside the same tolerance as long as the codebook's values are
  * normal fp16 numbers (|c| >= 2^-14).  Books of up to 2^12 entries (one or
- * two, d = 6 or 8) get a table kernel without slices.  Batches of 2 (2^16
- * book) or up to 8 (small books) run one table pass per row of x.
- * Batches of 2..16 (3..16 in the tiled order) of layers with one 2^16-entry
- * d = 8 book run the tensor-core kernel: per 128 rows of W and step of eight
- * vectors, the centroids are gathered into a shared-memory tile and
- * multiplied on the tcgen05 tensor cores with x, each row of x scaled by a
- * power of two into fp16 (exact products, fp32 accumulation); values of a
- * row below 2^-29 of its largest lose precision as fp16 subnormals.  The
- * first 32-bit word of its workspace is a status word: VQ_OK, or
- * VQ_ERR_TIMEOUT if a bounded device-side wait gave up (readable after the
- * stream completes).  Every other case runs the split-K gather kernel, which
- * reads either index order.  The environment variables VQ_LUT_MAX_BATCH (0
- * turns the table kernels off) and VQ_TC_MIN_BATCH (above 16 turns the
- * tensor-core kernel off) move those limits, for measurements.
+ * two, d = 6 or 8) get a table kernel without slices.  Tiled layers run one
+ * table pass per row of x up to batch 2 (2^16 book), 3 (small books, rows of
+ * at most 1024 vectors) or 5 (small books, longer rows).
+ * Larger batches (from 2 in row order) of layers with one 2^16-entry d = 8
+ * book, or with books of up to 2^12 + 2^12 entries and d = 6 or 8 (from 3 in
+ * row order), run the tensor-core kernels: per 128 rows of W and step of
+ * eight vectors, the centroids (the sum of both books' centroids, rounded
+ * once to fp16) are gathered into a shared-memory tile and multiplied on the
+ * tcgen05 tensor cores with x, each row of x scaled by a power of two into
+ * fp16 (exact products, fp32 accumulation); values of a row below 2^-29 of
+ * its largest lose precision as fp16 subnormals.  The first 32-bit word of
+ * their workspace is a status word: VQ_OK, or VQ_ERR_TIMEOUT if a bounded
+ * device-side wait gave up (readable after the stream completes).  Every
+ * other case runs the split-K gather kernel, which reads either index order.
+ * The environment variables VQ_LUT_MAX_BATCH (0 turns the table kernels
+ * off), VQ_TC_MIN_BATCH and VQ_TCS_MIN_BATCH (above 16 turns the 2^16-book or
+ * the small-book tensor-core kernel off) move those limits, for
+ * measurements.
  * Errors: VQ_ERR_INVALID_ARG, VQ_ERR_UNSUPPORTED (batch > 16), VQ_ERR_ALIGNMENT
  * (x or y not aligned to its element size), VQ_ERR_WORKSPACE, VQ_ERR_CUDA.
  */

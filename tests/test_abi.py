@@ -151,6 +151,20 @@ def test_table_batch_limit_needs_no_device(lib, monkeypatch):
     assert not table(n.value)
 
 
+def test_small_book_table_limit_needs_no_device(lib):
+    """Tiled layers with a 2^12 book take the per-row table passes up to
+    batch 3 when rows hold at most 1024 vectors and up to batch 5 when they
+    hold more; larger batches plan the small-book tensor-core kernel (status
+    word, scaled x, per-row scales; no per-block row sums)."""
+    n = C.c_size_t(0)
+    table = lambda v: v > 0 and v % (1001 * 4) == 0
+    for kin, last in ((8 * 1024, 3), (8 * 1025, 5)):
+        d = _tiled_desc(n=1000, kin=kin, b=12)
+        for batch in range(1, 9):
+            assert lib.vq_gemv_workspace_size(C.byref(d), batch, C.byref(n)) == vq.VQ_OK
+            assert table(n.value) == (batch <= last), (kin, batch, n.value)
+
+
 def test_encode_workspace_and_validation_need_no_device(lib):
     """vq_encode_workspace_size: control words + per book the prepared operand
     (K padded to 1024, 32 bytes per centroid) and the fp64 copy (8 bytes per
