@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(Layer L, uint16_t* 
                                                              int64_t ldw, int smem_mask,
                                                              int vec_store) {
   extern __shared__ __align__(16) uint8_t smem[];
+  // reads only the layer: a programmatic dependent may be scheduled at once
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   BookView bv[2];
   {
     size_t off = 0;
@@ -122,23 +124,24 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(Layer L, uint16_t* 
 
 template <int D, int NB>
 cudaError_t launch_dq(const Layer& L, uint16_t* w, int64_t ldw, int smem_mask, size_t smem,
-                      int vec_store, int grid, cudaStream_t stream) {
+                      int vec_store, int grid, cudaStream_t stream, bool pdl) {
   auto k = dequant_kernel<D, NB>;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = set_func_attr(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
   count_launch();
+  if (pdl) return launch_pdl(k, grid, kDqThreads, smem, stream, L, w, ldw, smem_mask, vec_store);
   k<<<grid, kDqThreads, smem, stream>>>(L, w, ldw, smem_mask, vec_store);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-vq_status launch_dequant(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream) {
+vq_status launch_dequant(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream, bool pdl) {
   if (L.n == 0 || L.kin == 0) return VQ_OK;
-  if (L.layout == VQ_IDX_TILE4) return launch_dequant_tile4(L, w, ldw, stream);
+  if (L.layout == VQ_IDX_TILE4) return launch_dequant_tile4(L, w, ldw, stream, pdl);
   int smem_mask = 0;
   const size_t smem = stage_plan(L, std::min<size_t>(kDqSmemBooks, device_smem_optin()), &smem_mask);
   const int vec_store = aligned(w, 16) && (ldw % 8 == 0);
@@ -147,15 +150,30 @@ vq_status launch_dequant(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t 
   cudaError_t e;
   const int D = (L.d == 8) ? 8 : (L.d == 6 ? 6 : 0);
   if (L.nb == 1) {
-    e = D == 8 ? launch_dq<8, 1>(L, w, ldw, smem_mask, smem, vec_store, grid, stream)
-      : D == 6 ? launch_dq<6, 1>(L, w, ldw, smem_mask, smem, vec_store, grid, stream)
-               : launch_dq<0, 1>(L, w, ldw, smem_mask, smem, vec_store, grid, stream);
+    e = D == 8 ? launch_dq<8, 1>(L, w, ldw, smem_mask, smem, vec_store, grid, stream, pdl)
+      : D == 6 ? launch_dq<6, 1>(L, w, ldw, smem_mask, smem, vec_store, grid, stream, pdl)
+               : launch_dq<0, 1>(L, w, ldw, smem_mask, smem, vec_store, grid, stream, pdl);
   } else {
-    e = D == 8 ? launch_dq<8, 2>(L, w, ldw, smem_mask, smem, vec_store, grid, stream)
-      : D == 6 ? launch_dq<6, 2>(L, w, ldw, smem_mask, smem, vec_store, grid, stream)
-               : launch_dq<0, 2>(L, w, ldw, smem_mask, smem, vec_store, grid, stream);
+    e = D == 8 ? launch_dq<8, 2>(L, w, ldw, smem_mask, smem, vec_store, grid, stream, pdl)
+      : D == 6 ? launch_dq<6, 2>(L, w, ldw, smem_mask, smem, vec_store, grid, stream, pdl)
+               : launch_dq<0, 2>(L, w, ldw, smem_mask, smem, vec_store, grid, stream, pdl);
   }
   return cuda_status(e);
+}
+
+Layer layer_rows(const Layer& L, int n0, int n1) {
+  Layer v = L;
+  v.n = n1 - n0;
+  for (int m = 0; m < 2; ++m) {
+    if (L.layout == VQ_IDX_TILE4)   // records of row o start at bit 4 o b of every tile
+      v.idx[m] = L.idx[m] + static_cast<int64_t>(n0) * 4 * L.b[m] / 32;
+    else
+      v.idx[m] = L.idx[m] + static_cast<int64_t>(n0) * L.rw[m];
+  }
+  if (L.scale) v.scale = L.scale + n0;
+  if (L.bias) v.bias = L.bias + n0;
+  if (L.ob) v.ob = L.ob + n0;
+  return v;
 }
 
 }  // namespace vqk

@@ -1043,7 +1043,7 @@ vq_status vq_encode(const vq_encode_desc* desc, void* workspace, size_t workspac
 
   const int smem = static_cast<int>(sizeof(EncCtrl)) + 1024 + kEncATile + kEncStages * kEncBlockBytes;
   auto tck = p.hw ? enc_tc_kernel<true> : enc_tc_kernel<false>;
-  e = cudaFuncSetAttribute(tck, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  e = set_func_attr(reinterpret_cast<const void*>(tck), cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_status(e);
   int* list = reinterpret_cast<int*>(ws + p.off_list);
   for (int m = 0; m < p.nb; ++m) {
@@ -1102,7 +1102,7 @@ vq_status vq_encode(const vq_encode_desc* desc, void* workspace, size_t workspac
     const int xsmem = kEncExactTile * p.d * static_cast<int>(sizeof(double));
     auto xk = p.hw ? enc_exact_kernel<true> : enc_exact_kernel<false>;
     if (m == 0) {
-      e = cudaFuncSetAttribute(xk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = set_func_attr(reinterpret_cast<const void*>(xk), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kEncExactTile * kEncMaxD * static_cast<int>(sizeof(double)));
       if (e != cudaSuccess) return cuda_status(e);
     }

@@ -280,6 +280,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctrl->tmem_base;
+  // As a programmatic dependent (the staged form's slabs), the weight tiles
+  // come from the launch before: wait for it; then let the next launch (the
+  // next slab's dequantisation) be scheduled.  No-ops for a plain launch.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == 0) {
     if (lane == 0) {                                   // TMA producer
@@ -603,11 +608,12 @@ GemmLayout layout_for(const Layer& L, int m, bool x_fp16) {
 
 template <int MODE, int B1, int B2, int MSUB>
 cudaError_t launch_kernel(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g,
-                          size_t smem, dim3 grid, cudaStream_t stream) {
+                          size_t smem, dim3 grid, cudaStream_t stream, bool pdl = false) {
   auto k = vq_gemm_kernel<MODE, B1, B2, MSUB>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cudaError_t e = set_func_attr(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   count_launch();
+  if (pdl) return launch_pdl(k, grid, kThreads, smem, stream, ma, mb, g);
   k<<<grid, kThreads, smem, stream>>>(ma, mb, g);
   return cudaGetLastError();
 }
@@ -631,8 +637,8 @@ void choose_tiles(int m, int n, int sms, int* msub, int* bn) {
 
 template <int MSUB>
 cudaError_t dispatch(const Layer& L, int mode, const CUtensorMap& ma, const CUtensorMap& mb,
-                     const GemmArgs& g, size_t smem, dim3 grid, cudaStream_t stream) {
-  if (mode == kStaged) return launch_kernel<kStaged, 0, 0, MSUB>(ma, mb, g, smem, grid, stream);
+                     const GemmArgs& g, size_t smem, dim3 grid, cudaStream_t stream, bool pdl = false) {
+  if (mode == kStaged) return launch_kernel<kStaged, 0, 0, MSUB>(ma, mb, g, smem, grid, stream, pdl);
   if (L.d == 8 && L.nb == 1 && L.b[0] == 16)
     return launch_kernel<kFused, 16, 0, MSUB>(ma, mb, g, smem, grid, stream);
   if (L.d == 8 && L.nb == 2 && L.b[0] == 16 && L.b[1] == 8)
@@ -715,6 +721,25 @@ size_t gemm_workspace_bytes(const Layer& L, int m, bool x_fp16) {
   return layout_for(L, m, x_fp16).total;
 }
 
+// Closes the staged form's chain of dependent launches.  A slab's product
+// waits only for its own dequantisation, so products can finish out of
+// order; this plain launch starts after all of them, so whatever the stream
+// runs next sees the whole of y.
+__global__ void gemm_join() {}
+
+// Slabs of the staged form.  One by default: splitting measured slower at
+// every size tried (8192^2, M = 2048: 299 us in one slab, 355 / 421 / 736 in
+// 2 / 4 / 8), because a product's CTAs hold most of an SM's shared memory,
+// so the next slab's product cannot share SMs with the running one and the
+// slabs run one after another, each on a partial wave.  VQ_GEMM_SLABS sets
+// the count, for measurements (each slab a whole number of tile widths).
+int gemm_slabs(int n, int bn) {
+  const int tiles = (n + bn - 1) / bn;
+  int s = 1;
+  if (const char* env = std::getenv("VQ_GEMM_SLABS")) s = std::max(1, std::atoi(env));
+  return std::max(1, std::min(s, tiles / 2));
+}
+
 vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t ldx, void* y,
                       vq_dtype yt, int64_t ldy, void* ws, size_t ws_bytes, cudaStream_t stream) {
   if (L.kin == 0) return launch_empty_rows(L, y, yt, ldy, m, stream);
@@ -753,23 +778,25 @@ vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t
       if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
     }
   }
-  if (lay.mode == kStaged) {
-    vq_status st = launch_dequant(L, what, lay.kp, stream);
-    if (st != VQ_OK) return st;
-  }
   int msub = 1, bn = BN;
   choose_tiles(m, L.n, device_sm_count(), &msub, &bn);
+  // Staged form: W_hat is written in slabs of output rows (one by default,
+  // see gemm_slabs).  Each slab's product is launched as a programmatic
+  // dependent of its dequantisation, and the next slab's dequantisation as a
+  // dependent of that product, so that the two may run side by side.
+  const int nslab = lay.mode == kStaged ? gemm_slabs(L.n, bn) : 1;
+  const int slab_rows = lay.mode == kStaged ? ((L.n + nslab - 1) / nslab + bn - 1) / bn * bn : L.n;
+  if (lay.mode == kStaged) {
+    vq_status st = launch_dequant(layer_rows(L, 0, std::min(L.n, slab_rows)), what, lay.kp, stream);
+    if (st != VQ_OK) return st;
+  }
   CUtensorMap ma, mb;
   if (lay.copy_x) {
     if (!make_map(&ma, x16, L.kin, m, lay.kp, BM)) return VQ_ERR_CUDA;
   } else {
     if (!make_map(&ma, x, L.kin, m, ldx, BM)) return VQ_ERR_CUDA;
   }
-  if (lay.mode == kStaged) {
-    if (!make_map(&mb, what, L.kin, L.n, lay.kp, bn)) return VQ_ERR_CUDA;
-  } else {
-    mb = ma;
-  }
+  if (lay.mode != kStaged) mb = ma;
 
   GemmArgs g{};
   g.L = L;
@@ -804,9 +831,34 @@ vq_status launch_gemm(const Layer& L, const void* x, bool x_fp16, int m, int64_t
   const size_t smem = fixed + static_cast<size_t>(g.stages) * kStageBytes + g.book_bytes;
   g.bn = bn;
   g.idesc = f16_idesc(BM, bn);
-  dim3 grid((m + BM * msub - 1) / (BM * msub), (L.n + bn - 1) / bn);
-  return cuda_status(msub == 2 ? dispatch<2>(L, lay.mode, ma, mb, g, smem, grid, stream)
-                               : dispatch<1>(L, lay.mode, ma, mb, g, smem, grid, stream));
+  if (lay.mode != kStaged) {
+    dim3 grid((m + BM * msub - 1) / (BM * msub), (L.n + bn - 1) / bn);
+    return cuda_status(msub == 2 ? dispatch<2>(L, lay.mode, ma, mb, g, smem, grid, stream)
+                                 : dispatch<1>(L, lay.mode, ma, mb, g, smem, grid, stream));
+  }
+  for (int n0 = 0; n0 < L.n; n0 += slab_rows) {
+    const int n1 = std::min(L.n, n0 + slab_rows);
+    GemmArgs gs = g;
+    gs.L = layer_rows(L, n0, n1);
+    gs.y = static_cast<uint8_t*>(y) + static_cast<size_t>(n0) * (yt == VQ_FP32 ? 4 : 2);
+    uint16_t* wslab = what + static_cast<size_t>(n0) * lay.kp;
+    if (!make_map(&mb, wslab, L.kin, n1 - n0, lay.kp, bn)) return VQ_ERR_CUDA;
+    dim3 grid((m + BM * msub - 1) / (BM * msub), (n1 - n0 + bn - 1) / bn);
+    cudaError_t e = msub == 2 ? dispatch<2>(gs.L, kStaged, ma, mb, gs, smem, grid, stream, true)
+                              : dispatch<1>(gs.L, kStaged, ma, mb, gs, smem, grid, stream, true);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (n1 < L.n) {
+      vq_status st = launch_dequant(layer_rows(L, n1, std::min(L.n, n1 + slab_rows)),
+                                    what + static_cast<size_t>(n1) * lay.kp, lay.kp, stream, true);
+      if (st != VQ_OK) return st;
+    }
+  }
+  if (nslab > 1) {
+    count_launch();
+    gemm_join<<<1, 32, 0, stream>>>();
+    return cuda_status(cudaGetLastError());
+  }
+  return VQ_OK;
 }
 
 }  // namespace vqk

@@ -204,7 +204,7 @@ cudaError_t launch_bt(const Layer& L, const GemvPlan& p, const void* x, bool x_f
                       int64_t ldx, void* y, vq_dtype yt, int64_t ldy, float* ws,
                       cudaStream_t stream) {
   auto k = L.layout == VQ_IDX_TILE4 ? gemv_kernel<D, NB, BT, true> : gemv_kernel<D, NB, BT, false>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
+  cudaError_t e = set_func_attr(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.grid_x, p.nsplit);
   count_launch();

@@ -280,10 +280,10 @@ template <int D, int B1, int B2, bool SM1, bool SM2>
 cudaError_t launch1(const Layer& L, const GemvPlan& p, const void* x, bool xf, void* y,
                     vq_dtype yt, float* ws, cudaStream_t stream) {
   auto k = gemv1_kernel<D, B1, B2, SM1, SM2>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
+  cudaError_t e = set_func_attr(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
   if (e != cudaSuccess) return e;
   if (!SM1) {   // L2-served book: keep shared memory small so L1 is as large as possible
-    e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 10);
+    e = set_func_attr(reinterpret_cast<const void*>(k), cudaFuncAttributePreferredSharedMemoryCarveout, 10);
     if (e != cudaSuccess) return e;
   }
   dim3 grid(p.grid_x, p.nsplit);

@@ -606,19 +606,51 @@ __global__ void __launch_bounds__(TsShape<LAYOUT>::threads, 1) gemv_tcs_kernel(c
 // value overflows fp16 and values above max * 2^-29 stay exact.  x' holds
 // vector j of the layer (d elements) at columns 8 j .. 8 j + d - 1 and zeros
 // in the rest of its 8 columns (d = 8: x' is x itself, scaled).
-__global__ void gemv_tc_prep(const uint16_t* __restrict__ x, int x_fp16, int64_t ldx, int kin, int kp, int batch,
-                             int d, uint16_t* __restrict__ xh, float* __restrict__ xe, float* __restrict__ xsum) {
-  __shared__ float s_max[32], s_sum[32];
-  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// Grid (16, kPrepChunks): every block of row b reads the whole row for its
+// maximum and sum (the same order in each, so the same result), then writes
+// its share of the row's columns, 8 at a time; block (b, 0) stores 2^e_b and
+// the sum.  vec: x is 16-byte aligned with ldx a multiple of 8.
+constexpr int kPrepChunks = 8;
+
+__global__ void __launch_bounds__(256) gemv_tc_prep(const uint16_t* __restrict__ x, int x_fp16, int64_t ldx,
+                                                    int kin, int kp, int batch, int d, int vec,
+                                                    uint16_t* __restrict__ xh, float* __restrict__ xe,
+                                                    float* __restrict__ xsum) {
+  __shared__ float s_max[8], s_sum[8];
+  const int b = blockIdx.x, c = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool live = b < batch;
+  const uint16_t* xr = x + static_cast<int64_t>(b) * ldx;
+  auto val = [&](uint16_t u) { return x_fp16 ? h2f(u) : bf2f(u); };
   float mx = 0.0f, sm = 0.0f;
-  if (live)
-    for (int k = tid; k < kin; k += blockDim.x) {
-      const uint16_t u = x[b * ldx + k];
-      const float v = x_fp16 ? h2f(u) : bf2f(u);
-      mx = fmaxf(mx, fabsf(v));
-      sm += v;
+  if (live) {
+    if (vec) {
+      for (int k = 8 * tid; k < kin; k += 8 * 256) {
+        if (k + 8 <= kin) {
+          const uint4 q = __ldg(reinterpret_cast<const uint4*>(xr + k));
+          const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float lo = val(static_cast<uint16_t>(w[i] & 0xFFFFu)), hi = val(static_cast<uint16_t>(w[i] >> 16));
+            mx = fmaxf(mx, fmaxf(fabsf(lo), fabsf(hi)));
+            sm += lo;
+            sm += hi;
+          }
+        } else {
+          for (int i = k; i < kin; ++i) {
+            const float v = val(xr[i]);
+            mx = fmaxf(mx, fabsf(v));
+            sm += v;
+          }
+        }
+      }
+    } else {
+      for (int k = tid; k < kin; k += 256) {
+        const float v = val(xr[k]);
+        mx = fmaxf(mx, fabsf(v));
+        sm += v;
+      }
     }
+  }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
@@ -626,37 +658,40 @@ __global__ void gemv_tc_prep(const uint16_t* __restrict__ x, int x_fp16, int64_t
   }
   if (lane == 0) { s_max[warp] = mx; s_sum[warp] = sm; }
   __syncthreads();
-  if (warp == 0) {
-    mx = lane < static_cast<int>(blockDim.x / 32) ? s_max[lane] : 0.0f;
-    sm = lane < static_cast<int>(blockDim.x / 32) ? s_sum[lane] : 0.0f;
+  mx = 0.0f;
+  sm = 0.0f;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      sm += __shfl_xor_sync(0xffffffffu, sm, off);
-    }
-    if (lane == 0) { s_max[0] = mx; s_sum[0] = sm; }
+  for (int w = 0; w < 8; ++w) {
+    mx = fmaxf(mx, s_max[w]);
+    sm += s_sum[w];
   }
-  __syncthreads();
-  mx = s_max[0];
   // max = m * 2^E with 0.5 <= m < 1; e = E - 15, kept in [-126, 127] (values
   // below 2^-111 scale to fp16 subnormals or zero).
   int e = 0;
   if (mx > 0.0f && mx < INFINITY) e = max(-126, min(127, static_cast<int>(__float_as_uint(mx) >> 23) - 126 - 15));
   const float f1 = __uint_as_float(static_cast<uint32_t>(127 - e / 2) << 23);
   const float f2 = __uint_as_float(static_cast<uint32_t>(127 - (e - e / 2)) << 23);
-  for (int k = tid; k < kp; k += blockDim.x) {
-    float v = 0.0f;
-    const int e8 = k & 7;
-    const int src = (k >> 3) * d + e8;               // element of x in column k
-    if (live && e8 < d && src < kin) {
-      const uint16_t u = x[b * ldx + src];
-      v = (x_fp16 ? h2f(u) : bf2f(u)) * f1 * f2;
+  // this block's columns: groups of 8 (one vector of the layer each)
+  const int ngroups = kp / 8;
+  const int g0 = c * ngroups / kPrepChunks, g1 = (c + 1) * ngroups / kPrepChunks;
+  for (int g = g0 + tid; g < g1; g += 256) {
+    uint32_t h[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float v2[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int e8 = 2 * i + q;
+        const int src = g * d + e8;                  // element of x in column 8 g + e8
+        v2[q] = (live && e8 < d && src < kin) ? val(xr[src]) * f1 * f2 : 0.0f;
+      }
+      h[i] = f2h(v2[0]) | (static_cast<uint32_t>(f2h(v2[1])) << 16);
     }
-    xh[static_cast<int64_t>(b) * kp + k] = f2h(v);
+    *reinterpret_cast<uint4*>(xh + static_cast<int64_t>(b) * kp + 8 * g) = make_uint4(h[0], h[1], h[2], h[3]);
   }
-  if (tid == 0) {
+  if (c == 0 && tid == 0) {
     xe[b] = live ? __uint_as_float(static_cast<uint32_t>(127 + e) << 23) : 0.0f;
-    xsum[b] = live ? s_sum[0] : 0.0f;
+    xsum[b] = live ? sm : 0.0f;
   }
 }
 
@@ -771,8 +806,9 @@ vq_status launch_gemv_tc(const Layer& L, const GemvPlan& p, const void* x, bool 
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), stream);
   if (e != cudaSuccess) return cuda_status(e);
   count_launch();
-  gemv_tc_prep<<<kTcN, 256, 0, stream>>>(static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, ldx, L.kin, t.kp, batch,
-                                          L.d, xh, xe, xsum);
+  const int vec = aligned(x, 16) && ldx % 8 == 0;
+  gemv_tc_prep<<<dim3(kTcN, kPrepChunks), 256, 0, stream>>>(static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, ldx,
+                                                            L.kin, t.kp, batch, L.d, vec, xh, xe, xsum);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   CUtensorMap xmap;
   if (!make_map_f16_sw128(&xmap, xh, t.kp, kTcN, t.kp, kTcN)) return VQ_ERR_CUDA;
@@ -794,7 +830,7 @@ vq_status launch_gemv_tc(const Layer& L, const GemvPlan& p, const void* x, bool 
   const int threads = small ? (L.layout == VQ_IDX_TILE4 ? TsShape<VQ_IDX_TILE4>::threads
                                                       : TsShape<VQ_IDX_ROWS>::threads)
                             : kTcThreads;
-  if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem)) != cudaSuccess)
+  if ((e = set_func_attr(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem)) != cudaSuccess)
     return cuda_status(e);
   g.tiles = t.tiles;
   g.nitems = t.tiles * t.nsplit;

@@ -153,14 +153,14 @@ cudaError_t launch_rht(const void* in, vq_dtype in_t, int rows, int n, int64_t l
     const int smem = 32 * E < b ? b * static_cast<int>(sizeof(float)) : 0;
     const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b)));
     auto k = E == 8 ? rht_big_kernel<8> : E == 16 ? rht_big_kernel<16> : rht_big_kernel<32>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = set_func_attr(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     count_launch();
     return launch_pdl(k, dim3(n / b, rows), T, smem, stream, in, static_cast<int>(in_t), ld_in, b, signs,
                       inverse ? 1 : 0, scale, out, static_cast<int>(out_t), ld_out, add);
   }
   const int smem = b * static_cast<int>(sizeof(float));
-  cudaError_t e = cudaFuncSetAttribute(rht_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = set_func_attr(reinterpret_cast<const void*>(rht_kernel), cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int threads = std::min(1024, std::max(32, b / 2));
   const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b)));

@@ -73,6 +73,8 @@ __global__ void repack_tile4_kernel(const uint32_t* __restrict__ src, int64_t sr
 template <int D, int NB>
 __global__ void dequant_tile4_kernel(Layer L, uint16_t* __restrict__ w, int64_t ldw, int vec_store,
                                      int smem_mask) {
+  // reads only the layer: a programmatic dependent may be scheduled at once
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ __align__(16) uint8_t smem[];
   BookView bv[2];
   {
@@ -163,12 +165,12 @@ __global__ void dequant_tile4_kernel(Layer L, uint16_t* __restrict__ w, int64_t 
 constexpr size_t kDq4SmemBooks = 96 * 1024;   // stage books up to this size
 
 template <int D, int NB>
-cudaError_t launch_dq4(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream) {
+cudaError_t launch_dq4(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream, bool pdl) {
   int smem_mask = 0;
   const size_t smem = stage_plan(L, std::min<size_t>(kDq4SmemBooks, device_smem_optin()), &smem_mask);
   auto k = dequant_tile4_kernel<D, NB>;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaError_t e = set_func_attr(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
   const int per_sm = smem ? std::max(1, std::min(8, static_cast<int>((228 * 1024) / (smem + 1024)))) : 8;
@@ -178,6 +180,7 @@ cudaError_t launch_dq4(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t st
   // 2: 16-byte rows of 8 halves aligned; 1: 4-byte pairs aligned (rows of even length)
   const int vec_store = (aligned(w, 16) && ldw % 8 == 0) ? 2 : (aligned(w, 4) && ldw % 2 == 0) ? 1 : 0;
   count_launch();
+  if (pdl) return launch_pdl(k, grid, 256, smem, stream, L, w, ldw, vec_store, smem_mask);
   k<<<grid, 256, smem, stream>>>(L, w, ldw, vec_store, smem_mask);
   return cudaGetLastError();
 }
@@ -197,15 +200,15 @@ vq_status launch_repack_tile4(const Layer& L, uint32_t* const dst[2], const int6
   return VQ_OK;
 }
 
-vq_status launch_dequant_tile4(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream) {
+vq_status launch_dequant_tile4(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream, bool pdl) {
   if (L.n == 0 || L.kin == 0) return VQ_OK;
   cudaError_t e;
   if (L.nb == 1)
-    e = L.d == 8 ? launch_dq4<8, 1>(L, w, ldw, stream)
-      : L.d == 6 ? launch_dq4<6, 1>(L, w, ldw, stream) : launch_dq4<0, 1>(L, w, ldw, stream);
+    e = L.d == 8 ? launch_dq4<8, 1>(L, w, ldw, stream, pdl)
+      : L.d == 6 ? launch_dq4<6, 1>(L, w, ldw, stream, pdl) : launch_dq4<0, 1>(L, w, ldw, stream, pdl);
   else
-    e = L.d == 8 ? launch_dq4<8, 2>(L, w, ldw, stream)
-      : L.d == 6 ? launch_dq4<6, 2>(L, w, ldw, stream) : launch_dq4<0, 2>(L, w, ldw, stream);
+    e = L.d == 8 ? launch_dq4<8, 2>(L, w, ldw, stream, pdl)
+      : L.d == 6 ? launch_dq4<6, 2>(L, w, ldw, stream, pdl) : launch_dq4<0, 2>(L, w, ldw, stream, pdl);
   return cuda_status(e);
 }
 
@@ -1025,7 +1028,7 @@ template <int RB8, int LB>
 cudaError_t launch_lut_set(const LutSet& S, const LutOut& out, int grid, const void* x, bool x_fp16,
                            vq_dtype yt, float* ws, cudaStream_t stream) {
   auto k = gemv_lut_kernel<RB8, LB>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutSmem);
+  cudaError_t e = set_func_attr(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize, kLutSmem);
   if (e != cudaSuccess) return e;
   const int ntot = S.row0[S.nl];
   float* part = ws;
@@ -1057,7 +1060,7 @@ template <int RB8, int D, int NB>
 cudaError_t launch_lut_small_t(const Layer& L, const GemvPlan& p, const void* x, bool x_fp16, float* ws,
                                cudaStream_t stream) {
   auto k = gemv_lut_small_kernel<RB8, D, NB>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
+  cudaError_t e = set_func_attr(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
   if (e != cudaSuccess) return e;
   count_launch();
   return launch_pdl(k, p.grid_x, kLutThreads, p.smem, stream, L, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0,
@@ -1073,7 +1076,7 @@ template <int RB8, int D, int B2, int LB>
 cudaError_t launch_lut_pair_set(const LutSet& S, int grid, int smem, const void* x, bool x_fp16, float* ws,
                                 cudaStream_t stream) {
   auto k = gemv_lut_pair_kernel<RB8, D, B2, LB>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = set_func_attr(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   count_launch();
   return launch_pdl(k, grid, kLutThreads, smem, stream, S, static_cast<const uint16_t*>(x), x_fp16 ? 1 : 0, ws,

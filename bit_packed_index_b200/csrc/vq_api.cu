@@ -53,6 +53,36 @@ vq_status cuda_status(cudaError_t e) {
 void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
 int device_sm_count() { return attrs_for_current_device().sms; }
+
+cudaError_t set_func_attr(const void* func, cudaFuncAttribute attr, int value) {
+  struct Entry {
+    int dev;
+    const void* func;
+    cudaFuncAttribute attr;
+    int value;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& e : done)
+      if (e.dev == dev && e.func == func && e.attr == attr &&
+          (e.value == value || (attr == cudaFuncAttributeMaxDynamicSharedMemorySize && e.value >= value)))
+        return cudaSuccess;
+  }
+  const cudaError_t err = cudaFuncSetAttribute(func, attr, value);
+  if (err != cudaSuccess) return err;
+  std::lock_guard<std::mutex> lock(mu);
+  for (Entry& e : done)
+    if (e.dev == dev && e.func == func && e.attr == attr) {
+      if (attr != cudaFuncAttributeMaxDynamicSharedMemorySize || value > e.value) e.value = value;
+      return cudaSuccess;
+    }
+  done.push_back({dev, func, attr, value});
+  return cudaSuccess;
+}
 int device_smem_optin() { return attrs_for_current_device().smem_optin; }
 
 vq_status check_layer(const vq_layer_desc* desc, Layer* out) {

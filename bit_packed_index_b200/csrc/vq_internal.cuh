@@ -51,6 +51,9 @@ vq_status gemv_run(const vq_layer_desc* layer, const void* x, vq_dtype x_dtype, 
 vq_status cuda_status(cudaError_t e);  // records e, returns VQ_ERR_CUDA (or VQ_OK)
 void count_launch(int n = 1);          // adds to the process-wide kernel launch counter
 int device_sm_count();
+// cudaFuncSetAttribute, remembered per (device, kernel, attribute): a call
+// that would not change the value launches nothing and costs a table lookup.
+cudaError_t set_func_attr(const void* func, cudaFuncAttribute attr, int value);
 int device_smem_optin();               // max dynamic shared memory per block, bytes
 
 __host__ __device__ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -79,7 +82,11 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // ---------------------------------------------------------------------------
 // Kernel launchers (one per .cu file).
 // ---------------------------------------------------------------------------
-vq_status launch_dequant(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream);
+// pdl: launched as a programmatic dependent (it reads only the layer, so it
+// may overlap the kernel before it; that kernel must not read w).
+vq_status launch_dequant(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream, bool pdl = false);
+// Rows n0 .. n1-1 of L as a layer of their own (n0 a multiple of 32).
+Layer layer_rows(const Layer& L, int n0, int n1);
 // y of a layer without inputs (Kin = 0): its output bias, else zeros (gemv.cu).
 vq_status launch_empty_rows(const Layer& L, void* y, vq_dtype yt, int64_t ldy, int rows,
                             cudaStream_t stream);
@@ -87,7 +94,7 @@ vq_status launch_empty_rows(const Layer& L, void* y, vq_dtype yt, int64_t ldy, i
 // Tiled index order (tile4.cu).
 vq_status launch_repack_tile4(const Layer& src, uint32_t* const dst[2], const int64_t tile_words[2],
                               cudaStream_t stream);
-vq_status launch_dequant_tile4(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream);
+vq_status launch_dequant_tile4(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t stream, bool pdl = false);
 
 struct GemvPlan {
   int bt;        // batch tile (power of two >= batch)
