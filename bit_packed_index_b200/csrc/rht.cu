@@ -16,10 +16,14 @@
 #include <algorithm>
 #include <cmath>
 
+#include <cooperative_groups.h>
+
 #include "vq_internal.cuh"
 
 namespace vqk {
 namespace {
+
+namespace cg = cooperative_groups;
 
 constexpr int kRhtMaxBlock = 32768;
 
@@ -144,10 +148,121 @@ __global__ void __launch_bounds__(1024) rht_big_kernel(const void* __restrict__ 
   }
 }
 
+// Blocks of b = 1024 C (C = 2, 4 or 8): a cluster of C CTAs transforms one
+// block, 1024 elements per CTA (128 threads x 8).  Stages h < 1024 run
+// inside each CTA as in rht_big_kernel (registers, shuffles, two through
+// shared memory); the last log2(C) stages pair CTA r with CTA r ^ (h / 1024)
+// and read the partner's elements through distributed shared memory, from a
+// second buffer so no CTA overwrites what its partner still reads.  One
+// thread block per Hadamard block leaves one SM to do all the work at batch 1
+// (8192 elements: 10.6 us); the cluster spreads it over C SMs.
+constexpr int kRhtClThreads = 128;
+constexpr int kRhtClElems = 1024;
+
+template <int C>
+__global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kRhtClThreads)
+    rht_cluster_kernel(const void* __restrict__ in, int in_t, int64_t ld_in, const uint32_t* __restrict__ signs,
+                       int inverse, float scale, void* __restrict__ out, int out_t, int64_t ld_out,
+                       const uint16_t* __restrict__ add) {
+  constexpr int E = 8;
+  __shared__ float hv[2][kRhtClElems];
+  asm volatile("griddepcontrol.wait;" ::: "memory");      // as rht_kernel
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int t = threadIdx.x;
+  const int64_t row = blockIdx.y;
+  const int64_t k0 = static_cast<int64_t>(blockIdx.x / C) * (C * kRhtClElems) + static_cast<int64_t>(rank) * kRhtClElems;
+  const int64_t base = k0 + static_cast<int64_t>(t) * E;
+  float v[E];
+#pragma unroll
+  for (int r = 0; r < E; ++r) {
+    v[r] = rht_load(in, in_t, row * ld_in + base + r);
+    if (!inverse) v[r] *= rht_sign(signs, base + r);
+  }
+#pragma unroll
+  for (int h = 1; h < E; h <<= 1) {
+#pragma unroll
+    for (int r = 0; r < E; ++r) {
+      if ((r & h) == 0) {
+        const float a = v[r], c = v[r + h];
+        v[r] = a + c;
+        v[r + h] = a - c;
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {                 // h = 8 .. 128
+    const bool upper = (t & m) != 0;
+#pragma unroll
+    for (int r = 0; r < E; ++r) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[r], m);
+      v[r] = upper ? o - v[r] : v[r] + o;
+    }
+  }
+  // h = 256 and 512 through shared memory (element i at hv[0][i])
+#pragma unroll
+  for (int r = 0; r < E; ++r) hv[0][t * E + r] = v[r];
+  __syncthreads();
+#pragma unroll
+  for (int lh = 8; lh < 10; ++lh) {
+    const int h = 1 << lh;
+#pragma unroll
+    for (int q = 0; q < kRhtClElems / 2 / kRhtClThreads; ++q) {
+      const int p = t + q * kRhtClThreads;
+      const int i = ((p >> lh) << (lh + 1)) | (p & (h - 1));
+      const float a = hv[0][i], c = hv[0][i + h];
+      hv[0][i] = a + c;
+      hv[0][i + h] = a - c;
+    }
+    __syncthreads();
+  }
+  // h = 1024 C' for C' < C: across the cluster
+  int cur = 0;
+#pragma unroll
+  for (int q = 1; q < C; q <<= 1) {
+    cluster.sync();                                   // every CTA's buffer `cur` is complete
+    const float* peer = cluster.map_shared_rank(&hv[cur][0], rank ^ q);
+    const bool upper = (rank & q) != 0;
+#pragma unroll
+    for (int r = 0; r < E; ++r) {
+      const int i = t * E + r;
+      const float mine = hv[cur][i], other = peer[i];
+      hv[cur ^ 1][i] = upper ? other - mine : mine + other;
+    }
+    cur ^= 1;
+  }
+  cluster.sync();                                     // no CTA exits while a peer still reads it
+#pragma unroll
+  for (int r = 0; r < E; ++r) {
+    float y = hv[cur][t * E + r] * scale;
+    if (inverse) y *= rht_sign(signs, base + r);
+    y += out_bias_of(add, static_cast<int>(base + r));
+    store_out(out, static_cast<vq_dtype>(out_t), row * ld_out + base + r, y);
+  }
+}
+
+template <int C>
+cudaError_t launch_rht_cluster(const void* in, vq_dtype in_t, int rows, int n, int64_t ld_in,
+                               const uint32_t* signs, bool inverse, void* out, vq_dtype out_t, int64_t ld_out,
+                               cudaStream_t stream, const uint16_t* add) {
+  const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(C * kRhtClElems)));
+  count_launch();
+  return launch_pdl(rht_cluster_kernel<C>, dim3(n / kRhtClElems, rows), kRhtClThreads, 0, stream, in,
+                    static_cast<int>(in_t), ld_in, signs, inverse ? 1 : 0, scale, out, static_cast<int>(out_t),
+                    ld_out, add);
+}
+
 cudaError_t launch_rht(const void* in, vq_dtype in_t, int rows, int n, int64_t ld_in, const uint32_t* signs,
                        bool inverse, void* out, vq_dtype out_t, int64_t ld_out, cudaStream_t stream,
                        const uint16_t* add = nullptr) {
   const int b = rht_block(n);
+  // Few rows: spread each block over a cluster (rows * n / 1024 CTAs)
+  if (rows <= 16 && (b == 2048 || b == 4096 || b == 8192)) {
+    if (b == 2048) return launch_rht_cluster<2>(in, in_t, rows, n, ld_in, signs, inverse, out, out_t, ld_out, stream, add);
+    if (b == 4096) return launch_rht_cluster<4>(in, in_t, rows, n, ld_in, signs, inverse, out, out_t, ld_out, stream, add);
+    return launch_rht_cluster<8>(in, in_t, rows, n, ld_in, signs, inverse, out, out_t, ld_out, stream, add);
+  }
   if (b >= 256) {
     const int T = std::min(1024, b / 8), E = b / T;
     const int smem = 32 * E < b ? b * static_cast<int>(sizeof(float)) : 0;

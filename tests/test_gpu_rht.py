@@ -37,7 +37,7 @@ def _rand(rows, n, dtype, seed):
     return x, x.double().cpu().numpy()
 
 
-@pytest.mark.parametrize("n", [1, 6, 24, 96, 1000, 8192, 28672, 65536])
+@pytest.mark.parametrize("n", [1, 6, 24, 96, 1000, 6144, 8192, 28672, 65536])
 @pytest.mark.parametrize("dtype", ["bf16", "fp16", "fp32"])
 def test_rht_matches_the_oracle(n, dtype):
     vq = _vq()
