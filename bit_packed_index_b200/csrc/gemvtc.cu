@@ -85,6 +85,7 @@ struct TcArgs {
   int* status;
   long long budget;
   int tiles, nitems;      // small-book kernel: work items (row tile, split), split-major
+  int xs;                 // small-book kernel: slots of the x ring
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -297,12 +298,13 @@ constexpr int kTsTmemCols = 2 * 16 * kTsNacc < 32 ? 32 : 2 * 16 * kTsNacc;
 #endif
 constexpr int kTsPf = VQ_TS_PF;                  // steps of index words a producer keeps in flight
 constexpr int kTsMaxEntries = 8192;              // K1 + K2 staged (128 KB)
-#ifndef VQ_TS_XS
-#define VQ_TS_XS 8
-#endif
-constexpr int kTsXs = VQ_TS_XS;                  // x tiles in flight (their own ring, deeper than the A ring)
-constexpr int kTsFixed = 2048 + kTcStages * kTcATile + kTsXs * kTcXTile;   // control, slack, A ring, x ring
-static_assert(kTsXs >= 2 && kTsXs <= 16, "x ring of 2..16 tiles");
+// The x ring: per slot the step's x tile (2 KB) and, in the tiled order,
+// the step's index records of the CTA's 128 rows (two tiles of each book,
+// 64 b bytes per tile and book: at most 3 KB), brought in by bulk copies on
+// the same barrier.  As many slots as shared memory leaves, 4..12.
+constexpr int kTsSlot = 5 * 1024;
+constexpr int kTsXsMin = 4, kTsXsMax = 12;
+constexpr int kTsFixed = 2048 + kTcStages * kTcATile;   // control, slack, A ring; x ring and books follow
 
 // Words holding the TsShape<LAYOUT>::vpt fields of book m for vectors 8 kt + TsShape<LAYOUT>::vpt p ..
 // of row o, and the bit position of the first (fields are b bits, LSB
@@ -358,10 +360,13 @@ __global__ void __launch_bounds__(TsShape<LAYOUT>::threads, 1) gemv_tcs_kernel(c
   uint8_t* base = align1024(smem_raw);
   TcCtrl* ctrl = reinterpret_cast<TcCtrl*>(base);
   uint8_t* stages = base + 1024;
-  uint8_t* xring = stages + kTcStages * kTcATile;   // kTsXs x tiles
-  uint8_t* books = xring + kTsXs * kTcXTile;        // [K1][16 B], then [K2][16 B]
+  uint8_t* xring = stages + kTcStages * kTcATile;   // g.xs slots of kTsSlot bytes
+  uint8_t* books = xring + g.xs * kTsSlot;          // [K1][16 B], then [K2][16 B]
+  const int xs = g.xs;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Layer& L = g.L;
+  // index records of a slot (tiled order): book 1 tiles 0 and 1, then book 2's
+  const int rb1 = 64 * L.b[0], rb2 = L.nb == 2 ? 64 * L.b[1] : 0;
   volatile int* abort_flag = &ctrl->abort;
   const int k1 = 1 << L.b[0];
   const int k2 = L.nb == 2 ? 1 << L.b[1] : 0;
@@ -377,7 +382,7 @@ __global__ void __launch_bounds__(TsShape<LAYOUT>::threads, 1) gemv_tcs_kernel(c
       mbar_init(&ctrl->accf[b], 1);
       mbar_init(&ctrl->acce[b], 4);              // the four epilogue warps
     }
-    for (int q = 0; q < kTsXs; ++q) {
+    for (int q = 0; q < xs; ++q) {
       mbar_init(&ctrl->xf[q], 1);
       mbar_init(&ctrl->xe[q], 1);
     }
@@ -416,20 +421,49 @@ __global__ void __launch_bounds__(TsShape<LAYOUT>::threads, 1) gemv_tcs_kernel(c
       for (int item = blockIdx.x; item < g.nitems && !stop; item += gridDim.x) {
         const int kt0 = (item / g.tiles) * g.kt_per_split;
         const int nkt = min(g.num_kt, kt0 + g.kt_per_split) - kt0;
+        const int row0 = (item % g.tiles) * kTcRows;
         for (int i = 0; i < nkt; ++i, ++gs) {
-          const int q = gs % kTsXs;
-          const uint32_t ph = (gs / kTsXs) & 1;
+          const int q = gs % xs;
+          const uint32_t ph = (gs / xs) & 1;
           if (!bounded_wait(&ctrl->xe[q], ph ^ 1, abort_flag, g.status, g.budget)) {
             stop = true;
             break;
           }
-          mbar_arrive_expect_tx(&ctrl->xf[q], kTcXTile);
-          tma_load_2d(xring + q * kTcXTile, &xmap, &ctrl->xf[q], (kt0 + i) * kTcK, 0);
+          uint8_t* slot = xring + q * kTsSlot;
+          // the records of tiles 2 kt and 2 kt + 1 for rows row0 .. row0+127
+          // (fewer bytes at the end of a tile; none past the last tile)
+          uint32_t bytes[2][2] = {{0u, 0u}, {0u, 0u}};
+          const uint32_t* src[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+          if (LAYOUT == VQ_IDX_TILE4) {
+            const int ntile = (L.nvec + 3) / 4;
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+              if (m >= L.nb) break;
+              const int64_t off = static_cast<int64_t>(row0) * L.b[m] / 8;   // words before row0's record
+              const int64_t avail = (L.rw[m] - off) * 4;
+#pragma unroll
+              for (int tt = 0; tt < 2; ++tt) {
+                const int t = 2 * (kt0 + i) + tt;
+                if (t >= ntile) continue;
+                bytes[m][tt] = static_cast<uint32_t>(avail < 64 * L.b[m] ? avail : 64 * L.b[m]);
+                src[m][tt] = L.idx[m] + static_cast<int64_t>(t) * L.rw[m] + off;
+              }
+            }
+          }
+          mbar_arrive_expect_tx(&ctrl->xf[q], kTcXTile + bytes[0][0] + bytes[0][1] + bytes[1][0] + bytes[1][1]);
+          tma_load_2d(slot, &xmap, &ctrl->xf[q], (kt0 + i) * kTcK, 0);
+#pragma unroll
+          for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt)
+              if (bytes[m][tt])
+                bulk_load(slot + kTcXTile + (m == 0 ? tt * rb1 : 2 * rb1 + tt * rb2), src[m][tt], bytes[m][tt],
+                          &ctrl->xf[q]);
         }
       }
       if (*abort_flag) {   // let loads already in flight land before the block exits
-        for (int i = max(0, gs - kTsXs); i < gs; ++i)
-          drain_phase(&ctrl->xf[i % kTsXs], (i / kTsXs) & 1, 4000000000LL);
+        for (int i = max(0, gs - xs); i < gs; ++i)
+          drain_phase(&ctrl->xf[i % xs], (i / xs) & 1, 4000000000LL);
       }
     }
   } else if (warp == 1) {
@@ -448,15 +482,15 @@ __global__ void __launch_bounds__(TsShape<LAYOUT>::threads, 1) gemv_tcs_kernel(c
         for (int i = 0; i < nkt; ++i, ++gs) {
           const int s = gs % kTcStages;
           const uint32_t ph = (gs / kTcStages) & 1;
-          const int xq = gs % kTsXs;
+          const int xq = gs % xs;
           if (!bounded_wait(&ctrl->full[s], ph, abort_flag, g.status, g.budget) ||
-              !bounded_wait(&ctrl->xf[xq], (gs / kTsXs) & 1, abort_flag, g.status, g.budget)) {
+              !bounded_wait(&ctrl->xf[xq], (gs / xs) & 1, abort_flag, g.status, g.budget)) {
             stop = true;
             break;
           }
           tc_fence_after();
           const uint32_t a = smem_addr(stages + s * kTcATile);
-          const uint32_t b = smem_addr(xring + xq * kTcXTile);
+          const uint32_t b = smem_addr(xring + xq * kTsSlot);
           // consecutive products go to different accumulators, so none waits
           // for the previous one to finish accumulating
 #pragma unroll
@@ -492,44 +526,80 @@ __global__ void __launch_bounds__(TsShape<LAYOUT>::threads, 1) gemv_tcs_kernel(c
       const int kt0 = split * g.kt_per_split;
       const int nkt = min(g.num_kt, kt0 + g.kt_per_split) - kt0;
       const int64_t o = min(row0 + r, L.n - 1);
-      // index words of the next kTsPf steps in flight (a register window
-      // that slides by one step per iteration)
-      uint32_t pw[kTsPf][2][3];
-      int psh[kTsPf][2];
+      // Row order: index words of the next kTsPf steps in flight in
+      // registers (a window that slides by one step per iteration).  Tiled
+      // order: the step's records arrive with x in the x ring (bulk copies).
+      constexpr bool kRec = LAYOUT == VQ_IDX_TILE4;
+      constexpr int PF = kRec ? 1 : kTsPf;
+      constexpr int VPT = TsShape<LAYOUT>::vpt;
+      uint32_t pw[PF][2][3];
+      int psh[PF][2];
 #pragma unroll
-      for (int q = 0; q < kTsPf; ++q) {
+      for (int q = 0; q < PF; ++q) {
+        pw[q][0][0] = pw[q][0][1] = pw[q][0][2] = 0u;
         pw[q][1][0] = pw[q][1][1] = pw[q][1][2] = 0u;
-        psh[q][1] = 0;
-        if (q < nkt) {
+        psh[q][0] = psh[q][1] = 0;
+        if (!kRec && q < nkt) {
           tcs_words<LAYOUT>(L, 0, o, kt0 + q, p, pw[q][0], psh[q][0]);
           if (L.nb == 2) tcs_words<LAYOUT>(L, 1, o, kt0 + q, p, pw[q][1], psh[q][1]);
-        } else {
-          pw[q][0][0] = pw[q][0][1] = pw[q][0][2] = 0u;
-          psh[q][0] = 0;
         }
       }
       for (int i = 0; i < nkt; ++i, ++gs) {
         const int s = gs % kTcStages;
         const uint32_t ph = (gs / kTcStages) & 1;
-        uint32_t f1[TsShape<LAYOUT>::vpt], f2[TsShape<LAYOUT>::vpt];
-#pragma unroll
-        for (int v = 0; v < TsShape<LAYOUT>::vpt; ++v) {
-          f1[v] = tcs_field(pw[0][0], psh[0][0] + v * b1, m1);
-          f2[v] = L.nb == 2 ? tcs_field(pw[0][1], psh[0][1] + v * b2, m2) : 0u;
-        }
-#pragma unroll
-        for (int q = 0; q + 1 < kTsPf; ++q) {
+        uint32_t f1[VPT], f2[VPT];
+        if constexpr (kRec) {
+          const int q = gs % xs;
+          if (!__all_sync(0xffffffffu, bounded_wait(&ctrl->xf[q], (gs / xs) & 1, abort_flag, g.status, g.budget))) {
+            stop = true;
+            break;
+          }
+          // this thread's VPT fields of row r: tile (VPT p) / 4 of the step,
+          // starting at field (VPT p) % 4 of the row's record
+          const uint8_t* slot = xring + q * kTsSlot + kTcXTile;
+          const int tt = (VPT * p) >> 2, f0 = (VPT * p) & 3;
 #pragma unroll
           for (int m = 0; m < 2; ++m) {
-            pw[q][m][0] = pw[q + 1][m][0];
-            pw[q][m][1] = pw[q + 1][m][1];
-            pw[q][m][2] = pw[q + 1][m][2];
-            psh[q][m] = psh[q + 1][m];
+            if (m == 1 && L.nb != 2) break;
+            const int bm = m == 0 ? b1 : b2;
+            const uint32_t* rec =
+                reinterpret_cast<const uint32_t*>(slot + (m == 0 ? tt * rb1 : 2 * rb1 + tt * rb2));
+            const int bit = r * 4 * bm + f0 * bm;
+            uint32_t w3[3];
+            w3[0] = rec[bit >> 5];
+            w3[1] = (bit & 31) + VPT * bm > 32 ? rec[(bit >> 5) + 1] : 0u;
+            w3[2] = 0u;
+#pragma unroll
+            for (int v = 0; v < VPT; ++v) {
+              const uint32_t f = tcs_field(w3, (bit & 31) + v * bm, m == 0 ? m1 : m2);
+              if (m == 0) f1[v] = f;
+              else f2[v] = f;
+            }
           }
-        }
-        if (i + kTsPf < nkt) {
-          tcs_words<LAYOUT>(L, 0, o, kt0 + i + kTsPf, p, pw[kTsPf - 1][0], psh[kTsPf - 1][0]);
-          if (L.nb == 2) tcs_words<LAYOUT>(L, 1, o, kt0 + i + kTsPf, p, pw[kTsPf - 1][1], psh[kTsPf - 1][1]);
+          if (L.nb != 2) {
+#pragma unroll
+            for (int v = 0; v < VPT; ++v) f2[v] = 0u;
+          }
+        } else {
+#pragma unroll
+          for (int v = 0; v < VPT; ++v) {
+            f1[v] = tcs_field(pw[0][0], psh[0][0] + v * b1, m1);
+            f2[v] = L.nb == 2 ? tcs_field(pw[0][1], psh[0][1] + v * b2, m2) : 0u;
+          }
+#pragma unroll
+          for (int q = 0; q + 1 < PF; ++q) {
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+              pw[q][m][0] = pw[q + 1][m][0];
+              pw[q][m][1] = pw[q + 1][m][1];
+              pw[q][m][2] = pw[q + 1][m][2];
+              psh[q][m] = psh[q + 1][m];
+            }
+          }
+          if (i + PF < nkt) {
+            tcs_words<LAYOUT>(L, 0, o, kt0 + i + PF, p, pw[PF - 1][0], psh[PF - 1][0]);
+            if (L.nb == 2) tcs_words<LAYOUT>(L, 1, o, kt0 + i + PF, p, pw[PF - 1][1], psh[PF - 1][1]);
+          }
         }
         uint4 c[TsShape<LAYOUT>::vpt];
 #pragma unroll
@@ -765,7 +835,16 @@ bool tcs_supported(const Layer& L) {
   if (!(L.d == 6 || L.d == 8) || L.b[0] > 12 || (L.nb == 2 && L.b[1] > 12)) return false;
   return (1 << L.b[0]) + (L.nb == 2 ? 1 << L.b[1] : 0) <= kTsMaxEntries;
 }
-int tcs_smem(const Layer& L) { return kTsFixed + ((1 << L.b[0]) + (L.nb == 2 ? 1 << L.b[1] : 0)) * 16; }
+// x-ring slots that fit beside the books (0 when fewer than kTsXsMin do).
+int tcs_slots(const Layer& L) {
+  const int books = ((1 << L.b[0]) + (L.nb == 2 ? 1 << L.b[1] : 0)) * 16;
+  const int room = device_smem_optin() - kTsFixed - books;
+  const int xs = std::min(kTsXsMax, room / kTsSlot);
+  return xs >= kTsXsMin ? xs : 0;
+}
+int tcs_smem(const Layer& L) {
+  return kTsFixed + tcs_slots(L) * kTsSlot + ((1 << L.b[0]) + (L.nb == 2 ? 1 << L.b[1] : 0)) * 16;
+}
 
 long long tc_wait_budget() {
   if (const char* env = std::getenv("VQ_WAIT_BUDGET")) return std::atoll(env);
@@ -777,7 +856,7 @@ long long tc_wait_budget() {
 bool plan_gemv_tc(const Layer& L, int batch, size_t ws_cap, GemvPlan* p) {
   if (!(L.layout == VQ_IDX_ROWS || L.layout == VQ_IDX_TILE4) || L.n < 1 || L.nvec < 1 || batch > kTcN) return false;
   const bool big = L.nb == 1 && L.d == 8 && L.b[0] == 16;
-  const bool small = !big && tcs_supported(L);
+  const bool small = !big && tcs_supported(L) && tcs_slots(L) > 0;
   if (!big && !small) return false;
   if (batch < std::max(1, big ? tc_min_batch() : tcs_min_batch())) return false;
   const int smem = big ? kTcSmem : tcs_smem(L);
@@ -834,6 +913,7 @@ vq_status launch_gemv_tc(const Layer& L, const GemvPlan& p, const void* x, bool 
     return cuda_status(e);
   g.tiles = t.tiles;
   g.nitems = t.tiles * t.nsplit;
+  g.xs = small ? tcs_slots(L) : 0;
   const dim3 grid = small ? dim3(std::min(g.nitems, device_sm_count())) : dim3(t.tiles, t.nsplit);
   count_launch();
   k<<<grid, threads, p.smem, stream>>>(xmap, g);

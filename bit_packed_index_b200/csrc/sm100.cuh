@@ -111,6 +111,16 @@ __device__ __forceinline__ void tma_prefetch(const CUtensorMap* map) {
 
 // 2-D tiled TMA load (no multicast) of box {x .. x+bx, y .. y+by} into dst,
 // completing `bytes` on bar.  x * element size must be a multiple of 16 bytes.
+// Plain bulk copy global -> shared (no multicast), `bytes` a multiple of 16
+// and both addresses 16-byte aligned, completing on bar's transaction count.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int x, int y) {
   asm volatile(
