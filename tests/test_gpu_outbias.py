@@ -162,14 +162,16 @@ def _signs(n, seed):
 
 
 @pytest.mark.parametrize("layout", ["rows", "tile4"])
-def test_gemv_rht_output_bias_lands_on_y(layout):
-    """y = U^T (W~ (V x)) + b_out: the bias is not rotated."""
+@pytest.mark.parametrize("batch", [1, 3])
+def test_gemv_rht_output_bias_lands_on_y(layout, batch):
+    """y = U^T (W~ (V x)) + b_out: the bias is not rotated (batch 1 in the
+    tiled order builds x~ inside the table kernel)."""
     vq = _vq()
     spec = LayerSpec(1024, 8 * 128, 8, (16,), (0.02,))
     data, with_b, _ = _pair(spec, 990, layout)
     s_in, d_in = _signs(spec.in_features, 991)
     s_out, d_out = _signs(spec.out_features, 992)
-    x = synth.make_x(993, 3, spec.in_features)
+    x = synth.make_x(993, batch, spec.in_features)
     w = oracle.f16_to_f32(oracle.dequant(data)).astype(np.float64)
     xt = oracle.rht(oracle.bf16_to_f32(x).astype(np.float64), s_in)
     ref = oracle.rht(xt @ w.T, s_out, inverse=True)
