@@ -550,7 +550,14 @@ __device__ __forceinline__ uint64_t load_record(const uint32_t* __restrict__ til
   return r;
 }
 
-// Table of one book for the task's four vectors: T[k][4] = <x'_j, C[k]>.
+// Table of one book for the task's four vectors: T[k][j] = <x'_j, C[k]>, in
+// two planes of K 4-byte words (plane p, word k: T[k][2p], T[k][2p+1]) that
+// start small_plane(K) halves apart.  A lookup instruction's lanes (one j,
+// random k) then spread over all 32 banks -- one 8-byte row T[k][0..3] per
+// centroid would put a given j in only 16 of them -- and a warp's stores
+// (8 consecutive words in each plane) hit 16 distinct banks.
+__device__ __forceinline__ int small_plane(int K) { return 2 * K + 32; }
+
 template <int D>
 __device__ __forceinline__ void build_small_table(const uint16_t* __restrict__ book, int K, uint32_t bfrag,
                                                   uint16_t* __restrict__ tab, int warp, int lane) {
@@ -577,8 +584,9 @@ __device__ __forceinline__ void build_small_table(const uint16_t* __restrict__ b
         : "r"(a[i][0]), "r"(a[i][1]), "r"(bfrag), "f"(0.0f), "f"(0.0f), "f"(0.0f), "f"(0.0f));
     const int r0 = tile * 16 + g;
     if (t < 2) {
-      if (r0 < K) *reinterpret_cast<__half2*>(tab + r0 * 4 + 2 * t) = __floats2half2_rn(d0, d1);
-      if (r0 + 8 < K) *reinterpret_cast<__half2*>(tab + (r0 + 8) * 4 + 2 * t) = __floats2half2_rn(d2, d3);
+      uint16_t* plane = tab + t * small_plane(K);
+      if (r0 < K) *reinterpret_cast<__half2*>(plane + r0 * 2) = __floats2half2_rn(d0, d1);
+      if (r0 + 8 < K) *reinterpret_cast<__half2*>(plane + (r0 + 8) * 2) = __floats2half2_rn(d2, d3);
     }
   }
 }
@@ -632,8 +640,8 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_small_kernel(Layer L,
   constexpr int TCOLS = 8 * CPW;
   extern __shared__ __align__(128) uint8_t smem[];
   const int K1 = 1 << L.b[0], K2 = NB == 2 ? (1 << L.b[1]) : 0;
-  uint16_t* tab1 = reinterpret_cast<uint16_t*>(smem);   // T1[K1][4]
-  uint16_t* tab2 = tab1 + K1 * 4;                        // T2[K2][4]
+  uint16_t* tab1 = reinterpret_cast<uint16_t*>(smem);   // T1, two planes
+  uint16_t* tab2 = tab1 + 2 * small_plane(K1);           // T2, two planes
   __shared__ uint32_t s_tmem;
   __shared__ float s_scale;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -719,8 +727,12 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_small_kernel(Layer L,
           float v = 0.0f;
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj) {
-            float u = h2f(tab1[(static_cast<uint32_t>(rec1[r] >> (jj * b1)) & m1) * 4 + jj]);
-            if constexpr (NB == 2) u += h2f(tab2[(static_cast<uint32_t>(rec2[r] >> (jj * b2)) & m2) * 4 + jj]);
+            const uint16_t* p1 = tab1 + (jj >> 1) * small_plane(K1) + (jj & 1);
+            float u = h2f(p1[(static_cast<uint32_t>(rec1[r] >> (jj * b1)) & m1) * 2]);
+            if constexpr (NB == 2) {
+              const uint16_t* p2 = tab2 + (jj >> 1) * small_plane(K2) + (jj & 1);
+              u += h2f(p2[(static_cast<uint32_t>(rec2[r] >> (jj * b2)) & m2) * 2]);
+            }
             v += u;
           }
           acc[r] = fmaf(v, sc, acc[r]);
@@ -1115,11 +1127,11 @@ cudaError_t launch_lut_small(const Layer& L, const GemvPlan& p, const void* x, b
                          stream);
 }
 
-// Tables of the small-book kernels: fp16 [K][4] per book, or fp32 [4][K] on
-// the paired-row path.
+// Tables of the small-book kernels: fp16 [K][4] per book in two padded
+// planes (small_plane), or fp32 [4][K] on the paired-row path.
 size_t lut_small_smem(const Layer& L) {
   const size_t k = (static_cast<size_t>(1) << L.b[0]) + (L.nb == 2 ? (static_cast<size_t>(1) << L.b[1]) : 0);
-  return k * 4 * (lut_pair_path(L) ? 4 : 2);
+  return lut_pair_path(L) ? k * 4 * 4 : k * 4 * 2 + 2 * 128;
 }
 
 bool lut_small_supported(const Layer& L) {
