@@ -122,15 +122,20 @@ __global__ void __launch_bounds__(kDqThreads) dequant_kernel(Layer L, uint16_t* 
   }
 }
 
+// One wave of persistent blocks: as many as the SMs hold at once (registers
+// bound this kernel: 40-44 per thread leave room for 5-6 blocks of 256, not
+// 8), at most one per row.
 template <int D, int NB>
 cudaError_t launch_dq(const Layer& L, uint16_t* w, int64_t ldw, int smem_mask, size_t smem,
-                      int vec_store, int grid, cudaStream_t stream, bool pdl) {
+                      int vec_store, cudaStream_t stream, bool pdl) {
   auto k = dequant_kernel<D, NB>;
   if (smem > 48 * 1024) {
     cudaError_t e = set_func_attr(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
+  const int per_sm = std::min(8, resident_blocks_per_sm(reinterpret_cast<const void*>(k), kDqThreads, smem));
+  const int grid = static_cast<int>(std::min<int64_t>(L.n, static_cast<int64_t>(device_sm_count()) * per_sm));
   count_launch();
   if (pdl) return launch_pdl(k, grid, kDqThreads, smem, stream, L, w, ldw, smem_mask, vec_store);
   k<<<grid, kDqThreads, smem, stream>>>(L, w, ldw, smem_mask, vec_store);
@@ -145,18 +150,16 @@ vq_status launch_dequant(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t 
   int smem_mask = 0;
   const size_t smem = stage_plan(L, std::min<size_t>(kDqSmemBooks, device_smem_optin()), &smem_mask);
   const int vec_store = aligned(w, 16) && (ldw % 8 == 0);
-  const int per_sm = smem ? std::max(1, std::min(8, static_cast<int>((228 * 1024) / (smem + 1024)))) : 8;
-  const int grid = static_cast<int>(std::min<int64_t>(L.n, static_cast<int64_t>(device_sm_count()) * per_sm));
   cudaError_t e;
   const int D = (L.d == 8) ? 8 : (L.d == 6 ? 6 : 0);
   if (L.nb == 1) {
-    e = D == 8 ? launch_dq<8, 1>(L, w, ldw, smem_mask, smem, vec_store, grid, stream, pdl)
-      : D == 6 ? launch_dq<6, 1>(L, w, ldw, smem_mask, smem, vec_store, grid, stream, pdl)
-               : launch_dq<0, 1>(L, w, ldw, smem_mask, smem, vec_store, grid, stream, pdl);
+    e = D == 8 ? launch_dq<8, 1>(L, w, ldw, smem_mask, smem, vec_store, stream, pdl)
+      : D == 6 ? launch_dq<6, 1>(L, w, ldw, smem_mask, smem, vec_store, stream, pdl)
+               : launch_dq<0, 1>(L, w, ldw, smem_mask, smem, vec_store, stream, pdl);
   } else {
-    e = D == 8 ? launch_dq<8, 2>(L, w, ldw, smem_mask, smem, vec_store, grid, stream, pdl)
-      : D == 6 ? launch_dq<6, 2>(L, w, ldw, smem_mask, smem, vec_store, grid, stream, pdl)
-               : launch_dq<0, 2>(L, w, ldw, smem_mask, smem, vec_store, grid, stream, pdl);
+    e = D == 8 ? launch_dq<8, 2>(L, w, ldw, smem_mask, smem, vec_store, stream, pdl)
+      : D == 6 ? launch_dq<6, 2>(L, w, ldw, smem_mask, smem, vec_store, stream, pdl)
+               : launch_dq<0, 2>(L, w, ldw, smem_mask, smem, vec_store, stream, pdl);
   }
   return cuda_status(e);
 }

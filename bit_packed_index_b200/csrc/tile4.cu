@@ -173,7 +173,8 @@ cudaError_t launch_dq4(const Layer& L, uint16_t* w, int64_t ldw, cudaStream_t st
     cudaError_t e = set_func_attr(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  const int per_sm = smem ? std::max(1, std::min(8, static_cast<int>((228 * 1024) / (smem + 1024)))) : 8;
+  // one wave: a grid-stride loop past what the SMs hold runs a partial second wave
+  const int per_sm = std::min(8, resident_blocks_per_sm(reinterpret_cast<const void*>(k), 256, smem));
   const int64_t total = static_cast<int64_t>((((L.nvec + 3) / 4) + 3) / 4) * L.n * 4;
   const int grid = static_cast<int>(std::min<int64_t>((total + 255) / 256,
                                                       static_cast<int64_t>(device_sm_count()) * per_sm));

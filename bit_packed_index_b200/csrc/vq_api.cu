@@ -85,6 +85,34 @@ cudaError_t set_func_attr(const void* func, cudaFuncAttribute attr, int value) {
 }
 int device_smem_optin() { return attrs_for_current_device().smem_optin; }
 
+int resident_blocks_per_sm(const void* func, int threads, size_t smem) {
+  struct Entry {
+    int dev;
+    const void* func;
+    int threads;
+    size_t smem;
+    int blocks;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& e : done)
+      if (e.dev == dev && e.func == func && e.threads == threads && e.smem == smem) return e.blocks;
+  }
+  int blocks = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, func, threads, smem) != cudaSuccess) {
+    cudaGetLastError();   // leave no sticky error for the launch to report
+    blocks = 1;
+  }
+  blocks = std::max(1, blocks);
+  std::lock_guard<std::mutex> lock(mu);
+  done.push_back({dev, func, threads, smem, blocks});
+  return blocks;
+}
+
 vq_status check_layer(const vq_layer_desc* desc, Layer* out) {
   if (!desc || !out) return VQ_ERR_INVALID_ARG;
   const vq_layer_desc& D = *desc;

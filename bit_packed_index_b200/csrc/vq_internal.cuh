@@ -55,6 +55,11 @@ int device_sm_count();
 // that would not change the value launches nothing and costs a table lookup.
 cudaError_t set_func_attr(const void* func, cudaFuncAttribute attr, int value);
 int device_smem_optin();               // max dynamic shared memory per block, bytes
+// Blocks of `func` (threads per block, dynamic shared memory) that one SM
+// holds at once, from the occupancy calculator (registers, shared memory,
+// threads), remembered per (device, kernel, shape); at least 1.  A
+// grid-stride kernel sized past SMs x this runs a partial second wave.
+int resident_blocks_per_sm(const void* func, int threads, size_t smem);
 
 __host__ __device__ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
