@@ -486,15 +486,20 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(LutSet S, cons
         sm100::tmem_ld8(tb, acc);
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
-          float v[kLutNJ];
+          // uniform: no thread has this row (a 28672-row layer's last batch
+          // is half empty; its lookups would be an eighth of the work).  Not
+          // compiled for one-batch layers: the test alone slowed the 8192-row
+          // down_proj by 3 %, which has no such rows.
+          if constexpr (LB > 1)
+            if ((b * 8 + r) * kLutThreads >= n) break;
+          float v = 0.0f;
 #pragma unroll
           for (int jj = 0; jj < kLutNJ; ++jj) {
             const uint32_t k = ((jj < 2 ? w[cur][r].x : w[cur][r].y) >> (16 * (jj & 1))) & 0xFFFFu;
-            v[jj] = 0.0f;
             const uint32_t t = k - static_cast<uint32_t>(s * kLutS);   // wraps when below
-            if (t < static_cast<uint32_t>(kLutS)) v[jj] = h2f(lut[t * kLutNJ + jj]);
+            if (t < static_cast<uint32_t>(kLutS)) v += h2f(lut[t * kLutNJ + jj]);
           }
-          acc[r] = fmaf((v[0] + v[1]) + (v[2] + v[3]), sc, acc[r]);
+          acc[r] = fmaf(v, sc, acc[r]);
         }
         sm100::tmem_st8(tb, acc);
       }
