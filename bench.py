@@ -129,6 +129,42 @@ def alg_bytes(spec, batch: int) -> float:
 
 # -- distributed plumbing (timing only; no collective on the data path) ------
 
+# The lookup-table GEMV's own attainable bound (2^16 book, d = 8, batch 1,
+# tiled order): its two phases run one after the other on every SM.
+#  - Table products: every (group of four vectors, slice) task streams its
+#    slice of the codebook from L2 into the SM, so each layer moves the whole
+#    book once per group; at best at the 31 TB/s that 148 SMs reading one
+#    1 MiB buffer with coalesced 16-byte loads reach (probe; 24 TB/s low end).
+#  - Lookups: every index is examined once per slice (LUT_SLICES), each
+#    examination at least a field extract, the slice subtraction, the range
+#    compare and one shared-memory load (4 instructions) at 4 warp
+#    instructions per clock per SM; the HBM read of the index stream at the
+#    measured copy bandwidth overlaps with it.
+LUT_SLICES = 3
+LUT_L2_TBS = (24.0, 31.0)
+LUT_MIN_INSTR_PER_EXAM = 4
+SM_COUNT = 148
+SM_MAX_GHZ = 1.965
+
+
+def lut_design_bound(specs, peak_hbm_gbs: float) -> dict:
+    """Microseconds the table design cannot beat for one launch over `specs`
+    (layers sharing x, batch 1)."""
+    book_bytes = exams = 0
+    for sp in specs:
+        nvec = -(-sp.in_features // sp.d)
+        groups = -(-nvec // 4)
+        book_bytes += groups * (1 << sp.log2k[0]) * sp.d * 2
+        exams += sp.out_features * nvec * LUT_SLICES
+    a_us = [book_bytes / (tbs * 1e12) * 1e6 for tbs in LUT_L2_TBS]
+    b_issue_us = exams * LUT_MIN_INSTR_PER_EXAM / 32 / (SM_COUNT * 4 * SM_MAX_GHZ * 1e9) * 1e6
+    hbm_us = sum(alg_bytes(sp, 1) for sp in specs) / (peak_hbm_gbs * 1e9) * 1e6
+    b_us = max(b_issue_us, hbm_us)
+    return {"bound_us": a_us[1] + b_us, "bound_us_at_24tbs": a_us[0] + b_us,
+            "codebook_l2_bytes": book_bytes, "table_phase_us": a_us[1],
+            "slice_examinations": exams, "lookup_phase_issue_us": b_issue_us, "hbm_us": hbm_us}
+
+
 def dist_env():
     return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
             int(os.environ.get("LOCAL_RANK", "0")))
@@ -381,6 +417,7 @@ def run_gpu(args):
     gu_bytes = alg_bytes(specs[0], BATCH) + alg_bytes(specs[1], BATCH)
     achieved = gu_bytes / (call_ms[0] * 1e-3) / 1e9
     rec = profiled_traffic("gemv_lut_kernel")
+    lut_bound = lut_design_bound(specs[:2], peaks["hbm_gbs"])
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"],
                 "traffic": rec["dram_bytes_per_launch"] if rec else None,
@@ -392,9 +429,14 @@ def run_gpu(args):
                 "per_call_us": {"gate_proj+up_proj": call_ms[0] * 1e3, "down_proj": call_ms[1] * 1e3},
                 "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                 "row_order_gather_ceiling_us": 120.0,
+                "design_bound": dict(lut_bound, frac=lut_bound["bound_us"] / (call_ms[0] * 1e3)),
                 "note": "not HBM-bound: the table kernel is bound by instruction issue and "
                         "shared-memory lookups (3 slice tests per index), the row-order kernel "
-                        "by random 16-byte centroid gathers through L1/L2 (0.84/clk/SM)"}
+                        "by random 16-byte centroid gathers through L1/L2 (0.84/clk/SM); "
+                        "design_bound: the table design's own floor (codebook slices streamed "
+                        "from L2 at 31 TB/s, then 4 instructions per slice examination of an "
+                        "index or the HBM read, whichever is longer) and the fraction of it "
+                        "the measured call reaches"}
 
     # e2e through the public API with pinned host activations and outputs:
     # each step copies all three layers' inputs to the device in one transfer,
